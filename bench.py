@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Throughput of the FLARE++ mixer forward on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one full forward call (synthesis, gate, encode, decode: every
+launch of the hot path) over one batch of the workload's synthetic inputs,
+already resident in HBM.  The default workload is the 1M-token scaling case
+(B=1, H=8, N=1048576, M=512, D=64, bf16); its inputs (1 GiB per [B,H,N,D]
+tensor) are larger than the 126 MB L2, so steps run back to back.  Smaller
+workloads get an L2 flush (a 512 MiB write) between steps and the step times
+are summed.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+problem of the same size (weak scaling, no collective on the data path); the
+timed region is bracketed by a barrier and a device synchronise, the elapsed
+device time is the maximum over ranks, and ``value`` counts the tokens of all
+ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FLARE++ mixer fwd Mtokens/s on 1 B200 + % of roofline (HBM GB/s or TFLOP/s)"
+UNIT = "Mtokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES_GATED = ["split_partial(synthesis)", "merge(q)", "split_partial(encode)", "merge(z)", "decode"]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="scale1m_bf16")
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- ranks
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own problem (independent batches: weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity on one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_mtokens(tokens_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: tokens processed by all ranks over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (max_ms * 1e-3) / 1e6
+
+
+# --------------------------------------------------------------------------- peaks, clocks, traffic
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_latent_attention_mixer_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock, max clock, utilisation and clock-event reasons through
+    NVML every `period` seconds while running (read-only queries)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period: float = 0.05):
+        self.period = period
+        self.samples = []
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            self.nvml = pynvml
+            pynvml.nvmlInit()
+            self.handle = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = repr(e)
+            self.handle = None
+            self.max_mhz = None
+
+    def _handle(self, device_index):
+        import torch
+        pynvml = self.nvml
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        pynvml = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+                util = pynvml.nvmlDeviceGetUtilizationRates(self.handle).gpu
+                try:
+                    reasons = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    reasons = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                self.samples.append((sm, util, reasons))
+            except Exception as e:  # pragma: no cover
+                self.error = repr(e)
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": self.error}
+        loaded = [s for s in self.samples if s[1] >= 50] or self.samples
+        reasons = set()
+        for _, _, r in loaded:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "samples_under_load": len(loaded)}
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(x_cpu_head, w, n_tokens: int):
+    """Times the oracle on one (b, h) slice restricted to the first n_tokens
+    tokens: synthesis and encode over those tokens, decode of every one."""
+    import numpy as np
+    import oracle
+    sl = slice(0, n_tokens)
+    q0, qf, g, k0, k, v = x_cpu_head
+    toks = np.arange(n_tokens, dtype=np.int64)
+    args = (q0, qf, g, k0[sl], k[sl], v[sl], toks)
+    t0 = time.perf_counter()
+    oracle.flarepp_head(*args)
+    return time.perf_counter() - t0
+
+
+def head_slice_cpu(x, w):
+    return (x["q0"][0].cpu(), x["q_fixed"][0].cpu(), float(x["gate"][0]), x["k0"][0, 0].cpu(),
+            x["k"][0, 0].cpu(), x["v"][0, 0].cpu())
+
+
+def cpu_baseline(x, w, target_s: float):
+    """Bounded sample of the workload on the host cores; returns the entry and
+    the per-step sample size.  Tokens/s covers all H heads of the workload:
+    the sample runs one head, so its per-token time is multiplied by H."""
+    import oracle
+    head = head_slice_cpu(x, w)
+    n_cal = min(w.N, 1024)
+    t_cal = oracle_sample(head, w, n_cal)
+    per_tok = max(t_cal / n_cal, 1e-9)
+    n = int(min(w.N, max(n_cal, target_s / per_tok)))
+    t = oracle_sample(head, w, n)
+    value = n / (t * w.H) / 1e6 if t > 0 else None
+    return {
+        "value": value,
+        "unit": UNIT,
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": (f"{w.name}: batch 0, head 0 of {w.H}, first {n} of {w.N} tokens, all M={w.M} latents, "
+                   f"D={w.D}, fp64; synthesis and encode over the sample, every sample token decoded; "
+                   f"tokens/s = sample tokens / (time x {w.H} heads)"),
+        "seconds": t,
+    }, n
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from rank_latent_attention_mixer_b200 import binding as fb
+    from rank_latent_attention_mixer_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    w = w.with_shape(seed=rank_seed(w.seed, rank))
+    x = W.make_inputs(w, device=str(dev))
+    path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
+    dtype_code = fb.F32 if w.dtype == "f32" else fb.BF16
+    used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
+    ws = torch.empty(fb.workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, True, path), dtype=torch.uint8,
+                     device=dev)
+    y = torch.empty_like(x["k"])
+    n_launch = fb.launches_per_call(True)
+    fits_l2 = 5 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
+
+    def step(events=None):
+        fb.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], y, path=path, workspace=ws,
+                     stage_events=events)
+
+    for _ in range(args.warmup):
+        step()
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize()
+    assert fb.check_device_status() == 0
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            step(evs[i])
+            if flush is not None:
+                flush.zero_()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    status = fb.check_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+
+    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_launch)] for i in range(K)]
+    if flush is None:
+        local_ms = evs[0][0].elapsed_time(evs[K - 1][n_launch])
+    else:
+        local_ms = sum(evs[i][0].elapsed_time(evs[i][n_launch]) for i in range(K))
+    max_ms = reduce_max(local_ms, world, dev)
+    counts = W.algorithmic_counts(w)
+    value = aggregate_mtokens(counts["tokens"], world, K, max_ms)
+    ms_per_step = max_ms / K
+
+    # live per-kernel figures (this rank)
+    avg_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(n_launch)]
+    total_stage = sum(avg_stage)
+    stages = {STAGES_GATED[j]: {"ms": round(avg_stage[j], 4), "share": round(avg_stage[j] / total_stage, 4)}
+              for j in range(n_launch)}
+    split_ms = statistics.mean([avg_stage[0], avg_stage[2]])
+    bhnmd = w.B * w.H * w.N * w.M * w.D
+    flops_per_split_launch = 4.0 * bhnmd
+    peaks, peak_src = load_peaks()
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved_t = flops_per_split_launch / (split_ms * 1e-3) / 1e12
+    roofline = {
+        "bound": "tensor",
+        "kernel": "split_partial" if used_path == fb.PATH_TCGEN05 else "split_partial_simt",
+        "achieved": round(achieved_t, 2),
+        "peak": peak_t,
+        "unit": "TFLOP/s",
+        "frac": round(achieved_t / peak_t, 4),
+        "traffic": ncu_traffic("split_partial", w.name),
+        "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside back-to-back steps)",
+        "algorithmic_per_launch": {"flops": flops_per_split_launch,
+                                   "bytes": 2 * w.B * w.H * w.N * w.D * (4 if w.dtype == 'f32' else 2)},
+        "launch_ms": round(split_ms, 4),
+    }
+    decode_ms = avg_stage[4]
+    dec_t = 4.0 * bhnmd / (decode_ms * 1e-3) / 1e12
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
+                   "gate": "open (FLARE++)", "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
+                   "l2": ("flushed between steps (512 MiB write)" if flush is not None
+                          else "inputs larger than L2 (back-to-back steps)"),
+                   "parallelism": f"replicas x{world} (independent problems per rank)",
+                   "seed_rank0": W.WORKLOADS[args.workload].seed},
+        "tflops": round(counts["flops"] / (ms_per_step * 1e-3) / 1e12 * world, 2),
+        "hbm_gbs_algorithmic": round(counts["bytes"] / (ms_per_step * 1e-3) / 1e9 * world, 1),
+        "gpu_launches": K * n_launch,
+        "roofline": roofline,
+        "stages": stages,
+        "decode": {"tflops": round(dec_t, 2), "frac_of_peak": round(dec_t / peak_t, 4)},
+        "clocks": sampler.summary(),
+    }
+
+    # end-to-end through the public API with host buffers
+    if not args.no_e2e:
+        hx = {}
+        for name in ("q0", "q_fixed", "gate", "k0", "k", "v"):
+            hx[name] = torch.empty(x[name].shape, dtype=x[name].dtype, pin_memory=True)
+            hx[name].copy_(x[name])
+        hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        ke = max(1, min(K, 5))
+        fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hx["gate"], hx["k0"], hx["k"], hx["v"], hy)  # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(ke):
+            fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hx["gate"], hx["k0"], hx["k"], hx["v"], hy)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
+        h2d = sum(hx[n].numel() * hx[n].element_size() for n in hx)
+        out["e2e"] = {"value": round(aggregate_mtokens(counts["tokens"], world, ke, e2e_ms), 4), "unit": UNIT,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hy.numel() * hy.element_size(),
+                      "steps": ke, "api": "flarepp_mixer_fwd_host (pinned host buffers)"}
+        del hx, hy
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb, _ = cpu_baseline(x, w, args.cpu_seconds)
+        out["cpu_baseline"] = cb
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# --------------------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return  # rank 0 alone runs the CPU reference
+    import torch
+    from rank_latent_attention_mixer_b200 import workloads as W
+    w = W.WORKLOADS[args.workload]
+    if w.device_rng:
+        # The CPU generator takes minutes for 2.7 G numbers; the sample needs
+        # one head, so draw that slice with the same recipe on the CPU.
+        x = _cpu_head_inputs(w)
+    else:
+        x = W.make_inputs(w)
+    budget = min(15.0, 150.0 / max(1, args.steps + args.warmup))
+    head = head_slice_cpu(x, w)
+    n_avail = head[3].shape[0]
+    n_cal = min(n_avail, 1024)
+    per_tok = max(oracle_sample(head, w, n_cal) / n_cal, 1e-9)
+    n = int(min(n_avail, max(n_cal, budget / per_tok)))
+    for _ in range(args.warmup):
+        oracle_sample(head, w, n)
+    times = [oracle_sample(head, w, n) for _ in range(args.steps)]
+    t = statistics.mean(times)
+    value = n / (t * w.H) / 1e6
+    import oracle
+    sample = (f"{w.name}: batch 0, head 0 of {w.H}, first {n} of {w.N} tokens, M={w.M}, D={w.D}, fp64 oracle; "
+              f"tokens/s = sample tokens / (time x {w.H} heads)")
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.num_threads(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def _cpu_head_inputs(w):
+    """Head-0 slice of a device-drawn workload, drawn on the CPU with the same
+    recipe (used only when no GPU runs: the reference arm)."""
+    import torch
+    from rank_latent_attention_mixer_b200 import workloads as W
+    n = min(w.N, 262144)
+    small = W.Workload(w.name + "_head0", 1, 1, n, w.M, w.D, w.dtype, w.seed, w.recipe, w.rms_q0, w.rms_k0)
+    return W.make_inputs(small)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

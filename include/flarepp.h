@@ -1,0 +1,154 @@
+/*
+ * flarepp.h -- C ABI of the B200 (sm_100a) FLARE++ token-mixer forward.
+ *
+ * The operation (FLARE.py README, "FLARE++" code block, flarepp_multihead_mixer;
+ * shapes from its docstring):
+ *
+ *     q_dyn = SDPA(q0, k0, k0)          synthesis: M latent seeds read the N tokens
+ *     q     = q_fixed + gate * q_dyn    routing queries (physicsnemo issue #2024,
+ *                                       "Fixed reference and gate")
+ *     z     = SDPA(q, k, v)             encode:  N tokens -> M latents
+ *     y     = SDPA(k, q, z)             decode:  M latents -> N tokens
+ *
+ * SDPA(Q, K, V)_i = sum_j softmax_j(scale * <Q_i, K_j>) V_j, no mask, no dropout,
+ * not causal; scale = 1/sqrt(D) unless an options struct says otherwise.  With
+ * the gate closed the mixer is FLARE (FLARE.py README, "FLARE" code block,
+ * flare_multihead_mixer): z = SDPA(q_fixed, k, v), y = SDPA(k, q_fixed, z).
+ *
+ * Layout and ownership (every entry point):
+ *   - All tensor pointers are caller-owned DEVICE pointers (except the *_host
+ *     entry), row-major and contiguous, 16-byte aligned:
+ *       q0, q_fixed   [H, M, D]     shared by every batch element
+ *       k0, k, v, y   [B, H, N, D]
+ *     in the I/O dtype (FLAREPP_F32 = fp32, FLAREPP_BF16 = bf16).
+ *   - gate: DEVICE float[H], the gate value sigmoid(g) per head (never the
+ *     logit; the library applies no sigmoid).  gate == NULL closes the gate:
+ *     the synthesis is skipped and the result is FLARE with q = q_fixed
+ *     (q0 and k0 may then be NULL).  A gate of zeros still runs the synthesis
+ *     and gives the same y.
+ *   - y must not overlap any input.
+ *   - stream is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Every call is asynchronous on it except the *_host entry and
+ *     flarepp_check_device_status, which synchronise the stream.
+ *   - Accumulation is fp32 for both dtypes.  bf16 I/O rounds q, z and the
+ *     softmax weights to bf16 where they feed the tensor cores; y is rounded
+ *     to the I/O dtype once, at the end.
+ *
+ * Errors: every entry returns a flarepp_status_t and never throws or aborts.
+ * Arguments are checked before any CUDA call or launch; a failed check
+ * launches nothing.  Launch failures are reported as FLAREPP_ERR_CUDA.  A
+ * kernel whose bounded wait runs out records FLAREPP_ERR_TIMEOUT in a device
+ * status word, returns early (its output is then undefined) and leaves the
+ * context usable; flarepp_check_device_status() reads and clears that word.
+ *
+ * Limits: 1 <= B*H <= 65535, 1 <= N <= 2^31-1, 1 <= M <= 4096,
+ * D in {16, 32, 64, 128}; other values give FLAREPP_ERR_UNSUPPORTED.
+ */
+#ifndef FLAREPP_H_
+#define FLAREPP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLAREPP_ABI_VERSION 1
+
+typedef enum flarepp_dtype {
+    FLAREPP_F32 = 0,
+    FLAREPP_BF16 = 1
+} flarepp_dtype_t;
+
+typedef enum flarepp_status {
+    FLAREPP_OK = 0,
+    FLAREPP_ERR_INVALID_ARG = 1,   /* NULL pointer, misaligned pointer, overlap, bad size */
+    FLAREPP_ERR_UNSUPPORTED = 2,   /* valid but outside the limits above (e.g. D = 48) */
+    FLAREPP_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    FLAREPP_ERR_WORKSPACE = 4,     /* caller workspace too small, or allocation failed */
+    FLAREPP_ERR_TIMEOUT = 5        /* a kernel's bounded wait ran out (device status word) */
+} flarepp_status_t;
+
+/* Kernel family.  AUTO picks the tcgen05 tensor-core kernels for bf16 with
+ * D in {16,32,64} and the SIMT (FFMA) kernels otherwise (all fp32 I/O: TF32
+ * products would not meet fp32 accuracy). */
+typedef enum flarepp_path {
+    FLAREPP_PATH_AUTO = 0,
+    FLAREPP_PATH_SIMT = 1,
+    FLAREPP_PATH_TCGEN05 = 2
+} flarepp_path_t;
+
+/* Optional controls for the _ex entry.  Zero-initialise and set what you need. */
+typedef struct flarepp_options {
+    float scale;             /* softmax scale; <= 0 selects 1/sqrt(D)                        */
+    int path;                /* flarepp_path_t; TCGEN05 on an unsupported shape -> UNSUPPORTED */
+    int force_chunks;        /* 0 = planned; > 0 forces the number of token chunks per (b,h)
+                                in the synthesis and encode passes (clamped to the tile count) */
+    int n_stage_events;      /* length of stage_events (0 = none)                            */
+    float* q_out;            /* optional DEVICE fp32 [B,H,M,D]: the routing queries q        */
+    float* z_out;            /* optional DEVICE fp32 [B,H,M,D]: the latents z                */
+    void* workspace;         /* optional DEVICE scratch, 256-byte aligned; NULL = the library
+                                allocates stream-ordered (cudaMallocAsync/cudaFreeAsync)      */
+    size_t workspace_bytes;  /* size of `workspace`; must be >= flarepp_workspace_bytes()    */
+    void* const* stage_events; /* optional caller-created cudaEvent_t handles (as void*):
+                                  [0] is recorded on `stream` before the first kernel launch
+                                  and [i] after the i-th launch, for i < n_stage_events; lets a
+                                  caller time each kernel on the stream it runs on            */
+} flarepp_options_t;
+
+/* Kernel launches one forward call makes (gated = 0: closed gate / FLARE).
+ * Launch order: gated -> split partial (synthesis), merge (q), split partial
+ * (encode), merge (z), decode; closed gate -> the last three. */
+int flarepp_launches_per_call(int gated);
+
+/* FLARE++ mixer forward (see the top of this file).  gate == NULL -> FLARE. */
+int flarepp_mixer_fwd(const void* q0, const void* q_fixed, const float* gate,
+                      const void* k0, const void* k, const void* v, void* y,
+                      int B, int H, int N, int M, int D, int dtype, void* stream);
+
+/* FLARE (closed gate): z = SDPA(q, k, v), y = SDPA(k, q, z), q [H,M,D] shared over B.
+ * Same result as flarepp_mixer_fwd(NULL, q, NULL, NULL, k, v, y, ...). */
+int flare_fwd(const void* q, const void* k, const void* v, void* y,
+              int B, int H, int N, int M, int D, int dtype, void* stream);
+
+/* flarepp_mixer_fwd with options (opts may be NULL = all defaults). */
+int flarepp_mixer_fwd_ex(const void* q0, const void* q_fixed, const float* gate,
+                         const void* k0, const void* k, const void* v, void* y,
+                         int B, int H, int N, int M, int D, int dtype,
+                         const flarepp_options_t* opts, void* stream);
+
+/* Bytes of device scratch one call needs (partial softmax triples per token
+ * chunk, and q, z in fp32 and bf16).  gated = 0 for the closed-gate form.
+ * Returns 0 for arguments the forward entries would reject. */
+size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
+                               const flarepp_options_t* opts);
+
+/* Same operation with HOST buffers (end-to-end form): copies the inputs to the
+ * device on `stream`, runs the mixer, copies y back and synchronises `stream`
+ * before returning.  Device memory is taken stream-ordered and released before
+ * return.  Pinned host memory lets the copies run at full speed; pageable
+ * memory works but is slower.  gate is a HOST float[H] here (NULL = FLARE). */
+int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate,
+                           const void* k0, const void* k, const void* v, void* y,
+                           int B, int H, int N, int M, int D, int dtype, void* stream);
+
+/* Which kernel family AUTO would run for this shape (flarepp_path_t), or 0 for
+ * arguments the forward entries would reject. */
+int flarepp_selected_path(int B, int H, int N, int M, int D, int dtype);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * (FLAREPP_OK when no kernel recorded a failure on the current device). */
+int flarepp_check_device_status(void* stream);
+
+/* Static text for a status code. */
+const char* flarepp_status_string(int status);
+
+/* FLAREPP_ABI_VERSION of the loaded library. */
+int flarepp_abi_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* FLAREPP_H_ */

@@ -1,0 +1,212 @@
+"""Thin ctypes binding of the C ABI in include/flarepp.h.
+
+Argument marshalling only: every step of the mixer runs in the CUDA library
+``libflarepp.so`` built in this directory.  PyTorch provides device memory,
+the current stream and scratch from its caching allocator.  There is no CPU
+fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflarepp.so")
+
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TCGEN05 = 0, 1, 2
+STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
+          4: "ERR_WORKSPACE", 5: "ERR_TIMEOUT"}
+EXPORTS = ["flarepp_mixer_fwd", "flare_fwd", "flarepp_mixer_fwd_ex", "flarepp_workspace_bytes",
+           "flarepp_mixer_fwd_host", "flarepp_selected_path", "flarepp_check_device_status",
+           "flarepp_status_string", "flarepp_abi_version", "flarepp_launches_per_call"]
+
+
+class FlareppError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class Options(ctypes.Structure):
+    """flarepp_options_t."""
+    _fields_ = [("scale", ctypes.c_float), ("path", ctypes.c_int), ("force_chunks", ctypes.c_int),
+                ("n_stage_events", ctypes.c_int), ("q_out", ctypes.c_void_p), ("z_out", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m rank_latent_attention_mixer_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    sig = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i]
+    lib.flarepp_mixer_fwd.argtypes = sig + [vp]
+    lib.flarepp_mixer_fwd_ex.argtypes = sig + [ctypes.POINTER(Options), vp]
+    lib.flarepp_mixer_fwd_host.argtypes = sig + [vp]
+    lib.flare_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.flarepp_workspace_bytes.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(Options)]
+    lib.flarepp_workspace_bytes.restype = ctypes.c_size_t
+    lib.flarepp_selected_path.argtypes = [i, i, i, i, i, i]
+    lib.flarepp_check_device_status.argtypes = [vp]
+    lib.flarepp_status_string.argtypes = [i]
+    lib.flarepp_status_string.restype = ctypes.c_char_p
+    lib.flarepp_launches_per_call.argtypes = [i]
+    for name in ("flarepp_mixer_fwd", "flarepp_mixer_fwd_ex", "flarepp_mixer_fwd_host", "flare_fwd",
+                 "flarepp_selected_path", "flarepp_check_device_status", "flarepp_abi_version",
+                 "flarepp_launches_per_call"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.flarepp_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; the mixer takes float32 or bfloat16")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise FlareppError(rc, where)
+
+
+def _shapes(q_fixed: torch.Tensor, k: torch.Tensor):
+    if k.dim() != 4 or q_fixed.dim() != 3:
+        raise ValueError("expected q_fixed [H,M,D] and k [B,H,N,D]")
+    B, H, N, D = k.shape
+    if q_fixed.shape[0] != H or q_fixed.shape[2] != D:
+        raise ValueError(f"q_fixed {tuple(q_fixed.shape)} does not match k {tuple(k.shape)}")
+    return B, H, N, q_fixed.shape[1], D
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (the mixer reads row-major [.., D] rows)")
+
+
+def launches_per_call(gated: bool = True) -> int:
+    return int(lib.flarepp_launches_per_call(int(gated)))
+
+
+def workspace_bytes(B, H, N, M, D, dtype=BF16, gated=True, path=PATH_AUTO, force_chunks=0) -> int:
+    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None)
+    return int(lib.flarepp_workspace_bytes(B, H, N, M, D, dtype, int(gated), ctypes.byref(o)))
+
+
+def selected_path(B, H, N, M, D, dtype=BF16) -> int:
+    return int(lib.flarepp_selected_path(B, H, N, M, D, dtype))
+
+
+def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: int = PATH_AUTO,
+              force_chunks: int = 0, return_qz: bool = False, workspace: Optional[torch.Tensor] = None,
+              stage_events=None):
+    """FLARE++ mixer forward on the current CUDA stream.  ``gate=None`` is FLARE.
+
+    q0, q_fixed [H,M,D]; gate fp32 [H] (sigmoid already applied); k0, k, v [B,H,N,D];
+    all on the same CUDA device, contiguous, fp32 or bf16.  Returns y (and q, z
+    fp32 [B,H,M,D] when ``return_qz``).  ``stage_events``: torch.cuda.Event objects
+    (created with enable_timing) recorded before the first launch and after each
+    launch on the current stream."""
+    B, H, N, M, D = _shapes(q_fixed, k)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    dt = _dtype_code(k)
+    if y is None:
+        y = torch.empty_like(k)
+    q_out = z_out = None
+    if return_qz:
+        q_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
+        z_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
+    if gate is not None and gate.dtype != torch.float32:
+        raise TypeError("gate must be float32 [H]")
+    need = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks)
+    if need == 0:
+        ws_ptr, ws_len = None, 0
+    else:
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+        ws_ptr, ws_len = workspace.data_ptr(), workspace.numel()
+    ev_arr, n_ev = None, 0
+    if stage_events:
+        handles = []
+        for e in stage_events:
+            if e.cuda_event == 0:          # torch creates the CUDA event lazily
+                e.record()
+            handles.append(e.cuda_event)
+        n_ev = len(handles)
+        ev_arr = (ctypes.c_void_p * n_ev)(*handles)
+    o = Options(float(scale), int(path), int(force_chunks), n_ev, _ptr(q_out), _ptr(z_out), ws_ptr, ws_len,
+                ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None)
+    rc = lib.flarepp_mixer_fwd_ex(_ptr(q0) if gate is not None else None, _ptr(q_fixed), _ptr(gate),
+                                  _ptr(k0) if gate is not None else None, _ptr(k), _ptr(v), _ptr(y),
+                                  B, H, N, M, D, dt, ctypes.byref(o), _stream(k.device))
+    _check(rc, "flarepp_mixer_fwd_ex")
+    return (y, q_out, z_out) if return_qz else y
+
+
+def mixer_fwd_plain(q0, q_fixed, gate, k0, k, v, y):
+    """flarepp_mixer_fwd exactly as a C caller would make it (library-managed scratch)."""
+    B, H, N, M, D = _shapes(q_fixed, k)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    rc = lib.flarepp_mixer_fwd(_ptr(q0), _ptr(q_fixed), _ptr(gate), _ptr(k0), _ptr(k), _ptr(v), _ptr(y),
+                               B, H, N, M, D, _dtype_code(k), _stream(k.device))
+    _check(rc, "flarepp_mixer_fwd")
+    return y
+
+
+def flare_fwd(q, k, v, y=None):
+    """FLARE (closed gate): z = SDPA(q,k,v), y = SDPA(k,q,z); q [H,M,D]."""
+    B, H, N, M, D = _shapes(q, k)
+    _contig(q, k, v, y)
+    if y is None:
+        y = torch.empty_like(k)
+    rc = lib.flare_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(y), B, H, N, M, D, _dtype_code(k), _stream(k.device))
+    _check(rc, "flare_fwd")
+    return y
+
+
+def mixer_fwd_host(q0, q_fixed, gate, k0, k, v, y, stream: Optional[torch.cuda.Stream] = None):
+    """End-to-end form on HOST tensors (pinned for full copy speed): the library
+    copies inputs in, runs, copies y out and synchronises the stream."""
+    B, H, N, M, D = _shapes(q_fixed, k)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    for t in (q0, q_fixed, gate, k0, k, v, y):
+        if t is not None and t.is_cuda:
+            raise ValueError("mixer_fwd_host takes host tensors")
+    st = (stream or torch.cuda.current_stream()).cuda_stream
+    rc = lib.flarepp_mixer_fwd_host(_ptr(q0), _ptr(q_fixed), _ptr(gate), _ptr(k0), _ptr(k), _ptr(v), _ptr(y),
+                                    B, H, N, M, D, _dtype_code(k), st)
+    _check(rc, "flarepp_mixer_fwd_host")
+    return y
+
+
+def check_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    st = (stream or torch.cuda.current_stream()).cuda_stream
+    return int(lib.flarepp_check_device_status(st))
+
+
+def raw_call(name: str, *args) -> int:
+    """Calls an exported entry with already-marshalled arguments (tests)."""
+    return int(getattr(lib, name)(*args))

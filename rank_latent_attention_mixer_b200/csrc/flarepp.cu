@@ -1,0 +1,406 @@
+// C ABI of the FLARE++ mixer forward: argument checks, planning, workspace
+// and the launch sequence.  The operation and the ABI contract are documented
+// in include/flarepp.h.
+//
+// Launch sequence for one call (gate open):
+//   1. split partial   Q = q0 [H,M,D],  K = V = k0     (synthesis, V = K)
+//   2. merge           q = q_fixed + gate * q_dyn       -> q fp32 + bf16
+//   3. split partial   Q = q,           K = k, V = v    (encode)
+//   4. merge           z                                -> z fp32 + bf16
+//   5. decode          y = SDPA(k, q, z)
+// With the gate closed, steps 1-2 are skipped and q_fixed is used as q.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/flarepp.h"
+#include "common.cuh"
+#include "kernels_simt.cuh"
+#include "kernels_tc.cuh"
+
+namespace flarepp {
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Shape {
+    int B, H, N, M, D, dtype;
+    int64_t bh() const { return (int64_t)B * H; }
+    size_t elem() const { return dtype == FLAREPP_F32 ? 4 : 2; }
+    size_t tok_bytes() const { return (size_t)B * H * (size_t)N * D * elem(); }
+    size_t lat_bytes() const { return (size_t)H * M * D * elem(); }
+};
+
+// Work split and scratch layout of one call.
+struct Plan {
+    int path;            // flarepp_path_t (SIMT or TCGEN05)
+    int chunks;          // token chunks per (b, h) in the split passes
+    int chunk_len;       // tokens per chunk
+    int row_blocks;      // latent-row blocks per (b, h, chunk) (SIMT)
+    float scale_log2;
+    // byte offsets into the workspace
+    size_t off_part_O, off_part_ml, off_q32, off_q16, off_z32, off_z16, total;
+};
+
+int check_shape(const Shape& s) {
+    if (s.B < 1 || s.H < 1 || s.N < 1 || s.M < 1) return FLAREPP_ERR_INVALID_ARG;
+    if (s.dtype != FLAREPP_F32 && s.dtype != FLAREPP_BF16) return FLAREPP_ERR_INVALID_ARG;
+    if (s.bh() > 65535 || s.M > 4096) return FLAREPP_ERR_UNSUPPORTED;
+    if (s.D != 16 && s.D != 32 && s.D != 64 && s.D != 128) return FLAREPP_ERR_UNSUPPORTED;
+    return FLAREPP_OK;
+}
+
+int tile_tokens_simt(int D) { return 2048 / D; }
+
+bool tc_supported(const Shape& s) { return tc::supported(s.dtype == FLAREPP_BF16, s.D, s.M); }
+
+int choose_path(const Shape& s, int requested) {
+    if (requested == FLAREPP_PATH_SIMT) return FLAREPP_PATH_SIMT;
+    if (requested == FLAREPP_PATH_TCGEN05) return tc_supported(s) ? FLAREPP_PATH_TCGEN05 : -1;
+    if (requested != FLAREPP_PATH_AUTO) return -1;
+    return tc_supported(s) ? FLAREPP_PATH_TCGEN05 : FLAREPP_PATH_SIMT;
+}
+
+int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    const int requested = o ? o->path : FLAREPP_PATH_AUTO;
+    const int path = choose_path(s, requested);
+    if (path < 0) return requested == FLAREPP_PATH_TCGEN05 ? FLAREPP_ERR_UNSUPPORTED : FLAREPP_ERR_INVALID_ARG;
+    if (o && o->n_stage_events < 0) return FLAREPP_ERR_INVALID_ARG;
+    if (o && o->n_stage_events > 0 && !o->stage_events) return FLAREPP_ERR_INVALID_ARG;
+    if (o && o->force_chunks < 0) return FLAREPP_ERR_INVALID_ARG;
+    pl->path = path;
+    const float scale = (o && o->scale > 0.f) ? o->scale : 1.f / std::sqrt((float)s.D);
+    if (!std::isfinite(scale)) return FLAREPP_ERR_INVALID_ARG;
+    pl->scale_log2 = scale * kLog2e;
+
+    int tile, units_per_bh;
+    if (path == FLAREPP_PATH_SIMT) {
+        tile = tile_tokens_simt(s.D);
+        pl->row_blocks = (s.M + kSimtThreads - 1) / kSimtThreads;
+        units_per_bh = pl->row_blocks;
+    } else {
+        tile = tc::kTokTile;
+        pl->row_blocks = tc::row_groups(s.M);
+        units_per_bh = pl->row_blocks;
+    }
+    const int64_t tiles = (s.N + tile - 1) / tile;
+    int64_t chunks;
+    if (o && o->force_chunks > 0) {
+        chunks = std::min<int64_t>(o->force_chunks, tiles);
+    } else {
+        // Enough CTAs for several waves over the SMs, but chunks of >= 1 tile.
+        const int64_t target = path == FLAREPP_PATH_SIMT ? 4 * kNumSMs : tc::target_ctas();
+        chunks = (target + s.bh() * units_per_bh - 1) / (s.bh() * units_per_bh);
+        chunks = std::max<int64_t>(1, std::min<int64_t>(chunks, tiles));
+    }
+    int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
+    pl->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
+    pl->chunks = (int)((s.N + (int64_t)pl->chunk_len - 1) / pl->chunk_len);
+    const int parts = path == FLAREPP_PATH_SIMT ? pl->chunks : pl->chunks * tc::kPartsPerChunk;
+
+    const size_t rows = (size_t)s.bh() * s.M;
+    size_t off = 0;
+    pl->off_part_O = off;  off = align_up(off + (size_t)parts * rows * s.D * sizeof(float));
+    pl->off_part_ml = off; off = align_up(off + (size_t)parts * rows * sizeof(float2));
+    pl->off_q32 = off;     off = align_up(off + rows * s.D * sizeof(float));
+    pl->off_q16 = off;     off = align_up(off + rows * s.D * sizeof(__nv_bfloat16));
+    pl->off_z32 = off;     off = align_up(off + rows * s.D * sizeof(float));
+    pl->off_z16 = off;     off = align_up(off + rows * s.D * sizeof(__nv_bfloat16));
+    pl->total = off;
+    return FLAREPP_OK;
+}
+
+// Caller-provided events recorded around the launches (flarepp_options_t).
+struct StageEvents {
+    void* const* ev = nullptr;
+    int n = 0;
+    int next = 0;
+    void mark(cudaStream_t st) {
+        if (next < n && ev[next]) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[next]), st);
+        ++next;
+    }
+};
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int check_pointers(const Shape& s, const void* q0, const void* q_fixed, const float* gate,
+                   const void* k0, const void* k, const void* v, const void* y) {
+    const bool gated = gate != nullptr;
+    if (!q_fixed || !k || !v || !y) return FLAREPP_ERR_INVALID_ARG;
+    if (gated && (!q0 || !k0)) return FLAREPP_ERR_INVALID_ARG;
+    const void* tensors[] = {q_fixed, k, v, y, gated ? q0 : nullptr, gated ? k0 : nullptr};
+    for (const void* t : tensors)
+        if (t && !aligned16(t)) return FLAREPP_ERR_INVALID_ARG;
+    if (gated && (reinterpret_cast<uintptr_t>(gate) & 3u)) return FLAREPP_ERR_INVALID_ARG;
+    const size_t tb = s.tok_bytes(), lb = s.lat_bytes();
+    if (overlaps(y, tb, k, tb) || overlaps(y, tb, v, tb) || overlaps(y, tb, q_fixed, lb)) return FLAREPP_ERR_INVALID_ARG;
+    if (gated && (overlaps(y, tb, k0, tb) || overlaps(y, tb, q0, lb) ||
+                  overlaps(y, tb, gate, (size_t)s.H * sizeof(float))))
+        return FLAREPP_ERR_INVALID_ARG;
+    return FLAREPP_OK;
+}
+
+template <typename T>
+int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, const float* gate,
+             const void* k0, const void* k, const void* v, void* y, char* ws,
+             float* q_out, float* z_out, StageEvents& ev, cudaStream_t st) {
+    const bool gated = gate != nullptr;
+    float* part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
+    float2* part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+    float* q32 = reinterpret_cast<float*>(ws + pl.off_q32);
+    __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_q16);
+    float* z32 = reinterpret_cast<float*>(ws + pl.off_z32);
+    __nv_bfloat16* z16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_z16);
+
+    const dim3 split_grid(pl.chunks, (unsigned)s.bh(), pl.row_blocks);
+    const int64_t rows = s.bh() * s.M;
+    const dim3 merge_grid((unsigned)((rows + 7) / 8));
+    const dim3 dec_grid((unsigned)((s.N + kSimtThreads - 1) / kSimtThreads), (unsigned)s.bh());
+
+    SplitParams sp{};
+    sp.part_O = part_O; sp.part_ml = part_ml;
+    sp.B = s.B; sp.H = s.H; sp.N = s.N; sp.M = s.M;
+    sp.chunks = pl.chunks; sp.chunk_len = pl.chunk_len; sp.scale_log2 = pl.scale_log2;
+    MergeParams mp{};
+    mp.part_O = part_O; mp.part_ml = part_ml; mp.chunks = pl.chunks;
+    mp.B = s.B; mp.H = s.H; mp.M = s.M; mp.q_fixed = q_fixed; mp.gate = gate;
+    DecodeParams dp{};
+    dp.Ktok = k; dp.Z = z32; dp.Y = y; dp.B = s.B; dp.H = s.H; dp.N = s.N; dp.M = s.M;
+    dp.scale_log2 = pl.scale_log2;
+
+#define FLAREPP_SIMT_DISPATCH(DD)                                                                  \
+    case DD: {                                                                                     \
+        ev.mark(st);                                                                               \
+        if (gated) {                                                                               \
+            sp.Q = q0; sp.q_batch_heads = 0; sp.K = k0; sp.V = k0;                                 \
+            split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
+            ev.mark(st);                                                                           \
+            mp.mode = kMergeSynthesis; mp.out_f32 = q32; mp.out_bf16 = q16; mp.user_out = q_out;   \
+            mp.q_copy_out = nullptr;                                                               \
+            merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                 \
+            ev.mark(st);                                                                           \
+            sp.Q = q32; sp.q_batch_heads = s.H; sp.K = k; sp.V = v;                                \
+            split_partial_simt<float, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);             \
+            ev.mark(st);                                                                           \
+        } else {                                                                                   \
+            sp.Q = q_fixed; sp.q_batch_heads = 0; sp.K = k; sp.V = v;                              \
+            split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
+            ev.mark(st);                                                                           \
+        }                                                                                          \
+        mp.mode = kMergeEncode; mp.out_f32 = z32; mp.out_bf16 = z16; mp.user_out = z_out;          \
+        mp.q_copy_out = gated ? nullptr : q_out;                                                   \
+        merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                     \
+        ev.mark(st);                                                                               \
+        if (gated) {                                                                               \
+            dp.Qlat = q32; dp.q_batch_heads = s.H;                                                 \
+            decode_simt<T, float, DD><<<dec_grid, kSimtThreads, 0, st>>>(dp);                      \
+            ev.mark(st);                                                                           \
+        } else {                                                                                   \
+            dp.Qlat = q_fixed; dp.q_batch_heads = 0;                                               \
+            decode_simt<T, T, DD><<<dec_grid, kSimtThreads, 0, st>>>(dp);                          \
+            ev.mark(st);                                                                           \
+        }                                                                                          \
+        break;                                                                                     \
+    }
+    switch (s.D) {
+        FLAREPP_SIMT_DISPATCH(16)
+        FLAREPP_SIMT_DISPATCH(32)
+        FLAREPP_SIMT_DISPATCH(64)
+        FLAREPP_SIMT_DISPATCH(128)
+        default: return FLAREPP_ERR_UNSUPPORTED;
+    }
+#undef FLAREPP_SIMT_DISPATCH
+    (void)q16; (void)z16;
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
+int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, const float* gate,
+        const void* k0, const void* k, const void* v, void* y, char* ws,
+        float* q_out, float* z_out, StageEvents& ev, cudaStream_t st) {
+    if (pl.path == FLAREPP_PATH_TCGEN05) {
+        tc::Buffers bu{};
+        bu.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
+        bu.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+        bu.q32 = reinterpret_cast<float*>(ws + pl.off_q32);
+        bu.q16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_q16);
+        bu.z32 = reinterpret_cast<float*>(ws + pl.off_z32);
+        bu.z16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_z16);
+        tc::Problem pr{};
+        pr.B = s.B; pr.H = s.H; pr.N = s.N; pr.M = s.M; pr.D = s.D;
+        pr.chunks = pl.chunks; pr.chunk_len = pl.chunk_len; pr.scale_log2 = pl.scale_log2;
+        return tc::run(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out,
+                       [&ev](cudaStream_t t) { ev.mark(t); }, st);
+    }
+    if (s.dtype == FLAREPP_F32)
+        return run_simt<float>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+    return run_simt<__nv_bfloat16>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+}
+
+int forward(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+            const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
+            const flarepp_options_t* opts, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    int rc = make_plan(s, opts, &pl);
+    if (rc) return rc;
+    rc = check_pointers(s, q0, q_fixed, gate, k0, k, v, y);
+    if (rc) return rc;
+    float* q_out = opts ? opts->q_out : nullptr;
+    float* z_out = opts ? opts->z_out : nullptr;
+    if ((q_out && !aligned16(q_out)) || (z_out && !aligned16(z_out))) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = nullptr;
+    bool owned = false;
+    if (opts && opts->workspace) {
+        if (opts->workspace_bytes < pl.total) return FLAREPP_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(opts->workspace) % kAlign) return FLAREPP_ERR_INVALID_ARG;
+        ws = static_cast<char*>(opts->workspace);
+    } else {
+        if (cudaMallocAsync(reinterpret_cast<void**>(&ws), pl.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return FLAREPP_ERR_WORKSPACE;
+        }
+        owned = true;
+    }
+    StageEvents ev;
+    if (opts && opts->n_stage_events > 0) {
+        ev.ev = opts->stage_events;
+        ev.n = opts->n_stage_events;
+    }
+    rc = run(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+    if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    return rc;
+}
+
+}  // namespace
+}  // namespace flarepp
+
+using namespace flarepp;
+
+extern "C" {
+
+int flarepp_abi_version(void) { return FLAREPP_ABI_VERSION; }
+
+int flarepp_launches_per_call(int gated) { return gated ? 5 : 3; }
+
+const char* flarepp_status_string(int status) {
+    switch (status) {
+        case FLAREPP_OK: return "ok";
+        case FLAREPP_ERR_INVALID_ARG: return "invalid argument";
+        case FLAREPP_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case FLAREPP_ERR_CUDA: return "CUDA error";
+        case FLAREPP_ERR_WORKSPACE: return "workspace too small or allocation failed";
+        case FLAREPP_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int flarepp_mixer_fwd_ex(const void* q0, const void* q_fixed, const float* gate, const void* k0,
+                         const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
+                         int dtype, const flarepp_options_t* opts, void* stream) {
+    return forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, opts, stream);
+}
+
+int flarepp_mixer_fwd(const void* q0, const void* q_fixed, const float* gate, const void* k0,
+                      const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
+                      int dtype, void* stream) {
+    return forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, nullptr, stream);
+}
+
+int flare_fwd(const void* q, const void* k, const void* v, void* y, int B, int H, int N, int M,
+              int D, int dtype, void* stream) {
+    return forward(nullptr, q, nullptr, nullptr, k, v, y, B, H, N, M, D, dtype, nullptr, stream);
+}
+
+size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
+                               const flarepp_options_t* opts) {
+    (void)gated;  // the same scratch serves both forms
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    if (make_plan(s, opts, &pl)) return 0;
+    return pl.total;
+}
+
+int flarepp_selected_path(int B, int H, int N, int M, int D, int dtype) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    if (make_plan(s, nullptr, &pl)) return 0;
+    return pl.path;
+}
+
+int flarepp_check_device_status(void* stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FLAREPP_ERR_CUDA;
+    int code = 0;
+    if (cudaMemcpyFromSymbol(&code, g_device_status, sizeof(int)) != cudaSuccess) return FLAREPP_ERR_CUDA;
+    if (code != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FLAREPP_ERR_CUDA;
+    }
+    return code;
+}
+
+int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate, const void* k0,
+                           const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
+                           int dtype, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    int rc = make_plan(s, nullptr, &pl);
+    if (rc) return rc;
+    const bool gated = gate != nullptr;
+    if (!q_fixed || !k || !v || !y || (gated && (!q0 || !k0))) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t tb = s.tok_bytes(), lb = s.lat_bytes(), gb = (size_t)H * sizeof(float);
+    // One stream-ordered block: inputs, output, then the mixer's workspace.
+    size_t off = 0;
+    const size_t o_qf = off; off = align_up(off + lb);
+    const size_t o_k = off;  off = align_up(off + tb);
+    const size_t o_v = off;  off = align_up(off + tb);
+    const size_t o_y = off;  off = align_up(off + tb);
+    size_t o_q0 = 0, o_k0 = 0, o_g = 0;
+    if (gated) {
+        o_q0 = off; off = align_up(off + lb);
+        o_k0 = off; off = align_up(off + tb);
+        o_g = off;  off = align_up(off + gb);
+    }
+    const size_t o_ws = off; off = align_up(off + pl.total);
+    char* d = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&d), off, st) != cudaSuccess) {
+        cudaGetLastError();
+        return FLAREPP_ERR_WORKSPACE;
+    }
+    bool ok = cudaMemcpyAsync(d + o_qf, q_fixed, lb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+              cudaMemcpyAsync(d + o_k, k, tb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+              cudaMemcpyAsync(d + o_v, v, tb, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    if (ok && gated)
+        ok = cudaMemcpyAsync(d + o_q0, q0, lb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+             cudaMemcpyAsync(d + o_k0, k0, tb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+             cudaMemcpyAsync(d + o_g, gate, gb, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    rc = ok ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+    if (rc == FLAREPP_OK) {
+        flarepp_options_t o{};
+        o.workspace = d + o_ws;
+        o.workspace_bytes = pl.total;
+        rc = forward(gated ? d + o_q0 : nullptr, d + o_qf, gated ? reinterpret_cast<float*>(d + o_g) : nullptr,
+                     gated ? d + o_k0 : nullptr, d + o_k, d + o_v, d + o_y, B, H, N, M, D, dtype, &o, stream);
+    }
+    if (rc == FLAREPP_OK && cudaMemcpyAsync(y, d + o_y, tb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = FLAREPP_ERR_CUDA;
+    if (cudaFreeAsync(d, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,268 @@
+// SIMT (FFMA, fp32) kernels of the FLARE++ mixer: the split-N partial pass used
+// by the synthesis and encode calls, the merge of the partial softmax triples,
+// and the decode.  They serve every fp32-I/O call (fp32 products keep the
+// 1e-4 accuracy that TF32 tensor-core products would not) and every shape the
+// tcgen05 kernels do not cover.
+//
+// Notation (FLARE.py README, "FLARE++" code block): for one (b, h) the score of
+// latent m and token n is S[m, n] = scale * <q[m], k[n]>.  The synthesis and
+// encode calls softmax S along n (per latent); the decode softmaxes the same
+// kind of score along m (per token).  All exponentials are taken base 2 on
+// scores pre-multiplied by scale*log2(e), which is the same softmax.
+#pragma once
+
+#include "common.cuh"
+
+namespace flarepp {
+
+constexpr int kSimtThreads = 128;
+
+// Split-N partial pass: for one (b, h), one chunk of tokens and one block of
+// latent rows, the online-softmax triple of every row over the chunk:
+// running max (log2 units), sum of weights, and the unnormalised weighted sum
+// of the value rows.  Chunks of the same (b, h) are combined by merge_partials;
+// this split of the token axis and the log-sum-exp merge is exact up to
+// rounding (physicsnemo issue #2024, section 2: the token-sharded encoder
+// rebuilds the globally normalised attention from latent-sized outputs and
+// log-sum-exp statistics).
+struct SplitParams {
+    const void* Q;       // latent query rows; (b, h) rows start at row (b*q_batch_heads + h)*M
+    int q_batch_heads;   // H when Q is [B,H,M,D]; 0 when Q is [H,M,D] (shared over b)
+    const void* K;       // [B,H,N,D] keys
+    const void* V;       // [B,H,N,D] values (may equal K: synthesis reads k0 twice)
+    float* part_O;       // [C][B*H][M][D]
+    float2* part_ml;     // [C][B*H][M]: (max in log2 units, sum of weights)
+    int B, H, N, M;
+    int chunks, chunk_len;
+    float scale_log2;    // softmax scale * log2(e)
+};
+
+template <int D> struct SimtTile { static constexpr int tokens = 2048 / D; };
+
+template <typename TQ, typename TKV, int D>
+__global__ void __launch_bounds__(kSimtThreads)
+split_partial_simt(SplitParams p) {
+    constexpr int TILE = SimtTile<D>::tokens;
+    __shared__ __align__(16) float sK[TILE * D];
+    __shared__ __align__(16) float sV[TILE * D];
+
+    const int c = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const int m = blockIdx.z * kSimtThreads + threadIdx.x;
+    const bool active = m < p.M;
+    const int n0 = c * p.chunk_len;
+    const int n1 = min(p.N, n0 + p.chunk_len);
+    const bool same_kv = p.K == p.V;
+
+    float q[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) q[d] = 0.f;
+    if (active) {
+        const TQ* qrow = reinterpret_cast<const TQ*>(p.Q) +
+                         ((int64_t)(b * p.q_batch_heads + h) * p.M + m) * D;
+        load_row_f32<TQ, D>(qrow, q);
+#pragma unroll
+        for (int d = 0; d < D; ++d) q[d] *= p.scale_log2;
+    }
+    float mx = -INFINITY, l = 0.f, acc[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) acc[d] = 0.f;
+
+    const TKV* Kbh = reinterpret_cast<const TKV*>(p.K) + (int64_t)bh * p.N * D;
+    const TKV* Vbh = reinterpret_cast<const TKV*>(p.V) + (int64_t)bh * p.N * D;
+    constexpr int VEC = 16 / sizeof(TKV);          // elements per 16-byte load
+    for (int t0 = n0; t0 < n1; t0 += TILE) {
+        const int cnt = min(TILE, n1 - t0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < cnt * D / VEC; i += kSimtThreads) {
+            float tmp[VEC];
+            load_row_f32<TKV, VEC>(Kbh + (int64_t)t0 * D + i * VEC, tmp);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) sK[i * VEC + e] = tmp[e];
+            if (!same_kv) {
+                load_row_f32<TKV, VEC>(Vbh + (int64_t)t0 * D + i * VEC, tmp);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) sV[i * VEC + e] = tmp[e];
+            }
+        }
+        __syncthreads();
+        const float* sVv = same_kv ? sK : sV;
+        if (active) {
+            for (int j = 0; j < cnt; ++j) {
+                const float* kr = sK + j * D;
+                float s = 0.f;
+#pragma unroll
+                for (int d = 0; d < D; ++d) s = fmaf(q[d], kr[d], s);
+                if (s > mx) {
+                    const float corr = ex2_mufu(mx - s);
+                    l *= corr;
+#pragma unroll
+                    for (int d = 0; d < D; ++d) acc[d] *= corr;
+                    mx = s;
+                }
+                const float w = ex2_mufu(s - mx);
+                l += w;
+                const float* vr = sVv + j * D;
+#pragma unroll
+                for (int d = 0; d < D; ++d) acc[d] = fmaf(w, vr[d], acc[d]);
+            }
+        }
+    }
+    if (active) {
+        const int64_t row = ((int64_t)c * p.B * p.H + bh) * p.M + m;
+        p.part_ml[row] = make_float2(mx, l);
+        store_row<float, D>(p.part_O + row * D, acc);
+    }
+}
+
+// Merge of the per-chunk triples of one latent row (one warp per row):
+// out = sum_c 2^(m_c - m*) O_c / sum_c 2^(m_c - m*) l_c with m* = max_c m_c.
+// Synthesis epilogue: q = q_fixed + gate[h] * out (FLARE.py README, FLARE++
+// block, second line).  Encode epilogue: z = out.
+enum MergeMode { kMergeSynthesis = 0, kMergeEncode = 1 };
+
+struct MergeParams {
+    const float* part_O;
+    const float2* part_ml;
+    int chunks;
+    int B, H, M;
+    int mode;                   // MergeMode
+    const void* q_fixed;        // [H,M,D] in the I/O dtype (synthesis epilogue, or copied to q_copy_out)
+    const float* gate;          // [H] (synthesis epilogue)
+    float* out_f32;             // [B,H,M,D]
+    __nv_bfloat16* out_bf16;    // [B,H,M,D]
+    float* user_out;            // optional [B,H,M,D]
+    float* q_copy_out;          // optional: closed gate, write q = q_fixed broadcast over b
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+merge_partials(MergeParams p) {
+    constexpr int PER = (D + 31) / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)p.B * p.H * p.M;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= rows) return;
+    const int m = (int)(row % p.M);
+    const int h = (int)((row / p.M) % p.H);
+    const int64_t cstride = rows;               // rows per chunk slab
+
+    float mstar = -INFINITY;
+    for (int c = lane; c < p.chunks; c += 32) mstar = fmaxf(mstar, p.part_ml[c * cstride + row].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+
+    float L = 0.f, acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    for (int c = 0; c < p.chunks; ++c) {
+        const float2 ml = p.part_ml[c * cstride + row];
+        if (ml.y <= 0.f) continue;               // empty chunk contributes nothing
+        const float w = ex2_mufu(ml.x - mstar);
+        L = fmaf(w, ml.y, L);
+        const float* o = p.part_O + (c * cstride + row) * D;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int d = lane + 32 * i;
+            if (d < D) acc[i] = fmaf(w, o[d], acc[i]);
+        }
+    }
+    const float inv = 1.f / L;
+    const T* qf = reinterpret_cast<const T*>(p.q_fixed) + ((int64_t)h * p.M + m) * D;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int d = lane + 32 * i;
+        if (d >= D) continue;
+        float val = acc[i] * inv;
+        if (p.mode == kMergeSynthesis) val = fmaf(p.gate[h], val, to_f32<T>(qf[d]));
+        p.out_f32[row * D + d] = val;
+        p.out_bf16[row * D + d] = __float2bfloat16_rn(val);
+        if (p.user_out) p.user_out[row * D + d] = val;
+        if (p.q_copy_out) p.q_copy_out[row * D + d] = to_f32<T>(qf[d]);
+    }
+}
+
+// Decode (FLARE.py README, FLARE++ block, last line: y = SDPA(k, q, z)): one
+// thread per token; the token's key row is the query, the M latent rows of q
+// are the keys and those of z the values.  Latent rows are staged through
+// shared memory in chunks of 2048/D rows and every thread reads the same row
+// (broadcast); the softmax over M is online across the chunks.
+struct DecodeParams {
+    const void* Ktok;     // [B,H,N,D]
+    const void* Qlat;     // latent keys; (b, h) rows start at row (b*q_batch_heads + h)*M
+    int q_batch_heads;
+    const float* Z;       // [B,H,M,D] fp32
+    void* Y;              // [B,H,N,D]
+    int B, H, N, M;
+    float scale_log2;
+};
+
+template <typename T, typename TQ, int D>
+__global__ void __launch_bounds__(kSimtThreads)
+decode_simt(DecodeParams p) {
+    constexpr int MC = 2048 / D;
+    __shared__ __align__(16) float sQ[MC * D];
+    __shared__ __align__(16) float sZ[MC * D];
+    const int bh = blockIdx.y;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const int n = blockIdx.x * kSimtThreads + threadIdx.x;
+    const bool active = n < p.N;
+
+    float kq[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) kq[d] = 0.f;
+    if (active) {
+        load_row_f32<T, D>(reinterpret_cast<const T*>(p.Ktok) + ((int64_t)bh * p.N + n) * D, kq);
+#pragma unroll
+        for (int d = 0; d < D; ++d) kq[d] *= p.scale_log2;
+    }
+    float mx = -INFINITY, l = 0.f, acc[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) acc[d] = 0.f;
+
+    const TQ* Qbh = reinterpret_cast<const TQ*>(p.Qlat) + (int64_t)(b * p.q_batch_heads + h) * p.M * D;
+    const float* Zbh = p.Z + (int64_t)bh * p.M * D;
+    constexpr int VEC = 16 / sizeof(TQ);
+    for (int m0 = 0; m0 < p.M; m0 += MC) {
+        const int cnt = min(MC, p.M - m0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < cnt * D / VEC; i += kSimtThreads) {
+            float tmp[VEC];
+            load_row_f32<TQ, VEC>(Qbh + (int64_t)m0 * D + i * VEC, tmp);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) sQ[i * VEC + e] = tmp[e];
+        }
+        for (int i = threadIdx.x; i < cnt * D / 4; i += kSimtThreads)
+            reinterpret_cast<float4*>(sZ)[i] = reinterpret_cast<const float4*>(Zbh + (int64_t)m0 * D)[i];
+        __syncthreads();
+        if (active) {
+            for (int j = 0; j < cnt; ++j) {
+                const float* qr = sQ + j * D;
+                float s = 0.f;
+#pragma unroll
+                for (int d = 0; d < D; ++d) s = fmaf(kq[d], qr[d], s);
+                if (s > mx) {
+                    const float corr = ex2_mufu(mx - s);
+                    l *= corr;
+#pragma unroll
+                    for (int d = 0; d < D; ++d) acc[d] *= corr;
+                    mx = s;
+                }
+                const float w = ex2_mufu(s - mx);
+                l += w;
+                const float* zr = sZ + j * D;
+#pragma unroll
+                for (int d = 0; d < D; ++d) acc[d] = fmaf(w, zr[d], acc[d]);
+            }
+        }
+    }
+    if (active) {
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int d = 0; d < D; ++d) acc[d] *= inv;
+        store_row<T, D>(reinterpret_cast<T*>(p.Y) + ((int64_t)bh * p.N + n) * D, acc);
+    }
+}
+
+}  // namespace flarepp

@@ -1,0 +1,118 @@
+"""The C-ABI library loads and exports what include/flarepp.h declares, and its
+host-side argument checks answer before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rank_latent_attention_mixer_b200 import build
+    build.build()
+    from rank_latent_attention_mixer_b200 import binding
+    return binding
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(flare[a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entries():
+    names = declared_functions()
+    for required in ("flarepp_mixer_fwd", "flare_fwd", "flarepp_workspace_bytes", "flarepp_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib.lib, name), f"libflarepp.so does not export {name}"
+    assert set(lib.EXPORTS) <= set(declared_functions())
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.lib.flarepp_abi_version() == 1
+    assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
+    for code in range(6):
+        assert lib.status_string(code) not in ("", "unknown status")
+    assert lib.status_string(99) == "unknown status"
+
+
+def _fwd(lib, ptrs, B=1, H=2, N=64, M=16, D=16, dtype=1):
+    return lib.lib.flarepp_mixer_fwd(*ptrs, B, H, N, M, D, dtype, None)
+
+
+FAKE = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]  # 16-byte aligned, never dereferenced
+
+
+def test_null_pointers_rejected(lib):
+    for i in (1, 4, 5, 6):        # q_fixed, k, v, y are always required
+        p = list(FAKE)
+        p[i] = None
+        assert _fwd(lib, p) == 1
+    p = list(FAKE)
+    p[0] = None                   # q0 required when the gate is open
+    assert _fwd(lib, p) == 1
+    p[3] = None                   # k0 as well
+    assert _fwd(lib, p) == 1
+
+
+def test_bad_sizes_and_dtype(lib):
+    assert _fwd(lib, FAKE, B=0) == 1
+    assert _fwd(lib, FAKE, N=0) == 1
+    assert _fwd(lib, FAKE, M=-3) == 1
+    assert _fwd(lib, FAKE, dtype=7) == 1
+    assert _fwd(lib, FAKE, D=48) == 2
+    assert _fwd(lib, FAKE, D=256) == 2
+    assert _fwd(lib, FAKE, M=5000) == 2
+    assert _fwd(lib, FAKE, B=300, H=300) == 2
+
+
+def test_misaligned_and_overlapping_rejected(lib):
+    p = list(FAKE)
+    p[4] = 0x20008                # k misaligned
+    assert _fwd(lib, p) == 1
+    p = list(FAKE)
+    p[6] = p[5] + 16              # y overlaps v
+    assert _fwd(lib, p) == 1
+    p = list(FAKE)
+    p[2] = 0x30002                # gate not 4-byte aligned
+    assert _fwd(lib, p) == 1
+
+
+def test_options_checked(lib):
+    o = lib.Options(0.0, 9, 0, 0, None, None, None, 0, None)
+    rc = lib.lib.flarepp_mixer_fwd_ex(*FAKE, 1, 2, 64, 16, 16, 1, ctypes.byref(o), None)
+    assert rc == 1
+    o = lib.Options(0.0, 0, 0, 5, None, None, None, 0, None)   # events promised, none given
+    rc = lib.lib.flarepp_mixer_fwd_ex(*FAKE, 1, 2, 64, 16, 16, 1, ctypes.byref(o), None)
+    assert rc == 1
+    o = lib.Options(0.0, 0, 0, 0, None, None, 0x1000, 16, None)   # workspace too small
+    rc = lib.lib.flarepp_mixer_fwd_ex(*FAKE, 1, 2, 64, 16, 16, 1, ctypes.byref(o), None)
+    assert rc == 4
+
+
+def test_workspace_and_path_queries(lib):
+    assert lib.workspace_bytes(1, 2, 1024, 16, 16, lib.F32) > 0
+    assert lib.workspace_bytes(1, 2, 1024, 16, 48, lib.F32) == 0
+    assert lib.selected_path(1, 2, 1024, 16, 16, lib.F32) == lib.PATH_SIMT
+    assert lib.selected_path(1, 2, 1024, 16, 48, lib.F32) == 0
+    # more forced chunks -> more partial triples -> more scratch
+    a = lib.workspace_bytes(1, 8, 100000, 64, 32, lib.BF16, force_chunks=1)
+    b = lib.workspace_bytes(1, 8, 100000, 64, 32, lib.BF16, force_chunks=16)
+    assert 0 < a < b
+
+
+def test_flare_entry_checks(lib):
+    assert lib.lib.flare_fwd(None, FAKE[4], FAKE[5], FAKE[6], 1, 2, 64, 16, 16, 1, None) == 1
+    assert lib.lib.flare_fwd(FAKE[1], FAKE[4], FAKE[5], FAKE[6], 1, 2, 64, 16, 40, 1, None) == 2

@@ -1,0 +1,222 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs, through the C ABI.
+
+Covers the four workloads the oracle finishes in seconds (whole outputs y, q
+and z), the closed-gate FLARE form, every supported head dim, ragged and
+degenerate sizes, forced chunk counts (the token-split/log-sum-exp merge is
+exact up to rounding), both kernel families, and the ABI variants (explicit
+or library-managed scratch, host buffers)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_parity, metrics, to64
+from rank_latent_attention_mixer_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+_ORACLE_CACHE = {}
+
+
+def binding():
+    from rank_latent_attention_mixer_b200 import binding as b
+    return b
+
+
+def oracle_out(name, x, flare=False):
+    key = (name, flare)
+    if key not in _ORACLE_CACHE:
+        _ORACLE_CACHE[key] = oracle.flarepp(x["q0"], x["q_fixed"], None if flare else x["gate"],
+                                            x["k0"], x["k"], x["v"], flare=flare)
+    return _ORACLE_CACHE[key]
+
+
+def cuda_inputs(x):
+    return {k: v.to(DEV) for k, v in x.items()}
+
+
+def run(x, path=0, force_chunks=0, flare=False, scale=0.0):
+    b = binding()
+    d = cuda_inputs(x)
+    y, q, z = b.mixer_fwd(d["q0"], d["q_fixed"], None if flare else d["gate"], d["k0"], d["k"], d["v"],
+                          return_qz=True, path=path, force_chunks=force_chunks, scale=scale)
+    torch.cuda.synchronize()
+    assert b.check_device_status() == 0
+    return y, q, z
+
+
+SMALL = ["tiny_f32", "grid85_bf16", "grid129_peaky_bf16", "cloud40k_bf16"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+@pytest.mark.parametrize("path", [0, 1], ids=["auto", "simt"])
+def test_workload_parity(name, path):
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w)
+    y_ref, q_ref, z_ref = oracle_out(name, x)
+    y, q, z = run(x, path=path)
+    assert_parity(q, q_ref, w.dtype, "q")
+    assert_parity(z, z_ref, w.dtype, "z")
+    m = assert_parity(y, y_ref, w.dtype, "y")
+    print(name, path, m)
+
+
+@pytest.mark.parametrize("name", ["grid85_bf16", "tiny_f32"])
+def test_closed_gate_is_flare(name):
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w)
+    y_ref, _, _ = oracle_out(name, x, flare=True)
+    b = binding()
+    d = cuda_inputs(x)
+    y_flare = b.flare_fwd(d["q_fixed"], d["k"], d["v"])
+    y_null = b.mixer_fwd(d["q0"], d["q_fixed"], None, d["k0"], d["k"], d["v"])
+    y_zero = b.mixer_fwd(d["q0"], d["q_fixed"], torch.zeros_like(d["gate"]), d["k0"], d["k"], d["v"])
+    torch.cuda.synchronize()
+    assert_parity(y_flare, y_ref, w.dtype, "y(flare)")
+    assert torch.equal(y_flare, y_null)
+    assert torch.equal(y_flare, y_zero), "a zero gate must give exactly the FLARE result"
+
+
+EDGE = [
+    # B, H, N, M, D
+    (1, 1, 1, 1, 16),
+    (1, 2, 7, 5, 16),
+    (2, 1, 129, 17, 32),
+    (1, 3, 300, 64, 64),
+    (1, 1, 1000, 1, 64),
+    (1, 2, 257, 130, 128),
+    (3, 2, 513, 64, 16),
+    (1, 1, 4097, 256, 32),
+    (1, 2, 2000, 512, 64),
+    (1, 1, 640, 100, 32),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: "x".join(map(str, s)))
+def test_edge_shapes(shape, dtype):
+    B, H, N, M, D = shape
+    x = W.random_inputs(B, H, N, M, D, dtype=dtype, seed=sum(shape))
+    y_ref, q_ref, z_ref = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+    y, q, z = run(x)
+    assert_parity(q, q_ref, dtype, "q")
+    assert_parity(z, z_ref, dtype, "z")
+    assert_parity(y, y_ref, dtype, "y")
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["auto", "simt"])
+def test_chunk_invariance(path):
+    x = W.random_inputs(2, 2, 3001, 128, 32, dtype="bf16", seed=5)
+    y_ref, _, z_ref = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+    outs = []
+    for fc in (0, 1, 2, 7):
+        y, q, z = run(x, path=path, force_chunks=fc)
+        assert_parity(y, y_ref, "bf16")
+        outs.append((y, q, z))
+    for y, q, z in outs[1:]:
+        # the merge is exact up to fp32 rounding of the combination order
+        assert metrics(z, outs[0][2])["max_abs"] < 1e-4
+        assert metrics(q, outs[0][1])["max_abs"] < 1e-4
+
+
+def test_scale_argument_flare_scale_one():
+    """The FLARE block printed with scale=1.0, via the options' scale."""
+    x = W.random_inputs(1, 2, 500, 32, 16, dtype="f32", seed=3)
+    y_ref, _, _ = oracle.flarepp(None, x["q_fixed"], None, None, x["k"], x["v"], scale=1.0, flare=True)
+    y, _, _ = run(x, flare=True, scale=1.0)
+    assert_parity(y, y_ref, "f32")
+
+
+def test_deterministic_and_abi_variants():
+    w = W.WORKLOADS["grid85_bf16"]
+    x = W.make_inputs(w)
+    d = cuda_inputs(x)
+    b = binding()
+    y1 = b.mixer_fwd(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"])
+    y2 = b.mixer_fwd(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"])
+    y3 = b.mixer_fwd_plain(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"], torch.empty_like(d["k"]))
+    hx = {k: v.pin_memory() for k, v in x.items()}
+    y4 = torch.empty_like(hx["k"]).pin_memory()
+    b.mixer_fwd_host(hx["q0"], hx["q_fixed"], hx["gate"], hx["k0"], hx["k"], hx["v"], y4)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert torch.equal(y1, y3)
+    assert torch.equal(y1.cpu(), y4)
+
+
+def test_invariants_on_gpu():
+    # single latent: every token gets the latent's value
+    x = W.random_inputs(1, 2, 999, 1, 32, dtype="f32", seed=11)
+    y, _, z = run(x)
+    assert torch.allclose(y, z.expand_as(y), rtol=1e-5, atol=1e-6)
+    # identical keys: encode returns the mean of v
+    x = W.random_inputs(1, 2, 777, 16, 32, dtype="f32", seed=12)
+    x["k"][:] = x["k"][:, :, :1]
+    _, _, z = run(x)
+    mean_v = x["v"].double().mean(dim=2, keepdim=True).expand(-1, -1, 16, -1)
+    assert metrics(z, mean_v)["max_abs"] < 1e-5
+    # convex hull: each y coordinate within the latents' range
+    x = W.random_inputs(2, 2, 3000, 64, 16, dtype="bf16", seed=13)
+    y, _, z = run(x)
+    lo = z.min(dim=2, keepdim=True).values
+    hi = z.max(dim=2, keepdim=True).values
+    tol = 2 ** -7 * z.abs().max()
+    yf = y.float()
+    assert bool(((yf >= lo - tol) & (yf <= hi + tol)).all())
+
+
+def test_permutation_equivariance_gpu():
+    x = W.random_inputs(1, 2, 2500, 64, 32, dtype="f32", seed=21)
+    perm = torch.randperm(2500, generator=torch.Generator().manual_seed(0))
+    xp = dict(x)
+    for kname in ("k0", "k", "v"):
+        xp[kname] = x[kname][:, :, perm].contiguous()
+    y, q, z = run(x)
+    yp, qp, zp = run(xp)
+    assert metrics(qp, q)["max_rel"] < 1e-4 and metrics(zp, z)["max_rel"] < 1e-4
+    assert metrics(yp, y[:, :, perm.to(y.device)])["max_rel"] < 1e-4
+
+
+def test_scale1m_sampled():
+    """The 1M-token workload in the launch configuration the benchmark times:
+    one head checked in full for q and z, and 256 sampled tokens of y."""
+    w = W.WORKLOADS["scale1m_bf16"]
+    x = W.make_inputs(w, device=DEV)
+    b = binding()
+    y, q, z = b.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], return_qz=True)
+    torch.cuda.synchronize()
+    assert b.check_device_status() == 0
+    h = 5
+    toks = torch.randint(0, w.N, (256,), generator=torch.Generator().manual_seed(1)).numpy()
+    toks[:2] = [0, w.N - 1]
+    y_ref, q_ref, z_ref = oracle.flarepp_head(x["q0"][h], x["q_fixed"][h], float(x["gate"][h]),
+                                              x["k0"][0, h], x["k"][0, h], x["v"][0, h], toks)
+    assert_parity(q[0, h], q_ref, "bf16", "q")
+    assert_parity(z[0, h], z_ref, "bf16", "z")
+    assert_parity(y[0, h, torch.from_numpy(toks).to(DEV)], y_ref, "bf16", "y")
+    assert bool(torch.isfinite(y.float()).all())
+
+
+def test_golden_fixture_gpu():
+    from test_golden import load_golden
+    c, x, ref = load_golden()
+    t = {k: torch.from_numpy(v) for k, v in x.items()}
+    for k in ("q0", "q_fixed", "k0", "k", "v"):
+        t[k] = t[k].to(torch.bfloat16)
+    t["gate"] = t["gate"].float()
+    y, q, z = run(t)
+    assert_parity(y, ref["y"], "bf16")
+    assert_parity(q, ref["q"], "bf16")
+
+
+def test_invalid_args_on_gpu():
+    b = binding()
+    x = cuda_inputs(W.random_inputs(1, 2, 64, 16, 16, dtype="bf16"))
+    with pytest.raises(b.FlareppError) as e:
+        b.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], y=x["k"])  # y aliases k
+    assert e.value.status == 1
+    xf = cuda_inputs(W.random_inputs(1, 2, 64, 16, 16, dtype="f32"))
+    with pytest.raises(b.FlareppError) as e:       # fp32 I/O has no tensor-core path
+        b.mixer_fwd(xf["q0"], xf["q_fixed"], xf["gate"], xf["k0"], xf["k"], xf["v"], path=b.PATH_TCGEN05)
+    assert e.value.status == 2
