@@ -1,13 +1,695 @@
-// tcgen05 (5th-generation tensor core) kernels of the FLARE++ mixer.
+// tcgen05 (5th-generation tensor core) kernels of the FLARE++ mixer, bf16 I/O.
+//
+// One warp-specialised attention kernel serves all three SDPA calls of the
+// FLARE++ block (FLARE.py README, "FLARE++" code block):
+//   * split mode  -- synthesis q_dyn = SDPA(q0, k0, k0) and encode
+//                    z = SDPA(q, k, v): the query rows are the M latents, the
+//                    key/value rows are one chunk of the N tokens, and the
+//                    output is the online-softmax triple (row max, row sum,
+//                    unnormalised weighted sum) of every latent over the chunk,
+//                    merged across chunks by merge_partials (log-sum-exp
+//                    combine; physicsnemo issue #2024, section 2);
+//   * decode mode -- y = SDPA(k, q, z): the query rows are tokens, the
+//                    key/value rows are the M latents of q and z, and the
+//                    output is the normalised y row in bf16.
+//
+// Per CTA (persistent, one per SM, 320 threads):
+//   warps 0-3  softmax warpgroup 0  (query-row tile 0, TMEM lanes 0-127)
+//   warps 4-7  softmax warpgroup 1  (query-row tile 1)
+//   warp  8    TMA producer: query tiles and a ring of key/value tiles
+//   warp  9    MMA issuer: S_w = Q_w K^T into TMEM, O_w += P_w V into TMEM
+// Each softmax thread owns one query row: it reads its 128 scores from TMEM,
+// takes exponentials base 2, writes the bf16 weights P to shared memory in the
+// tcgen05 K-major 128-byte-swizzled layout, and rescales its O row in TMEM
+// only when its running max grows by more than 2^8 (the final normalisation
+// uses the same stale max, so the result is exact up to rounding).
+// The MMA warp runs the score MMA of the job two ahead before the value MMA of
+// the current job, so the two warpgroups' softmaxes alternate with the tensor
+// core (ping-pong).
+//
+// Every wait on an mbarrier is bounded (about 2 s of %globaltimer); on expiry
+// the kernel records FLAREPP_ERR_TIMEOUT in the device status word, raises a
+// CTA-wide abort flag that every other wait checks, drains its outstanding
+// tensor-core work (bounded), frees its TMEM and returns.
 #pragma once
 
+#include <cuda.h>
+#include <mutex>
+
 #include "common.cuh"
+#include "kernels_simt.cuh"
 
 namespace flarepp {
 namespace tc {
 
-constexpr int kTokTile = 128;        // tokens per K/V tile
-constexpr int kPartsPerChunk = 2;    // partial triples written per token chunk
+constexpr int kTokTile = 128;        // rows per key/value tile and per query tile
+constexpr int kPartsPerChunk = 2;    // upper bound of partial triples per token chunk
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kStatusTimeout = 5;    // FLAREPP_ERR_TIMEOUT
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits until the phase with the given parity has completed.  Returns false
+// if the CTA's abort flag is up or the wait ran past kWaitLimitNs (then it
+// raises the flag and records the timeout).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
+                *abort_flag = 1;
+                record_status(kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on `bar` when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane -> 32 registers.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of tcgen05: start address, leading and
+// stride byte offsets (16-byte units), descriptor version 1, layout type.
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
+    return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, bf16 A
+// and B, A K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------ kernel parameters
+
+enum Mode { kSplit = 0, kDecode = 1 };
+
+struct Params {
+    int mode;             // Mode
+    int B, H;
+    int M, N;             // latents, tokens
+    int q_rows;           // rows of the query tensor per (b, h)  (M in split mode, N in decode)
+    int kv_rows;          // rows of the key/value tensors per (b, h) (N in split mode, M in decode)
+    int kv_tiles;         // ceil(kv_rows / 128)
+    int q_shared;         // query map's z coordinate is h (tensor [H, rows, D]) instead of b*H+h
+    int k_shared;         // key map's z coordinate is h
+    int kv_same;          // values are the keys (synthesis): load one tile per stage
+    int interleave;       // split mode with M <= 128: both warpgroups share query tile 0 and take
+                          // alternate key/value tiles, each writing its own partial triple
+    int row_groups;       // split mode, not interleaved: 256-row latent groups per (b, h)
+    int chunks;           // split mode: token chunks per (b, h)
+    int chunk_tiles;      // split mode: 128-token tiles per chunk
+    int q_pairs;          // decode mode: 256-token query groups per (b, h)
+    int items;
+    float scale_log2;
+    float* part_O;        // split: [parts][B*H][M][D]
+    float2* part_ml;      // split: [parts][B*H][M]
+    __nv_bfloat16* y;     // decode: [B,H,N,D]
+};
+
+struct Item {
+    int bh, qz, kz, vz;
+    int qrow0;            // first query row of the item
+    int t_begin, t_end;   // key/value tile range
+    int part;             // split mode: partial index of warpgroup 0 (interleaved: 2c, else c)
+};
+
+__device__ __forceinline__ Item decode_item(const Params& p, int item) {
+    Item it;
+    if (p.mode == kSplit) {
+        const int G = p.interleave ? 1 : p.row_groups;
+        const int g = item % G;
+        const int rest = item / G;
+        const int c = rest % p.chunks;
+        it.bh = rest / p.chunks;
+        it.qrow0 = g * 256;
+        it.t_begin = c * p.chunk_tiles;
+        it.t_end = min(p.kv_tiles, it.t_begin + p.chunk_tiles);
+        it.part = p.interleave ? 2 * c : c;
+    } else {
+        const int pi = item % p.q_pairs;
+        it.bh = item / p.q_pairs;
+        it.qrow0 = pi * 256;
+        it.t_begin = 0;
+        it.t_end = p.kv_tiles;
+        it.part = 0;
+    }
+    const int h = it.bh % p.H;
+    it.qz = p.q_shared ? h : it.bh;
+    it.kz = p.k_shared ? h : it.bh;
+    it.vz = it.bh;
+    return it;
+}
+
+// Shared-memory plan for head dim D, NST key/value stages, QS query slots.
+template <int D, int NST, int QS>
+struct Smem {
+    static constexpr int kTileBytes = kTokTile * D * 2;             // one [128 x D] bf16 tile
+    static constexpr int kQ = 0;                                     // QS slots x 2 tiles
+    static constexpr int kKV = kQ + QS * 2 * kTileBytes;             // NST stages x (K, V)
+    static constexpr int kP = kKV + NST * 2 * kTileBytes;            // 2 warpgroups x [128 x 128] bf16
+    static constexpr int kPBytes = 128 * 128 * 2;
+    static constexpr int kBar = kP + 2 * kPBytes;
+    // barriers: kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull[2], sfree[2], pfull[2], pfree[2], drain
+    static constexpr int kNumBars = 2 * NST + 2 * QS + 8 + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;               // tmem base (u32), abort flag (int)
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kLaunchBytes = kBytes + 1024;              // + alignment slack
+};
+
+template <int D>
+struct Layout {
+    // swizzle of a [rows x D] bf16 tile whose rows are D*2 bytes
+    static constexpr uint32_t kType = D == 64 ? kLayoutSw128 : (D == 32 ? kLayoutSw64 : kLayoutSw32);
+    static constexpr uint32_t kRowBytes = D * 2;
+    static constexpr uint32_t kSbo = 8 * kRowBytes;                  // 8-row group stride
+    // TMEM column stride between the two warpgroups' O accumulators: at least
+    // 32 so that 32-column TMEM loads/stores of one never touch the other's
+    static constexpr int kOStride = D < 32 ? 32 : D;
+};
+
+// ------------------------------------------------------------------ the kernel
+
+template <int D, int NST, int QS>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+            const __grid_constant__ CUtensorMap map_v, const Params p) {
+    static_assert(D == 16 || D == 32 || D == 64, "tcgen05 path covers D in {16, 32, 64}");
+    static_assert(NST >= 3, "the score MMA runs two jobs ahead: at least three key/value stages");
+    using SM = Smem<D, NST, QS>;
+    using LY = Layout<D>;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+    uint64_t* kv_full = bars;
+    uint64_t* kv_empty = bars + NST;
+    uint64_t* q_full = bars + 2 * NST;
+    uint64_t* q_empty = q_full + QS;
+    uint64_t* sfull = q_empty + QS;
+    uint64_t* sfree = sfull + 2;
+    uint64_t* pfull = sfree + 2;
+    uint64_t* pfree = pfull + 2;
+    uint64_t* drain = pfree + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+        for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&sfull[w], 1);
+            mbar_init(&sfree[w], 4);
+            mbar_init(&pfull[w], 4);
+            mbar_init(&pfree[w], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        prefetch_tensormap(&map_q);
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+    }
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kTmaWarp) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            uint32_t kv_load = 0, q_load = 0;
+            int kv_last_phase[NST], q_last_phase[QS];
+            for (int i = 0; i < NST; ++i) kv_last_phase[i] = -1;
+            for (int i = 0; i < QS; ++i) q_last_phase[i] = -1;
+            const uint32_t kv_bytes = (p.kv_same ? 1 : 2) * SM::kTileBytes;
+            const uint32_t q_bytes = (p.interleave ? 1 : 2) * SM::kTileBytes;
+            bool ok = true;
+            for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+                const Item it = decode_item(p, item);
+                const int slot = q_load % QS;
+                ok = mbar_wait(&q_empty[slot], ((q_load / QS) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                mbar_expect_tx(&q_full[slot], q_bytes);
+                uint8_t* qdst = smem + SM::kQ + slot * 2 * SM::kTileBytes;
+                tma_load_3d(qdst, &map_q, &q_full[slot], 0, it.qrow0, it.qz);
+                if (!p.interleave)
+                    tma_load_3d(qdst + SM::kTileBytes, &map_q, &q_full[slot], 0, it.qrow0 + kTokTile, it.qz);
+                q_last_phase[slot] = (q_load / QS) & 1;
+                ++q_load;
+                for (int t = it.t_begin; t < it.t_end; ++t) {
+                    const int st = kv_load % NST;
+                    ok = mbar_wait(&kv_empty[st], ((kv_load / NST) & 1) ^ 1, abort_flag);
+                    if (!ok) break;
+                    mbar_expect_tx(&kv_full[st], kv_bytes);
+                    uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kTileBytes;
+                    tma_load_3d(kdst, &map_k, &kv_full[st], 0, t * kTokTile, it.kz);
+                    if (!p.kv_same)
+                        tma_load_3d(kdst + SM::kTileBytes, &map_v, &kv_full[st], 0, t * kTokTile, it.vz);
+                    kv_last_phase[st] = (kv_load / NST) & 1;
+                    ++kv_load;
+                }
+            }
+            if (!ok) {
+                // Let the copies already issued land before the CTA exits (bounded):
+                // the last phase issued on each barrier completes when its bytes arrive.
+                const unsigned long long t0 = globaltimer_ns();
+                for (int s = 0; s < NST; ++s)
+                    while (kv_last_phase[s] >= 0 && !mbar_try_wait(&kv_full[s], kv_last_phase[s]) &&
+                           globaltimer_ns() - t0 < 100000000ull) {
+                    }
+                for (int s = 0; s < QS; ++s)
+                    while (q_last_phase[s] >= 0 && !mbar_try_wait(&q_full[s], q_last_phase[s]) &&
+                           globaltimer_ns() - t0 < 100000000ull) {
+                    }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = make_idesc(128, 128, false);   // S = Q K^T: [128 q x 128 kv]
+            constexpr uint32_t idesc_o = make_idesc(128, D, true);      // O += P V:  [128 q x D], V MN-major
+            // Job stream: (item, warpgroup, tile).  Two cursors over the same
+            // stream: `sc` issues score MMAs two jobs ahead of `pc`, which
+            // issues the value MMAs.
+            struct Cursor {
+                int item, t, w, njobs_w[2];
+                bool valid;
+                Item info;
+                uint32_t tile_count, item_count;
+            };
+            auto first_job = [&](Cursor& c) {
+                c.item = blockIdx.x;
+                c.tile_count = 0;
+                c.item_count = 0;
+                c.valid = c.item < p.items;
+                if (c.valid) {
+                    c.info = decode_item(p, c.item);
+                    c.t = c.info.t_begin;
+                    c.w = 0;
+                    c.njobs_w[0] = c.njobs_w[1] = 0;
+                }
+            };
+            auto next_job = [&](Cursor& c) {
+                // advance within the item
+                bool tile_done;
+                if (p.interleave) {
+                    tile_done = true;
+                } else {
+                    tile_done = (c.w == 1);
+                }
+                c.njobs_w[c.w]++;
+                if (!tile_done) {
+                    c.w = 1;
+                    return;
+                }
+                ++c.tile_count;
+                ++c.t;
+                if (c.t < c.info.t_end) {
+                    c.w = p.interleave ? ((c.t - c.info.t_begin) & 1) : 0;
+                    return;
+                }
+                ++c.item_count;
+                c.item += gridDim.x;
+                c.valid = c.item < p.items;
+                if (c.valid) {
+                    c.info = decode_item(p, c.item);
+                    c.t = c.info.t_begin;
+                    c.w = 0;
+                    c.njobs_w[0] = c.njobs_w[1] = 0;
+                }
+            };
+            uint32_t s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
+            bool ok = true;
+            Cursor sc, pc;
+            first_job(sc);
+            first_job(pc);
+            auto issue_s = [&](const Cursor& c) -> bool {
+                const int w = c.w;
+                const bool first_of_item = (c.t == c.info.t_begin) && (w == 0);
+                const bool first_use = p.interleave || w == 0;
+                const int slot = c.item_count % QS;
+                if (first_of_item) {
+                    if (!mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag)) return false;
+                }
+                const int st = c.tile_count % NST;
+                if (first_use) {
+                    if (!mbar_wait(&kv_full[st], (c.tile_count / NST) & 1, abort_flag)) return false;
+                }
+                if (!mbar_wait(&sfree[w], (s_issued[w] & 1) ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t qaddr = smem_u32(smem + SM::kQ + slot * 2 * SM::kTileBytes +
+                                                (p.interleave ? 0 : w * SM::kTileBytes));
+                const uint32_t kaddr = smem_u32(smem + SM::kKV + st * 2 * SM::kTileBytes);
+                const uint32_t d_tmem = tmem + w * 128;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = smem_desc(qaddr + kk * 32, 16, LY::kSbo, LY::kType);
+                    const uint64_t bd = smem_desc(kaddr + kk * 32, 16, LY::kSbo, LY::kType);
+                    umma_bf16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&sfull[w]);
+                ++s_issued[w];
+                // last score MMA of the item frees the query slot once it completes
+                const bool last_of_item = (c.t == c.info.t_end - 1) && (p.interleave || w == 1);
+                if (last_of_item) umma_commit(&q_empty[slot]);
+                return true;
+            };
+            auto issue_pv = [&](const Cursor& c) -> bool {
+                const int w = c.w;
+                if (!mbar_wait(&pfull[w], pv_issued[w] & 1, abort_flag)) return false;
+                tc_fence_after();
+                const int st = c.tile_count % NST;
+                const uint32_t paddr = smem_u32(smem + SM::kP + w * SM::kPBytes);
+                const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kTileBytes + (p.kv_same ? 0 : SM::kTileBytes);
+                const uint32_t vaddr = smem_u32(vbase);
+                const uint32_t d_tmem = tmem + 256 + w * LY::kOStride;
+                const bool first_of_w = c.njobs_w[w] == 0;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // A = P: K-major, 128B swizzle, two 64-column atoms of 16 KB
+                    const uint64_t ad = smem_desc(paddr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSw128);
+                    // B = V tile [128 kv x D], D contiguous: MN-major; 16 kv rows per step
+                    // (D fits one swizzle atom along MN, so the leading offset is never used)
+                    const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kTileBytes,
+                                                  LY::kSbo, LY::kType);
+                    umma_bf16(d_tmem, ad, bd, idesc_o, (first_of_w && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&pfree[w]);
+                ++pv_issued[w];
+                const bool last_use = p.interleave || w == 1;
+                if (last_use) umma_commit(&kv_empty[st]);
+                return true;
+            };
+            // prologue: two score MMAs
+            for (int k = 0; k < 2 && sc.valid && ok; ++k) {
+                ok = issue_s(sc);
+                next_job(sc);
+            }
+            while (pc.valid && ok) {
+                if (sc.valid) {
+                    ok = issue_s(sc);
+                    if (!ok) break;
+                    next_job(sc);
+                }
+                ok = issue_pv(pc);
+                next_job(pc);
+            }
+            // drain: wait until every issued MMA has completed before TMEM is released
+            umma_commit(drain);
+            const unsigned long long t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- softmax warpgroups
+        const int wg = warp >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base + wg * 128;
+        const uint32_t tO = tmem + lane_base + 256 + wg * LY::kOStride;
+        uint8_t* pbuf = smem + SM::kP + wg * SM::kPBytes;
+        const float sl2 = p.scale_log2;
+        uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+            const Item it = decode_item(p, item);
+            float m_run = -INFINITY, l_run = 0.f;
+            int njobs = 0;
+            const int tstep = p.interleave ? 2 : 1;
+            for (int t = it.t_begin + (p.interleave ? wg : 0); t < it.t_end; t += tstep) {
+                if (!mbar_wait(&sfull[wg], sfull_waits & 1, abort_flag)) { ok = false; break; }
+                ++sfull_waits;
+                tc_fence_after();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[wg]);
+
+                const int valid = p.kv_rows - t * kTokTile;      // key/value rows of this tile that exist
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        float s = __uint_as_float(sr[c][j]);
+                        if (c * 32 + j >= valid) s = -INFINITY;
+                        sr[c][j] = __float_as_uint(s);
+                        mx = fmaxf(mx, s);
+                    }
+                }
+                const float m_new = fmaxf(m_run, mx * sl2);
+                float factor = 1.f;
+                const bool resc = m_new > m_run + kRescaleLog2;
+                if (resc) {
+                    factor = ex2_mufu(m_run - m_new);
+                    m_run = m_new;
+                }
+                const float neg_m = -m_run;
+                float rs = 0.f;
+                uint32_t pk[64];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float p0 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j]), sl2, neg_m));
+                        const float p1 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j + 1]), sl2, neg_m));
+                        rs += p0 + p1;
+                        pk[c * 16 + j] = pack_bf16x2(p0, p1);
+                    }
+                }
+                l_run = l_run * factor + rs;
+
+                // the previous value MMA of this warpgroup must be done before P and O are touched
+                while (pfree_waits < jobs_done) {
+                    if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                    ++pfree_waits;
+                }
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, resc && njobs > 0)) {
+                    const float f = njobs > 0 ? factor : 1.f;
+#pragma unroll
+                    for (int c = 0; c < D / 32 + (D % 32 ? 1 : 0); ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+                        tmem_st32(tO + c * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+                // P row -> shared memory, K-major 128-byte swizzle: 16-byte chunk c of a
+                // 128-byte row r sits at chunk position c ^ (r % 8)
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) {
+                    const int atom = ch >> 3, c8 = ch & 7;
+                    uint8_t* dst = pbuf + atom * 16384 + row * 128 + ((c8 ^ (row & 7)) << 4);
+                    *reinterpret_cast<uint4*>(dst) =
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pfull[wg]);
+                ++jobs_done;
+                ++njobs;
+            }
+            if (!ok) break;
+
+            // ---------------- epilogue of the item
+            uint32_t o[(D + 31) / 32][32];
+            if (njobs > 0) {
+                while (pfree_waits < jobs_done) {
+                    if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                    ++pfree_waits;
+                }
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < (D + 31) / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+                tmem_wait_ld();
+                tc_fence_before();
+            } else {
+#pragma unroll
+                for (int c = 0; c < (D + 31) / 32; ++c)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[c][j] = 0u;
+            }
+            // with D = 16 only the first 16 columns of the 32-column load are O (the
+            // rest belong to the other warpgroup's O or are unused)
+            if (p.mode == kSplit) {
+                const int r = p.interleave ? row : it.qrow0 + wg * kTokTile + row;
+                const int part = p.interleave ? it.part + wg : it.part;
+                if (r < p.M) {
+                    const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
+                    p.part_ml[ridx] = make_float2(njobs > 0 ? m_run : -INFINITY, l_run);
+                    float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D);
+#pragma unroll
+                    for (int i = 0; i < D / 4; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
+                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
+                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
+                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 3]));
+                }
+            } else {
+                const int n = it.qrow0 + wg * kTokTile + row;
+                if (n < p.N) {
+                    const float inv = 1.f / l_run;
+                    uint4* dst = reinterpret_cast<uint4*>(p.y + ((int64_t)it.bh * p.N + n) * D);
+#pragma unroll
+                    for (int i = 0; i < D / 8; ++i) {
+                        const int c = i / 4, j = (i % 4) * 8;
+                        dst[i] = make_uint4(
+                            pack_bf16x2(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
 
 struct Buffers {
     float* part_O;
@@ -24,14 +706,173 @@ struct Problem {
     float scale_log2;
 };
 
-inline bool supported(bool bf16, int D, int M) { (void)bf16; (void)D; (void)M; return false; }
-inline int row_groups(int M) { return (M + 255) / 256; }
+inline bool supported(bool bf16, int D, int M) {
+    (void)M;
+    return bf16 && (D == 16 || D == 32 || D == 64);
+}
+
+// latent-row groups handled per (b, h, chunk): one 256-row group per item,
+// or a single shared 128-row tile when M <= 128 (interleaved)
+inline int row_groups(int M) { return M <= 128 ? 1 : (M + 255) / 256; }
+inline bool interleaved(int M) { return M <= 128; }
+inline int parts_per_chunk(int M) { return interleaved(M) ? 2 : 1; }
 inline int target_ctas() { return 4 * kNumSMs; }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over a [planes, rows, D] bf16 tensor, box [1, 128, D], swizzle = D*2 bytes.
+inline bool make_map(CUtensorMap* map, const void* base, int planes, int rows, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)kTokTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                          : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int sm_count() {
+    int dev = 0, n = kNumSMs;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : kNumSMs;
+}
+
+template <int D>
+struct Config {
+    static constexpr int NST = D == 64 ? 3 : 4;
+    static constexpr int QS = 2;
+    using SM = Smem<D, NST, QS>;
+    // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
+    static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
+};
+
+template <int D>
+int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& prm,
+                cudaStream_t st) {
+    using C = Config<D>;
+    auto kern = attn_kernel<D, C::NST, C::QS>;
+    static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
+        return 3;
+    const int grid = prm.items < sm_count() ? prm.items : sm_count();
+    kern<<<grid, kThreads, C::kSmemLaunch, st>>>(mq, mk, mv, prm);
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
+inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const Params& prm, cudaStream_t st) {
+    switch (D) {
+        case 16: return launch_attn<16>(mq, mk, mv, prm, st);
+        case 32: return launch_attn<32>(mq, mk, mv, prm, st);
+        case 64: return launch_attn<64>(mq, mk, mv, prm, st);
+        default: return 2;
+    }
+}
+
+template <int D>
+void launch_merge(const MergeParams& mp, int64_t rows, cudaStream_t st) {
+    merge_partials<__nv_bfloat16, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
+}
+
+inline void launch_merge_d(int D, const MergeParams& mp, int64_t rows, cudaStream_t st) {
+    switch (D) {
+        case 16: launch_merge<16>(mp, rows, st); break;
+        case 32: launch_merge<32>(mp, rows, st); break;
+        default: launch_merge<64>(mp, rows, st); break;
+    }
+}
+
+// The whole FLARE++ forward on the tcgen05 path; `mark(stream)` is called
+// before the first launch and after each launch.
 template <typename Mark>
-inline int run(const Problem&, const Buffers&, const void*, const void*, const float*, const void*,
-               const void*, const void*, void*, float*, float*, Mark&&, cudaStream_t) {
-    return 2;  // FLAREPP_ERR_UNSUPPORTED
+int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixed, const float* gate,
+        const void* k0, const void* k, const void* v, void* y, float* q_out, float* z_out, Mark&& mark,
+        cudaStream_t st) {
+    const bool gated = gate != nullptr;
+    const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
+    CUtensorMap m_q0, m_qf, m_q16, m_z16, m_k0, m_k, m_v;
+    bool ok = make_map(&m_qf, q_fixed, H, M, D) && make_map(&m_q16, bu.q16, BH, M, D) &&
+              make_map(&m_z16, bu.z16, BH, M, D) && make_map(&m_k, k, BH, N, D) && make_map(&m_v, v, BH, N, D);
+    if (gated) ok = ok && make_map(&m_q0, q0, H, M, D) && make_map(&m_k0, k0, BH, N, D);
+    if (!ok) return 3;
+
+    const int kv_tiles = (N + kTokTile - 1) / kTokTile;
+    const int chunk_tiles = pr.chunk_len / kTokTile;
+    Params sp{};
+    sp.mode = kSplit;
+    sp.B = B; sp.H = H; sp.M = M; sp.N = N;
+    sp.q_rows = M; sp.kv_rows = N; sp.kv_tiles = kv_tiles;
+    sp.interleave = interleaved(M) ? 1 : 0;
+    sp.row_groups = row_groups(M);
+    sp.chunks = pr.chunks;
+    sp.chunk_tiles = chunk_tiles;
+    sp.items = BH * pr.chunks * (sp.interleave ? 1 : sp.row_groups);
+    sp.scale_log2 = pr.scale_log2;
+    sp.part_O = bu.part_O;
+    sp.part_ml = bu.part_ml;
+    const int parts = pr.chunks * parts_per_chunk(M);
+
+    MergeParams mp{};
+    mp.part_O = bu.part_O; mp.part_ml = bu.part_ml; mp.chunks = parts;
+    mp.B = B; mp.H = H; mp.M = M; mp.q_fixed = q_fixed; mp.gate = gate;
+    const int64_t rows = (int64_t)BH * M;
+
+    int rc = 0;
+    mark(st);
+    if (gated) {
+        Params s1 = sp;
+        s1.q_shared = 1; s1.k_shared = 0; s1.kv_same = 1;
+        rc = launch_attn_d(D, m_q0, m_k0, m_k0, s1, st);
+        if (rc) return rc;
+        mark(st);
+        mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_bf16 = bu.q16; mp.user_out = q_out;
+        mp.q_copy_out = nullptr;
+        launch_merge_d(D, mp, rows, st);
+        mark(st);
+    }
+    Params s2 = sp;
+    s2.q_shared = gated ? 0 : 1; s2.k_shared = 0; s2.kv_same = 0;
+    rc = launch_attn_d(D, gated ? m_q16 : m_qf, m_k, m_v, s2, st);
+    if (rc) return rc;
+    mark(st);
+    mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_bf16 = bu.z16; mp.user_out = z_out;
+    mp.q_copy_out = gated ? nullptr : q_out;
+    launch_merge_d(D, mp, rows, st);
+    mark(st);
+
+    Params dp{};
+    dp.mode = kDecode;
+    dp.B = B; dp.H = H; dp.M = M; dp.N = N;
+    dp.q_rows = N; dp.kv_rows = M; dp.kv_tiles = (M + kTokTile - 1) / kTokTile;
+    dp.q_shared = 0; dp.k_shared = gated ? 0 : 1; dp.kv_same = 0;
+    dp.interleave = 0;
+    dp.q_pairs = (N + 255) / 256;
+    dp.items = BH * dp.q_pairs;
+    dp.scale_log2 = pr.scale_log2;
+    dp.y = static_cast<__nv_bfloat16*>(y);
+    rc = launch_attn_d(D, m_k, gated ? m_q16 : m_qf, m_z16, dp, st);
+    if (rc) return rc;
+    mark(st);
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
 }  // namespace tc
