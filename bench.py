@@ -47,6 +47,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="scale1m_bf16")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override N of the workload (a smaller case of the same kernels, e.g. for ncu)")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
@@ -255,6 +257,8 @@ def run_ours(args):
 
     w = W.WORKLOADS[args.workload]
     w = w.with_shape(seed=rank_seed(w.seed, rank))
+    if args.tokens:
+        w = w.with_shape(N=args.tokens, name=f"{w.name}_n{args.tokens}")
     x = W.make_inputs(w, device=str(dev))
     path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
     dtype_code = fb.F32 if w.dtype == "f32" else fb.BF16

@@ -115,9 +115,16 @@ def test_chunk_invariance(path):
         assert_parity(y, y_ref, "bf16")
         outs.append((y, q, z))
     for y, q, z in outs[1:]:
-        # the merge is exact up to fp32 rounding of the combination order
-        assert metrics(z, outs[0][2])["max_abs"] < 1e-4
-        assert metrics(q, outs[0][1])["max_abs"] < 1e-4
+        # The split/merge is exact up to rounding.  The SIMT path keeps the
+        # softmax weights in fp32, so chunkings agree to fp32 roundoff; the
+        # tcgen05 path rounds the weights to bf16 relative to a running max
+        # that depends on the chunking, so they agree to bf16 rounding.
+        if path == 1:
+            assert metrics(z, outs[0][2])["max_abs"] < 1e-4
+            assert metrics(q, outs[0][1])["max_abs"] < 1e-4
+        else:
+            assert metrics(z, outs[0][2])["rel_l2"] < 6e-3
+            assert metrics(q, outs[0][1])["rel_l2"] < 6e-3
 
 
 def test_scale_argument_flare_scale_one():
