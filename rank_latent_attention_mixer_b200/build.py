@@ -6,6 +6,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -35,13 +36,48 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+# The tcgen05 kernel splits its launch registers between warpgroups with
+# setmaxnreg (softmax warpgroups grow, the producer warpgroup shrinks).  The
+# split is sized for exactly this many registers per thread at launch; a
+# smaller launch allocation would leave the growing warpgroups waiting, so the
+# build refuses any other count.
+ATTN_LAUNCH_REGS = 168
+
+
+def check_registers(ptxas_log: str) -> None:
+    current = None
+    found = 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current and "attn_kernel" in current:
+            found += 1
+            regs = int(m.group(1))
+            if regs != ATTN_LAUNCH_REGS:
+                raise RuntimeError(f"{current}: ptxas allocated {regs} registers per thread, the register split "
+                                   f"needs exactly {ATTN_LAUNCH_REGS}; refusing to build")
+    if found == 0:
+        raise RuntimeError("no attn_kernel register report found in the ptxas log")
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose_ptxas else []), "-o", tmp, *sources()]
-    subprocess.run(cmd, check=True)
+    cmd = [nvcc, *NVCC_FLAGS, "-Xptxas", "-v", "-o", tmp, *sources()]
+    res = subprocess.run(cmd, check=True, capture_output=True, text=True)
+    log = res.stdout + res.stderr
+    if verbose_ptxas:
+        print(log)
+    try:
+        check_registers(log)
+    except Exception:
+        os.remove(tmp)
+        raise
     os.replace(tmp, LIB)
     return LIB
 

@@ -104,7 +104,7 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
     pl->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
     pl->chunks = (int)((s.N + (int64_t)pl->chunk_len - 1) / pl->chunk_len);
-    const int parts = path == FLAREPP_PATH_SIMT ? pl->chunks : pl->chunks * tc::kPartsPerChunk;
+    const int parts = path == FLAREPP_PATH_SIMT ? pl->chunks : pl->chunks * tc::parts_per_chunk(s.M);
 
     const size_t rows = (size_t)s.bh() * s.M;
     size_t off = 0;

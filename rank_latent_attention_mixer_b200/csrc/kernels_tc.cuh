@@ -13,16 +13,24 @@
 //                    key/value rows are the M latents of q and z, and the
 //                    output is the normalised y row in bf16.
 //
-// Per CTA (persistent, one per SM, 320 threads):
+// Per CTA (persistent, one per SM, 384 threads = three warpgroups):
 //   warps 0-3  softmax warpgroup 0  (query-row tile 0, TMEM lanes 0-127)
 //   warps 4-7  softmax warpgroup 1  (query-row tile 1)
 //   warp  8    TMA producer: query tiles and a ring of key/value tiles
 //   warp  9    MMA issuer: S_w = Q_w K^T into TMEM, O_w += P_w V into TMEM
+//   warps 10-11 idle
+// The launch gives every thread 168 registers (384 x 168 = 64512); the third
+// warpgroup gives back down to 56 and the softmax warpgroups take up to 224
+// (256 x 224 + 128 x 56 = 64512): the split never asks for more than the
+// launch holds.  The build checks that ptxas allocated exactly 168.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 and O_1 from 256 (stride
+// max(D,32)), P_0 and P_1 (128 bf16 = 64 columns each) after them.
 // Each softmax thread owns one query row: it reads its 128 scores from TMEM,
-// takes exponentials base 2, writes the bf16 weights P to shared memory in the
-// tcgen05 K-major 128-byte-swizzled layout, and rescales its O row in TMEM
-// only when its running max grows by more than 2^8 (the final normalisation
-// uses the same stale max, so the result is exact up to rounding).
+// takes exponentials base 2, writes the bf16 weights P back to TMEM (its own
+// columns; the value MMA reads its A operand from TMEM), and rescales its O
+// row in TMEM only when its running max grows by more than 2^8 (the final
+// normalisation uses the same stale max, so the result is exact up to
+// rounding).
 // The MMA warp runs the score MMA of the job two ahead before the value MMA of
 // the current job, so the two warpgroups' softmaxes alternate with the tensor
 // core (ping-pong).
@@ -43,8 +51,12 @@ namespace flarepp {
 namespace tc {
 
 constexpr int kTokTile = 128;        // rows per key/value tile and per query tile
-constexpr int kPartsPerChunk = 2;    // upper bound of partial triples per token chunk
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;     // registers per thread at launch (checked at build time)
+constexpr int kProducerRegs = 56;    // warpgroup 2 after setmaxnreg.dec
+constexpr int kSoftmaxRegs = 224;    // warpgroups 0-1 after setmaxnreg.inc
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -92,7 +104,7 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 // Waits until the phase with the given parity has completed.  Returns false
 // if the CTA's abort flag is up or the wait ran past kWaitLimitNs (then it
 // raises the flag and records the timeout).
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -134,6 +146,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x K bf16, K-major) read from TMEM.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -262,9 +285,7 @@ struct Smem {
     static constexpr int kTileBytes = kTokTile * D * 2;             // one [128 x D] bf16 tile
     static constexpr int kQ = 0;                                     // QS slots x 2 tiles
     static constexpr int kKV = kQ + QS * 2 * kTileBytes;             // NST stages x (K, V)
-    static constexpr int kP = kKV + NST * 2 * kTileBytes;            // 2 warpgroups x [128 x 128] bf16
-    static constexpr int kPBytes = 128 * 128 * 2;
-    static constexpr int kBar = kP + 2 * kPBytes;
+    static constexpr int kBar = kKV + NST * 2 * kTileBytes;
     // barriers: kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull[2], sfree[2], pfull[2], pfree[2], drain
     static constexpr int kNumBars = 2 * NST + 2 * QS + 8 + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;               // tmem base (u32), abort flag (int)
@@ -281,6 +302,9 @@ struct Layout {
     // TMEM column stride between the two warpgroups' O accumulators: at least
     // 32 so that 32-column TMEM loads/stores of one never touch the other's
     static constexpr int kOStride = D < 32 ? 32 : D;
+    static constexpr int kOCol = 256;                                 // O_0
+    static constexpr int kPCol = kOCol + 2 * kOStride;               // P_0; P_1 at +64
+    static_assert(kPCol + 128 <= 512, "TMEM plan exceeds 512 columns");
 };
 
 // ------------------------------------------------------------------ the kernel
@@ -340,7 +364,9 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kTmaWarp) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+      if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
             uint32_t kv_load = 0, q_load = 0;
@@ -389,7 +415,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     }
             }
         }
-    } else if (warp == kMmaWarp) {
+      } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = make_idesc(128, 128, false);   // S = Q K^T: [128 q x 128 kv]
@@ -485,20 +511,19 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 if (!mbar_wait(&pfull[w], pv_issued[w] & 1, abort_flag)) return false;
                 tc_fence_after();
                 const int st = c.tile_count % NST;
-                const uint32_t paddr = smem_u32(smem + SM::kP + w * SM::kPBytes);
                 const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kTileBytes + (p.kv_same ? 0 : SM::kTileBytes);
                 const uint32_t vaddr = smem_u32(vbase);
-                const uint32_t d_tmem = tmem + 256 + w * LY::kOStride;
+                const uint32_t d_tmem = tmem + LY::kOCol + w * LY::kOStride;
+                const uint32_t p_tmem = tmem + LY::kPCol + w * 64;
                 const bool first_of_w = c.njobs_w[w] == 0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    // A = P: K-major, 128B swizzle, two 64-column atoms of 16 KB
-                    const uint64_t ad = smem_desc(paddr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSw128);
+                    // A = P in TMEM: 16 key/value columns = 8 packed bf16x2 columns per step
                     // B = V tile [128 kv x D], D contiguous: MN-major; 16 kv rows per step
                     // (D fits one swizzle atom along MN, so the leading offset is never used)
                     const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kTileBytes,
                                                   LY::kSbo, LY::kType);
-                    umma_bf16(d_tmem, ad, bd, idesc_o, (first_of_w && kk == 0) ? 0u : 1u);
+                    umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (first_of_w && kk == 0) ? 0u : 1u);
                 }
                 umma_commit(&pfree[w]);
                 ++pv_issued[w];
@@ -526,15 +551,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
             }
         }
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ---------------------------------------------------------- softmax warpgroups
         const int wg = warp >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + wg * 128;
-        const uint32_t tO = tmem + lane_base + 256 + wg * LY::kOStride;
-        uint8_t* pbuf = smem + SM::kP + wg * SM::kPBytes;
+        const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride;
+        const uint32_t tP = tmem + lane_base + LY::kPCol + wg * 64;
         const float sl2 = p.scale_log2;
         uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0;
         bool ok = true;
@@ -556,17 +583,18 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 if (lane == 0) mbar_arrive(&sfree[wg]);
 
                 const int valid = p.kv_rows - t * kTokTile;      // key/value rows of this tile that exist
+                if (valid < kTokTile) {                           // ragged last tile only (warp-uniform)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c * 32 + j >= valid) sr[c][j] = __float_as_uint(-INFINITY);
+                }
                 float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float s = __uint_as_float(sr[c][j]);
-                        if (c * 32 + j >= valid) s = -INFINITY;
-                        sr[c][j] = __float_as_uint(s);
-                        mx = fmaxf(mx, s);
-                    }
-                }
+                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(sr[c][j]));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
@@ -576,7 +604,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 const float neg_m = -m_run;
                 float rs = 0.f;
-                uint32_t pk[64];
+                uint32_t pk[2][32];                  // [half][j]: columns 64*half + 2j, 2j+1
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -584,7 +612,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         const float p0 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j]), sl2, neg_m));
                         const float p1 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j + 1]), sl2, neg_m));
                         rs += p0 + p1;
-                        pk[c * 16 + j] = pack_bf16x2(p0, p1);
+                        pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(p0, p1);
                     }
                 }
                 l_run = l_run * factor + rs;
@@ -607,18 +635,11 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
                         tmem_st32(tO + c * 32, o);
                     }
-                    tmem_wait_st();
                 }
-                // P row -> shared memory, K-major 128-byte swizzle: 16-byte chunk c of a
-                // 128-byte row r sits at chunk position c ^ (r % 8)
-#pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {
-                    const int atom = ch >> 3, c8 = ch & 7;
-                    uint8_t* dst = pbuf + atom * 16384 + row * 128 + ((c8 ^ (row & 7)) << 4);
-                    *reinterpret_cast<uint4*>(dst) =
-                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                }
-                fence_async_smem();
+                // P row -> TMEM (this thread's lane, 64 columns of bf16 pairs)
+                tmem_st32(tP, pk[0]);
+                tmem_st32(tP + 32, pk[1]);
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pfull[wg]);
@@ -758,7 +779,7 @@ inline int sm_count() {
 
 template <int D>
 struct Config {
-    static constexpr int NST = D == 64 ? 3 : 4;
+    static constexpr int NST = D == 64 ? 4 : 6;
     static constexpr int QS = 2;
     using SM = Smem<D, NST, QS>;
     // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
