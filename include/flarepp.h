@@ -133,6 +133,31 @@ int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gat
                            const void* k0, const void* k, const void* v, void* y,
                            int B, int H, int N, int M, int D, int dtype, void* stream);
 
+/* FLARE++ mixer forward that allocates no memory: the same operation, arguments
+ * and result as flarepp_mixer_fwd (up to rounding: it may split the token axis
+ * into fewer chunks), with its scratch taken from a fixed device array inside
+ * the library instead of cudaMallocAsync.  (This entry has no counterpart in
+ * the FLARE++ paper or pages; it serves callers that cannot allocate device
+ * memory during the call: code whose memory belongs to another allocator,
+ * such as a framework's caching allocator or a pre-reserved arena that may
+ * not be bypassed, and code that must not run the implicit synchronisation a
+ * cudaMalloc/cudaFree can bring.)
+ *   - The array holds FLAREPP_NOALLOC_SCRATCH_BYTES and every GPU that loads
+ *     the library keeps it until the process exits.  A problem whose scratch
+ *     does not fit even with one token chunk returns FLAREPP_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress) and caches it; make that first call before
+ *     any stream capture.
+ *   - All calls share the array.  Calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads on one device) race on
+ *     it and give undefined results: serialise them.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+#define FLAREPP_NOALLOC_SCRATCH_BYTES (32u << 20)
+int flarepp_mixer_fwd_noalloc(const void* q0, const void* q_fixed, const float* gate,
+                              const void* k0, const void* k, const void* v, void* y,
+                              int B, int H, int N, int M, int D, int dtype, void* stream);
+
 /* Which kernel family AUTO would run for this shape (flarepp_path_t), or 0 for
  * arguments the forward entries would reject. */
 int flarepp_selected_path(int B, int H, int N, int M, int D, int dtype);

@@ -202,6 +202,23 @@ def mixer_fwd_host(q0, q_fixed, gate, k0, k, v, y, stream: Optional[torch.cuda.S
     return y
 
 
+def mixer_fwd_noalloc(q0, q_fixed, gate, k0, k, v, y):
+    """flarepp_mixer_fwd_noalloc: the mixer with no device allocation during
+    the call (scratch comes from a fixed array inside the library; calls that
+    overlap on the GPU race on it).  Same arguments and result as mixer_fwd_plain."""
+    fn = lib.flarepp_mixer_fwd_noalloc
+    if fn.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        fn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        fn.restype = ctypes.c_int
+    B, H, N, M, D = _shapes(q_fixed, k)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    rc = fn(_ptr(q0), _ptr(q_fixed), _ptr(gate), _ptr(k0), _ptr(k), _ptr(v), _ptr(y),
+            B, H, N, M, D, _dtype_code(k), _stream(k.device))
+    _check(rc, "flarepp_mixer_fwd_noalloc")
+    return y
+
+
 def check_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     st = (stream or torch.cuda.current_stream()).cuda_stream
     return int(lib.flarepp_check_device_status(st))

@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/flarepp.h"
 #include "common.cuh"
@@ -284,6 +285,63 @@ int forward(const void* q0, const void* q_fixed, const float* gate, const void* 
     return rc;
 }
 
+// ------------------------------------------------------------------ fixed device scratch
+//
+// Scratch for flarepp_mixer_fwd_noalloc: a file-scope device array, so that
+// entry point never allocates.  Every GPU that loads this library holds the
+// array until the process exits.  All calls share it; each call overwrites the
+// part it uses, and nothing in it needs to start at zero (every byte a kernel
+// reads was written earlier in the same call).  Two such calls whose kernels
+// overlap on the GPU race on it.
+constexpr size_t kStaticScratchBytes = FLAREPP_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is asked from the
+// runtime once per device, with that device current, and cached.
+void* static_scratch_address() {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+// Largest token-chunk count whose scratch fits the fixed array (0: none fits).
+int chunks_fitting_static_scratch(const Shape& s) {
+    Plan pl{};
+    if (make_plan(s, nullptr, &pl)) return 0;
+    if (pl.total <= kStaticScratchBytes) return pl.chunks;
+    int lo = 1, hi = pl.chunks, best = 0;
+    while (lo <= hi) {
+        const int mid = lo + (hi - lo) / 2;
+        flarepp_options_t o{};
+        o.force_chunks = mid;
+        Plan q{};
+        if (make_plan(s, &o, &q)) return 0;
+        if (q.total <= kStaticScratchBytes) {
+            best = mid;
+            lo = mid + 1;
+        } else {
+            hi = mid - 1;
+        }
+    }
+    return best;
+}
+
 }  // namespace
 }  // namespace flarepp
 
@@ -322,6 +380,23 @@ int flarepp_mixer_fwd(const void* q0, const void* q_fixed, const float* gate, co
 int flare_fwd(const void* q, const void* k, const void* v, void* y, int B, int H, int N, int M,
               int D, int dtype, void* stream) {
     return forward(nullptr, q, nullptr, nullptr, k, v, y, B, H, N, M, D, dtype, nullptr, stream);
+}
+
+int flarepp_mixer_fwd_noalloc(const void* q0, const void* q_fixed, const float* gate, const void* k0,
+                              const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
+                              int dtype, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    int rc = check_shape(s);
+    if (rc) return rc;
+    const int chunks = chunks_fitting_static_scratch(s);
+    if (chunks < 1) return FLAREPP_ERR_WORKSPACE;   // needs more than FLAREPP_NOALLOC_SCRATCH_BYTES
+    void* scratch = static_scratch_address();
+    if (!scratch) return FLAREPP_ERR_CUDA;
+    flarepp_options_t o{};
+    o.force_chunks = chunks;
+    o.workspace = scratch;
+    o.workspace_bytes = kStaticScratchBytes;
+    return forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, &o, stream);
 }
 
 size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
