@@ -18,7 +18,7 @@
 //   warps 4-7  softmax warpgroup 1  (query-row tile 1)
 //   warp  8    TMA producer: query tiles and a ring of key/value tiles
 //   warp  9    MMA issuer: S_w = Q_w K^T into TMEM, O_w += P_w V into TMEM
-//   warps 10-11 idle
+//   warp  11   idle
 // The launch gives every thread 168 registers (384 x 168 = 64512); the third
 // warpgroup gives back down to 56 and the softmax warpgroups take up to 224
 // (256 x 224 + 128 x 56 = 64512): the split never asks for more than the
@@ -31,9 +31,9 @@
 // row in TMEM only when its running max grows by more than 2^8 (the final
 // normalisation uses the same stale max, so the result is exact up to
 // rounding).
-// The MMA warp runs the score MMA of the job two ahead before the value MMA of
-// the current job, so the two warpgroups' softmaxes alternate with the tensor
-// core (ping-pong).
+// Each MMA warp issues its warpgroup's next score MMA as soon as the softmax
+// has read the previous scores, before that job's value MMA, so the tensor
+// core works ahead of the softmax; the two warpgroups run independently.
 //
 // Every wait on an mbarrier is bounded (about 2 s of %globaltimer); on expiry
 // the kernel records FLAREPP_ERR_TIMEOUT in the device status word, raises a
@@ -213,6 +213,13 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major)
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -286,8 +293,8 @@ struct Smem {
     static constexpr int kQ = 0;                                     // QS slots x 2 tiles
     static constexpr int kKV = kQ + QS * 2 * kTileBytes;             // NST stages x (K, V)
     static constexpr int kBar = kKV + NST * 2 * kTileBytes;
-    // barriers: kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull[2], sfree[2], pfull[2], pfree[2], drain
-    static constexpr int kNumBars = 2 * NST + 2 * QS + 8 + 1;
+    // barriers: kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull[2], sfree[2], pfull[2], pfree[2], drain[2]
+    static constexpr int kNumBars = 2 * NST + 2 * QS + 8 + 2;
     static constexpr int kMisc = kBar + kNumBars * 8;               // tmem base (u32), abort flag (int)
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kLaunchBytes = kBytes + 1024;              // + alignment slack
@@ -337,15 +344,18 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
-        for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+        // a key/value stage is released by every warpgroup that consumes it; a
+        // query slot by both warpgroups
+        for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], p.interleave ? 1 : 2); }
+        for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 2); }
         for (int w = 0; w < 2; ++w) {
             mbar_init(&sfull[w], 1);
             mbar_init(&sfree[w], 4);
             mbar_init(&pfull[w], 4);
             mbar_init(&pfree[w], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -415,79 +425,72 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     }
             }
         }
-      } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------- MMA issuer
+      } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+        // ---------------------------------------------------------- MMA issuers
+        // Warp 9 issues for softmax warpgroup 0, warp 10 for warpgroup 1, so the
+        // two warpgroups' pipelines never wait on each other's softmax.
         if (lane == 0) {
+            const int w = warp - kMmaWarp;
             constexpr uint32_t idesc_s = make_idesc(128, 128, false);   // S = Q K^T: [128 q x 128 kv]
             constexpr uint32_t idesc_o = make_idesc(128, D, true);      // O += P V:  [128 q x D], V MN-major
-            // Job stream: (item, warpgroup, tile).  Two cursors over the same
-            // stream: `sc` issues score MMAs two jobs ahead of `pc`, which
-            // issues the value MMAs.
+            // This warpgroup's jobs: the key/value tiles it consumes, item by item
+            // (every tile, or alternate tiles when interleaved).  Two cursors over
+            // the stream: `sc` issues the score MMA one job ahead of `pc`.
             struct Cursor {
-                int item, t, w, njobs_w[2];
+                int item, t, njobs;
                 bool valid;
                 Item info;
-                uint32_t tile_count, item_count;
+                uint32_t tiles_before, item_count;
             };
-            auto first_job = [&](Cursor& c) {
-                c.item = blockIdx.x;
-                c.tile_count = 0;
-                c.item_count = 0;
-                c.valid = c.item < p.items;
-                if (c.valid) {
+            bool ok = true;
+            // Settles on the next item (from c.item on) that has a job for this
+            // warpgroup.  An item without one still takes part in freeing its
+            // query slot, after the slot's load has landed (so the release is
+            // counted in the right phase); only the score cursor does that.
+            auto settle = [&](Cursor& c, bool score_cursor) {
+                while (c.item < p.items) {
                     c.info = decode_item(p, c.item);
-                    c.t = c.info.t_begin;
-                    c.w = 0;
-                    c.njobs_w[0] = c.njobs_w[1] = 0;
+                    c.t = c.info.t_begin + (p.interleave ? w : 0);
+                    c.njobs = 0;
+                    if (c.t < c.info.t_end) {
+                        c.valid = true;
+                        return;
+                    }
+                    if (score_cursor && ok) {
+                        const int slot = c.item_count % QS;
+                        ok = mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag);
+                        if (ok) umma_commit(&q_empty[slot]);
+                    }
+                    c.tiles_before += c.info.t_end - c.info.t_begin;
+                    ++c.item_count;
+                    c.item += gridDim.x;
                 }
+                c.valid = false;
             };
-            auto next_job = [&](Cursor& c) {
-                // advance within the item
-                bool tile_done;
-                if (p.interleave) {
-                    tile_done = true;
-                } else {
-                    tile_done = (c.w == 1);
-                }
-                c.njobs_w[c.w]++;
-                if (!tile_done) {
-                    c.w = 1;
-                    return;
-                }
-                ++c.tile_count;
-                ++c.t;
-                if (c.t < c.info.t_end) {
-                    c.w = p.interleave ? ((c.t - c.info.t_begin) & 1) : 0;
-                    return;
-                }
+            auto first = [&](Cursor& c, bool score_cursor) {
+                c.item = blockIdx.x;
+                c.tiles_before = 0;
+                c.item_count = 0;
+                settle(c, score_cursor);
+            };
+            auto next = [&](Cursor& c, bool score_cursor) {
+                ++c.njobs;
+                c.t += p.interleave ? 2 : 1;
+                if (c.t < c.info.t_end) return;
+                c.tiles_before += c.info.t_end - c.info.t_begin;
                 ++c.item_count;
                 c.item += gridDim.x;
-                c.valid = c.item < p.items;
-                if (c.valid) {
-                    c.info = decode_item(p, c.item);
-                    c.t = c.info.t_begin;
-                    c.w = 0;
-                    c.njobs_w[0] = c.njobs_w[1] = 0;
-                }
+                settle(c, score_cursor);
             };
-            uint32_t s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
-            bool ok = true;
-            Cursor sc, pc;
-            first_job(sc);
-            first_job(pc);
+            auto stage_of = [&](const Cursor& c) { return (c.tiles_before + (c.t - c.info.t_begin)); };
+            uint32_t s_issued = 0;
             auto issue_s = [&](const Cursor& c) -> bool {
-                const int w = c.w;
-                const bool first_of_item = (c.t == c.info.t_begin) && (w == 0);
-                const bool first_use = p.interleave || w == 0;
                 const int slot = c.item_count % QS;
-                if (first_of_item) {
-                    if (!mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag)) return false;
-                }
-                const int st = c.tile_count % NST;
-                if (first_use) {
-                    if (!mbar_wait(&kv_full[st], (c.tile_count / NST) & 1, abort_flag)) return false;
-                }
-                if (!mbar_wait(&sfree[w], (s_issued[w] & 1) ^ 1, abort_flag)) return false;
+                if (c.njobs == 0 && !mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag)) return false;
+                const uint32_t tile = stage_of(c);
+                const int st = tile % NST;
+                if (!mbar_wait(&kv_full[st], (tile / NST) & 1, abort_flag)) return false;
+                if (!mbar_wait(&sfree[w], (s_issued & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t qaddr = smem_u32(smem + SM::kQ + slot * 2 * SM::kTileBytes +
                                                 (p.interleave ? 0 : w * SM::kTileBytes));
@@ -500,22 +503,20 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     umma_bf16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sfull[w]);
-                ++s_issued[w];
-                // last score MMA of the item frees the query slot once it completes
-                const bool last_of_item = (c.t == c.info.t_end - 1) && (p.interleave || w == 1);
-                if (last_of_item) umma_commit(&q_empty[slot]);
+                ++s_issued;
+                // this warpgroup's last score MMA of the item releases its share of the query slot
+                if (c.t + (p.interleave ? 2 : 1) >= c.info.t_end) umma_commit(&q_empty[slot]);
                 return true;
             };
+            uint32_t pv_issued = 0;
             auto issue_pv = [&](const Cursor& c) -> bool {
-                const int w = c.w;
-                if (!mbar_wait(&pfull[w], pv_issued[w] & 1, abort_flag)) return false;
+                if (!mbar_wait(&pfull[w], pv_issued & 1, abort_flag)) return false;
                 tc_fence_after();
-                const int st = c.tile_count % NST;
+                const int st = stage_of(c) % NST;
                 const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kTileBytes + (p.kv_same ? 0 : SM::kTileBytes);
                 const uint32_t vaddr = smem_u32(vbase);
                 const uint32_t d_tmem = tmem + LY::kOCol + w * LY::kOStride;
                 const uint32_t p_tmem = tmem + LY::kPCol + w * 64;
-                const bool first_of_w = c.njobs_w[w] == 0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     // A = P in TMEM: 16 key/value columns = 8 packed bf16x2 columns per step
@@ -523,32 +524,33 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     // (D fits one swizzle atom along MN, so the leading offset is never used)
                     const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kTileBytes,
                                                   LY::kSbo, LY::kType);
-                    umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (first_of_w && kk == 0) ? 0u : 1u);
+                    umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
                 }
                 umma_commit(&pfree[w]);
-                ++pv_issued[w];
-                const bool last_use = p.interleave || w == 1;
-                if (last_use) umma_commit(&kv_empty[st]);
+                ++pv_issued;
+                umma_commit(&kv_empty[st]);     // this warpgroup is done with the stage
                 return true;
             };
-            // prologue: two score MMAs
-            for (int k = 0; k < 2 && sc.valid && ok; ++k) {
+            Cursor sc, pc;
+            first(sc, true);
+            first(pc, false);
+            if (sc.valid && ok) {
                 ok = issue_s(sc);
-                next_job(sc);
+                next(sc, true);
             }
             while (pc.valid && ok) {
                 if (sc.valid) {
                     ok = issue_s(sc);
                     if (!ok) break;
-                    next_job(sc);
+                    next(sc, true);
                 }
                 ok = issue_pv(pc);
-                next_job(pc);
+                next(pc, false);
             }
             // drain: wait until every issued MMA has completed before TMEM is released
-            umma_commit(drain);
+            umma_commit(&drain[w]);
             const unsigned long long t0 = globaltimer_ns();
-            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            while (!mbar_try_wait(&drain[w], 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
             }
         }
       }
@@ -590,11 +592,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         for (int j = 0; j < 32; ++j)
                             if (c * 32 + j >= valid) sr[c][j] = __float_as_uint(-INFINITY);
                 }
-                float mx = -INFINITY;
+                // row max: four independent chains of 3-input maxima (short dependency chains)
+                float mc[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 4; ++c) {
+                    mc[c] = __uint_as_float(sr[c][0]);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(sr[c][j]));
+                    for (int j = 1; j < 31; j += 2)
+                        mc[c] = max3f(mc[c], __uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1]));
+                    mc[c] = fmaxf(mc[c], __uint_as_float(sr[c][31]));
+                }
+                const float mx = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
@@ -602,20 +610,26 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     factor = ex2_mufu(m_run - m_new);
                     m_run = m_new;
                 }
-                const float neg_m = -m_run;
-                float rs = 0.f;
+                // exponent arguments in pairs (packed fp32 FMA), row sum in four packed chains
+                const float2 sl2v = make_float2(sl2, sl2);
+                const float2 negm = make_float2(-m_run, -m_run);
+                float2 acc[4];
                 uint32_t pk[2][32];                  // [half][j]: columns 64*half + 2j, 2j+1
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    acc[c] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const float p0 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j]), sl2, neg_m));
-                        const float p1 = ex2_mufu(fmaf(__uint_as_float(sr[c][2 * j + 1]), sl2, neg_m));
-                        rs += p0 + p1;
-                        pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(p0, p1);
+                        const float2 sv = make_float2(__uint_as_float(sr[c][2 * j]), __uint_as_float(sr[c][2 * j + 1]));
+                        const float2 xv = __ffma2_rn(sv, sl2v, negm);
+                        const float2 pv = make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
+                        acc[c] = __fadd2_rn(acc[c], pv);
+                        pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(pv.x, pv.y);
                     }
                 }
-                l_run = l_run * factor + rs;
+                const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+                const float2 a = __fadd2_rn(a01, a23);
+                l_run = l_run * factor + (a.x + a.y);
 
                 // the previous value MMA of this warpgroup must be done before P and O are touched
                 while (pfree_waits < jobs_done) {
