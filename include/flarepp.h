@@ -124,11 +124,16 @@ int flarepp_mixer_fwd_ex(const void* q0, const void* q_fixed, const float* gate,
 size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
                                const flarepp_options_t* opts);
 
-/* Same operation with HOST buffers (end-to-end form): copies the inputs to the
- * device on `stream`, runs the mixer, copies y back and synchronises `stream`
- * before returning.  Device memory is taken stream-ordered and released before
- * return.  Pinned host memory lets the copies run at full speed; pageable
- * memory works but is slower.  gate is a HOST float[H] here (NULL = FLARE). */
+/* Same operation with HOST buffers (end-to-end form): streams the (b, h)
+ * slices through the GPU -- the copy-in of one slice, the forward of the
+ * previous one (on `stream`) and the copy-out of the one before overlap, on two
+ * library-owned copy streams -- and synchronises `stream` before returning.
+ * Device staging (two slices of inputs and output, the latent inputs, scratch)
+ * comes from a library-owned memory pool that keeps it reserved between calls.
+ * Pinned host memory lets the copies run at full speed; pageable memory works
+ * but is slower.  gate is a HOST float[H] here (NULL = FLARE).  The result is
+ * identical to flarepp_mixer_fwd's up to the token-chunk split, which is
+ * planned per slice here. */
 int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate,
                            const void* k0, const void* k, const void* v, void* y,
                            int B, int H, int N, int M, int D, int dtype, void* stream);

@@ -342,6 +342,149 @@ int chunks_fitting_static_scratch(const Shape& s) {
     return best;
 }
 
+// ------------------------------------------------------------------ host-buffer entry
+//
+// The (b, h) slices of the mixer are independent problems, so the host entry
+// streams them: the copy-in of slice i+1 (stream `in`), the forward of slice
+// i (the caller's stream) and the copy-out of slice i-1 (stream `out`) overlap,
+// with two device slots for a slice's inputs and output.  Staging comes from
+// a library-owned memory pool that keeps its memory reserved between calls,
+// so repeated calls do not map and unmap device memory.
+struct HostResources {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaMemPool_t pool = nullptr;
+    bool ready = false;
+};
+
+HostResources* host_resources() {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static HostResources res[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    HostResources& r = res[dev];
+    if (!r.ready) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        if ((!r.in && cudaStreamCreateWithFlags(&r.in, cudaStreamNonBlocking) != cudaSuccess) ||
+            (!r.out && cudaStreamCreateWithFlags(&r.out, cudaStreamNonBlocking) != cudaSuccess) ||
+            (!r.pool && cudaMemPoolCreate(&r.pool, &props) != cudaSuccess)) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolSetAttribute(r.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        r.ready = true;
+    }
+    return &r;
+}
+
+int host_forward(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+                 const void* v, void* y, int B, int H, int N, int M, int D, int dtype, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    int rc = make_plan(s, nullptr, &pl);
+    if (rc) return rc;
+    const bool gated = gate != nullptr;
+    if (!q_fixed || !k || !v || !y || (gated && (!q0 || !k0))) return FLAREPP_ERR_INVALID_ARG;
+    const Shape s1{1, 1, N, M, D, dtype};
+    Plan p1{};
+    rc = make_plan(s1, nullptr, &p1);
+    if (rc) return rc;
+    HostResources* hr = host_resources();
+    if (!hr) return FLAREPP_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    const size_t t1 = (size_t)N * D * s.elem(), l1 = (size_t)M * D * s.elem();
+    const int slices = B * H;
+    // device layout: latent inputs of all heads, then two slots of
+    // [k0 (gated), k, v, y, scratch] for one (b, h) slice each
+    size_t off = 0;
+    const size_t o_qf = off; off = align_up(off + (size_t)H * l1);
+    const size_t o_q0 = off; if (gated) off = align_up(off + (size_t)H * l1);
+    const size_t o_g = off;  if (gated) off = align_up(off + (size_t)H * sizeof(float));
+    size_t o_slot[2], o_k0 = 0, o_k, o_v, o_y, o_ws;
+    {
+        size_t so = 0;
+        o_k0 = so; if (gated) so = align_up(so + t1);
+        o_k = so;  so = align_up(so + t1);
+        o_v = so;  so = align_up(so + t1);
+        o_y = so;  so = align_up(so + t1);
+        o_ws = so; so = align_up(so + p1.total);
+        o_slot[0] = off; off += so;
+        o_slot[1] = off; off += so;
+    }
+    char* d = nullptr;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void**>(&d), off, hr->pool, st) != cudaSuccess) {
+        cudaGetLastError();
+        return FLAREPP_ERR_WORKSPACE;
+    }
+    cudaEvent_t ev_lat = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+    bool ok = cudaEventCreateWithFlags(&ev_lat, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+        ok = cudaEventCreateWithFlags(&in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(d + o_qf, q_fixed, (size_t)H * l1, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    if (ok && gated)
+        ok = cudaMemcpyAsync(d + o_q0, q0, (size_t)H * l1, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+             cudaMemcpyAsync(d + o_g, gate, (size_t)H * sizeof(float), cudaMemcpyHostToDevice, st) == cudaSuccess;
+    // the copy streams may touch the block only after its stream-ordered allocation
+    ok = ok && cudaEventRecord(ev_lat, st) == cudaSuccess && cudaStreamWaitEvent(hr->in, ev_lat, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(hr->out, ev_lat, 0) == cudaSuccess;
+    rc = ok ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+    const char* hk0 = static_cast<const char*>(k0);
+    const char* hk = static_cast<const char*>(k);
+    const char* hv = static_cast<const char*>(v);
+    char* hy = static_cast<char*>(y);
+    for (int si = 0; si < slices && rc == FLAREPP_OK; ++si) {
+        const int slot = si & 1, h = si % H;
+        char* base = d + o_slot[slot];
+        const size_t ho = (size_t)si * t1;
+        ok = si < 2 || cudaStreamWaitEvent(hr->in, comp_done[slot], 0) == cudaSuccess;   // slot inputs consumed
+        if (ok && gated) ok = cudaMemcpyAsync(base + o_k0, hk0 + ho, t1, cudaMemcpyHostToDevice, hr->in) == cudaSuccess;
+        ok = ok && cudaMemcpyAsync(base + o_k, hk + ho, t1, cudaMemcpyHostToDevice, hr->in) == cudaSuccess &&
+             cudaMemcpyAsync(base + o_v, hv + ho, t1, cudaMemcpyHostToDevice, hr->in) == cudaSuccess &&
+             cudaEventRecord(in_done[slot], hr->in) == cudaSuccess &&
+             cudaStreamWaitEvent(st, in_done[slot], 0) == cudaSuccess &&
+             (si < 2 || cudaStreamWaitEvent(st, out_done[slot], 0) == cudaSuccess);        // slot output drained
+        if (!ok) { rc = FLAREPP_ERR_CUDA; break; }
+        flarepp_options_t o{};
+        o.workspace = base + o_ws;
+        o.workspace_bytes = p1.total;
+        rc = forward(gated ? d + o_q0 + (size_t)h * l1 : nullptr, d + o_qf + (size_t)h * l1,
+                     gated ? reinterpret_cast<float*>(d + o_g) + h : nullptr, gated ? base + o_k0 : nullptr,
+                     base + o_k, base + o_v, base + o_y, 1, 1, N, M, D, dtype, &o, stream);
+        if (rc) break;
+        ok = cudaEventRecord(comp_done[slot], st) == cudaSuccess &&
+             cudaStreamWaitEvent(hr->out, comp_done[slot], 0) == cudaSuccess &&
+             cudaMemcpyAsync(hy + ho, base + o_y, t1, cudaMemcpyDeviceToHost, hr->out) == cudaSuccess &&
+             cudaEventRecord(out_done[slot], hr->out) == cudaSuccess;
+        if (!ok) rc = FLAREPP_ERR_CUDA;
+    }
+    // join the copy streams back into the caller's stream, release, synchronise
+    for (int i = 0; i < 2; ++i) {
+        if (in_done[i] && cudaStreamWaitEvent(st, in_done[i], 0) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+        if (out_done[i] && cudaStreamWaitEvent(st, out_done[i], 0) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    }
+    if (cudaFreeAsync(d, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    cudaEvent_t evs[] = {ev_lat, in_done[0], in_done[1], comp_done[0], comp_done[1], out_done[0], out_done[1]};
+    for (cudaEvent_t e : evs)
+        if (e) cudaEventDestroy(e);
+    return rc;
+}
+
 }  // namespace
 }  // namespace flarepp
 
@@ -430,52 +573,7 @@ int flarepp_check_device_status(void* stream) {
 int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate, const void* k0,
                            const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
                            int dtype, void* stream) {
-    const Shape s{B, H, N, M, D, dtype};
-    Plan pl{};
-    int rc = make_plan(s, nullptr, &pl);
-    if (rc) return rc;
-    const bool gated = gate != nullptr;
-    if (!q_fixed || !k || !v || !y || (gated && (!q0 || !k0))) return FLAREPP_ERR_INVALID_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t tb = s.tok_bytes(), lb = s.lat_bytes(), gb = (size_t)H * sizeof(float);
-    // One stream-ordered block: inputs, output, then the mixer's workspace.
-    size_t off = 0;
-    const size_t o_qf = off; off = align_up(off + lb);
-    const size_t o_k = off;  off = align_up(off + tb);
-    const size_t o_v = off;  off = align_up(off + tb);
-    const size_t o_y = off;  off = align_up(off + tb);
-    size_t o_q0 = 0, o_k0 = 0, o_g = 0;
-    if (gated) {
-        o_q0 = off; off = align_up(off + lb);
-        o_k0 = off; off = align_up(off + tb);
-        o_g = off;  off = align_up(off + gb);
-    }
-    const size_t o_ws = off; off = align_up(off + pl.total);
-    char* d = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&d), off, st) != cudaSuccess) {
-        cudaGetLastError();
-        return FLAREPP_ERR_WORKSPACE;
-    }
-    bool ok = cudaMemcpyAsync(d + o_qf, q_fixed, lb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-              cudaMemcpyAsync(d + o_k, k, tb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-              cudaMemcpyAsync(d + o_v, v, tb, cudaMemcpyHostToDevice, st) == cudaSuccess;
-    if (ok && gated)
-        ok = cudaMemcpyAsync(d + o_q0, q0, lb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-             cudaMemcpyAsync(d + o_k0, k0, tb, cudaMemcpyHostToDevice, st) == cudaSuccess &&
-             cudaMemcpyAsync(d + o_g, gate, gb, cudaMemcpyHostToDevice, st) == cudaSuccess;
-    rc = ok ? FLAREPP_OK : FLAREPP_ERR_CUDA;
-    if (rc == FLAREPP_OK) {
-        flarepp_options_t o{};
-        o.workspace = d + o_ws;
-        o.workspace_bytes = pl.total;
-        rc = forward(gated ? d + o_q0 : nullptr, d + o_qf, gated ? reinterpret_cast<float*>(d + o_g) : nullptr,
-                     gated ? d + o_k0 : nullptr, d + o_k, d + o_v, d + o_y, B, H, N, M, D, dtype, &o, stream);
-    }
-    if (rc == FLAREPP_OK && cudaMemcpyAsync(y, d + o_y, tb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        rc = FLAREPP_ERR_CUDA;
-    if (cudaFreeAsync(d, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
-    return rc;
+    return host_forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, stream);
 }
 
 }  // extern "C"

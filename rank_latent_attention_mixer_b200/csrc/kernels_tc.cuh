@@ -213,6 +213,37 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major)
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit.
+// Range reduction: n = round(x) by adding 1.5 * 2^23 (the addition rounds x
+// to an integer held in the low mantissa bits of t), f = x - n in [-1/2, 1/2]
+// exactly; 2^f from the cubic c0 + f (c1 + f (c2 + f c3)), the minimax
+// approximation of 2^f on [-1/2, 1/2] for relative error, fitted by the Remez
+// exchange algorithm (max relative error 7.5e-5; exp2_poly.py); then 2^n is
+// applied by adding n to the exponent field (t's bits shifted left by 23 are
+// n << 23).  Arguments below -120 are clamped there: such weights (< 2^-120)
+// cannot matter next to the row's largest weight, which is >= 1.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ float2 ex2_fma_pair(float2 x) {
+    x.x = fmaxf(x.x, -120.f);
+    x.y = fmaxf(x.y, -120.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+    q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+    q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Column pairs (of the 64 per 128-column score tile) whose exponentials run on
+// the FMA pipe; the rest use the MUFU unit.  Balances the two pipes.
+constexpr int kFmaExpPairs = 16;
+
 // max(a, b, c) in one instruction (three-input max.f32)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
@@ -622,7 +653,9 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     for (int j = 0; j < 16; ++j) {
                         const float2 sv = make_float2(__uint_as_float(sr[c][2 * j]), __uint_as_float(sr[c][2 * j + 1]));
                         const float2 xv = __ffma2_rn(sv, sl2v, negm);
-                        const float2 pv = make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
+                        const float2 pv = (c * 16 + j >= 64 - kFmaExpPairs)
+                                              ? ex2_fma_pair(xv)
+                                              : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
                         pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(pv.x, pv.y);
                     }

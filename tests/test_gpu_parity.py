@@ -149,7 +149,10 @@ def test_deterministic_and_abi_variants():
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
     assert torch.equal(y1, y3)
-    assert torch.equal(y1.cpu(), y4)
+    # the host entry plans its token chunks per (b, h) slice: equal up to rounding
+    assert_parity(y4, y1.cpu(), w.dtype, "host entry vs device entry")
+    y_ref, _, _ = oracle_out("grid85_bf16", x)
+    assert_parity(y4, y_ref, w.dtype, "host entry vs oracle")
 
 
 def test_invariants_on_gpu():
