@@ -38,10 +38,18 @@ def _stale() -> bool:
 
 # The tcgen05 kernel splits its launch registers between warpgroups with
 # setmaxnreg (softmax warpgroups grow, the producer warpgroup shrinks).  The
-# split is sized for exactly this many registers per thread at launch; a
-# smaller launch allocation would leave the growing warpgroups waiting, so the
-# build refuses any other count.
-ATTN_LAUNCH_REGS = 168
+# split is sized for exactly 65536 / threads registers per thread at launch
+# (rounded down to a multiple of 8); a smaller launch allocation would leave
+# the growing warpgroups waiting, so the build refuses any other count.  The
+# kernel's template arguments are <D, NW, KT, NST, QS>, threads = (NW+1)*128.
+
+
+def expected_launch_regs(kernel_name: str) -> int:
+    m = re.search(r"attn_kernelILi(\d+)ELi(\d+)ELi(\d+)E", kernel_name)
+    if not m:
+        raise RuntimeError(f"cannot read the warpgroup count from {kernel_name}")
+    nw = int(m.group(2))
+    return (65536 // ((nw + 1) * 128)) // 8 * 8
 
 
 def check_registers(ptxas_log: str) -> None:
@@ -56,9 +64,10 @@ def check_registers(ptxas_log: str) -> None:
         if m and current and "attn_kernel" in current:
             found += 1
             regs = int(m.group(1))
-            if regs != ATTN_LAUNCH_REGS:
+            want = expected_launch_regs(current)
+            if regs != want:
                 raise RuntimeError(f"{current}: ptxas allocated {regs} registers per thread, the register split "
-                                   f"needs exactly {ATTN_LAUNCH_REGS}; refusing to build")
+                                   f"needs exactly {want}; refusing to build")
     if found == 0:
         raise RuntimeError("no attn_kernel register report found in the ptxas log")
 

@@ -88,7 +88,7 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
         pl->row_blocks = (s.M + kSimtThreads - 1) / kSimtThreads;
         units_per_bh = pl->row_blocks;
     } else {
-        tile = tc::kTokTile;
+        tile = tc::kv_tile();
         pl->row_blocks = tc::row_groups(s.M);
         units_per_bh = pl->row_blocks;
     }
@@ -96,11 +96,13 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     int64_t chunks;
     if (o && o->force_chunks > 0) {
         chunks = std::min<int64_t>(o->force_chunks, tiles);
-    } else {
+    } else if (path == FLAREPP_PATH_SIMT) {
         // Enough CTAs for several waves over the SMs, but chunks of >= 1 tile.
-        const int64_t target = path == FLAREPP_PATH_SIMT ? 4 * kNumSMs : tc::target_ctas();
+        const int64_t target = 4 * kNumSMs;
         chunks = (target + s.bh() * units_per_bh - 1) / (s.bh() * units_per_bh);
         chunks = std::max<int64_t>(1, std::min<int64_t>(chunks, tiles));
+    } else {
+        chunks = tc::choose_chunks(s.bh() * units_per_bh, tiles, kNumSMs);
     }
     int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
     pl->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);

@@ -13,27 +13,35 @@
 //                    key/value rows are the M latents of q and z, and the
 //                    output is the normalised y row in bf16.
 //
-// Per CTA (persistent, one per SM, 384 threads = three warpgroups):
-//   warps 0-3  softmax warpgroup 0  (query-row tile 0, TMEM lanes 0-127)
-//   warps 4-7  softmax warpgroup 1  (query-row tile 1)
-//   warp  8    TMA producer: query tiles and a ring of key/value tiles
-//   warp  9    MMA issuer: S_w = Q_w K^T into TMEM, O_w += P_w V into TMEM
-//   warp  11   idle
-// The launch gives every thread 168 registers (384 x 168 = 64512); the third
-// warpgroup gives back down to 56 and the softmax warpgroups take up to 224
-// (256 x 224 + 128 x 56 = 64512): the split never asks for more than the
-// launch holds.  The build checks that ptxas allocated exactly 168.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 and O_1 from 256 (stride
-// max(D,32)), P_0 and P_1 (128 bf16 = 64 columns each) after them.
-// Each softmax thread owns one query row: it reads its 128 scores from TMEM,
-// takes exponentials base 2, writes the bf16 weights P back to TMEM (its own
-// columns; the value MMA reads its A operand from TMEM), and rescales its O
-// row in TMEM only when its running max grows by more than 2^8 (the final
-// normalisation uses the same stale max, so the result is exact up to
-// rounding).
-// Each MMA warp issues its warpgroup's next score MMA as soon as the softmax
-// has read the previous scores, before that job's value MMA, so the tensor
-// core works ahead of the softmax; the two warpgroups run independently.
+// Per CTA (persistent, one per SM): NW softmax warpgroups and one producer
+// warpgroup, (NW + 1) x 128 threads.
+//   warps 0 .. 4NW-1   softmax warpgroup w = warp / 4 (query-row tile, TMEM lanes
+//                      32 (warp % 4) .. +31)
+//   warp  4NW          TMA producer: query tiles and a ring of key/value tiles of
+//                      KT rows
+//   warps 4NW+1 ..     one MMA issuer per softmax warpgroup w:
+//                      S_w = Q_w K^T and O_w += P_w V, into TMEM
+// TMEM columns: S_w at KT w, O_w at NW KT + OS w (OS = max(D, 32)), P_w (KT
+// bf16 = KT/2 columns) after them; NW (KT + OS + KT/2) <= 512.
+// Each softmax thread owns one query row: it reads its KT scores from TMEM,
+// takes exponentials base 2, writes the bf16 weights P back to TMEM (the value
+// MMA reads its A operand from TMEM), and rescales its O row in TMEM only when
+// its running max grows by more than 2^8 (the final normalisation uses the
+// same stale max, so the result is exact up to rounding).  Each MMA warp
+// issues its warpgroup's next score MMA as soon as the softmax has read the
+// previous scores, before that job's value MMA, so the tensor core works ahead
+// of the softmax; the warpgroups run independently.
+// Query tiles and key/value tiles are shared in one of two ways:
+//   * shared key/value tiles (decode, and split with one 128-latent group per
+//     warpgroup): each warpgroup has its own query tile and every warpgroup
+//     consumes every key/value tile of the item;
+//   * interleaved (split otherwise): the warpgroups share one query tile and
+//     take the item's key/value tiles round-robin, each writing its own
+//     partial triple.
+// The launch gives every thread R0 = 65536 / threads registers; the producer
+// warpgroup gives back down to 56 and the softmax warpgroups take the rest
+// (setmaxnreg), never more than the launch holds.  The build checks ptxas's
+// launch allocation for each configuration.
 //
 // Every wait on an mbarrier is bounded (about 2 s of %globaltimer); on expiry
 // the kernel records FLAREPP_ERR_TIMEOUT in the device status word, raises a
@@ -50,19 +58,23 @@
 namespace flarepp {
 namespace tc {
 
-constexpr int kTokTile = 128;        // rows per key/value tile and per query tile
-constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;     // registers per thread at launch (checked at build time)
-constexpr int kProducerRegs = 56;    // warpgroup 2 after setmaxnreg.dec
-constexpr int kSoftmaxRegs = 224;    // warpgroups 0-1 after setmaxnreg.inc
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kQTile = 128;          // query rows per tile (the tcgen05.mma M)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kStatusTimeout = 5;    // FLAREPP_ERR_TIMEOUT
+constexpr int kProducerRegs = 56;    // producer warpgroup after setmaxnreg.dec
+
+// Threads, launch registers and the softmax warpgroups' register share of a
+// configuration with NW softmax warpgroups.
+template <int NW>
+struct Regs {
+    static constexpr int kThreads = (NW + 1) * 128;
+    static constexpr int kLaunch = (65536 / kThreads) / 8 * 8;           // 168 (NW=2), 128 (NW=3)
+    static constexpr int kSoftmax = ((kThreads * kLaunch - 128 * kProducerRegs) / (NW * 128)) / 8 * 8;
+    static_assert(NW * 128 * kSoftmax + 128 * kProducerRegs <= kThreads * kLaunch,
+                  "register split exceeds the launch allocation");
+};
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -240,9 +252,9 @@ __device__ __forceinline__ float2 ex2_fma_pair(float2 x) {
                        __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-// Column pairs (of the 64 per 128-column score tile) whose exponentials run on
-// the FMA pipe; the rest use the MUFU unit.  Balances the two pipes.
-constexpr int kFmaExpPairs = 16;
+// Share of the exponentials that run on the FMA pipe instead of the MUFU unit:
+// this many column pairs out of every 64 (scaled to the tile width).
+constexpr int kFmaExpPairsPer64 = 16;
 
 // max(a, b, c) in one instruction (three-input max.f32)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -264,18 +276,16 @@ struct Params {
     int mode;             // Mode
     int B, H;
     int M, N;             // latents, tokens
-    int q_rows;           // rows of the query tensor per (b, h)  (M in split mode, N in decode)
     int kv_rows;          // rows of the key/value tensors per (b, h) (N in split mode, M in decode)
-    int kv_tiles;         // ceil(kv_rows / 128)
+    int kv_tiles;         // ceil(kv_rows / KT)
     int q_shared;         // query map's z coordinate is h (tensor [H, rows, D]) instead of b*H+h
     int k_shared;         // key map's z coordinate is h
     int kv_same;          // values are the keys (synthesis): load one tile per stage
-    int interleave;       // split mode with M <= 128: both warpgroups share query tile 0 and take
-                          // alternate key/value tiles, each writing its own partial triple
-    int row_groups;       // split mode, not interleaved: 256-row latent groups per (b, h)
+    int interleave;       // warpgroups share one query tile and take the key/value tiles round-robin
+    int row_groups;       // split mode: query-row groups per (b, h) (128 rows, or 128 NW when not interleaved)
     int chunks;           // split mode: token chunks per (b, h)
-    int chunk_tiles;      // split mode: 128-token tiles per chunk
-    int q_pairs;          // decode mode: 256-token query groups per (b, h)
+    int chunk_tiles;      // split mode: KT-token tiles per chunk
+    int q_groups;         // decode mode: (128 NW)-token query groups per (b, h)
     int items;
     float scale_log2;
     float* part_O;        // split: [parts][B*H][M][D]
@@ -287,25 +297,25 @@ struct Item {
     int bh, qz, kz, vz;
     int qrow0;            // first query row of the item
     int t_begin, t_end;   // key/value tile range
-    int part;             // split mode: partial index of warpgroup 0 (interleaved: 2c, else c)
+    int part;             // split mode: partial index of warpgroup 0 (interleaved: NW c, else c)
 };
 
+template <int NW>
 __device__ __forceinline__ Item decode_item(const Params& p, int item) {
     Item it;
     if (p.mode == kSplit) {
-        const int G = p.interleave ? 1 : p.row_groups;
-        const int g = item % G;
-        const int rest = item / G;
+        const int g = item % p.row_groups;
+        const int rest = item / p.row_groups;
         const int c = rest % p.chunks;
         it.bh = rest / p.chunks;
-        it.qrow0 = g * 256;
+        it.qrow0 = g * (p.interleave ? kQTile : NW * kQTile);
         it.t_begin = c * p.chunk_tiles;
         it.t_end = min(p.kv_tiles, it.t_begin + p.chunk_tiles);
-        it.part = p.interleave ? 2 * c : c;
+        it.part = p.interleave ? NW * c : c;
     } else {
-        const int pi = item % p.q_pairs;
-        it.bh = item / p.q_pairs;
-        it.qrow0 = pi * 256;
+        const int gi = item % p.q_groups;
+        it.bh = item / p.q_groups;
+        it.qrow0 = gi * NW * kQTile;
         it.t_begin = 0;
         it.t_end = p.kv_tiles;
         it.part = 0;
@@ -317,44 +327,59 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item) {
     return it;
 }
 
-// Shared-memory plan for head dim D, NST key/value stages, QS query slots.
-template <int D, int NST, int QS>
+// Shared-memory plan: QS query slots of NW [128 x D] tiles, NST stages of a
+// [KT x D] key tile and value tile, then the barriers.
+template <int D, int NW, int KT, int NST, int QS>
 struct Smem {
-    static constexpr int kTileBytes = kTokTile * D * 2;             // one [128 x D] bf16 tile
-    static constexpr int kQ = 0;                                     // QS slots x 2 tiles
-    static constexpr int kKV = kQ + QS * 2 * kTileBytes;             // NST stages x (K, V)
-    static constexpr int kBar = kKV + NST * 2 * kTileBytes;
-    // barriers: kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull[2], sfree[2], pfull[2], pfree[2], drain[2]
-    static constexpr int kNumBars = 2 * NST + 2 * QS + 8 + 2;
+    static constexpr int kQTileBytes = kQTile * D * 2;
+    static constexpr int kKVTileBytes = KT * D * 2;
+    static constexpr int kQ = 0;
+    static constexpr int kKV = kQ + QS * NW * kQTileBytes;
+    static constexpr int kBar = kKV + NST * 2 * kKVTileBytes;
+    // kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull, sfree, pfull, pfree, drain [NW each]
+    static constexpr int kNumBars = 2 * NST + 2 * QS + 5 * NW;
     static constexpr int kMisc = kBar + kNumBars * 8;               // tmem base (u32), abort flag (int)
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kLaunchBytes = kBytes + 1024;              // + alignment slack
 };
 
-template <int D>
+template <int D, int NW, int KT>
 struct Layout {
     // swizzle of a [rows x D] bf16 tile whose rows are D*2 bytes
     static constexpr uint32_t kType = D == 64 ? kLayoutSw128 : (D == 32 ? kLayoutSw64 : kLayoutSw32);
     static constexpr uint32_t kRowBytes = D * 2;
     static constexpr uint32_t kSbo = 8 * kRowBytes;                  // 8-row group stride
-    // TMEM column stride between the two warpgroups' O accumulators: at least
-    // 32 so that 32-column TMEM loads/stores of one never touch the other's
+    // TMEM: O accumulators at least 32 columns apart so that 32-column TMEM
+    // loads/stores of one never touch another's
     static constexpr int kOStride = D < 32 ? 32 : D;
-    static constexpr int kOCol = 256;                                 // O_0
-    static constexpr int kPCol = kOCol + 2 * kOStride;               // P_0; P_1 at +64
-    static_assert(kPCol + 128 <= 512, "TMEM plan exceeds 512 columns");
+    static constexpr int kOCol = NW * KT;
+    static constexpr int kPCol = kOCol + NW * kOStride;
+    static_assert(kPCol + NW * (KT / 2) <= 512, "TMEM plan exceeds 512 columns");
+    static constexpr int kChunks = KT / 32;                          // 32-column score chunks per row
+    static constexpr int kPairs = KT / 2;                            // column pairs per row
+    static constexpr int kFmaPairs = kFmaExpPairsPer64 * kPairs / 64;
 };
 
 // ------------------------------------------------------------------ the kernel
 
-template <int D, int NST, int QS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int NW, int KT, int NST, int QS>
+__global__ void __launch_bounds__(Regs<NW>::kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const Params p) {
     static_assert(D == 16 || D == 32 || D == 64, "tcgen05 path covers D in {16, 32, 64}");
-    static_assert(NST >= 3, "the score MMA runs two jobs ahead: at least three key/value stages");
-    using SM = Smem<D, NST, QS>;
-    using LY = Layout<D>;
+    static_assert(KT == 64 || KT == 128, "key/value tiles of 64 or 128 rows");
+    static_assert(NW >= 1 && NW <= 3, "the producer warpgroup holds one TMA warp and NW MMA warps");
+    static_assert(NST >= 3, "at least three key/value stages");
+    static_assert(NST % NW == 0, "interleaved mode splits the stages into one ring per warpgroup");
+    // Interleaved mode: warpgroup w owns stages [w R, w R + R) and consumes them in
+    // order, so no consumer can wait on a stage two fills ahead (a parity wait
+    // cannot tell phase k+1 from phase k-1).  Shared mode: one ring of NST stages
+    // that every warpgroup consumes in order.
+    constexpr int R = NST / NW;
+    using SM = Smem<D, NW, KT, NST, QS>;
+    using LY = Layout<D, NW, KT>;
+    constexpr int kTmaWarp = 4 * NW;
+    constexpr int kMmaWarp0 = 4 * NW + 1;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -364,10 +389,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     uint64_t* q_full = bars + 2 * NST;
     uint64_t* q_empty = q_full + QS;
     uint64_t* sfull = q_empty + QS;
-    uint64_t* sfree = sfull + 2;
-    uint64_t* pfull = sfree + 2;
-    uint64_t* pfree = pfull + 2;
-    uint64_t* drain = pfree + 2;
+    uint64_t* sfree = sfull + NW;
+    uint64_t* pfull = sfree + NW;
+    uint64_t* pfree = pfull + NW;
+    uint64_t* drain = pfree + NW;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kMisc + 4);
 
@@ -375,18 +400,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        // a key/value stage is released by every warpgroup that consumes it; a
-        // query slot by both warpgroups
-        for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], p.interleave ? 1 : 2); }
-        for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 2); }
-        for (int w = 0; w < 2; ++w) {
+        // a key/value stage is released by every warpgroup that consumes it;
+        // a query slot by every warpgroup
+        for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], p.interleave ? 1 : NW); }
+        for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], NW); }
+        for (int w = 0; w < NW; ++w) {
             mbar_init(&sfull[w], 1);
             mbar_init(&sfree[w], 4);
             mbar_init(&pfull[w], 4);
             mbar_init(&pfree[w], 1);
+            mbar_init(&drain[w], 1);
         }
-        mbar_init(&drain[0], 1);
-        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -395,7 +419,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
     }
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -404,41 +428,51 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int q_tiles = p.interleave ? 1 : NW;                         // query tiles per item
 
-    if (warp >= 8) {
+    if (warp >= 4 * NW) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
       if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t kv_load = 0, q_load = 0;
+            uint32_t kv_load = 0, q_load = 0, wg_load[NW] = {};
             int kv_last_phase[NST], q_last_phase[QS];
             for (int i = 0; i < NST; ++i) kv_last_phase[i] = -1;
             for (int i = 0; i < QS; ++i) q_last_phase[i] = -1;
-            const uint32_t kv_bytes = (p.kv_same ? 1 : 2) * SM::kTileBytes;
-            const uint32_t q_bytes = (p.interleave ? 1 : 2) * SM::kTileBytes;
+            const uint32_t kv_bytes = (p.kv_same ? 1 : 2) * SM::kKVTileBytes;
+            const uint32_t q_bytes = q_tiles * SM::kQTileBytes;
             bool ok = true;
             for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-                const Item it = decode_item(p, item);
+                const Item it = decode_item<NW>(p, item);
                 const int slot = q_load % QS;
                 ok = mbar_wait(&q_empty[slot], ((q_load / QS) & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 mbar_expect_tx(&q_full[slot], q_bytes);
-                uint8_t* qdst = smem + SM::kQ + slot * 2 * SM::kTileBytes;
-                tma_load_3d(qdst, &map_q, &q_full[slot], 0, it.qrow0, it.qz);
-                if (!p.interleave)
-                    tma_load_3d(qdst + SM::kTileBytes, &map_q, &q_full[slot], 0, it.qrow0 + kTokTile, it.qz);
+                uint8_t* qdst = smem + SM::kQ + slot * NW * SM::kQTileBytes;
+                for (int qt = 0; qt < q_tiles; ++qt)
+                    tma_load_3d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, it.qrow0 + qt * kQTile, it.qz);
                 q_last_phase[slot] = (q_load / QS) & 1;
                 ++q_load;
                 for (int t = it.t_begin; t < it.t_end; ++t) {
-                    const int st = kv_load % NST;
-                    ok = mbar_wait(&kv_empty[st], ((kv_load / NST) & 1) ^ 1, abort_flag);
+                    int st;
+                    uint32_t fill;                     // fills of this stage before this one
+                    if (p.interleave) {
+                        const int ow = (t - it.t_begin) % NW;
+                        st = ow * R + (int)(wg_load[ow] % R);
+                        fill = wg_load[ow] / R;
+                        ++wg_load[ow];
+                    } else {
+                        st = kv_load % NST;
+                        fill = kv_load / NST;
+                    }
+                    ok = mbar_wait(&kv_empty[st], (fill & 1) ^ 1, abort_flag);
                     if (!ok) break;
                     mbar_expect_tx(&kv_full[st], kv_bytes);
-                    uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kTileBytes;
-                    tma_load_3d(kdst, &map_k, &kv_full[st], 0, t * kTokTile, it.kz);
+                    uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kKVTileBytes;
+                    tma_load_3d(kdst, &map_k, &kv_full[st], 0, t * KT, it.kz);
                     if (!p.kv_same)
-                        tma_load_3d(kdst + SM::kTileBytes, &map_v, &kv_full[st], 0, t * kTokTile, it.vz);
-                    kv_last_phase[st] = (kv_load / NST) & 1;
+                        tma_load_3d(kdst + SM::kKVTileBytes, &map_v, &kv_full[st], 0, t * KT, it.vz);
+                    kv_last_phase[st] = fill & 1;
                     ++kv_load;
                 }
             }
@@ -456,17 +490,19 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     }
             }
         }
-      } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+      } else if (warp >= kMmaWarp0 && warp < kMmaWarp0 + NW) {
         // ---------------------------------------------------------- MMA issuers
-        // Warp 9 issues for softmax warpgroup 0, warp 10 for warpgroup 1, so the
-        // two warpgroups' pipelines never wait on each other's softmax.
+        // Warp kMmaWarp0 + w issues for softmax warpgroup w, so the warpgroups'
+        // pipelines never wait on each other's softmax.
         if (lane == 0) {
-            const int w = warp - kMmaWarp;
-            constexpr uint32_t idesc_s = make_idesc(128, 128, false);   // S = Q K^T: [128 q x 128 kv]
-            constexpr uint32_t idesc_o = make_idesc(128, D, true);      // O += P V:  [128 q x D], V MN-major
-            // This warpgroup's jobs: the key/value tiles it consumes, item by item
-            // (every tile, or alternate tiles when interleaved).  Two cursors over
-            // the stream: `sc` issues the score MMA one job ahead of `pc`.
+            const int w = warp - kMmaWarp0;
+            constexpr uint32_t idesc_s = make_idesc(kQTile, KT, false);   // S = Q K^T: [128 q x KT kv]
+            constexpr uint32_t idesc_o = make_idesc(kQTile, D, true);     // O += P V:  [128 q x D], V MN-major
+            const int tstep = p.interleave ? NW : 1;
+            const int tfirst = p.interleave ? w : 0;
+            // This warpgroup's jobs: the key/value tiles it consumes, item by item.
+            // Two cursors over the stream: `sc` issues the score MMA one job ahead
+            // of `pc`, which issues the value MMAs.
             struct Cursor {
                 int item, t, njobs;
                 bool valid;
@@ -480,8 +516,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             // counted in the right phase); only the score cursor does that.
             auto settle = [&](Cursor& c, bool score_cursor) {
                 while (c.item < p.items) {
-                    c.info = decode_item(p, c.item);
-                    c.t = c.info.t_begin + (p.interleave ? w : 0);
+                    c.info = decode_item<NW>(p, c.item);
+                    c.t = c.info.t_begin + tfirst;
                     c.njobs = 0;
                     if (c.t < c.info.t_end) {
                         c.valid = true;
@@ -506,27 +542,37 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             };
             auto next = [&](Cursor& c, bool score_cursor) {
                 ++c.njobs;
-                c.t += p.interleave ? 2 : 1;
+                c.t += tstep;
                 if (c.t < c.info.t_end) return;
                 c.tiles_before += c.info.t_end - c.info.t_begin;
                 ++c.item_count;
                 c.item += gridDim.x;
                 settle(c, score_cursor);
             };
-            auto stage_of = [&](const Cursor& c) { return (c.tiles_before + (c.t - c.info.t_begin)); };
+            // stage and fill count of the cursor's tile: this warpgroup's own ring in
+            // interleaved mode (its j-th tile), else the shared ring (global tile count)
+            auto stage_of = [&](const Cursor& c, uint32_t j, uint32_t& fill) -> int {
+                if (p.interleave) {
+                    fill = j / R;
+                    return w * R + (int)(j % R);
+                }
+                const uint32_t g = c.tiles_before + (c.t - c.info.t_begin);
+                fill = g / NST;
+                return (int)(g % NST);
+            };
             uint32_t s_issued = 0;
             auto issue_s = [&](const Cursor& c) -> bool {
                 const int slot = c.item_count % QS;
                 if (c.njobs == 0 && !mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag)) return false;
-                const uint32_t tile = stage_of(c);
-                const int st = tile % NST;
-                if (!mbar_wait(&kv_full[st], (tile / NST) & 1, abort_flag)) return false;
+                uint32_t fill;
+                const int st = stage_of(c, s_issued, fill);
+                if (!mbar_wait(&kv_full[st], fill & 1, abort_flag)) return false;
                 if (!mbar_wait(&sfree[w], (s_issued & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t qaddr = smem_u32(smem + SM::kQ + slot * 2 * SM::kTileBytes +
-                                                (p.interleave ? 0 : w * SM::kTileBytes));
-                const uint32_t kaddr = smem_u32(smem + SM::kKV + st * 2 * SM::kTileBytes);
-                const uint32_t d_tmem = tmem + w * 128;
+                const uint32_t qaddr = smem_u32(smem + SM::kQ + slot * NW * SM::kQTileBytes +
+                                                (p.interleave ? 0 : w * SM::kQTileBytes));
+                const uint32_t kaddr = smem_u32(smem + SM::kKV + st * 2 * SM::kKVTileBytes);
+                const uint32_t d_tmem = tmem + w * KT;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = smem_desc(qaddr + kk * 32, 16, LY::kSbo, LY::kType);
@@ -536,24 +582,25 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 umma_commit(&sfull[w]);
                 ++s_issued;
                 // this warpgroup's last score MMA of the item releases its share of the query slot
-                if (c.t + (p.interleave ? 2 : 1) >= c.info.t_end) umma_commit(&q_empty[slot]);
+                if (c.t + tstep >= c.info.t_end) umma_commit(&q_empty[slot]);
                 return true;
             };
             uint32_t pv_issued = 0;
             auto issue_pv = [&](const Cursor& c) -> bool {
                 if (!mbar_wait(&pfull[w], pv_issued & 1, abort_flag)) return false;
                 tc_fence_after();
-                const int st = stage_of(c) % NST;
-                const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kTileBytes + (p.kv_same ? 0 : SM::kTileBytes);
+                uint32_t fill;
+                const int st = stage_of(c, pv_issued, fill);
+                const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kKVTileBytes + (p.kv_same ? 0 : SM::kKVTileBytes);
                 const uint32_t vaddr = smem_u32(vbase);
                 const uint32_t d_tmem = tmem + LY::kOCol + w * LY::kOStride;
-                const uint32_t p_tmem = tmem + LY::kPCol + w * 64;
+                const uint32_t p_tmem = tmem + LY::kPCol + w * (KT / 2);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < KT / 16; ++kk) {
                     // A = P in TMEM: 16 key/value columns = 8 packed bf16x2 columns per step
-                    // B = V tile [128 kv x D], D contiguous: MN-major; 16 kv rows per step
+                    // B = V tile [KT kv x D], D contiguous: MN-major; 16 kv rows per step
                     // (D fits one swizzle atom along MN, so the leading offset is never used)
-                    const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kTileBytes,
+                    const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kKVTileBytes,
                                                   LY::kSbo, LY::kType);
                     umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
                 }
@@ -586,54 +633,57 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         }
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Regs<NW>::kSoftmax));
         // ---------------------------------------------------------- softmax warpgroups
         const int wg = warp >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_base + wg * 128;
+        const uint32_t tS = tmem + lane_base + wg * KT;
         const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride;
-        const uint32_t tP = tmem + lane_base + LY::kPCol + wg * 64;
+        const uint32_t tP = tmem + lane_base + LY::kPCol + wg * (KT / 2);
         const float sl2 = p.scale_log2;
+        const int tstep = p.interleave ? NW : 1;
+        const int tfirst = p.interleave ? wg : 0;
         uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-            const Item it = decode_item(p, item);
+            const Item it = decode_item<NW>(p, item);
             float m_run = -INFINITY, l_run = 0.f;
             int njobs = 0;
-            const int tstep = p.interleave ? 2 : 1;
-            for (int t = it.t_begin + (p.interleave ? wg : 0); t < it.t_end; t += tstep) {
+            for (int t = it.t_begin + tfirst; t < it.t_end; t += tstep) {
                 if (!mbar_wait(&sfull[wg], sfull_waits & 1, abort_flag)) { ok = false; break; }
                 ++sfull_waits;
                 tc_fence_after();
-                uint32_t sr[4][32];
+                uint32_t sr[LY::kChunks][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                for (int c = 0; c < LY::kChunks; ++c) tmem_ld32(tS + c * 32, sr[c]);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sfree[wg]);
 
-                const int valid = p.kv_rows - t * kTokTile;      // key/value rows of this tile that exist
-                if (valid < kTokTile) {                           // ragged last tile only (warp-uniform)
+                const int valid = p.kv_rows - t * KT;             // key/value rows of this tile that exist
+                if (valid < KT) {                                 // ragged last tile only (warp-uniform)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < LY::kChunks; ++c)
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (c * 32 + j >= valid) sr[c][j] = __float_as_uint(-INFINITY);
                 }
-                // row max: four independent chains of 3-input maxima (short dependency chains)
-                float mc[4];
+                // row max: one chain of 3-input maxima per 32-column chunk (short dependency chains)
+                float mc[LY::kChunks];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < LY::kChunks; ++c) {
                     mc[c] = __uint_as_float(sr[c][0]);
 #pragma unroll
                     for (int j = 1; j < 31; j += 2)
                         mc[c] = max3f(mc[c], __uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1]));
                     mc[c] = fmaxf(mc[c], __uint_as_float(sr[c][31]));
                 }
-                const float mx = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+                float mx = mc[0];
+#pragma unroll
+                for (int c = 1; c < LY::kChunks; ++c) mx = fmaxf(mx, mc[c]);
                 const float m_new = fmaxf(m_run, mx * sl2);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
@@ -641,28 +691,29 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     factor = ex2_mufu(m_run - m_new);
                     m_run = m_new;
                 }
-                // exponent arguments in pairs (packed fp32 FMA), row sum in four packed chains
+                // exponent arguments in pairs (packed fp32 FMA), row sum in packed chains
                 const float2 sl2v = make_float2(sl2, sl2);
                 const float2 negm = make_float2(-m_run, -m_run);
-                float2 acc[4];
-                uint32_t pk[2][32];                  // [half][j]: columns 64*half + 2j, 2j+1
+                float2 acc[LY::kChunks];
+                uint32_t pk[KT / 64][32];            // [half][j]: columns 64*half + 2j, 2j+1
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < LY::kChunks; ++c) {
                     acc[c] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float2 sv = make_float2(__uint_as_float(sr[c][2 * j]), __uint_as_float(sr[c][2 * j + 1]));
                         const float2 xv = __ffma2_rn(sv, sl2v, negm);
-                        const float2 pv = (c * 16 + j >= 64 - kFmaExpPairs)
+                        const float2 pv = (c * 16 + j >= LY::kPairs - LY::kFmaPairs)
                                               ? ex2_fma_pair(xv)
                                               : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
                         pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(pv.x, pv.y);
                     }
                 }
-                const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-                const float2 a = __fadd2_rn(a01, a23);
-                l_run = l_run * factor + (a.x + a.y);
+                float2 asum = acc[0];
+#pragma unroll
+                for (int c = 1; c < LY::kChunks; ++c) asum = __fadd2_rn(asum, acc[c]);
+                l_run = l_run * factor + (asum.x + asum.y);
 
                 // the previous value MMA of this warpgroup must be done before P and O are touched
                 while (pfree_waits < jobs_done) {
@@ -683,9 +734,9 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         tmem_st32(tO + c * 32, o);
                     }
                 }
-                // P row -> TMEM (this thread's lane, 64 columns of bf16 pairs)
-                tmem_st32(tP, pk[0]);
-                tmem_st32(tP + 32, pk[1]);
+                // P row -> TMEM (this thread's lane, KT/2 columns of bf16 pairs)
+#pragma unroll
+                for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -714,10 +765,9 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[c][j] = 0u;
             }
-            // with D = 16 only the first 16 columns of the 32-column load are O (the
-            // rest belong to the other warpgroup's O or are unused)
+            // with D = 16 only the first 16 columns of the 32-column load are O
             if (p.mode == kSplit) {
-                const int r = p.interleave ? row : it.qrow0 + wg * kTokTile + row;
+                const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
                 const int part = p.interleave ? it.part + wg : it.part;
                 if (r < p.M) {
                     const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
@@ -731,7 +781,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                                              __uint_as_float(o[i / 8][(i % 8) * 4 + 3]));
                 }
             } else {
-                const int n = it.qrow0 + wg * kTokTile + row;
+                const int n = it.qrow0 + wg * kQTile + row;
                 if (n < p.N) {
                     const float inv = 1.f / l_run;
                     uint4* dst = reinterpret_cast<uint4*>(p.y + ((int64_t)it.bh * p.N + n) * D);
@@ -751,7 +801,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
@@ -774,17 +824,49 @@ struct Problem {
     float scale_log2;
 };
 
+// Kernel configurations: NW softmax warpgroups, KT-row key/value tiles, NST
+// key/value stages, QS query slots.  The split passes (synthesis, encode) use
+// two warpgroups on 128-row key/value tiles that both consume (each tile read
+// from L2 once per 256 latents); the decode uses three warpgroups on 64-row
+// latent tiles (more softmax warps per SM sub-partition to hide latency).
+template <int D, int NW_, int KT_>
+struct Config {
+    static constexpr int NW = NW_;
+    static constexpr int KT = KT_;
+    static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 64 ? 4 : 6);
+    static constexpr int QS = 2;
+    using SM = Smem<D, NW, KT, NST, QS>;
+    // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
+    static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
+};
+constexpr int kSplitNW = 2, kSplitKT = 128;
+constexpr int kDecodeNW = 3, kDecodeKT = 64;
+
 inline bool supported(bool bf16, int D, int M) {
     (void)M;
     return bf16 && (D == 16 || D == 32 || D == 64);
 }
 
-// latent-row groups handled per (b, h, chunk): one 256-row group per item,
-// or a single shared 128-row tile when M <= 128 (interleaved)
-inline int row_groups(int M) { return M <= 128 ? 1 : (M + 255) / 256; }
-inline bool interleaved(int M) { return M <= 128; }
-inline int parts_per_chunk(int M) { return interleaved(M) ? 2 : 1; }
-inline int target_ctas() { return 4 * kNumSMs; }
+// Split-pass plan.  With one 128-row tile holding all M latents, the two
+// warpgroups share it and take the key/value tiles round-robin (interleaved,
+// two partial triples per chunk); otherwise each takes its own 128 latents.
+inline int kv_tile() { return kSplitKT; }
+inline bool interleaved(int M) { return M <= kQTile; }
+inline int row_groups(int M) {
+    return interleaved(M) ? (M + kQTile - 1) / kQTile : (M + kSplitNW * kQTile - 1) / (kSplitNW * kQTile);
+}
+inline int parts_per_chunk(int M) { return interleaved(M) ? kSplitNW : 1; }
+
+// Token chunks per (b, h): at least `min_items` items in all, preferring a
+// count that makes the items a whole number of waves over the SMs.
+inline int64_t choose_chunks(int64_t units, int64_t tiles, int sms) {
+    const int64_t min_items = 4LL * sms;
+    int64_t c0 = (min_items + units - 1) / units;
+    c0 = std::max<int64_t>(1, std::min<int64_t>(c0, tiles));
+    for (int64_t c = c0; c <= std::min<int64_t>(tiles, 4 * c0); ++c)
+        if ((units * c) % sms == 0) return c;
+    return c0;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -803,13 +885,13 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D map over a [planes, rows, D] bf16 tensor, box [1, 128, D], swizzle = D*2 bytes.
-inline bool make_map(CUtensorMap* map, const void* base, int planes, int rows, int D) {
+// 3-D map over a [planes, rows, D] bf16 tensor, box [1, box_rows, D], swizzle = D*2 bytes.
+inline bool make_map(CUtensorMap* map, const void* base, int planes, int rows, int D, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)kTokTile, 1};
+    const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                           : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -824,34 +906,26 @@ inline int sm_count() {
     return n > 0 ? n : kNumSMs;
 }
 
-template <int D>
-struct Config {
-    static constexpr int NST = D == 64 ? 4 : 6;
-    static constexpr int QS = 2;
-    using SM = Smem<D, NST, QS>;
-    // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
-    static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
-};
-
-template <int D>
+template <int D, int NW, int KT>
 int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& prm,
                 cudaStream_t st) {
-    using C = Config<D>;
-    auto kern = attn_kernel<D, C::NST, C::QS>;
+    using C = Config<D, NW, KT>;
+    auto kern = attn_kernel<D, C::NW, C::KT, C::NST, C::QS>;
     static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = prm.items < sm_count() ? prm.items : sm_count();
-    kern<<<grid, kThreads, C::kSmemLaunch, st>>>(mq, mk, mv, prm);
+    kern<<<grid, Regs<C::NW>::kThreads, C::kSmemLaunch, st>>>(mq, mk, mv, prm);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
+template <int NW, int KT>
 inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const Params& prm, cudaStream_t st) {
     switch (D) {
-        case 16: return launch_attn<16>(mq, mk, mv, prm, st);
-        case 32: return launch_attn<32>(mq, mk, mv, prm, st);
-        case 64: return launch_attn<64>(mq, mk, mv, prm, st);
+        case 16: return launch_attn<16, NW, KT>(mq, mk, mv, prm, st);
+        case 32: return launch_attn<32, NW, KT>(mq, mk, mv, prm, st);
+        case 64: return launch_attn<64, NW, KT>(mq, mk, mv, prm, st);
         default: return 2;
     }
 }
@@ -877,23 +951,27 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
         cudaStream_t st) {
     const bool gated = gate != nullptr;
     const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
-    CUtensorMap m_q0, m_qf, m_q16, m_z16, m_k0, m_k, m_v;
-    bool ok = make_map(&m_qf, q_fixed, H, M, D) && make_map(&m_q16, bu.q16, BH, M, D) &&
-              make_map(&m_z16, bu.z16, BH, M, D) && make_map(&m_k, k, BH, N, D) && make_map(&m_v, v, BH, N, D);
-    if (gated) ok = ok && make_map(&m_q0, q0, H, M, D) && make_map(&m_k0, k0, BH, N, D);
+    // query maps use 128-row boxes, key/value maps the pass's tile height; the
+    // token keys k serve as key/value tiles (split) and as query tiles (decode)
+    CUtensorMap m_q0, m_qf_q, m_qf_kv, m_q16_q, m_q16_kv, m_z16, m_k0, m_k_kv, m_k_q, m_v;
+    bool ok = make_map(&m_qf_q, q_fixed, H, M, D, kQTile) && make_map(&m_qf_kv, q_fixed, H, M, D, kDecodeKT) &&
+              make_map(&m_q16_q, bu.q16, BH, M, D, kQTile) && make_map(&m_q16_kv, bu.q16, BH, M, D, kDecodeKT) &&
+              make_map(&m_z16, bu.z16, BH, M, D, kDecodeKT) && make_map(&m_k_kv, k, BH, N, D, kSplitKT) &&
+              make_map(&m_k_q, k, BH, N, D, kQTile) && make_map(&m_v, v, BH, N, D, kSplitKT);
+    if (gated) ok = ok && make_map(&m_q0, q0, H, M, D, kQTile) && make_map(&m_k0, k0, BH, N, D, kSplitKT);
     if (!ok) return 3;
 
-    const int kv_tiles = (N + kTokTile - 1) / kTokTile;
-    const int chunk_tiles = pr.chunk_len / kTokTile;
+    const int kv_tiles = (N + kSplitKT - 1) / kSplitKT;
+    const int chunk_tiles = pr.chunk_len / kSplitKT;
     Params sp{};
     sp.mode = kSplit;
     sp.B = B; sp.H = H; sp.M = M; sp.N = N;
-    sp.q_rows = M; sp.kv_rows = N; sp.kv_tiles = kv_tiles;
+    sp.kv_rows = N; sp.kv_tiles = kv_tiles;
     sp.interleave = interleaved(M) ? 1 : 0;
     sp.row_groups = row_groups(M);
     sp.chunks = pr.chunks;
     sp.chunk_tiles = chunk_tiles;
-    sp.items = BH * pr.chunks * (sp.interleave ? 1 : sp.row_groups);
+    sp.items = BH * pr.chunks * sp.row_groups;
     sp.scale_log2 = pr.scale_log2;
     sp.part_O = bu.part_O;
     sp.part_ml = bu.part_ml;
@@ -909,7 +987,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     if (gated) {
         Params s1 = sp;
         s1.q_shared = 1; s1.k_shared = 0; s1.kv_same = 1;
-        rc = launch_attn_d(D, m_q0, m_k0, m_k0, s1, st);
+        rc = launch_attn_d<kSplitNW, kSplitKT>(D, m_q0, m_k0, m_k0, s1, st);
         if (rc) return rc;
         mark(st);
         mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_bf16 = bu.q16; mp.user_out = q_out;
@@ -919,7 +997,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     }
     Params s2 = sp;
     s2.q_shared = gated ? 0 : 1; s2.k_shared = 0; s2.kv_same = 0;
-    rc = launch_attn_d(D, gated ? m_q16 : m_qf, m_k, m_v, s2, st);
+    rc = launch_attn_d<kSplitNW, kSplitKT>(D, gated ? m_q16_q : m_qf_q, m_k_kv, m_v, s2, st);
     if (rc) return rc;
     mark(st);
     mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_bf16 = bu.z16; mp.user_out = z_out;
@@ -930,14 +1008,14 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     Params dp{};
     dp.mode = kDecode;
     dp.B = B; dp.H = H; dp.M = M; dp.N = N;
-    dp.q_rows = N; dp.kv_rows = M; dp.kv_tiles = (M + kTokTile - 1) / kTokTile;
+    dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
     dp.q_shared = 0; dp.k_shared = gated ? 0 : 1; dp.kv_same = 0;
     dp.interleave = 0;
-    dp.q_pairs = (N + 255) / 256;
-    dp.items = BH * dp.q_pairs;
+    dp.q_groups = (N + kDecodeNW * kQTile - 1) / (kDecodeNW * kQTile);
+    dp.items = BH * dp.q_groups;
     dp.scale_log2 = pr.scale_log2;
     dp.y = static_cast<__nv_bfloat16*>(y);
-    rc = launch_attn_d(D, m_k, gated ? m_q16 : m_qf, m_z16, dp, st);
+    rc = launch_attn_d<kDecodeNW, kDecodeKT>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
     if (rc) return rc;
     mark(st);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
