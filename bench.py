@@ -39,6 +39,7 @@ UNIT = "Mtokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES_GATED = ["split_partial(synthesis)", "merge(q)", "split_partial(encode)", "merge(z)", "decode"]
+STAGES_FLARE = ["split_partial(encode)", "merge(z)", "decode"]
 
 
 def parse_args(argv=None):
@@ -51,6 +52,7 @@ def parse_args(argv=None):
                    help="override N of the workload (a smaller case of the same kernels, e.g. for ncu)")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
+    p.add_argument("--flare", action="store_true", help="closed gate: the two-call FLARE form (flare_fwd)")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -268,16 +270,18 @@ def run_ours(args):
     path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
     dtype_code = fb.F32 if w.dtype == "f32" else fb.BF16
     used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
-    ws = torch.empty(fb.workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, True, path), dtype=torch.uint8,
+    gated = not args.flare
+    ws = torch.empty(fb.workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, gated, path), dtype=torch.uint8,
                      device=dev)
     y = torch.empty_like(x["k"])
-    n_launch = fb.launches_per_call(True)
+    n_launch = fb.launches_per_call(gated)
+    stage_names = STAGES_GATED if gated else STAGES_FLARE
     fits_l2 = 5 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
 
     def step(events=None):
-        fb.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], y, path=path, workspace=ws,
-                     stage_events=events)
+        fb.mixer_fwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y, path=path,
+                     workspace=ws, stage_events=events)
 
     for _ in range(args.warmup):
         step()
@@ -310,36 +314,43 @@ def run_ours(args):
     else:
         local_ms = sum(evs[i][0].elapsed_time(evs[i][n_launch]) for i in range(K))
     max_ms = reduce_max(local_ms, world, dev)
-    counts = W.algorithmic_counts(w)
+    counts = W.algorithmic_counts(w, flare=not gated)
     value = aggregate_mtokens(counts["tokens"], world, K, max_ms)
     ms_per_step = max_ms / K
 
     # live per-kernel figures (this rank)
     avg_stage = [statistics.mean(s[j] for s in stage_ms) for j in range(n_launch)]
     total_stage = sum(avg_stage)
-    stages = {STAGES_GATED[j]: {"ms": round(avg_stage[j], 4), "share": round(avg_stage[j] / total_stage, 4)}
+    stages = {stage_names[j]: {"ms": round(avg_stage[j], 4), "share": round(avg_stage[j] / total_stage, 4)}
               for j in range(n_launch)}
-    split_ms = statistics.mean([avg_stage[0], avg_stage[2]])
+    split_ms = statistics.mean([avg_stage[0], avg_stage[2]]) if gated else avg_stage[0]
     bhnmd = w.B * w.H * w.N * w.M * w.D
     flops_per_split_launch = 4.0 * bhnmd
     peaks, peak_src = load_peaks()
     peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_b = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    # bytes: mean of the split launches (synthesis reads k0 once, encode reads k and v)
+    bytes_per_split_launch = (1.5 if gated else 2.0) * w.B * w.H * w.N * w.D * (4 if w.dtype == "f32" else 2)
     achieved_t = flops_per_split_launch / (split_ms * 1e-3) / 1e12
+    achieved_b = bytes_per_split_launch / (split_ms * 1e-3) / 1e9
+    # the binding roof: tensor pipe when the launch's FLOP/byte is above the measured ridge, else HBM
+    tensor_bound = flops_per_split_launch / bytes_per_split_launch > peak_t * 1e12 / (peak_b * 1e9)
     roofline = {
-        "bound": "tensor",
+        "bound": "tensor" if tensor_bound else "hbm",
         "kernel": "split_partial" if used_path == fb.PATH_TCGEN05 else "split_partial_simt",
-        "achieved": round(achieved_t, 2),
-        "peak": peak_t,
-        "unit": "TFLOP/s",
-        "frac": round(achieved_t / peak_t, 4),
+        "achieved": round(achieved_t if tensor_bound else achieved_b, 2),
+        "peak": peak_t if tensor_bound else peak_b,
+        "unit": "TFLOP/s" if tensor_bound else "GB/s",
+        "frac": round(achieved_t / peak_t if tensor_bound else achieved_b / peak_b, 4),
         "traffic": ncu_traffic("split_partial", w.name),
-        "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside back-to-back steps)",
-        # bytes: mean of the two split launches (synthesis reads k0 once, encode reads k and v)
-        "algorithmic_per_launch": {"flops": flops_per_split_launch,
-                                   "bytes": 1.5 * w.B * w.H * w.N * w.D * (4 if w.dtype == 'f32' else 2)},
+        "peak_kind": (f"{peak_src} bf16 sustained (kernel timed inside back-to-back steps)" if tensor_bound
+                      else f"{peak_src} HBM copy bandwidth"),
+        "algorithmic_per_launch": {"flops": flops_per_split_launch, "bytes": bytes_per_split_launch},
         "launch_ms": round(split_ms, 4),
+        "tensor_frac": round(achieved_t / peak_t, 4),
+        "hbm_frac": round(achieved_b / peak_b, 4),
     }
-    decode_ms = avg_stage[4]
+    decode_ms = avg_stage[n_launch - 1]
     dec_t = 4.0 * bhnmd / (decode_ms * 1e-3) / 1e12
 
     out = {
@@ -356,7 +367,8 @@ def run_ours(args):
         "dtype": w.dtype,
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
-                   "gate": "open (FLARE++)", "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
+                   "gate": "open (FLARE++)" if gated else "closed (FLARE, flare_fwd)",
+                   "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)"),
                    "parallelism": f"replicas x{world} (independent problems per rank)",
@@ -378,18 +390,20 @@ def run_ours(args):
             hx[name].copy_(x[name])
         hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
         ke = max(1, min(K, 5))
-        fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hx["gate"], hx["k0"], hx["k"], hx["v"], hy)  # warm-up
+        hg = hx["gate"] if gated else None
+        fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hg, hx["k0"], hx["k"], hx["v"], hy)  # warm-up
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
         e0.record()
         for _ in range(ke):
-            fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hx["gate"], hx["k0"], hx["k"], hx["v"], hy)
+            fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hg, hx["k0"], hx["k"], hx["v"], hy)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev)
-        h2d = sum(hx[n].numel() * hx[n].element_size() for n in hx)
+        h2d = sum(hx[n].numel() * hx[n].element_size() for n in hx
+                  if gated or n in ("q_fixed", "k", "v"))
         out["e2e"] = {"value": round(aggregate_mtokens(counts["tokens"], world, ke, e2e_ms), 4), "unit": UNIT,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hy.numel() * hy.element_size(),
                       "steps": ke, "api": "flarepp_mixer_fwd_host (pinned host buffers)"}

@@ -167,6 +167,14 @@ int flarepp_mixer_fwd_noalloc(const void* q0, const void* q_fixed, const float* 
  * arguments the forward entries would reject. */
 int flarepp_selected_path(int B, int H, int N, int M, int D, int dtype);
 
+/* Diagnostic for the failure path: launches on `stream` one thread that waits,
+ * with the kernels' bounded wait and a limit of limit_us microseconds
+ * (1 .. 1e6), on an mbarrier nothing ever arrives at.  The wait gives up and
+ * records FLAREPP_ERR_TIMEOUT in the device status word, which the next
+ * flarepp_check_device_status returns (and clears); the context stays usable.
+ * Returns the launch status. */
+int flarepp_selftest_wait_timeout(void* stream, unsigned int limit_us);
+
 /* Synchronises `stream`, then returns and clears the device status word
  * (FLAREPP_OK when no kernel recorded a failure on the current device). */
 int flarepp_check_device_status(void* stream);

@@ -219,6 +219,15 @@ def mixer_fwd_noalloc(q0, q_fixed, gate, k0, k, v, y):
     return y
 
 
+def selftest_wait_timeout(limit_us: int = 20000, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Launches the bounded-wait self-test (a wait nothing satisfies); returns the launch status."""
+    fn = lib.flarepp_selftest_wait_timeout
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_uint]
+    fn.restype = ctypes.c_int
+    st = (stream or torch.cuda.current_stream()).cuda_stream
+    return int(fn(st, int(limit_us)))
+
+
 def check_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     st = (stream or torch.cuda.current_stream()).cuda_stream
     return int(lib.flarepp_check_device_status(st))

@@ -560,6 +560,13 @@ int flarepp_selected_path(int B, int H, int N, int M, int D, int dtype) {
     return pl.path;
 }
 
+int flarepp_selftest_wait_timeout(void* stream, unsigned int limit_us) {
+    if (limit_us == 0 || limit_us > 1000000u) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    tc::wait_timeout_selftest<<<1, 32, 0, st>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
 int flarepp_check_device_status(void* stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return FLAREPP_ERR_CUDA;

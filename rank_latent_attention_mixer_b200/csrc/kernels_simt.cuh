@@ -139,7 +139,13 @@ struct MergeParams {
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 merge_partials(MergeParams p) {
-    constexpr int PER = (D + 31) / 32;
+    // A warp merges one latent row.  Each lane loads one float4 of a chunk's O
+    // row, so LPC = D/4 lanes cover a chunk and the warp takes CPI = 32/LPC
+    // chunks per iteration (D = 128: one chunk in four float4s per lane).
+    constexpr int V4 = D / 4;
+    constexpr int LPC = V4 < 32 ? V4 : 32;
+    constexpr int CPI = 32 / LPC;
+    constexpr int F4PL = V4 / LPC;              // float4s per lane per chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t rows = (int64_t)p.B * p.H * p.M;
     const int64_t row = (int64_t)blockIdx.x * 8 + warp;
@@ -153,33 +159,54 @@ merge_partials(MergeParams p) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
 
-    float L = 0.f, acc[PER];
+    const int sub = lane / LPC, li = lane % LPC;
+    float L = 0.f;
+    float4 acc[F4PL];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    for (int c = 0; c < p.chunks; ++c) {
-        const float2 ml = p.part_ml[c * cstride + row];
-        if (ml.y <= 0.f) continue;               // empty chunk contributes nothing
-        const float w = ex2_mufu(ml.x - mstar);
-        L = fmaf(w, ml.y, L);
-        const float* o = p.part_O + (c * cstride + row) * D;
+    for (int i = 0; i < F4PL; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < p.chunks; c0 += CPI) {
+        const int c = c0 + sub;
+        if (c < p.chunks) {
+            const float2 ml = p.part_ml[c * cstride + row];
+            const float4* o4 = reinterpret_cast<const float4*>(p.part_O + (c * cstride + row) * D);
+            const float w = ml.y > 0.f ? ex2_mufu(ml.x - mstar) : 0.f;   // empty chunk contributes nothing
+            L = fmaf(w, ml.y, L);
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int d = lane + 32 * i;
-            if (d < D) acc[i] = fmaf(w, o[d], acc[i]);
+            for (int i = 0; i < F4PL; ++i) {
+                const float4 v = o4[li + LPC * i];
+                acc[i].x = fmaf(w, v.x, acc[i].x); acc[i].y = fmaf(w, v.y, acc[i].y);
+                acc[i].z = fmaf(w, v.z, acc[i].z); acc[i].w = fmaf(w, v.w, acc[i].w);
+            }
         }
     }
+    // combine the CPI chunk groups of the warp (lanes li, li + LPC, ...)
+#pragma unroll
+    for (int o = 16; o >= LPC; o >>= 1) {
+        L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+        for (int i = 0; i < F4PL; ++i) {
+            acc[i].x += __shfl_xor_sync(0xffffffffu, acc[i].x, o);
+            acc[i].y += __shfl_xor_sync(0xffffffffu, acc[i].y, o);
+            acc[i].z += __shfl_xor_sync(0xffffffffu, acc[i].z, o);
+            acc[i].w += __shfl_xor_sync(0xffffffffu, acc[i].w, o);
+        }
+    }
+    if (sub != 0) return;
     const float inv = 1.f / L;
     const T* qf = reinterpret_cast<const T*>(p.q_fixed) + ((int64_t)h * p.M + m) * D;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int d = lane + 32 * i;
-        if (d >= D) continue;
-        float val = acc[i] * inv;
-        if (p.mode == kMergeSynthesis) val = fmaf(p.gate[h], val, to_f32<T>(qf[d]));
-        p.out_f32[row * D + d] = val;
-        p.out_bf16[row * D + d] = __float2bfloat16_rn(val);
-        if (p.user_out) p.user_out[row * D + d] = val;
-        if (p.q_copy_out) p.q_copy_out[row * D + d] = to_f32<T>(qf[d]);
+    for (int i = 0; i < F4PL; ++i) {
+        const int d0 = 4 * (li + LPC * i);
+        float val[4] = {acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int d = d0 + e;
+            if (p.mode == kMergeSynthesis) val[e] = fmaf(p.gate[h], val[e], to_f32<T>(qf[d]));
+            p.out_f32[row * D + d] = val[e];
+            p.out_bf16[row * D + d] = __float2bfloat16_rn(val[e]);
+            if (p.user_out) p.user_out[row * D + d] = val[e];
+            if (p.q_copy_out) p.q_copy_out[row * D + d] = to_f32<T>(qf[d]);
+        }
     }
 }
 

@@ -116,14 +116,15 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 // Waits until the phase with the given parity has completed.  Returns false
 // if the CTA's abort flag is up or the wait ran past kWaitLimitNs (then it
 // raises the flag and records the timeout).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
+            if (globaltimer_ns() - t0 > limit_ns || it > (1u << 30)) {
                 *abort_flag = 1;
                 record_status(kStatusTimeout);
                 return false;
@@ -647,6 +648,56 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         const int tfirst = p.interleave ? wg : 0;
         uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0;
         bool ok = true;
+        // Item outputs from this thread's O row (o == nullptr: the warpgroup had no
+        // job in the item).  With D = 16 only the first 16 of 32 loaded columns are O.
+        auto write_outputs = [&](const Item& it, int njobs, float m, float l, const uint32_t (*o)[32]) {
+            if (p.mode == kSplit) {
+                const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
+                const int part = p.interleave ? it.part + wg : it.part;
+                if (r < p.M) {
+                    const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
+                    p.part_ml[ridx] = make_float2(njobs > 0 ? m : -INFINITY, l);
+                    float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D);
+#pragma unroll
+                    for (int i = 0; i < D / 4; ++i)
+                        dst[i] = o ? make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
+                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
+                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
+                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 3]))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            } else {
+                const int n = it.qrow0 + wg * kQTile + row;
+                if (n < p.N && o) {
+                    const float inv = 1.f / l;
+                    uint4* dst = reinterpret_cast<uint4*>(p.y + ((int64_t)it.bh * p.N + n) * D);
+#pragma unroll
+                    for (int i = 0; i < D / 8; ++i) {
+                        const int c = i / 4, j = (i % 4) * 8;
+                        dst[i] = make_uint4(
+                            pack_bf16x2(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                    }
+                }
+            }
+        };
+        // O row of the finished item -> outputs (every value MMA of the item has completed)
+        auto flush = [&](const Item& it, int njobs, float m, float l) {
+            uint32_t o[(D + 31) / 32][32];
+#pragma unroll
+            for (int c = 0; c < (D + 31) / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+            tmem_wait_ld();
+            write_outputs(it, njobs, m, l, o);
+        };
+        // The epilogue of an item is deferred into the next item's first job:
+        // its last value MMA finishes while the next exponentials are computed,
+        // and its O row is read just before the next value MMA overwrites it.
+        bool pend = false;
+        Item pend_it{};
+        int pend_jobs = 0;
+        float pend_m = 0.f, pend_l = 0.f;
         for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const Item it = decode_item<NW>(p, item);
             float m_run = -INFINITY, l_run = 0.f;
@@ -722,6 +773,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 if (!ok) break;
                 tc_fence_after();
+                if (pend) {
+                    flush(pend_it, pend_jobs, pend_m, pend_l);
+                    pend = false;
+                }
                 if (__any_sync(0xffffffffu, resc && njobs > 0)) {
                     const float f = njobs > 0 ? factor : 1.f;
 #pragma unroll
@@ -746,55 +801,25 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             }
             if (!ok) break;
 
-            // ---------------- epilogue of the item
-            uint32_t o[(D + 31) / 32][32];
+            // ---------------- end of the item: defer its epilogue
             if (njobs > 0) {
-                while (pfree_waits < jobs_done) {
-                    if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
-                    ++pfree_waits;
-                }
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < (D + 31) / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
-                tmem_wait_ld();
-                tc_fence_before();
+                pend = true;
+                pend_it = it;
+                pend_jobs = njobs;
+                pend_m = m_run;
+                pend_l = l_run;
             } else {
-#pragma unroll
-                for (int c = 0; c < (D + 31) / 32; ++c)
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) o[c][j] = 0u;
+                write_outputs(it, 0, m_run, l_run, nullptr);
             }
-            // with D = 16 only the first 16 columns of the 32-column load are O
-            if (p.mode == kSplit) {
-                const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
-                const int part = p.interleave ? it.part + wg : it.part;
-                if (r < p.M) {
-                    const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
-                    p.part_ml[ridx] = make_float2(njobs > 0 ? m_run : -INFINITY, l_run);
-                    float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D);
-#pragma unroll
-                    for (int i = 0; i < D / 4; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
-                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
-                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
-                                             __uint_as_float(o[i / 8][(i % 8) * 4 + 3]));
-                }
-            } else {
-                const int n = it.qrow0 + wg * kQTile + row;
-                if (n < p.N) {
-                    const float inv = 1.f / l_run;
-                    uint4* dst = reinterpret_cast<uint4*>(p.y + ((int64_t)it.bh * p.N + n) * D);
-#pragma unroll
-                    for (int i = 0; i < D / 8; ++i) {
-                        const int c = i / 4, j = (i % 4) * 8;
-                        dst[i] = make_uint4(
-                            pack_bf16x2(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
-                    }
-                }
+        }
+        if (ok && pend) {
+            while (pfree_waits < jobs_done) {
+                if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                ++pfree_waits;
+            }
+            if (ok) {
+                tc_fence_after();
+                flush(pend_it, pend_jobs, pend_m, pend_l);
             }
         }
     }
@@ -805,6 +830,19 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
+}
+
+// Self-test of the failure path: one thread waits, with a short limit, on an
+// mbarrier that nothing arrives at.  The bounded wait gives up, records
+// FLAREPP_ERR_TIMEOUT in the device status word and the kernel returns.
+__global__ void wait_timeout_selftest(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(&bar, 0, &abort_flag, limit_ns);
 }
 
 // ------------------------------------------------------------------ host side

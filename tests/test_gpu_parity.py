@@ -230,3 +230,18 @@ def test_invalid_args_on_gpu():
     with pytest.raises(b.FlareppError) as e:       # fp32 I/O has no tensor-core path
         b.mixer_fwd(xf["q0"], xf["q_fixed"], xf["gate"], xf["k0"], xf["k"], xf["v"], path=b.PATH_TCGEN05)
     assert e.value.status == 2
+
+
+def test_bounded_wait_reports_timeout():
+    """A wait that nothing satisfies gives up within its limit, records
+    FLAREPP_ERR_TIMEOUT in the device status word, and leaves the context
+    usable: the next forward runs and matches the oracle."""
+    b = binding()
+    assert b.check_device_status() == 0
+    assert b.selftest_wait_timeout(20000) == 0          # 20 ms limit
+    assert b.check_device_status() == 5                 # FLAREPP_ERR_TIMEOUT, then cleared
+    assert b.check_device_status() == 0
+    x = W.random_inputs(1, 2, 700, 64, 32, dtype="bf16", seed=31)
+    y_ref, _, _ = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+    y, _, _ = run(x)
+    assert_parity(y, y_ref, "bf16")
