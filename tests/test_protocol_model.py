@@ -1,0 +1,37 @@
+"""The attention kernel's mbarrier protocol, modelled on the CPU (see
+protocol_model.py), over shapes that exercise ragged tiles, one-tile and
+jobless items, interleaved and shared stage rings, and forced chunk counts,
+for both kernel configurations (two warpgroups on 128-row tiles for the
+split passes, three on 64-row tiles for the decode)."""
+import pytest
+
+from protocol_model import check
+
+SHAPES = [(1, 2, 1024, 16, 16), (1, 1, 1, 1, 16), (1, 2, 7, 5, 16), (2, 1, 129, 17, 32),
+          (1, 3, 300, 64, 64), (3, 2, 513, 64, 16), (1, 1, 4097, 256, 32), (1, 2, 2000, 512, 64),
+          (1, 1, 640, 100, 32), (1, 2, 1500, 384, 64)]
+
+
+@pytest.mark.parametrize("nw", [2, 3])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_protocol(shape, nw):
+    check(*shape, NW=nw, grid=37)
+
+
+@pytest.mark.parametrize("nw", [2, 3])
+@pytest.mark.parametrize("force", [1, 2, 7])
+def test_protocol_forced_chunks(nw, force):
+    check(2, 2, 3001, 128, 32, force_chunks=force, NW=nw, grid=37)
+
+
+def test_per_warpgroup_rings_on_the_16641_token_workload():
+    check(2, 8, 16641, 128, 32, NW=3, grid=148, mode="split")
+    check(2, 8, 16641, 128, 32, NW=2, grid=148, mode="split")
+
+
+def test_model_catches_the_shared_ring_race():
+    """With one shared stage ring in interleaved mode, consecutive fills of a
+    stage can belong to different warpgroups and a parity wait can pass on the
+    wrong fill; the model must see a stage holding the wrong tile."""
+    with pytest.raises(AssertionError, match="kv stage holds wrong tile"):
+        check(2, 8, 16641, 128, 32, NW=3, grid=148, mode="split", shared_ring=True)
