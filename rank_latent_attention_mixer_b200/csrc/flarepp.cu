@@ -102,7 +102,8 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
         chunks = (target + s.bh() * units_per_bh - 1) / (s.bh() * units_per_bh);
         chunks = std::max<int64_t>(1, std::min<int64_t>(chunks, tiles));
     } else {
-        chunks = tc::choose_chunks(s.bh() * units_per_bh, tiles, kNumSMs);
+        chunks = tc::choose_chunks(s.bh() * units_per_bh, tiles, kNumSMs,
+                                   tc::interleaved(s.M) ? tc::kSplitNW : 1);
     }
     int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
     pl->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);

@@ -895,15 +895,27 @@ inline int row_groups(int M) {
 }
 inline int parts_per_chunk(int M) { return interleaved(M) ? kSplitNW : 1; }
 
-// Token chunks per (b, h): at least `min_items` items in all, preferring a
-// count that makes the items a whole number of waves over the SMs.
-inline int64_t choose_chunks(int64_t units, int64_t tiles, int sms) {
-    const int64_t min_items = 4LL * sms;
-    int64_t c0 = (min_items + units - 1) / units;
-    c0 = std::max<int64_t>(1, std::min<int64_t>(c0, tiles));
-    for (int64_t c = c0; c <= std::min<int64_t>(tiles, 4 * c0); ++c)
-        if ((units * c) % sms == 0) return c;
-    return c0;
+// Token chunks per (b, h) for the split passes.  With `units` items per
+// chunk count step ((b, h) x latent groups) and `tiles` key/value tiles per
+// (b, h), c chunks give units*c items in ceil(units*c / sms) waves, each item
+// holding ceil(tiles / c) tiles, i.e. that many jobs per warpgroup (divided by
+// the warpgroup count when interleaved).  An item costs about two jobs of
+// fixed work (query load, first-tile max, epilogue), so the time is about
+// waves * (2 + jobs per item); take the cheapest c (the largest on ties).
+inline int64_t choose_chunks(int64_t units, int64_t tiles, int sms, int jobs_div) {
+    int64_t best_c = 1;
+    double best = 1e300;
+    for (int64_t c = 1; c <= tiles; ++c) {
+        const int64_t per = (tiles + c - 1) / c;
+        if (c > 1 && (tiles + per - 1) / per < c) continue;          // same split as a smaller c
+        const int64_t waves = (units * c + sms - 1) / sms;
+        const double cost = (double)waves * (2.0 + (double)((per + jobs_div - 1) / jobs_div));
+        if (cost <= best) {
+            best = cost;
+            best_c = c;
+        }
+    }
+    return best_c;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -287,12 +287,17 @@ def simulate(p, grid, NST, QS, seed):
         events.sort(key=lambda e: e[0]); events.pop(0)[1]()
 
 
-def choose_chunks(units, tiles, sms=148):
-    c0 = max(1, min(-(-4 * sms // units), tiles))
-    for c in range(c0, min(tiles, 4 * c0) + 1):
-        if (units * c) % sms == 0:
-            return c
-    return c0
+def choose_chunks(units, tiles, sms=148, jobs_div=1):
+    # Same cost model as the host planner: waves * (2 + jobs per item).
+    best_c, best = 1, float("inf")
+    for c in range(1, tiles + 1):
+        per = -(-tiles // c)
+        if c > 1 and -(-tiles // per) < c:
+            continue
+        cost = -(-units * c // sms) * (2 + -(-per // jobs_div))
+        if cost <= best:
+            best, best_c = cost, c
+    return best_c
 
 
 def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, shared_ring=False):
@@ -301,7 +306,7 @@ def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, sh
     kv_tiles = (N + KT - 1) // KT
     inter = NW == 3 or M <= 128
     rg = (M + 127) // 128 if inter else (M + NW * 128 - 1) // (NW * 128)
-    chunks = force_chunks or choose_chunks(BH * rg, kv_tiles)
+    chunks = force_chunks or choose_chunks(BH * rg, kv_tiles, jobs_div=NW if inter else 1)
     chunks = min(chunks, kv_tiles)
     tpc = -(-kv_tiles // chunks)
     chunks = -(-kv_tiles // tpc)

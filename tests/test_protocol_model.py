@@ -32,6 +32,8 @@ def test_per_warpgroup_rings_on_the_16641_token_workload():
 def test_model_catches_the_shared_ring_race():
     """With one shared stage ring in interleaved mode, consecutive fills of a
     stage can belong to different warpgroups and a parity wait can pass on the
-    wrong fill; the model must see a stage holding the wrong tile."""
+    wrong fill; the model must see a stage holding the wrong tile.  The chunk
+    count is pinned to 37 (592 items of 8 tiles), a split in which the model
+    interleaves the warpgroups closely enough to show the race."""
     with pytest.raises(AssertionError, match="kv stage holds wrong tile"):
-        check(2, 8, 16641, 128, 32, NW=3, grid=148, mode="split", shared_ring=True)
+        check(2, 8, 16641, 128, 32, NW=3, grid=148, mode="split", shared_ring=True, force_chunks=37)
