@@ -20,7 +20,9 @@
  *     entry), row-major and contiguous, 16-byte aligned:
  *       q0, q_fixed   [H, M, D]     shared by every batch element
  *       k0, k, v, y   [B, H, N, D]
- *     in the I/O dtype (FLAREPP_F32 = fp32, FLAREPP_BF16 = bf16).
+ *     in the I/O dtype (FLAREPP_F32 = fp32, FLAREPP_BF16 = bf16, FLAREPP_F16 =
+ *     fp16; the last for the fp16 forward that physicsnemo issue #1150, the
+ *     author's reply, "3. Scaling to 1 M points", calls essential at 1M points).
  *   - gate: DEVICE float[H], the gate value sigmoid(g) per head (never the
  *     logit; the library applies no sigmoid).  gate == NULL closes the gate:
  *     the synthesis is skipped and the result is FLARE with q = q_fixed
@@ -30,9 +32,12 @@
  *   - stream is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Every call is asynchronous on it except the *_host entry and
  *     flarepp_check_device_status, which synchronise the stream.
- *   - Accumulation is fp32 for both dtypes.  bf16 I/O rounds q, z and the
- *     softmax weights to bf16 where they feed the tensor cores; y is rounded
- *     to the I/O dtype once, at the end.
+ *   - Accumulation is fp32 for every dtype.  16-bit I/O (bf16 or fp16) rounds
+ *     q, z and the softmax weights to the I/O dtype where they feed the tensor
+ *     cores; y is rounded to the I/O dtype once, at the end.  With fp16 the
+ *     weights are taken relative to (running row max - 7 log2 units), so they
+ *     stay below 2^15 (fp16's largest finite value is 65504); weights below
+ *     about 2^-31 of the row's largest round to zero.
  *
  * Errors: every entry returns a flarepp_status_t and never throws or aborts.
  * Arguments are checked before any CUDA call or launch; a failed check
@@ -58,7 +63,8 @@ extern "C" {
 
 typedef enum flarepp_dtype {
     FLAREPP_F32 = 0,
-    FLAREPP_BF16 = 1
+    FLAREPP_BF16 = 1,
+    FLAREPP_F16 = 2
 } flarepp_dtype_t;
 
 typedef enum flarepp_status {
@@ -70,9 +76,9 @@ typedef enum flarepp_status {
     FLAREPP_ERR_TIMEOUT = 5        /* a kernel's bounded wait ran out (device status word) */
 } flarepp_status_t;
 
-/* Kernel family.  AUTO picks the tcgen05 tensor-core kernels for bf16 with
- * D in {16,32,64} and the SIMT (FFMA) kernels otherwise (all fp32 I/O: TF32
- * products would not meet fp32 accuracy). */
+/* Kernel family.  AUTO picks the tcgen05 tensor-core kernels for 16-bit I/O
+ * (bf16 or fp16) with D in {16,32,64} and the SIMT (FFMA) kernels otherwise
+ * (all fp32 I/O: TF32 products would not meet fp32 accuracy). */
 typedef enum flarepp_path {
     FLAREPP_PATH_AUTO = 0,
     FLAREPP_PATH_SIMT = 1,
@@ -119,7 +125,7 @@ int flarepp_mixer_fwd_ex(const void* q0, const void* q_fixed, const float* gate,
                          const flarepp_options_t* opts, void* stream);
 
 /* Bytes of device scratch one call needs (partial softmax triples per token
- * chunk, and q, z in fp32 and bf16).  gated = 0 for the closed-gate form.
+ * chunk, and q, z in fp32 and in the 16-bit I/O dtype).  gated = 0 for the closed-gate form.
  * Returns 0 for arguments the forward entries would reject. */
 size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
                                const flarepp_options_t* opts);

@@ -16,7 +16,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libflarepp.so")
 
-F32, BF16 = 0, 1
+F32, BF16, F16 = 0, 1, 2
 PATH_AUTO, PATH_SIMT, PATH_TCGEN05 = 0, 1, 2
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
           4: "ERR_WORKSPACE", 5: "ERR_TIMEOUT"}
@@ -76,7 +76,9 @@ def _dtype_code(t: torch.Tensor) -> int:
         return F32
     if t.dtype == torch.bfloat16:
         return BF16
-    raise TypeError(f"unsupported dtype {t.dtype}; the mixer takes float32 or bfloat16")
+    if t.dtype == torch.float16:
+        return F16
+    raise TypeError(f"unsupported dtype {t.dtype}; the mixer takes float32, bfloat16 or float16")
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

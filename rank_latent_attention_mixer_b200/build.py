@@ -45,7 +45,7 @@ def _stale() -> bool:
 
 
 def expected_launch_regs(kernel_name: str) -> int:
-    m = re.search(r"attn_kernelILi(\d+)ELi(\d+)ELi(\d+)E", kernel_name)
+    m = re.search(r"attn_kernelI\d+\w+?Li(\d+)ELi(\d+)ELi(\d+)E", kernel_name)
     if not m:
         raise RuntimeError(f"cannot read the warpgroup count from {kernel_name}")
     nw = int(m.group(2))

@@ -3,7 +3,10 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 namespace flarepp {
 
@@ -25,10 +28,34 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
     return __bfloat162float(x);
 }
 
+template <> __device__ __forceinline__ float to_f32<__half>(__half x) { return __half2float(x); }
+
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+
+// Two fp32 values rounded to nearest even into a packed pair of the 16-bit
+// type T (bf16 or fp16), `lo` in the low half.
+template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The packed pair of 16-bit values in `w` as two fp32 values (exact).
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t w);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
 // 2^x on the MUFU unit (PTX ex2.approx, flush-to-zero).
@@ -57,14 +84,15 @@ __device__ __forceinline__ void load_row_f32(const T* __restrict__ src, float (&
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                dst[8 * i + 2 * j + 0] = __uint_as_float(w[j] << 16);
-                dst[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+                const float2 f = unpack2<T>(w[j]);
+                dst[8 * i + 2 * j + 0] = f.x;
+                dst[8 * i + 2 * j + 1] = f.y;
             }
         }
     }
 }
 
-// Store `D` fp32 registers as type T (round to nearest even for bf16).
+// Store `D` fp32 registers as type T (round to nearest even for 16-bit types).
 template <typename T, int D>
 __device__ __forceinline__ void store_row(T* __restrict__ dst, const float (&src)[D]) {
     if constexpr (sizeof(T) == 4) {
@@ -78,10 +106,7 @@ __device__ __forceinline__ void store_row(T* __restrict__ dst, const float (&src
         for (int i = 0; i < D / 8; ++i) {
             uint32_t w[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 p = __floats2bfloat162_rn(src[8 * i + 2 * j], src[8 * i + 2 * j + 1]);
-                w[j] = *reinterpret_cast<uint32_t*>(&p);
-            }
+            for (int j = 0; j < 4; ++j) w[j] = pack2<T>(src[8 * i + 2 * j], src[8 * i + 2 * j + 1]);
             d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }

@@ -4,9 +4,9 @@
 //
 // Launch sequence for one call (gate open):
 //   1. split partial   Q = q0 [H,M,D],  K = V = k0     (synthesis, V = K)
-//   2. merge           q = q_fixed + gate * q_dyn       -> q fp32 + bf16
+//   2. merge           q = q_fixed + gate * q_dyn       -> q fp32 + I/O dtype
 //   3. split partial   Q = q,           K = k, V = v    (encode)
-//   4. merge           z                                -> z fp32 + bf16
+//   4. merge           z                                -> z fp32 + I/O dtype
 //   5. decode          y = SDPA(k, q, z)
 // With the gate closed, steps 1-2 are skipped and q_fixed is used as q.
 #include <algorithm>
@@ -51,7 +51,7 @@ struct Plan {
 
 int check_shape(const Shape& s) {
     if (s.B < 1 || s.H < 1 || s.N < 1 || s.M < 1) return FLAREPP_ERR_INVALID_ARG;
-    if (s.dtype != FLAREPP_F32 && s.dtype != FLAREPP_BF16) return FLAREPP_ERR_INVALID_ARG;
+    if (s.dtype != FLAREPP_F32 && s.dtype != FLAREPP_BF16 && s.dtype != FLAREPP_F16) return FLAREPP_ERR_INVALID_ARG;
     if (s.bh() > 65535 || s.M > 4096) return FLAREPP_ERR_UNSUPPORTED;
     if (s.D != 16 && s.D != 32 && s.D != 64 && s.D != 128) return FLAREPP_ERR_UNSUPPORTED;
     return FLAREPP_OK;
@@ -59,7 +59,7 @@ int check_shape(const Shape& s) {
 
 int tile_tokens_simt(int D) { return 2048 / D; }
 
-bool tc_supported(const Shape& s) { return tc::supported(s.dtype == FLAREPP_BF16, s.D, s.M); }
+bool tc_supported(const Shape& s) { return tc::supported(s.dtype != FLAREPP_F32, s.D, s.M); }
 
 int choose_path(const Shape& s, int requested) {
     if (requested == FLAREPP_PATH_SIMT) return FLAREPP_PATH_SIMT;
@@ -115,9 +115,9 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     pl->off_part_O = off;  off = align_up(off + (size_t)parts * rows * s.D * sizeof(float));
     pl->off_part_ml = off; off = align_up(off + (size_t)parts * rows * sizeof(float2));
     pl->off_q32 = off;     off = align_up(off + rows * s.D * sizeof(float));
-    pl->off_q16 = off;     off = align_up(off + rows * s.D * sizeof(__nv_bfloat16));
+    pl->off_q16 = off;     off = align_up(off + rows * s.D * sizeof(uint16_t));     // q in the 16-bit I/O dtype
     pl->off_z32 = off;     off = align_up(off + rows * s.D * sizeof(float));
-    pl->off_z16 = off;     off = align_up(off + rows * s.D * sizeof(__nv_bfloat16));
+    pl->off_z16 = off;     off = align_up(off + rows * s.D * sizeof(uint16_t));
     pl->total = off;
     return FLAREPP_OK;
 }
@@ -164,9 +164,9 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
     float* part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
     float2* part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
     float* q32 = reinterpret_cast<float*>(ws + pl.off_q32);
-    __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_q16);
+    void* q16 = ws + pl.off_q16;
     float* z32 = reinterpret_cast<float*>(ws + pl.off_z32);
-    __nv_bfloat16* z16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_z16);
+    void* z16 = ws + pl.off_z16;
 
     const dim3 split_grid(pl.chunks, (unsigned)s.bh(), pl.row_blocks);
     const int64_t rows = s.bh() * s.M;
@@ -191,7 +191,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
             sp.Q = q0; sp.q_batch_heads = 0; sp.K = k0; sp.V = k0;                                 \
             split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
             ev.mark(st);                                                                           \
-            mp.mode = kMergeSynthesis; mp.out_f32 = q32; mp.out_bf16 = q16; mp.user_out = q_out;   \
+            mp.mode = kMergeSynthesis; mp.out_f32 = q32; mp.out_16 = q16; mp.user_out = q_out;   \
             mp.q_copy_out = nullptr;                                                               \
             merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                 \
             ev.mark(st);                                                                           \
@@ -203,7 +203,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
             split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
             ev.mark(st);                                                                           \
         }                                                                                          \
-        mp.mode = kMergeEncode; mp.out_f32 = z32; mp.out_bf16 = z16; mp.user_out = z_out;          \
+        mp.mode = kMergeEncode; mp.out_f32 = z32; mp.out_16 = z16; mp.user_out = z_out;          \
         mp.q_copy_out = gated ? nullptr : q_out;                                                   \
         merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                     \
         ev.mark(st);                                                                               \
@@ -238,17 +238,21 @@ int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, con
         bu.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
         bu.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
         bu.q32 = reinterpret_cast<float*>(ws + pl.off_q32);
-        bu.q16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_q16);
+        bu.q16 = ws + pl.off_q16;
         bu.z32 = reinterpret_cast<float*>(ws + pl.off_z32);
-        bu.z16 = reinterpret_cast<__nv_bfloat16*>(ws + pl.off_z16);
+        bu.z16 = ws + pl.off_z16;
         tc::Problem pr{};
         pr.B = s.B; pr.H = s.H; pr.N = s.N; pr.M = s.M; pr.D = s.D;
         pr.chunks = pl.chunks; pr.chunk_len = pl.chunk_len; pr.scale_log2 = pl.scale_log2;
-        return tc::run(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out,
-                       [&ev](cudaStream_t t) { ev.mark(t); }, st);
+        auto mark = [&ev](cudaStream_t t) { ev.mark(t); };
+        if (s.dtype == FLAREPP_F16)
+            return tc::run<__half>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st);
+        return tc::run<__nv_bfloat16>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st);
     }
     if (s.dtype == FLAREPP_F32)
         return run_simt<float>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+    if (s.dtype == FLAREPP_F16)
+        return run_simt<__half>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
     return run_simt<__nv_bfloat16>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
 }
 

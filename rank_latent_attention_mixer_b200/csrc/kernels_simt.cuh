@@ -131,7 +131,7 @@ struct MergeParams {
     const void* q_fixed;        // [H,M,D] in the I/O dtype (synthesis epilogue, or copied to q_copy_out)
     const float* gate;          // [H] (synthesis epilogue)
     float* out_f32;             // [B,H,M,D]
-    __nv_bfloat16* out_bf16;    // [B,H,M,D]
+    void* out_16;               // [B,H,M,D] in the I/O dtype (16-bit I/O only; may be null)
     float* user_out;            // optional [B,H,M,D]
     float* q_copy_out;          // optional: closed gate, write q = q_fixed broadcast over b
 };
@@ -203,7 +203,9 @@ merge_partials(MergeParams p) {
             const int d = d0 + e;
             if (p.mode == kMergeSynthesis) val[e] = fmaf(p.gate[h], val[e], to_f32<T>(qf[d]));
             p.out_f32[row * D + d] = val[e];
-            p.out_bf16[row * D + d] = __float2bfloat16_rn(val[e]);
+            if constexpr (sizeof(T) == 2) {
+                if (p.out_16) reinterpret_cast<T*>(p.out_16)[row * D + d] = from_f32<T>(val[e]);
+            }
             if (p.user_out) p.user_out[row * D + d] = val[e];
             if (p.q_copy_out) p.q_copy_out[row * D + d] = to_f32<T>(qf[d]);
         }

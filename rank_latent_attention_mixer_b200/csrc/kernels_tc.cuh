@@ -1,4 +1,5 @@
-// tcgen05 (5th-generation tensor core) kernels of the FLARE++ mixer, bf16 I/O.
+// tcgen05 (5th-generation tensor core) kernels of the FLARE++ mixer, 16-bit
+// I/O (bf16 or fp16; the element type E is a template parameter throughout).
 //
 // One warp-specialised attention kernel serves all three SDPA calls of the
 // FLARE++ block (FLARE.py README, "FLARE++" code block):
@@ -11,7 +12,7 @@
 //                    combine; physicsnemo issue #2024, section 2);
 //   * decode mode -- y = SDPA(k, q, z): the query rows are tokens, the
 //                    key/value rows are the M latents of q and z, and the
-//                    output is the normalised y row in bf16.
+//                    output is the normalised y row in E.
 //
 // Per CTA (persistent, one per SM): NW softmax warpgroups and one producer
 // warpgroup, (NW + 1) x 128 threads.
@@ -22,9 +23,9 @@
 //   warps 4NW+1 ..     one MMA issuer per softmax warpgroup w:
 //                      S_w = Q_w K^T and O_w += P_w V, into TMEM
 // TMEM columns: S_w at KT w, O_w at NW KT + OS w (OS = max(D, 32)), P_w (KT
-// bf16 = KT/2 columns) after them; NW (KT + OS + KT/2) <= 512.
+// 16-bit values = KT/2 columns) after them; NW (KT + OS + KT/2) <= 512.
 // Each softmax thread owns one query row: it reads its KT scores from TMEM,
-// takes exponentials base 2, writes the bf16 weights P back to TMEM (the value
+// takes exponentials base 2, writes the weights P back to TMEM in E (the value
 // MMA reads its A operand from TMEM), and rescales its O row in TMEM only when
 // its running max grows by more than 2^8 (the final normalisation uses the
 // same stale max, so the result is exact up to rounding).  Each MMA warp
@@ -151,8 +152,8 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulation.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit inputs (the type is in idesc), fp32 accumulation.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -162,8 +163,8 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x K bf16, K-major) read from TMEM.
-__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x K 16-bit, K-major) read from TMEM.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                                  uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -219,12 +220,29 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, bf16 A
-// and B, A K-major, B K-major or MN-major, shape M x N.
-__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, A and B
+// both of the type `fmt` (0 = fp16, 1 = bf16; never mixed), A K-major, B
+// K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool b_mn_major, uint32_t fmt) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+
+// The 16-bit I/O element types.  kFmt: operand format of kind::f16.  kPBias:
+// the exponentials are taken against (running max - kPBias), so the weights P
+// lie below 2^(kPBias + 8): fp16 (largest finite 65504) gains 7 binades at
+// the small end (values below 2^-24 flush to zero there), bf16 needs none.
+template <typename E> struct Elem;
+template <> struct Elem<__nv_bfloat16> {
+    static constexpr uint32_t kFmt = 1;
+    static constexpr float kPBias = 0.f;
+    static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+template <> struct Elem<__half> {
+    static constexpr uint32_t kFmt = 0;
+    static constexpr float kPBias = 7.f;
+    static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+};
 
 // 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit.
 // Range reduction: n = round(x) by adding 1.5 * 2^23 (the addition rounds x
@@ -264,10 +282,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // ------------------------------------------------------------------ kernel parameters
 
@@ -291,7 +305,7 @@ struct Params {
     float scale_log2;
     float* part_O;        // split: [parts][B*H][M][D]
     float2* part_ml;      // split: [parts][B*H][M]
-    __nv_bfloat16* y;     // decode: [B,H,N,D]
+    void* y;              // decode: [B,H,N,D] in E
 };
 
 struct Item {
@@ -346,7 +360,7 @@ struct Smem {
 
 template <int D, int NW, int KT>
 struct Layout {
-    // swizzle of a [rows x D] bf16 tile whose rows are D*2 bytes
+    // swizzle of a [rows x D] 16-bit tile whose rows are D*2 bytes
     static constexpr uint32_t kType = D == 64 ? kLayoutSw128 : (D == 32 ? kLayoutSw64 : kLayoutSw32);
     static constexpr uint32_t kRowBytes = D * 2;
     static constexpr uint32_t kSbo = 8 * kRowBytes;                  // 8-row group stride
@@ -363,7 +377,7 @@ struct Layout {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int D, int NW, int KT, int NST, int QS>
+template <typename E, int D, int NW, int KT, int NST, int QS>
 __global__ void __launch_bounds__(Regs<NW>::kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const Params p) {
@@ -497,8 +511,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         // pipelines never wait on each other's softmax.
         if (lane == 0) {
             const int w = warp - kMmaWarp0;
-            constexpr uint32_t idesc_s = make_idesc(kQTile, KT, false);   // S = Q K^T: [128 q x KT kv]
-            constexpr uint32_t idesc_o = make_idesc(kQTile, D, true);     // O += P V:  [128 q x D], V MN-major
+            constexpr uint32_t idesc_s = make_idesc(kQTile, KT, false, Elem<E>::kFmt);   // S = Q K^T: [128 q x KT kv]
+            constexpr uint32_t idesc_o = make_idesc(kQTile, D, true, Elem<E>::kFmt);     // O += P V: [128 q x D], V MN-major
             const int tstep = p.interleave ? NW : 1;
             const int tfirst = p.interleave ? w : 0;
             // This warpgroup's jobs: the key/value tiles it consumes, item by item.
@@ -578,7 +592,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = smem_desc(qaddr + kk * 32, 16, LY::kSbo, LY::kType);
                     const uint64_t bd = smem_desc(kaddr + kk * 32, 16, LY::kSbo, LY::kType);
-                    umma_bf16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_f16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sfull[w]);
                 ++s_issued;
@@ -598,12 +612,12 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const uint32_t p_tmem = tmem + LY::kPCol + w * (KT / 2);
 #pragma unroll
                 for (int kk = 0; kk < KT / 16; ++kk) {
-                    // A = P in TMEM: 16 key/value columns = 8 packed bf16x2 columns per step
+                    // A = P in TMEM: 16 key/value columns = 8 columns of packed pairs per step
                     // B = V tile [KT kv x D], D contiguous: MN-major; 16 kv rows per step
                     // (D fits one swizzle atom along MN, so the leading offset is never used)
                     const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kKVTileBytes,
                                                   LY::kSbo, LY::kType);
-                    umma_bf16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
+                    umma_f16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
                 }
                 umma_commit(&pfree[w]);
                 ++pv_issued;
@@ -670,15 +684,15 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const int n = it.qrow0 + wg * kQTile + row;
                 if (n < p.N && o) {
                     const float inv = 1.f / l;
-                    uint4* dst = reinterpret_cast<uint4*>(p.y + ((int64_t)it.bh * p.N + n) * D);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + ((int64_t)it.bh * p.N + n) * D);
 #pragma unroll
                     for (int i = 0; i < D / 8; ++i) {
                         const int c = i / 4, j = (i % 4) * 8;
                         dst[i] = make_uint4(
-                            pack_bf16x2(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
-                            pack_bf16x2(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                            pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
                     }
                 }
             }
@@ -735,7 +749,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 float mx = mc[0];
 #pragma unroll
                 for (int c = 1; c < LY::kChunks; ++c) mx = fmaxf(mx, mc[c]);
-                const float m_new = fmaxf(m_run, mx * sl2);
+                const float m_new = fmaxf(m_run, mx * sl2 - Elem<E>::kPBias);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
                 if (resc) {
@@ -758,7 +772,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                                               ? ex2_fma_pair(xv)
                                               : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
-                        pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(pv.x, pv.y);
+                        pk[c >> 1][(c & 1) * 16 + j] = pack2<E>(pv.x, pv.y);
                     }
                 }
                 float2 asum = acc[0];
@@ -789,7 +803,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         tmem_st32(tO + c * 32, o);
                     }
                 }
-                // P row -> TMEM (this thread's lane, KT/2 columns of bf16 pairs)
+                // P row -> TMEM (this thread's lane, KT/2 columns of packed pairs)
 #pragma unroll
                 for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
                 tmem_wait_st();
@@ -851,9 +865,9 @@ struct Buffers {
     float* part_O;
     float2* part_ml;
     float* q32;
-    __nv_bfloat16* q16;
+    void* q16;            // q in E: the MMA operand
     float* z32;
-    __nv_bfloat16* z16;
+    void* z16;            // z in E
 };
 
 struct Problem {
@@ -880,9 +894,9 @@ struct Config {
 constexpr int kSplitNW = 2, kSplitKT = 128;
 constexpr int kDecodeNW = 3, kDecodeKT = 64;
 
-inline bool supported(bool bf16, int D, int M) {
+inline bool supported(bool io16, int D, int M) {
     (void)M;
-    return bf16 && (D == 16 || D == 32 || D == 64);
+    return io16 && (D == 16 || D == 32 || D == 64);
 }
 
 // Split-pass plan.  With one 128-row tile holding all M latents, the two
@@ -935,8 +949,9 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D map over a [planes, rows, D] bf16 tensor, box [1, box_rows, D], swizzle = D*2 bytes.
-inline bool make_map(CUtensorMap* map, const void* base, int planes, int rows, int D, int box_rows) {
+// 3-D map over a [planes, rows, D] tensor of 16-bit elements, box [1, box_rows, D], swizzle = D*2 bytes.
+inline bool make_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int planes, int rows, int D,
+                     int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
@@ -945,7 +960,7 @@ inline bool make_map(CUtensorMap* map, const void* base, int planes, int rows, i
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                           : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -956,11 +971,11 @@ inline int sm_count() {
     return n > 0 ? n : kNumSMs;
 }
 
-template <int D, int NW, int KT>
+template <typename E, int D, int NW, int KT>
 int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& prm,
                 cudaStream_t st) {
     using C = Config<D, NW, KT>;
-    auto kern = attn_kernel<D, C::NW, C::KT, C::NST, C::QS>;
+    auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS>;
     static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
         return 3;
@@ -969,33 +984,34 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
-template <int NW, int KT>
+template <typename E, int NW, int KT>
 inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const Params& prm, cudaStream_t st) {
     switch (D) {
-        case 16: return launch_attn<16, NW, KT>(mq, mk, mv, prm, st);
-        case 32: return launch_attn<32, NW, KT>(mq, mk, mv, prm, st);
-        case 64: return launch_attn<64, NW, KT>(mq, mk, mv, prm, st);
+        case 16: return launch_attn<E, 16, NW, KT>(mq, mk, mv, prm, st);
+        case 32: return launch_attn<E, 32, NW, KT>(mq, mk, mv, prm, st);
+        case 64: return launch_attn<E, 64, NW, KT>(mq, mk, mv, prm, st);
         default: return 2;
     }
 }
 
-template <int D>
+template <typename E, int D>
 void launch_merge(const MergeParams& mp, int64_t rows, cudaStream_t st) {
-    merge_partials<__nv_bfloat16, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
+    merge_partials<E, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
 }
 
+template <typename E>
 inline void launch_merge_d(int D, const MergeParams& mp, int64_t rows, cudaStream_t st) {
     switch (D) {
-        case 16: launch_merge<16>(mp, rows, st); break;
-        case 32: launch_merge<32>(mp, rows, st); break;
-        default: launch_merge<64>(mp, rows, st); break;
+        case 16: launch_merge<E, 16>(mp, rows, st); break;
+        case 32: launch_merge<E, 32>(mp, rows, st); break;
+        default: launch_merge<E, 64>(mp, rows, st); break;
     }
 }
 
 // The whole FLARE++ forward on the tcgen05 path; `mark(stream)` is called
 // before the first launch and after each launch.
-template <typename Mark>
+template <typename E, typename Mark>
 int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixed, const float* gate,
         const void* k0, const void* k, const void* v, void* y, float* q_out, float* z_out, Mark&& mark,
         cudaStream_t st) {
@@ -1004,11 +1020,13 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     // query maps use 128-row boxes, key/value maps the pass's tile height; the
     // token keys k serve as key/value tiles (split) and as query tiles (decode)
     CUtensorMap m_q0, m_qf_q, m_qf_kv, m_q16_q, m_q16_kv, m_z16, m_k0, m_k_kv, m_k_q, m_v;
-    bool ok = make_map(&m_qf_q, q_fixed, H, M, D, kQTile) && make_map(&m_qf_kv, q_fixed, H, M, D, kDecodeKT) &&
-              make_map(&m_q16_q, bu.q16, BH, M, D, kQTile) && make_map(&m_q16_kv, bu.q16, BH, M, D, kDecodeKT) &&
-              make_map(&m_z16, bu.z16, BH, M, D, kDecodeKT) && make_map(&m_k_kv, k, BH, N, D, kSplitKT) &&
-              make_map(&m_k_q, k, BH, N, D, kQTile) && make_map(&m_v, v, BH, N, D, kSplitKT);
-    if (gated) ok = ok && make_map(&m_q0, q0, H, M, D, kQTile) && make_map(&m_k0, k0, BH, N, D, kSplitKT);
+    const CUtensorMapDataType ty = Elem<E>::kMapType;
+    bool ok = make_map(&m_qf_q, ty, q_fixed, H, M, D, kQTile) && make_map(&m_qf_kv, ty, q_fixed, H, M, D, kDecodeKT) &&
+              make_map(&m_q16_q, ty, bu.q16, BH, M, D, kQTile) && make_map(&m_q16_kv, ty, bu.q16, BH, M, D, kDecodeKT) &&
+              make_map(&m_z16, ty, bu.z16, BH, M, D, kDecodeKT) && make_map(&m_k_kv, ty, k, BH, N, D, kSplitKT) &&
+              make_map(&m_k_q, ty, k, BH, N, D, kQTile) && make_map(&m_v, ty, v, BH, N, D, kSplitKT);
+    if (gated)
+        ok = ok && make_map(&m_q0, ty, q0, H, M, D, kQTile) && make_map(&m_k0, ty, k0, BH, N, D, kSplitKT);
     if (!ok) return 3;
 
     const int kv_tiles = (N + kSplitKT - 1) / kSplitKT;
@@ -1037,22 +1055,22 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     if (gated) {
         Params s1 = sp;
         s1.q_shared = 1; s1.k_shared = 0; s1.kv_same = 1;
-        rc = launch_attn_d<kSplitNW, kSplitKT>(D, m_q0, m_k0, m_k0, s1, st);
+        rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, m_q0, m_k0, m_k0, s1, st);
         if (rc) return rc;
         mark(st);
-        mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_bf16 = bu.q16; mp.user_out = q_out;
+        mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_16 = bu.q16; mp.user_out = q_out;
         mp.q_copy_out = nullptr;
-        launch_merge_d(D, mp, rows, st);
+        launch_merge_d<E>(D, mp, rows, st);
         mark(st);
     }
     Params s2 = sp;
     s2.q_shared = gated ? 0 : 1; s2.k_shared = 0; s2.kv_same = 0;
-    rc = launch_attn_d<kSplitNW, kSplitKT>(D, gated ? m_q16_q : m_qf_q, m_k_kv, m_v, s2, st);
+    rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, gated ? m_q16_q : m_qf_q, m_k_kv, m_v, s2, st);
     if (rc) return rc;
     mark(st);
-    mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_bf16 = bu.z16; mp.user_out = z_out;
+    mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_16 = bu.z16; mp.user_out = z_out;
     mp.q_copy_out = gated ? nullptr : q_out;
-    launch_merge_d(D, mp, rows, st);
+    launch_merge_d<E>(D, mp, rows, st);
     mark(st);
 
     Params dp{};
@@ -1064,8 +1082,8 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     dp.q_groups = (N + kDecodeNW * kQTile - 1) / (kDecodeNW * kQTile);
     dp.items = BH * dp.q_groups;
     dp.scale_log2 = pr.scale_log2;
-    dp.y = static_cast<__nv_bfloat16*>(y);
-    rc = launch_attn_d<kDecodeNW, kDecodeKT>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
+    dp.y = y;
+    rc = launch_attn_d<E, kDecodeNW, kDecodeKT>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
     if (rc) return rc;
     mark(st);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;

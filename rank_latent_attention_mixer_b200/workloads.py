@@ -48,7 +48,7 @@ class Workload:
     N: int
     M: int
     D: int
-    dtype: str          # "f32" or "bf16"
+    dtype: str          # "f32", "bf16" or "f16"
     seed: int
     recipe: str         # "iid", "peaky" or "clusters"
     rms_q0: bool
@@ -58,7 +58,7 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
-        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[self.dtype]
 
     @property
     def tokens(self) -> int:
@@ -81,6 +81,12 @@ WORKLOADS: Dict[str, Workload] = {
                  note="irregular point cloud, 32 key clusters, tokens randomly permuted"),
         Workload("scale1m_bf16", 1, 8, 1048576, 512, 64, "bf16", 4, "iid", True, True,
                  device_rng=True, note="1M-token scaling case, ~1 GiB per [B,H,N,D] tensor"),
+        # variants: the same draws rounded to fp16 (the fp16 forward of the
+        # 1M-point runs), and a small fp16 case for parity tests
+        Workload("scale1m_f16", 1, 8, 1048576, 512, 64, "f16", 4, "iid", True, True,
+                 device_rng=True, note="scale1m_bf16 with fp16 I/O"),
+        Workload("cloud40k_f16", 1, 8, 40000, 256, 32, "f16", 3, "clusters", False, False,
+                 note="cloud40k_bf16 with fp16 I/O"),
     ]
 }
 ORDER = ["tiny_f32", "grid85_bf16", "grid129_peaky_bf16", "cloud40k_bf16", "scale1m_bf16"]

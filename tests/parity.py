@@ -5,6 +5,10 @@ Tolerances of the FLARE++ mixer forward on B200:
              for every output row r (the D-vector of one token or latent),
              max_d |g - o| / max_d |o| <= 1e-4
   bf16 I/O : ||g - o||_2 / ||o||_2 <= 1e-2  and  max |g - o| <= 2e-2
+  fp16 I/O : ||g - o||_2 / ||o||_2 <= 2.5e-3 and  max |g - o| <= 5e-3
+             (the bf16 bounds scaled by 1/4: the errors come from rounding
+             q, z, the weights P and y to the 16-bit type, whose unit
+             roundoff is 8 times smaller in fp16; a factor 2 is kept as margin)
 An elementwise relative error is ill-conditioned here: z is a weighted mean of
 zero-mean values, so single entries cancel to near zero and fp32 rounding of
 the accumulation order alone gives them relative errors far above 1e-4.  The
@@ -16,6 +20,8 @@ import torch
 FP32_MAX_REL = 1e-4
 BF16_REL_L2 = 1e-2
 BF16_MAX_ABS = 2e-2
+F16_REL_L2 = 2.5e-3
+F16_MAX_ABS = 5e-3
 
 
 def to64(t):
@@ -47,6 +53,9 @@ def assert_parity(g, o, dtype: str, what: str = "y"):
     assert m["finite"], f"{what}: non-finite values"
     if dtype == "f32":
         assert m["row_max_rel"] <= FP32_MAX_REL, f"{what}: fp32 row max rel {m['row_max_rel']:.3e} > {FP32_MAX_REL} ({m})"
+    elif dtype == "f16":
+        assert m["rel_l2"] <= F16_REL_L2, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} > {F16_REL_L2} ({m})"
+        assert m["max_abs"] <= F16_MAX_ABS, f"{what}: fp16 max abs {m['max_abs']:.3e} > {F16_MAX_ABS} ({m})"
     else:
         assert m["rel_l2"] <= BF16_REL_L2, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} > {BF16_REL_L2} ({m})"
         assert m["max_abs"] <= BF16_MAX_ABS, f"{what}: bf16 max abs {m['max_abs']:.3e} > {BF16_MAX_ABS} ({m})"

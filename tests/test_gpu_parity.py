@@ -46,7 +46,7 @@ def run(x, path=0, force_chunks=0, flare=False, scale=0.0):
     return y, q, z
 
 
-SMALL = ["tiny_f32", "grid85_bf16", "grid129_peaky_bf16", "cloud40k_bf16"]
+SMALL = ["tiny_f32", "grid85_bf16", "grid129_peaky_bf16", "cloud40k_bf16", "cloud40k_f16"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -62,7 +62,7 @@ def test_workload_parity(name, path):
     print(name, path, m)
 
 
-@pytest.mark.parametrize("name", ["grid85_bf16", "tiny_f32"])
+@pytest.mark.parametrize("name", ["grid85_bf16", "tiny_f32", "cloud40k_f16"])
 def test_closed_gate_is_flare(name):
     w = W.WORKLOADS[name]
     x = W.make_inputs(w)
@@ -93,7 +93,7 @@ EDGE = [
 ]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("shape", EDGE, ids=lambda s: "x".join(map(str, s)))
 def test_edge_shapes(shape, dtype):
     B, H, N, M, D = shape
@@ -188,10 +188,11 @@ def test_permutation_equivariance_gpu():
     assert metrics(yp, y[:, :, perm.to(y.device)])["row_max_rel"] < 1e-4
 
 
-def test_scale1m_sampled():
+@pytest.mark.parametrize("name", ["scale1m_bf16", "scale1m_f16"])
+def test_scale1m_sampled(name):
     """The 1M-token workload in the launch configuration the benchmark times:
     one head checked in full for q and z, and 256 sampled tokens of y."""
-    w = W.WORKLOADS["scale1m_bf16"]
+    w = W.WORKLOADS[name]
     x = W.make_inputs(w, device=DEV)
     b = binding()
     y, q, z = b.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], return_qz=True)
@@ -202,9 +203,9 @@ def test_scale1m_sampled():
     toks[:2] = [0, w.N - 1]
     y_ref, q_ref, z_ref = oracle.flarepp_head(x["q0"][h], x["q_fixed"][h], float(x["gate"][h]),
                                               x["k0"][0, h], x["k"][0, h], x["v"][0, h], toks)
-    assert_parity(q[0, h], q_ref, "bf16", "q")
-    assert_parity(z[0, h], z_ref, "bf16", "z")
-    assert_parity(y[0, h, torch.from_numpy(toks).to(DEV)], y_ref, "bf16", "y")
+    assert_parity(q[0, h], q_ref, w.dtype, "q")
+    assert_parity(z[0, h], z_ref, w.dtype, "z")
+    assert_parity(y[0, h, torch.from_numpy(toks).to(DEV)], y_ref, w.dtype, "y")
     assert bool(torch.isfinite(y.float()).all())
 
 
