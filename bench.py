@@ -383,6 +383,25 @@ def run_ours(args):
         "clocks": sampler.summary(),
     }
 
+    # back-to-back calls (no L2 flush, no per-launch events between them): the
+    # launch sequence as a model calling the mixer layer after layer sees it,
+    # with consecutive kernels overlapping set-up and tail (programmatic
+    # dependent launch)
+    kb = max(1, min(K, 30))
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    b0.record()
+    for _ in range(kb):
+        step()
+    b1.record()
+    torch.cuda.synchronize()
+    b2b_ms = reduce_max(b0.elapsed_time(b1), world, dev) / kb
+    out["back_to_back"] = {"ms_per_call": round(b2b_ms, 4), "calls": kb,
+                           "value": round(aggregate_mtokens(counts["tokens"], world, 1, b2b_ms), 4), "unit": UNIT,
+                           "l2": "not flushed between calls"}
+
     # end-to-end through the public API with host buffers
     if not args.no_e2e:
         hx = {}

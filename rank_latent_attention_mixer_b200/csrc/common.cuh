@@ -58,6 +58,16 @@ template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t w) {
     return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still
+// running; it calls pdl_wait() before its first global-memory access, which
+// returns once that kernel has completed and its writes are visible.
+// pdl_launch_dependents() lets the next kernel of the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 2^x on the MUFU unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2_mufu(float x) {
     float y;

@@ -146,6 +146,8 @@ merge_partials(MergeParams p) {
     constexpr int LPC = V4 < 32 ? V4 : 32;
     constexpr int CPI = 32 / LPC;
     constexpr int F4PL = V4 / LPC;              // float4s per lane per chunk
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t rows = (int64_t)p.B * p.H * p.M;
     const int64_t row = (int64_t)blockIdx.x * 8 + warp;

@@ -52,6 +52,7 @@
 
 #include <cuda.h>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels_simt.cuh"
@@ -444,6 +445,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int q_tiles = p.interleave ? 1 : NW;                         // query tiles per item
+    // the set-up above overlaps the previous kernel's tail; global memory is
+    // touched only after it has completed
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp >= 4 * NW) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
@@ -965,6 +970,24 @@ inline bool make_map(CUtensorMap* map, CUtensorMapDataType type, const void* bas
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialization (the kernel calls pdl_wait()
+// before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 inline int sm_count() {
     int dev = 0, n = kNumSMs;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -980,8 +1003,10 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = prm.items < sm_count() ? prm.items : sm_count();
-    kern<<<grid, Regs<C::NW>::kThreads, C::kSmemLaunch, st>>>(mq, mk, mv, prm);
-    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+    return launch_pdl(kern, dim3(grid), dim3(Regs<C::NW>::kThreads), C::kSmemLaunch, st, mq, mk, mv, prm) ==
+                   cudaSuccess
+               ? 0
+               : 3;
 }
 
 template <typename E, int NW, int KT>
@@ -997,7 +1022,12 @@ inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, co
 
 template <typename E, int D>
 void launch_merge(const MergeParams& mp, int64_t rows, cudaStream_t st) {
-    merge_partials<E, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
+    // the attention kernels run with the largest shared-memory carveout; the
+    // merge asks for the same so that the SMs are not reconfigured in between
+    static const cudaError_t carveout = cudaFuncSetAttribute(
+        merge_partials<E, D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    (void)carveout;
+    launch_pdl(merge_partials<E, D>, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, mp);
 }
 
 template <typename E>
