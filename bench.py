@@ -53,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
     p.add_argument("--flare", action="store_true", help="closed gate: the two-call FLARE form (flare_fwd)")
+    p.add_argument("--layout", choices=["bhnd", "bnhd"], default="bhnd",
+                   help="memory layout of k0, k, v, y: [B,H,N,D] or [B,N,H,D] (read in place)")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -267,6 +269,9 @@ def run_ours(args):
     if args.tokens:
         w = w.with_shape(N=args.tokens, name=f"{w.name}_n{args.tokens}")
     x = W.make_inputs(w, device=str(dev))
+    if args.layout == "bnhd":
+        for name in ("k0", "k", "v"):
+            x[name] = x[name].transpose(1, 2).contiguous()
     path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
     dtype_code = {"f32": fb.F32, "bf16": fb.BF16, "f16": fb.F16}[w.dtype]
     used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
@@ -281,7 +286,7 @@ def run_ours(args):
 
     def step(events=None):
         fb.mixer_fwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y, path=path,
-                     workspace=ws, stage_events=events)
+                     workspace=ws, stage_events=events, layout=args.layout)
 
     for _ in range(args.warmup):
         step()
@@ -369,6 +374,7 @@ def run_ours(args):
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
                    "gate": "open (FLARE++)" if gated else "closed (FLARE, flare_fwd)",
+                   "layout": args.layout,
                    "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)"),
@@ -406,9 +412,10 @@ def run_ours(args):
     if not args.no_e2e:
         hx = {}
         for name in ("q0", "q_fixed", "gate", "k0", "k", "v"):
-            hx[name] = torch.empty(x[name].shape, dtype=x[name].dtype, pin_memory=True)
-            hx[name].copy_(x[name])
-        hy = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+            src = x[name].transpose(1, 2) if args.layout == "bnhd" and name in ("k0", "k", "v") else x[name]
+            hx[name] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+            hx[name].copy_(src)
+        hy = torch.empty(hx["k"].shape, dtype=y.dtype, pin_memory=True)
         ke = max(1, min(K, 5))
         hg = hx["gate"] if gated else None
         fb.mixer_fwd_host(hx["q0"], hx["q_fixed"], hg, hx["k0"], hx["k"], hx["v"], hy)  # warm-up
@@ -426,7 +433,7 @@ def run_ours(args):
                   if gated or n in ("q_fixed", "k", "v"))
         out["e2e"] = {"value": round(aggregate_mtokens(counts["tokens"], world, ke, e2e_ms), 4), "unit": UNIT,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hy.numel() * hy.element_size(),
-                      "steps": ke, "api": "flarepp_mixer_fwd_host (pinned host buffers)"}
+                      "steps": ke, "api": "flarepp_mixer_fwd_host (pinned host buffers, [B,H,N,D])"}
         del hx, hy
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

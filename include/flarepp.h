@@ -19,7 +19,10 @@
  *   - All tensor pointers are caller-owned DEVICE pointers (except the *_host
  *     entry), row-major and contiguous, 16-byte aligned:
  *       q0, q_fixed   [H, M, D]     shared by every batch element
- *       k0, k, v, y   [B, H, N, D]
+ *       k0, k, v, y   [B, H, N, D]  (or [B, N, H, D] with
+ *                                    flarepp_options_t.layout = FLAREPP_LAYOUT_BNHD:
+ *                                    the heads of one token adjacent, as a
+ *                                    [B, N, H*D] projection output viewed per head)
  *     in the I/O dtype (FLAREPP_F32 = fp32, FLAREPP_BF16 = bf16, FLAREPP_F16 =
  *     fp16; the last for the fp16 forward that physicsnemo issue #1150, the
  *     author's reply, "3. Scaling to 1 M points", calls essential at 1M points).
@@ -59,7 +62,7 @@
 extern "C" {
 #endif
 
-#define FLAREPP_ABI_VERSION 1
+#define FLAREPP_ABI_VERSION 2
 
 typedef enum flarepp_dtype {
     FLAREPP_F32 = 0,
@@ -85,6 +88,14 @@ typedef enum flarepp_path {
     FLAREPP_PATH_TCGEN05 = 2
 } flarepp_path_t;
 
+/* Memory layout of the token tensors k0, k, v and y (q0, q_fixed are always
+ * [H, M, D]; q_out and z_out always [B, H, M, D]). */
+typedef enum flarepp_layout {
+    FLAREPP_LAYOUT_BHND = 0,   /* [B, H, N, D]: one head's tokens contiguous           */
+    FLAREPP_LAYOUT_BNHD = 1    /* [B, N, H, D]: one token's heads contiguous; read and
+                                  written in place, no transpose pass                 */
+} flarepp_layout_t;
+
 /* Optional controls for the _ex entry.  Zero-initialise and set what you need. */
 typedef struct flarepp_options {
     float scale;             /* softmax scale; <= 0 selects 1/sqrt(D)                        */
@@ -101,6 +112,7 @@ typedef struct flarepp_options {
                                   [0] is recorded on `stream` before the first kernel launch
                                   and [i] after the i-th launch, for i < n_stage_events; lets a
                                   caller time each kernel on the stream it runs on            */
+    int layout;              /* flarepp_layout_t of k0, k, v, y; other values -> INVALID_ARG  */
 } flarepp_options_t;
 
 /* Kernel launches one forward call makes (gated = 0: closed gate / FLARE).

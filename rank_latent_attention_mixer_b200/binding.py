@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libflarepp.so")
 
 F32, BF16, F16 = 0, 1, 2
 PATH_AUTO, PATH_SIMT, PATH_TCGEN05 = 0, 1, 2
+LAYOUTS = {"bhnd": 0, "bnhd": 1}
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
           4: "ERR_WORKSPACE", 5: "ERR_TIMEOUT"}
 EXPORTS = ["flarepp_mixer_fwd", "flare_fwd", "flarepp_mixer_fwd_ex", "flarepp_workspace_bytes",
@@ -36,7 +37,7 @@ class Options(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("path", ctypes.c_int), ("force_chunks", ctypes.c_int),
                 ("n_stage_events", ctypes.c_int), ("q_out", ctypes.c_void_p), ("z_out", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("layout", ctypes.c_int)]
 
 
 def _load() -> ctypes.CDLL:
@@ -65,6 +66,8 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
+if lib.flarepp_abi_version() != 2:
+    raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs 2: rebuild it")
 
 
 def status_string(status: int) -> str:
@@ -94,10 +97,15 @@ def _check(rc: int, where: str):
         raise FlareppError(rc, where)
 
 
-def _shapes(q_fixed: torch.Tensor, k: torch.Tensor):
+def _shapes(q_fixed: torch.Tensor, k: torch.Tensor, layout: str = "bhnd"):
     if k.dim() != 4 or q_fixed.dim() != 3:
-        raise ValueError("expected q_fixed [H,M,D] and k [B,H,N,D]")
-    B, H, N, D = k.shape
+        raise ValueError(f"expected q_fixed [H,M,D] and k [{','.join(layout.upper())}]")
+    if layout == "bhnd":
+        B, H, N, D = k.shape
+    elif layout == "bnhd":
+        B, N, H, D = k.shape
+    else:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
     if q_fixed.shape[0] != H or q_fixed.shape[2] != D:
         raise ValueError(f"q_fixed {tuple(q_fixed.shape)} does not match k {tuple(k.shape)}")
     return B, H, N, q_fixed.shape[1], D
@@ -113,8 +121,8 @@ def launches_per_call(gated: bool = True) -> int:
     return int(lib.flarepp_launches_per_call(int(gated)))
 
 
-def workspace_bytes(B, H, N, M, D, dtype=BF16, gated=True, path=PATH_AUTO, force_chunks=0) -> int:
-    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None)
+def workspace_bytes(B, H, N, M, D, dtype=BF16, gated=True, path=PATH_AUTO, force_chunks=0, layout="bhnd") -> int:
+    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout])
     return int(lib.flarepp_workspace_bytes(B, H, N, M, D, dtype, int(gated), ctypes.byref(o)))
 
 
@@ -124,15 +132,16 @@ def selected_path(B, H, N, M, D, dtype=BF16) -> int:
 
 def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: int = PATH_AUTO,
               force_chunks: int = 0, return_qz: bool = False, workspace: Optional[torch.Tensor] = None,
-              stage_events=None):
+              stage_events=None, layout: str = "bhnd"):
     """FLARE++ mixer forward on the current CUDA stream.  ``gate=None`` is FLARE.
 
-    q0, q_fixed [H,M,D]; gate fp32 [H] (sigmoid already applied); k0, k, v [B,H,N,D];
-    all on the same CUDA device, contiguous, fp32 or bf16.  Returns y (and q, z
-    fp32 [B,H,M,D] when ``return_qz``).  ``stage_events``: torch.cuda.Event objects
-    (created with enable_timing) recorded before the first launch and after each
-    launch on the current stream."""
-    B, H, N, M, D = _shapes(q_fixed, k)
+    q0, q_fixed [H,M,D]; gate fp32 [H] (sigmoid already applied); k0, k, v and y
+    [B,H,N,D] (``layout="bhnd"``) or [B,N,H,D] (``layout="bnhd"``, read and
+    written in place); all on the same CUDA device, contiguous, fp32, bf16 or
+    fp16.  Returns y (and q, z fp32 [B,H,M,D] when ``return_qz``).
+    ``stage_events``: torch.cuda.Event objects (created with enable_timing)
+    recorded before the first launch and after each launch on the current stream."""
+    B, H, N, M, D = _shapes(q_fixed, k, layout)
     _contig(q0, q_fixed, gate, k0, k, v, y)
     dt = _dtype_code(k)
     if y is None:
@@ -143,7 +152,7 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
         z_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
     if gate is not None and gate.dtype != torch.float32:
         raise TypeError("gate must be float32 [H]")
-    need = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks)
+    need = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks, layout)
     if need == 0:
         ws_ptr, ws_len = None, 0
     else:
@@ -160,7 +169,8 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
         n_ev = len(handles)
         ev_arr = (ctypes.c_void_p * n_ev)(*handles)
     o = Options(float(scale), int(path), int(force_chunks), n_ev, _ptr(q_out), _ptr(z_out), ws_ptr, ws_len,
-                ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None)
+                ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None,
+                LAYOUTS[layout])
     rc = lib.flarepp_mixer_fwd_ex(_ptr(q0) if gate is not None else None, _ptr(q_fixed), _ptr(gate),
                                   _ptr(k0) if gate is not None else None, _ptr(k), _ptr(v), _ptr(y),
                                   B, H, N, M, D, dt, ctypes.byref(o), _stream(k.device))

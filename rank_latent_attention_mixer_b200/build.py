@@ -78,8 +78,11 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, "-Xptxas", "-v", "-o", tmp, *sources()]
-    res = subprocess.run(cmd, check=True, capture_output=True, text=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
     log = res.stdout + res.stderr
+    if res.returncode != 0:
+        errors = "\n".join(line for line in log.splitlines() if "error" in line) or log[-4000:]
+        raise RuntimeError(f"nvcc failed (exit {res.returncode}):\n{errors}")
     if verbose_ptxas:
         print(log)
     try:

@@ -45,6 +45,7 @@ struct Plan {
     int chunk_len;       // tokens per chunk
     int row_blocks;      // latent-row blocks per (b, h, chunk) (SIMT)
     float scale_log2;
+    tc::RowStrides tok;  // element strides of the token tensors k0, k, v, y (flarepp_layout_t)
     // byte offsets into the workspace
     size_t off_part_O, off_part_ml, off_q32, off_q16, off_z32, off_z16, total;
 };
@@ -77,6 +78,11 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     if (o && o->n_stage_events < 0) return FLAREPP_ERR_INVALID_ARG;
     if (o && o->n_stage_events > 0 && !o->stage_events) return FLAREPP_ERR_INVALID_ARG;
     if (o && o->force_chunks < 0) return FLAREPP_ERR_INVALID_ARG;
+    const int layout = o ? o->layout : FLAREPP_LAYOUT_BHND;
+    if (layout != FLAREPP_LAYOUT_BHND && layout != FLAREPP_LAYOUT_BNHD) return FLAREPP_ERR_INVALID_ARG;
+    pl->tok = layout == FLAREPP_LAYOUT_BNHD
+                  ? tc::RowStrides{(int64_t)s.H * s.D, s.D, (int64_t)s.N * s.H * s.D}
+                  : tc::contiguous_rows(s.N, s.H, s.D);
     pl->path = path;
     const float scale = (o && o->scale > 0.f) ? o->scale : 1.f / std::sqrt((float)s.D);
     if (!std::isfinite(scale)) return FLAREPP_ERR_INVALID_ARG;
@@ -174,6 +180,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
     const dim3 dec_grid((unsigned)((s.N + kSimtThreads - 1) / kSimtThreads), (unsigned)s.bh());
 
     SplitParams sp{};
+    sp.tok_row = pl.tok.row; sp.tok_h = pl.tok.h; sp.tok_b = pl.tok.b;
     sp.part_O = part_O; sp.part_ml = part_ml;
     sp.B = s.B; sp.H = s.H; sp.N = s.N; sp.M = s.M;
     sp.chunks = pl.chunks; sp.chunk_len = pl.chunk_len; sp.scale_log2 = pl.scale_log2;
@@ -182,6 +189,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
     mp.B = s.B; mp.H = s.H; mp.M = s.M; mp.q_fixed = q_fixed; mp.gate = gate;
     DecodeParams dp{};
     dp.Ktok = k; dp.Z = z32; dp.Y = y; dp.B = s.B; dp.H = s.H; dp.N = s.N; dp.M = s.M;
+    dp.tok_row = pl.tok.row; dp.tok_h = pl.tok.h; dp.tok_b = pl.tok.b;
     dp.scale_log2 = pl.scale_log2;
 
 #define FLAREPP_SIMT_DISPATCH(DD)                                                                  \
@@ -243,6 +251,7 @@ int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, con
         bu.z16 = ws + pl.off_z16;
         tc::Problem pr{};
         pr.B = s.B; pr.H = s.H; pr.N = s.N; pr.M = s.M; pr.D = s.D;
+        pr.tok = pl.tok;
         pr.chunks = pl.chunks; pr.chunk_len = pl.chunk_len; pr.scale_log2 = pl.scale_log2;
         auto mark = [&ev](cudaStream_t t) { ev.mark(t); };
         if (s.dtype == FLAREPP_F16)

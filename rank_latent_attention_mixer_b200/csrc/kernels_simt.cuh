@@ -28,8 +28,9 @@ constexpr int kSimtThreads = 128;
 struct SplitParams {
     const void* Q;       // latent query rows; (b, h) rows start at row (b*q_batch_heads + h)*M
     int q_batch_heads;   // H when Q is [B,H,M,D]; 0 when Q is [H,M,D] (shared over b)
-    const void* K;       // [B,H,N,D] keys
-    const void* V;       // [B,H,N,D] values (may equal K: synthesis reads k0 twice)
+    const void* K;       // token keys: row n of (b, h) at b*tok_b + h*tok_h + n*tok_row elements
+    const void* V;       // token values, same strides (may equal K: synthesis reads k0 twice)
+    int64_t tok_row, tok_h, tok_b;
     float* part_O;       // [C][B*H][M][D]
     float2* part_ml;     // [C][B*H][M]: (max in log2 units, sum of weights)
     int B, H, N, M;
@@ -69,19 +70,22 @@ split_partial_simt(SplitParams p) {
 #pragma unroll
     for (int d = 0; d < D; ++d) acc[d] = 0.f;
 
-    const TKV* Kbh = reinterpret_cast<const TKV*>(p.K) + (int64_t)bh * p.N * D;
-    const TKV* Vbh = reinterpret_cast<const TKV*>(p.V) + (int64_t)bh * p.N * D;
+    const int64_t base = (int64_t)b * p.tok_b + (int64_t)h * p.tok_h;
+    const TKV* Kbh = reinterpret_cast<const TKV*>(p.K) + base;
+    const TKV* Vbh = reinterpret_cast<const TKV*>(p.V) + base;
     constexpr int VEC = 16 / sizeof(TKV);          // elements per 16-byte load
+    constexpr int VPR = D / VEC;                   // 16-byte loads per row
     for (int t0 = n0; t0 < n1; t0 += TILE) {
         const int cnt = min(TILE, n1 - t0);
         __syncthreads();
-        for (int i = threadIdx.x; i < cnt * D / VEC; i += kSimtThreads) {
+        for (int i = threadIdx.x; i < cnt * VPR; i += kSimtThreads) {
             float tmp[VEC];
-            load_row_f32<TKV, VEC>(Kbh + (int64_t)t0 * D + i * VEC, tmp);
+            const int64_t off = (int64_t)(t0 + i / VPR) * p.tok_row + (i % VPR) * VEC;
+            load_row_f32<TKV, VEC>(Kbh + off, tmp);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) sK[i * VEC + e] = tmp[e];
             if (!same_kv) {
-                load_row_f32<TKV, VEC>(Vbh + (int64_t)t0 * D + i * VEC, tmp);
+                load_row_f32<TKV, VEC>(Vbh + off, tmp);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) sV[i * VEC + e] = tmp[e];
             }
@@ -220,11 +224,12 @@ merge_partials(MergeParams p) {
 // shared memory in chunks of 2048/D rows and every thread reads the same row
 // (broadcast); the softmax over M is online across the chunks.
 struct DecodeParams {
-    const void* Ktok;     // [B,H,N,D]
+    const void* Ktok;     // token keys: row n of (b, h) at b*tok_b + h*tok_h + n*tok_row elements
     const void* Qlat;     // latent keys; (b, h) rows start at row (b*q_batch_heads + h)*M
     int q_batch_heads;
     const float* Z;       // [B,H,M,D] fp32
-    void* Y;              // [B,H,N,D]
+    void* Y;              // output rows, same strides as Ktok
+    int64_t tok_row, tok_h, tok_b;
     int B, H, N, M;
     float scale_log2;
 };
@@ -244,7 +249,8 @@ decode_simt(DecodeParams p) {
 #pragma unroll
     for (int d = 0; d < D; ++d) kq[d] = 0.f;
     if (active) {
-        load_row_f32<T, D>(reinterpret_cast<const T*>(p.Ktok) + ((int64_t)bh * p.N + n) * D, kq);
+        load_row_f32<T, D>(reinterpret_cast<const T*>(p.Ktok) + (int64_t)b * p.tok_b + (int64_t)h * p.tok_h +
+                               (int64_t)n * p.tok_row, kq);
 #pragma unroll
         for (int d = 0; d < D; ++d) kq[d] *= p.scale_log2;
     }
@@ -292,7 +298,8 @@ decode_simt(DecodeParams p) {
         const float inv = 1.f / l;
 #pragma unroll
         for (int d = 0; d < D; ++d) acc[d] *= inv;
-        store_row<T, D>(reinterpret_cast<T*>(p.Y) + ((int64_t)bh * p.N + n) * D, acc);
+        store_row<T, D>(reinterpret_cast<T*>(p.Y) + (int64_t)b * p.tok_b + (int64_t)h * p.tok_h +
+                            (int64_t)n * p.tok_row, acc);
     }
 }
 

@@ -135,11 +135,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                            int z) {
+// Tile load from a 4-D map (x = element within a row, y = row, z = head,
+// w = batch), completing on `bar`.  x is always 0 here (whole rows).
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
+          "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -286,6 +290,15 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 
 // ------------------------------------------------------------------ kernel parameters
 
+// Element strides of a tensor of D-element rows: between consecutive rows,
+// heads and batch elements.
+struct RowStrides {
+    int64_t row, h, b;
+};
+inline RowStrides contiguous_rows(int rows, int H, int D) {
+    return {D, (int64_t)rows * D, (int64_t)H * rows * D};
+}
+
 enum Mode { kSplit = 0, kDecode = 1 };
 
 struct Params {
@@ -294,8 +307,8 @@ struct Params {
     int M, N;             // latents, tokens
     int kv_rows;          // rows of the key/value tensors per (b, h) (N in split mode, M in decode)
     int kv_tiles;         // ceil(kv_rows / KT)
-    int q_shared;         // query map's z coordinate is h (tensor [H, rows, D]) instead of b*H+h
-    int k_shared;         // key map's z coordinate is h
+    int q_shared;         // the query tensor is [H, rows, D], shared over the batch (map batch coordinate 0)
+    int k_shared;         // the key tensor is [H, rows, D]
     int kv_same;          // values are the keys (synthesis): load one tile per stage
     int interleave;       // warpgroups share one query tile and take the key/value tiles round-robin
     int row_groups;       // split mode: query-row groups per (b, h) (128 rows, or 128 NW when not interleaved)
@@ -306,11 +319,14 @@ struct Params {
     float scale_log2;
     float* part_O;        // split: [parts][B*H][M][D]
     float2* part_ml;      // split: [parts][B*H][M]
-    void* y;              // decode: [B,H,N,D] in E
+    int tok_heads_inner;  // the token tensor's map is ordered (D, H, rows, B): [B,N,H,D] layout
+    void* y;              // decode: token rows in E, addressed by the strides below
+    int64_t y_row, y_h, y_b;   // decode: element strides of y between tokens, heads, batch elements
 };
 
 struct Item {
-    int bh, qz, kz, vz;
+    int bh, h;
+    int qb, kb, vb;       // batch coordinate of the query, key and value maps (0 for a shared tensor)
     int qrow0;            // first query row of the item
     int t_begin, t_end;   // key/value tile range
     int part;             // split mode: partial index of warpgroup 0 (interleaved: NW c, else c)
@@ -336,10 +352,11 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item) {
         it.t_end = p.kv_tiles;
         it.part = 0;
     }
-    const int h = it.bh % p.H;
-    it.qz = p.q_shared ? h : it.bh;
-    it.kz = p.k_shared ? h : it.bh;
-    it.vz = it.bh;
+    it.h = it.bh % p.H;
+    const int b = it.bh / p.H;
+    it.qb = p.q_shared ? 0 : b;
+    it.kb = p.k_shared ? 0 : b;
+    it.vb = b;
     return it;
 }
 
@@ -469,8 +486,13 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 if (!ok) break;
                 mbar_expect_tx(&q_full[slot], q_bytes);
                 uint8_t* qdst = smem + SM::kQ + slot * NW * SM::kQTileBytes;
-                for (int qt = 0; qt < q_tiles; ++qt)
-                    tma_load_3d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, it.qrow0 + qt * kQTile, it.qz);
+                for (int qt = 0; qt < q_tiles; ++qt) {
+                    const int qrow = it.qrow0 + qt * kQTile;
+                    if (p.mode == kDecode && p.tok_heads_inner)      // token queries, [B,N,H,D]
+                        tma_load_4d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, it.h, qrow, it.qb);
+                    else
+                        tma_load_4d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, qrow, it.h, it.qb);
+                }
                 q_last_phase[slot] = (q_load / QS) & 1;
                 ++q_load;
                 for (int t = it.t_begin; t < it.t_end; ++t) {
@@ -489,9 +511,11 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     if (!ok) break;
                     mbar_expect_tx(&kv_full[st], kv_bytes);
                     uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kKVTileBytes;
-                    tma_load_3d(kdst, &map_k, &kv_full[st], 0, t * KT, it.kz);
+                    const bool hi = p.mode == kSplit && p.tok_heads_inner;   // token keys/values, [B,N,H,D]
+                    tma_load_4d(kdst, &map_k, &kv_full[st], 0, hi ? it.h : t * KT, hi ? t * KT : it.h, it.kb);
                     if (!p.kv_same)
-                        tma_load_3d(kdst + SM::kKVTileBytes, &map_v, &kv_full[st], 0, t * KT, it.vz);
+                        tma_load_4d(kdst + SM::kKVTileBytes, &map_v, &kv_full[st], 0, hi ? it.h : t * KT,
+                                    hi ? t * KT : it.h, it.vb);
                     kv_last_phase[st] = fill & 1;
                     ++kv_load;
                 }
@@ -689,7 +713,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const int n = it.qrow0 + wg * kQTile + row;
                 if (n < p.N && o) {
                     const float inv = 1.f / l;
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + ((int64_t)it.bh * p.N + n) * D);
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + (int64_t)(it.bh / p.H) * p.y_b +
+                                                          (int64_t)it.h * p.y_h + (int64_t)n * p.y_row);
 #pragma unroll
                     for (int i = 0; i < D / 8; ++i) {
                         const int c = i / 4, j = (i % 4) * 8;
@@ -877,6 +902,7 @@ struct Buffers {
 
 struct Problem {
     int B, H, N, M, D;
+    RowStrides tok;       // element strides of the token tensors k0, k, v, y
     int chunks, chunk_len;
     float scale_log2;
 };
@@ -954,20 +980,27 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D map over a [planes, rows, D] tensor of 16-bit elements, box [1, box_rows, D], swizzle = D*2 bytes.
-inline bool make_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int planes, int rows, int D,
-                     int box_rows) {
+// 4-D map over a tensor of 16-bit elements, box of box_rows whole rows of one
+// (b, h), swizzle = D*2 bytes.  The dimensions are ordered by increasing
+// stride: (D, rows, H, B) when a head's rows are contiguous ([B,H,rows,D]),
+// (D, H, rows, B) when a row's heads are ([B,rows,H,D]); the kernel passes its
+// coordinates in the same order (Params::tok_heads_inner).
+inline bool make_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rows, int H, int B, int D,
+                     const RowStrides& str, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
+    const bool heads_inner = str.h < str.row;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)(heads_inner ? H : rows),
+                                (cuuint64_t)(heads_inner ? rows : H), (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(heads_inner ? str.h : str.row) * 2,
+                                   (cuuint64_t)(heads_inner ? str.row : str.h) * 2, (cuuint64_t)str.b * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)D, heads_inner ? 1u : (cuuint32_t)box_rows,
+                               heads_inner ? (cuuint32_t)box_rows : 1u, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                           : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-    return fn(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(map, type, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Launch with programmatic stream serialization (the kernel calls pdl_wait()
@@ -1051,12 +1084,17 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     // token keys k serve as key/value tiles (split) and as query tiles (decode)
     CUtensorMap m_q0, m_qf_q, m_qf_kv, m_q16_q, m_q16_kv, m_z16, m_k0, m_k_kv, m_k_q, m_v;
     const CUtensorMapDataType ty = Elem<E>::kMapType;
-    bool ok = make_map(&m_qf_q, ty, q_fixed, H, M, D, kQTile) && make_map(&m_qf_kv, ty, q_fixed, H, M, D, kDecodeKT) &&
-              make_map(&m_q16_q, ty, bu.q16, BH, M, D, kQTile) && make_map(&m_q16_kv, ty, bu.q16, BH, M, D, kDecodeKT) &&
-              make_map(&m_z16, ty, bu.z16, BH, M, D, kDecodeKT) && make_map(&m_k_kv, ty, k, BH, N, D, kSplitKT) &&
-              make_map(&m_k_q, ty, k, BH, N, D, kQTile) && make_map(&m_v, ty, v, BH, N, D, kSplitKT);
+    const RowStrides lat1 = contiguous_rows(M, H, D), latb = contiguous_rows(M, H, D), tok = pr.tok;
+    bool ok = make_map(&m_qf_q, ty, q_fixed, M, H, 1, D, lat1, kQTile) &&
+              make_map(&m_qf_kv, ty, q_fixed, M, H, 1, D, lat1, kDecodeKT) &&
+              make_map(&m_q16_q, ty, bu.q16, M, H, B, D, latb, kQTile) &&
+              make_map(&m_q16_kv, ty, bu.q16, M, H, B, D, latb, kDecodeKT) &&
+              make_map(&m_z16, ty, bu.z16, M, H, B, D, latb, kDecodeKT) &&
+              make_map(&m_k_kv, ty, k, N, H, B, D, tok, kSplitKT) && make_map(&m_k_q, ty, k, N, H, B, D, tok, kQTile) &&
+              make_map(&m_v, ty, v, N, H, B, D, tok, kSplitKT);
     if (gated)
-        ok = ok && make_map(&m_q0, ty, q0, H, M, D, kQTile) && make_map(&m_k0, ty, k0, BH, N, D, kSplitKT);
+        ok = ok && make_map(&m_q0, ty, q0, M, H, 1, D, lat1, kQTile) &&
+             make_map(&m_k0, ty, k0, N, H, B, D, tok, kSplitKT);
     if (!ok) return 3;
 
     const int kv_tiles = (N + kSplitKT - 1) / kSplitKT;
@@ -1065,6 +1103,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     sp.mode = kSplit;
     sp.B = B; sp.H = H; sp.M = M; sp.N = N;
     sp.kv_rows = N; sp.kv_tiles = kv_tiles;
+    sp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
     sp.interleave = interleaved(M) ? 1 : 0;
     sp.row_groups = row_groups(M);
     sp.chunks = pr.chunks;
@@ -1113,6 +1152,8 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     dp.items = BH * dp.q_groups;
     dp.scale_log2 = pr.scale_log2;
     dp.y = y;
+    dp.y_row = tok.row; dp.y_h = tok.h; dp.y_b = tok.b;
+    dp.tok_heads_inner = tok.h < tok.row ? 1 : 0;
     rc = launch_attn_d<E, kDecodeNW, kDecodeKT>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
     if (rc) return rc;
     mark(st);

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.lib.flarepp_abi_version() == 1
+    assert lib.lib.flarepp_abi_version() == 2
     assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
     for code in range(6):
         assert lib.status_string(code) not in ("", "unknown status")
@@ -100,6 +100,10 @@ def test_options_checked(lib):
     o = lib.Options(0.0, 0, 0, 0, None, None, 0x1000, 16, None)   # workspace too small
     rc = lib.lib.flarepp_mixer_fwd_ex(*FAKE, 1, 2, 64, 16, 16, 1, ctypes.byref(o), None)
     assert rc == 4
+    o = lib.Options(0.0, 0, 0, 0, None, None, None, 0, None, 2)     # unknown token layout
+    assert lib.lib.flarepp_mixer_fwd_ex(*FAKE, 1, 2, 64, 16, 16, 1, ctypes.byref(o), None) == 1
+    assert lib.workspace_bytes(1, 2, 64, 16, 16, lib.BF16, layout="bnhd") == lib.workspace_bytes(1, 2, 64, 16, 16,
+                                                                                                  lib.BF16)
 
 
 def test_workspace_and_path_queries(lib):

@@ -105,6 +105,35 @@ def test_edge_shapes(shape, dtype):
     assert_parity(y, y_ref, dtype, "y")
 
 
+@pytest.mark.parametrize("dtype,path", [("bf16", 0), ("f16", 0), ("f32", 0), ("bf16", 1)],
+                         ids=["bf16-auto", "f16-auto", "f32", "bf16-simt"])
+@pytest.mark.parametrize("shape", [(2, 3, 1000, 64, 32), (1, 8, 3001, 256, 64), (2, 2, 300, 17, 16),
+                                   (1, 1, 777, 130, 64)], ids=lambda s: "x".join(map(str, s)))
+def test_bnhd_layout(shape, dtype, path):
+    """k0, k, v, y in [B,N,H,D] (one token's heads adjacent) give exactly the
+    [B,H,N,D] result: only the addressing differs."""
+    B, H, N, M, D = shape
+    x = W.random_inputs(B, H, N, M, D, dtype=dtype, seed=B * H + N)
+    y_ref, q_ref, z_ref = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+    y, q, z = run(x, path=path)
+    b = binding()
+    d = cuda_inputs(x)
+    t = lambda a: a.transpose(1, 2).contiguous()
+    for gated in (True, False):
+        yb, qb, zb = b.mixer_fwd(d["q0"], d["q_fixed"], d["gate"] if gated else None, t(d["k0"]), t(d["k"]),
+                                 t(d["v"]), return_qz=True, path=path, layout="bnhd")
+        torch.cuda.synchronize()
+        assert b.check_device_status() == 0
+        assert yb.shape == (B, N, H, D)
+        if gated:
+            assert torch.equal(yb.transpose(1, 2), y)
+            assert torch.equal(qb, q) and torch.equal(zb, z)
+            assert_parity(yb.transpose(1, 2), y_ref, dtype, "y (bnhd)")
+        else:
+            y_flare = b.mixer_fwd(d["q0"], d["q_fixed"], None, d["k0"], d["k"], d["v"], path=path)
+            assert torch.equal(yb.transpose(1, 2), y_flare)
+
+
 @pytest.mark.parametrize("path", [0, 1], ids=["auto", "simt"])
 def test_chunk_invariance(path):
     x = W.random_inputs(2, 2, 3001, 128, 32, dtype="bf16", seed=5)
