@@ -53,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
     p.add_argument("--flare", action="store_true", help="closed gate: the two-call FLARE form (flare_fwd)")
+    p.add_argument("--cp", action="store_true",
+                   help="token-sharded form: one global problem, each rank holds N/world tokens (strong scaling)")
     p.add_argument("--layout", choices=["bhnd", "bnhd"], default="bhnd",
                    help="memory layout of k0, k, v, y: [B,H,N,D] or [B,N,H,D] (read in place)")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
@@ -495,10 +497,132 @@ def _cpu_head_inputs(w):
     return W.make_inputs(small)
 
 
+# --------------------------------------------------------------------------- token-sharded arm
+
+def run_cp(args):
+    """One global problem with its tokens sharded over the ranks: each rank
+    runs the split passes on its N/world tokens, the latent-sized triples are
+    all-gathered over NCCL and merged, and each rank decodes its tokens
+    (strong scaling: total work fixed as the rank count grows)."""
+    import torch
+    rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from rank_latent_attention_mixer_b200 import binding as fb
+    from rank_latent_attention_mixer_b200 import cp
+    from rank_latent_attention_mixer_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]                  # the same global problem on every rank
+    if args.tokens:
+        w = w.with_shape(N=args.tokens, name=f"{w.name}_n{args.tokens}")
+    x = W.make_inputs(w, device=str(dev))
+    lo, hi = cp.shard_bounds(w.N, world, rank)
+    for name in ("k0", "k", "v"):
+        t = x[name][:, :, lo:hi]
+        x[name] = (t.transpose(1, 2) if args.layout == "bnhd" else t).contiguous()
+    torch.cuda.empty_cache()
+    n_local = hi - lo
+    path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
+    gated = not args.flare
+    y = torch.empty_like(x["k"])
+    fits_l2 = 5 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
+
+    class TimedOps:
+        """The library stages, with events around each split pass on the launching stream."""
+        def __init__(self):
+            self.marks = None
+
+        def __getattr__(self, name):
+            return getattr(fb, name)
+
+        def cp_partials(self, *a, **kw):
+            if self.marks is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fb.cp_partials(*a, **kw)
+                e1.record()
+                self.marks.append((e0, e1))
+            else:
+                fb.cp_partials(*a, **kw)
+
+    ops = TimedOps()
+
+    def step():
+        cp.mixer_fwd_cp(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y,
+                        layout=args.layout, path=path, _ops=ops)
+
+    for _ in range(args.warmup):
+        step()
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize()
+    assert fb.check_device_status() == 0
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ops.marks = []
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+            if flush is not None:
+                flush.zero_()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if fb.check_device_status() != 0:
+        raise SystemExit("device status after the timed region")
+    local_ms = sum(a.elapsed_time(b) for a, b in ev)
+    max_ms = reduce_max(local_ms, world, dev)
+    split_ms = statistics.mean(a.elapsed_time(b) for a, b in ops.marks)
+    counts = W.algorithmic_counts(w, flare=not gated)
+    value = counts["tokens"] * K / (max_ms * 1e-3) / 1e6          # the global problem's tokens
+    peaks, peak_src = load_peaks()
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    flops_split = 4.0 * w.B * w.H * n_local * w.M * w.D
+    achieved = flops_split / (split_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
+                   "gate": "open (FLARE++)" if gated else "closed (FLARE)", "layout": args.layout,
+                   "parallelism": f"token-sharded x{world} ({n_local} tokens on rank {rank}; NCCL all-gather of "
+                                  f"latent triples)",
+                   "l2": ("flushed between steps (512 MiB write)" if flush is not None
+                          else "inputs larger than L2 (back-to-back steps)")},
+        "tflops": round(counts["flops"] / (max_ms / K * 1e-3) / 1e12, 2),
+        "gpu_launches": K * ((5 if gated else 3) + (2 if gated else 1)),
+        "roofline": {"bound": "tensor", "kernel": "split_partial (+ local triple reduction)",
+                     "achieved": round(achieved, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_t, 4), "traffic": None,
+                     "peak_kind": f"{peak_src} bf16 sustained", "launch_ms": round(split_ms, 4)},
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.cp:
+        run_cp(args)
     else:
         run_ours(args)
 

@@ -200,6 +200,60 @@ int flarepp_check_device_status(void* stream);
 /* Static text for a status code. */
 const char* flarepp_status_string(int status);
 
+/* ---------------------------------------------------------------------------
+ * Token-sharded (context-parallel) form, physicsnemo issue #2024, section 2:
+ * the N tokens are split across ranks and no rank holds the whole sequence.
+ * Each rank runs the split softmax passes on its own tokens and reduces them
+ * to one unnormalised triple (row max in log2 units, row sum, weighted sum of
+ * the value rows) per latent row; the ranks' triples are all-gathered (by the
+ * caller, e.g. NCCL) and merged by log-sum-exp, which rebuilds the globally
+ * normalised attention exactly up to rounding; the decode stays local.  Per
+ * rank, for the gated form:
+ *     flarepp_cp_partials(q0, 1, k0, k0, T)   all-gather T -> Tg
+ *     flarepp_cp_merge(Tg, G, q_fixed, gate, Q)            routing queries q
+ *     flarepp_cp_partials(Q, 0, k, v, T)      all-gather T -> Tg
+ *     flarepp_cp_merge(Tg, G, NULL, NULL, Z)               latents z
+ *     flarepp_cp_decode(Q, 0, Z, k, y)
+ * and for the closed gate (FLARE) the encode and decode take q_fixed with
+ * q_shared = 1.  N is this rank's token count (>= 1); k0, k, v, y hold this
+ * rank's tokens in the layout of opts->layout.  Every rank must use the same
+ * B, H, M, D, dtype, scale and rank order.  Arguments, ownership, alignment,
+ * errors and asynchrony are as for flarepp_mixer_fwd_ex; opts (may be NULL)
+ * supplies scale, path, force_chunks, workspace and layout.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of one rank's triple buffer T: B*H*M*(D+2) fp32 -- the O rows
+ * [B,H,M,D] followed by (max, sum) pairs [B,H,M,2].  The all-gathered buffer
+ * Tg is G such buffers back to back in rank order.  0 for invalid sizes. */
+size_t flarepp_cp_triple_bytes(int B, int H, int M, int D);
+
+/* Bytes of a latent state Q or Z: [B,H,M,D] fp32, then (16-bit I/O) the same
+ * rows in the I/O dtype at a 256-byte-aligned offset.  0 for invalid sizes. */
+size_t flarepp_cp_latent_bytes(int B, int H, int M, int D, int dtype);
+
+/* One split pass over this rank's N tokens into `triple` (DEVICE, 16-byte
+ * aligned, flarepp_cp_triple_bytes).  q: q_shared = 1 -> [H,M,D] in the I/O
+ * dtype (q0 for the synthesis, q_fixed for the closed-gate encode);
+ * q_shared = 0 -> a latent state from flarepp_cp_merge.  v == k reads each key
+ * tile once and uses it as the value tile (the synthesis, V = K = k0). */
+int flarepp_cp_partials(const void* q, int q_shared, const void* k, const void* v, float* triple,
+                        int B, int H, int N, int M, int D, int dtype,
+                        const flarepp_options_t* opts, void* stream);
+
+/* Log-sum-exp merge of `ranks` gathered triples into the latent state `state`
+ * (DEVICE, flarepp_cp_latent_bytes).  gate != NULL: synthesis, state = q =
+ * q_fixed + gate * merged (q_fixed [H,M,D] in the I/O dtype, gate fp32 [H]);
+ * gate == NULL: encode, state = z = merged (q_fixed ignored). */
+int flarepp_cp_merge(const float* gathered, int ranks, const void* q_fixed, const float* gate, void* state,
+                     int B, int H, int M, int D, int dtype, void* stream);
+
+/* Decode of this rank's N tokens: y = SDPA(k, q, z) with q as in
+ * flarepp_cp_partials (the routing-query state, or q_fixed with q_shared = 1)
+ * and z_state from the encode merge; y in the token layout of opts. */
+int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const void* k, void* y,
+                      int B, int H, int N, int M, int D, int dtype,
+                      const flarepp_options_t* opts, void* stream);
+
 /* FLAREPP_ABI_VERSION of the loaded library. */
 int flarepp_abi_version(void);
 

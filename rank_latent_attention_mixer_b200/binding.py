@@ -231,6 +231,66 @@ def mixer_fwd_noalloc(q0, q_fixed, gate, k0, k, v, y):
     return y
 
 
+# ---------------------------------------------------------------- token-sharded stages
+
+def cp_triple_bytes(B, H, M, D) -> int:
+    fn = lib.flarepp_cp_triple_bytes
+    fn.argtypes = [ctypes.c_int] * 4
+    fn.restype = ctypes.c_size_t
+    return int(fn(B, H, M, D))
+
+
+def cp_latent_bytes(B, H, M, D, dtype) -> int:
+    fn = lib.flarepp_cp_latent_bytes
+    fn.argtypes = [ctypes.c_int] * 5
+    fn.restype = ctypes.c_size_t
+    return int(fn(B, H, M, D, dtype))
+
+
+def _cp_options(path, scale, force_chunks, layout, workspace=None):
+    ws_ptr, ws_len = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
+    return Options(float(scale), int(path), int(force_chunks), 0, None, None, ws_ptr, ws_len, None, LAYOUTS[layout])
+
+
+def cp_partials(q, q_shared: bool, k, v, triple, *, B, H, N, M, D, path=PATH_AUTO, scale=0.0, force_chunks=0,
+                layout="bhnd"):
+    """flarepp_cp_partials: this rank's split pass reduced to one triple per latent row."""
+    fn = lib.flarepp_cp_partials
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, ctypes.POINTER(Options), vp]
+    fn.restype = i
+    o = _cp_options(path, scale, force_chunks, layout)
+    rc = fn(_ptr(q), int(q_shared), _ptr(k), _ptr(v), _ptr(triple), B, H, N, M, D, _dtype_code(k),
+            ctypes.byref(o), _stream(k.device))
+    _check(rc, "flarepp_cp_partials")
+    return triple
+
+
+def cp_merge(gathered, ranks: int, q_fixed, gate, state, *, B, H, M, D, dtype):
+    """flarepp_cp_merge: log-sum-exp merge of the gathered triples into a latent state."""
+    fn = lib.flarepp_cp_merge
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, vp]
+    fn.restype = i
+    rc = fn(_ptr(gathered), int(ranks), _ptr(q_fixed), _ptr(gate), _ptr(state), B, H, M, D, dtype,
+            _stream(gathered.device))
+    _check(rc, "flarepp_cp_merge")
+    return state
+
+
+def cp_decode(q, q_shared: bool, z_state, k, y, *, B, H, N, M, D, path=PATH_AUTO, scale=0.0, layout="bhnd"):
+    """flarepp_cp_decode: this rank's tokens decoded against the merged latents."""
+    fn = lib.flarepp_cp_decode
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, ctypes.POINTER(Options), vp]
+    fn.restype = i
+    o = _cp_options(path, scale, 0, layout)
+    rc = fn(_ptr(q), int(q_shared), _ptr(z_state), _ptr(k), _ptr(y), B, H, N, M, D, _dtype_code(k),
+            ctypes.byref(o), _stream(k.device))
+    _check(rc, "flarepp_cp_decode")
+    return y
+
+
 def selftest_wait_timeout(limit_us: int = 20000, stream: Optional[torch.cuda.Stream] = None) -> int:
     """Launches the bounded-wait self-test (a wait nothing satisfies); returns the launch status."""
     fn = lib.flarepp_selftest_wait_timeout

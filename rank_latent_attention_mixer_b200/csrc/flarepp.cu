@@ -501,6 +501,238 @@ int host_forward(const void* q0, const void* q_fixed, const float* gate, const v
     return rc;
 }
 
+// ------------------------------------------------------------------ token-sharded stages
+//
+// A latent state (the routing queries q or the latents z after the merge
+// across ranks) is [B,H,M,D] fp32 followed, for 16-bit I/O, by the same rows
+// in the I/O dtype (the tensor-core operand) at latent_16_offset().
+
+size_t latent_16_offset(const Shape& s) { return align_up((size_t)s.bh() * s.M * s.D * sizeof(float)); }
+
+size_t latent_state_bytes(const Shape& s) {
+    return latent_16_offset(s) + (s.dtype == FLAREPP_F32 ? 0 : (size_t)s.bh() * s.M * s.D * 2);
+}
+
+// Workspace of one staged call: the caller's, or stream-ordered from the pool.
+struct StageScratch {
+    char* ws = nullptr;
+    bool owned = false;
+    cudaStream_t st = nullptr;
+    int acquire(const Plan& pl, const flarepp_options_t* opts, cudaStream_t stream) {
+        st = stream;
+        if (opts && opts->workspace) {
+            if (opts->workspace_bytes < pl.total) return FLAREPP_ERR_WORKSPACE;
+            if (reinterpret_cast<uintptr_t>(opts->workspace) % kAlign) return FLAREPP_ERR_INVALID_ARG;
+            ws = static_cast<char*>(opts->workspace);
+            return FLAREPP_OK;
+        }
+        if (cudaMallocAsync(reinterpret_cast<void**>(&ws), pl.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return FLAREPP_ERR_WORKSPACE;
+        }
+        owned = true;
+        return FLAREPP_OK;
+    }
+    int release(int rc) {
+        if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+        owned = false;
+        return rc;
+    }
+};
+
+template <typename T>
+void simt_triple(const Shape& s, const Plan& pl, char* ws, float* triple, cudaStream_t st) {
+    const int64_t rows = s.bh() * s.M;
+    MergeParams mp{};
+    mp.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
+    mp.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+    mp.chunks = pl.chunks;
+    mp.B = s.B; mp.H = s.H; mp.M = s.M;
+    mp.mode = kMergeTriple;
+    mp.out_f32 = triple;
+    mp.out_ml = reinterpret_cast<float2*>(triple + rows * s.D);
+    const dim3 grid((unsigned)((rows + 7) / 8));
+    switch (s.D) {
+        case 16: merge_partials<T, 16><<<grid, 256, 0, st>>>(mp); break;
+        case 32: merge_partials<T, 32><<<grid, 256, 0, st>>>(mp); break;
+        case 64: merge_partials<T, 64><<<grid, 256, 0, st>>>(mp); break;
+        default: merge_partials<T, 128><<<grid, 256, 0, st>>>(mp); break;
+    }
+}
+
+// SIMT split pass + local reduction.  The query rows are the I/O dtype T when
+// shared ([H,M,D]) and the fp32 part of a latent state otherwise.
+template <typename T>
+int simt_cp_partials(const Shape& s, const Plan& pl, const void* q, bool q_shared, const void* k, const void* v,
+                     float* triple, char* ws, cudaStream_t st) {
+    SplitParams sp{};
+    sp.Q = q; sp.q_batch_heads = q_shared ? 0 : s.H; sp.K = k; sp.V = v;
+    sp.tok_row = pl.tok.row; sp.tok_h = pl.tok.h; sp.tok_b = pl.tok.b;
+    sp.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
+    sp.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+    sp.B = s.B; sp.H = s.H; sp.N = s.N; sp.M = s.M;
+    sp.chunks = pl.chunks; sp.chunk_len = pl.chunk_len; sp.scale_log2 = pl.scale_log2;
+    const dim3 grid(pl.chunks, (unsigned)s.bh(), pl.row_blocks);
+#define FLAREPP_CP_SPLIT(DD)                                                                       \
+    case DD:                                                                                       \
+        if (q_shared) split_partial_simt<T, T, DD><<<grid, kSimtThreads, 0, st>>>(sp);             \
+        else split_partial_simt<float, T, DD><<<grid, kSimtThreads, 0, st>>>(sp);                  \
+        break;
+    switch (s.D) {
+        FLAREPP_CP_SPLIT(16)
+        FLAREPP_CP_SPLIT(32)
+        FLAREPP_CP_SPLIT(64)
+        FLAREPP_CP_SPLIT(128)
+        default: return FLAREPP_ERR_UNSUPPORTED;
+    }
+#undef FLAREPP_CP_SPLIT
+    simt_triple<T>(s, pl, ws, triple, st);
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
+template <typename T>
+int simt_cp_decode(const Shape& s, const Plan& pl, const void* q, bool q_shared, const float* z32, const void* k,
+                   void* y, cudaStream_t st) {
+    DecodeParams dp{};
+    dp.Ktok = k; dp.Qlat = q; dp.q_batch_heads = q_shared ? 0 : s.H; dp.Z = z32; dp.Y = y;
+    dp.B = s.B; dp.H = s.H; dp.N = s.N; dp.M = s.M;
+    dp.tok_row = pl.tok.row; dp.tok_h = pl.tok.h; dp.tok_b = pl.tok.b;
+    dp.scale_log2 = pl.scale_log2;
+    const dim3 grid((unsigned)((s.N + kSimtThreads - 1) / kSimtThreads), (unsigned)s.bh());
+#define FLAREPP_CP_DEC(DD)                                                                         \
+    case DD:                                                                                       \
+        if (q_shared) decode_simt<T, T, DD><<<grid, kSimtThreads, 0, st>>>(dp);                    \
+        else decode_simt<T, float, DD><<<grid, kSimtThreads, 0, st>>>(dp);                         \
+        break;
+    switch (s.D) {
+        FLAREPP_CP_DEC(16)
+        FLAREPP_CP_DEC(32)
+        FLAREPP_CP_DEC(64)
+        FLAREPP_CP_DEC(128)
+        default: return FLAREPP_ERR_UNSUPPORTED;
+    }
+#undef FLAREPP_CP_DEC
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
+tc::Problem tc_problem(const Shape& s, const Plan& pl) {
+    tc::Problem pr{};
+    pr.B = s.B; pr.H = s.H; pr.N = s.N; pr.M = s.M; pr.D = s.D;
+    pr.tok = pl.tok;
+    pr.chunks = pl.chunks; pr.chunk_len = pl.chunk_len; pr.scale_log2 = pl.scale_log2;
+    return pr;
+}
+
+tc::Buffers tc_buffers(const Plan& pl, char* ws) {
+    tc::Buffers bu{};
+    bu.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
+    bu.part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
+    return bu;
+}
+
+int cp_partials(const void* q, int q_shared, const void* k, const void* v, float* triple, int B, int H, int N,
+                int M, int D, int dtype, const flarepp_options_t* opts, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    int rc = make_plan(s, opts, &pl);
+    if (rc) return rc;
+    if (!q || !k || !v || !triple || (q_shared != 0 && q_shared != 1)) return FLAREPP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(triple)) return FLAREPP_ERR_INVALID_ARG;
+    const size_t tb = s.tok_bytes();
+    const size_t trb = (size_t)s.bh() * M * (D + 2) * sizeof(float);
+    if (overlaps(triple, trb, k, tb) || overlaps(triple, trb, v, tb)) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    StageScratch sc;
+    rc = sc.acquire(pl, opts, st);
+    if (rc) return rc;
+    // a latent state's operand part: the I/O-dtype copy (tensor cores) or fp32 (SIMT)
+    const void* q16 = q_shared ? q : static_cast<const char*>(q) + latent_16_offset(s);
+    if (pl.path == FLAREPP_PATH_TCGEN05) {
+        const tc::Problem pr = tc_problem(s, pl);
+        const tc::Buffers bu = tc_buffers(pl, sc.ws);
+        rc = dtype == FLAREPP_F16 ? tc::cp_split<__half>(pr, bu, q16, q_shared, k, v, triple, st)
+                                  : tc::cp_split<__nv_bfloat16>(pr, bu, q16, q_shared, k, v, triple, st);
+        if (rc) rc = rc == 2 ? FLAREPP_ERR_UNSUPPORTED : FLAREPP_ERR_CUDA;
+    } else if (dtype == FLAREPP_F32) {
+        rc = simt_cp_partials<float>(s, pl, q, q_shared, k, v, triple, sc.ws, st);
+    } else if (dtype == FLAREPP_F16) {
+        rc = simt_cp_partials<__half>(s, pl, q, q_shared, k, v, triple, sc.ws, st);
+    } else {
+        rc = simt_cp_partials<__nv_bfloat16>(s, pl, q, q_shared, k, v, triple, sc.ws, st);
+    }
+    return sc.release(rc);
+}
+
+int cp_merge(const float* gathered, int G, const void* q_fixed, const float* gate, void* state, int B, int H, int M,
+             int D, int dtype, void* stream) {
+    const Shape s{B, H, 1, M, D, dtype};
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (G < 1 || !gathered || !state || (gate && !q_fixed)) return FLAREPP_ERR_INVALID_ARG;
+    if (!aligned16(gathered) || !aligned16(state) || (q_fixed && !aligned16(q_fixed)) ||
+        (gate && (reinterpret_cast<uintptr_t>(gate) & 3u)))
+        return FLAREPP_ERR_INVALID_ARG;
+    const int64_t rows = s.bh() * M;
+    const size_t gb = (size_t)G * rows * (D + 2) * sizeof(float);
+    if (overlaps(state, latent_state_bytes(s), gathered, gb)) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    MergeParams mp{};
+    mp.part_O = gathered;
+    mp.o_part_stride = rows * (D + 2);
+    mp.part_ml = reinterpret_cast<const float2*>(gathered + rows * D);
+    mp.ml_part_stride = rows * (D + 2) / 2;
+    mp.chunks = G;
+    mp.B = B; mp.H = H; mp.M = M;
+    mp.mode = gate ? kMergeSynthesis : kMergeEncode;
+    mp.q_fixed = q_fixed; mp.gate = gate;
+    mp.out_f32 = static_cast<float*>(state);
+    mp.out_16 = dtype == FLAREPP_F32 ? nullptr : static_cast<char*>(state) + latent_16_offset(s);
+    const dim3 grid((unsigned)((rows + 7) / 8));
+#define FLAREPP_CP_MERGE(T)                                                                        \
+    switch (D) {                                                                                   \
+        case 16: merge_partials<T, 16><<<grid, 256, 0, st>>>(mp); break;                           \
+        case 32: merge_partials<T, 32><<<grid, 256, 0, st>>>(mp); break;                           \
+        case 64: merge_partials<T, 64><<<grid, 256, 0, st>>>(mp); break;                           \
+        default: merge_partials<T, 128><<<grid, 256, 0, st>>>(mp); break;                          \
+    }
+    if (dtype == FLAREPP_F32) {
+        FLAREPP_CP_MERGE(float)
+    } else if (dtype == FLAREPP_F16) {
+        FLAREPP_CP_MERGE(__half)
+    } else {
+        FLAREPP_CP_MERGE(__nv_bfloat16)
+    }
+#undef FLAREPP_CP_MERGE
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
+int cp_decode(const void* q, int q_shared, const void* z_state, const void* k, void* y, int B, int H, int N, int M,
+              int D, int dtype, const flarepp_options_t* opts, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    Plan pl{};
+    int rc = make_plan(s, opts, &pl);
+    if (rc) return rc;
+    if (!q || !z_state || !k || !y || (q_shared != 0 && q_shared != 1)) return FLAREPP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(z_state) || !aligned16(k) || !aligned16(y)) return FLAREPP_ERR_INVALID_ARG;
+    const size_t tb = s.tok_bytes();
+    if (overlaps(y, tb, k, tb) || overlaps(y, tb, z_state, latent_state_bytes(s)) ||
+        overlaps(y, tb, q, q_shared ? s.lat_bytes() : latent_state_bytes(s)))
+        return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const char* q16 = q_shared ? static_cast<const char*>(q) : static_cast<const char*>(q) + latent_16_offset(s);
+    const char* z16 = static_cast<const char*>(z_state) + latent_16_offset(s);
+    if (pl.path == FLAREPP_PATH_TCGEN05) {
+        const tc::Problem pr = tc_problem(s, pl);
+        rc = dtype == FLAREPP_F16 ? tc::cp_decode<__half>(pr, q16, q_shared, z16, k, y, st)
+                                  : tc::cp_decode<__nv_bfloat16>(pr, q16, q_shared, z16, k, y, st);
+        return rc ? (rc == 2 ? FLAREPP_ERR_UNSUPPORTED : FLAREPP_ERR_CUDA) : FLAREPP_OK;
+    }
+    const float* z32 = static_cast<const float*>(z_state);
+    if (dtype == FLAREPP_F32) return simt_cp_decode<float>(s, pl, q, q_shared, z32, k, y, st);
+    if (dtype == FLAREPP_F16) return simt_cp_decode<__half>(s, pl, q, q_shared, z32, k, y, st);
+    return simt_cp_decode<__nv_bfloat16>(s, pl, q, q_shared, z32, k, y, st);
+}
+
 }  // namespace
 }  // namespace flarepp
 
@@ -591,6 +823,33 @@ int flarepp_check_device_status(void* stream) {
         if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FLAREPP_ERR_CUDA;
     }
     return code;
+}
+
+size_t flarepp_cp_triple_bytes(int B, int H, int M, int D) {
+    const Shape s{B, H, 1, M, D, FLAREPP_F32};
+    if (check_shape(s)) return 0;
+    return (size_t)s.bh() * M * (D + 2) * sizeof(float);
+}
+
+size_t flarepp_cp_latent_bytes(int B, int H, int M, int D, int dtype) {
+    const Shape s{B, H, 1, M, D, dtype};
+    if (check_shape(s)) return 0;
+    return latent_state_bytes(s);
+}
+
+int flarepp_cp_partials(const void* q, int q_shared, const void* k, const void* v, float* triple, int B, int H,
+                        int N, int M, int D, int dtype, const flarepp_options_t* opts, void* stream) {
+    return cp_partials(q, q_shared, k, v, triple, B, H, N, M, D, dtype, opts, stream);
+}
+
+int flarepp_cp_merge(const float* gathered, int ranks, const void* q_fixed, const float* gate, void* state, int B,
+                     int H, int M, int D, int dtype, void* stream) {
+    return cp_merge(gathered, ranks, q_fixed, gate, state, B, H, M, D, dtype, stream);
+}
+
+int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const void* k, void* y, int B, int H, int N,
+                      int M, int D, int dtype, const flarepp_options_t* opts, void* stream) {
+    return cp_decode(q, q_shared, z_state, k, y, B, H, N, M, D, dtype, opts, stream);
 }
 
 int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate, const void* k0,

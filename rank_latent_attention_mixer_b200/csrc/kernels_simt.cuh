@@ -123,12 +123,18 @@ split_partial_simt(SplitParams p) {
 // Merge of the per-chunk triples of one latent row (one warp per row):
 // out = sum_c 2^(m_c - m*) O_c / sum_c 2^(m_c - m*) l_c with m* = max_c m_c.
 // Synthesis epilogue: q = q_fixed + gate[h] * out (FLARE.py README, FLARE++
-// block, second line).  Encode epilogue: z = out.
-enum MergeMode { kMergeSynthesis = 0, kMergeEncode = 1 };
+// block, second line).  Encode epilogue: z = out.  Triple mode writes the
+// combined triple itself (m*, L = sum_c 2^(m_c - m*) l_c, sum_c 2^(m_c - m*)
+// O_c) unnormalised: the local step of the token-sharded form, whose triples
+// are merged again across ranks.
+enum MergeMode { kMergeSynthesis = 0, kMergeEncode = 1, kMergeTriple = 2 };
 
 struct MergeParams {
-    const float* part_O;
-    const float2* part_ml;
+    const float* part_O;        // part c's O row r at part_O + c*o_part_stride + r*D
+    const float2* part_ml;      // part c's (m, l) of row r at part_ml[c*ml_part_stride + r]
+    int64_t o_part_stride;      // floats; 0 = B*H*M*D (parts stored back to back)
+    int64_t ml_part_stride;     // float2s; 0 = B*H*M
+    float2* out_ml;             // triple mode: combined (m*, L) per row
     int chunks;
     int B, H, M;
     int mode;                   // MergeMode
@@ -158,10 +164,11 @@ merge_partials(MergeParams p) {
     if (row >= rows) return;
     const int m = (int)(row % p.M);
     const int h = (int)((row / p.M) % p.H);
-    const int64_t cstride = rows;               // rows per chunk slab
+    const int64_t ostride = p.o_part_stride ? p.o_part_stride : rows * D;
+    const int64_t mlstride = p.ml_part_stride ? p.ml_part_stride : rows;
 
     float mstar = -INFINITY;
-    for (int c = lane; c < p.chunks; c += 32) mstar = fmaxf(mstar, p.part_ml[c * cstride + row].x);
+    for (int c = lane; c < p.chunks; c += 32) mstar = fmaxf(mstar, p.part_ml[c * mlstride + row].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
 
@@ -173,8 +180,8 @@ merge_partials(MergeParams p) {
     for (int c0 = 0; c0 < p.chunks; c0 += CPI) {
         const int c = c0 + sub;
         if (c < p.chunks) {
-            const float2 ml = p.part_ml[c * cstride + row];
-            const float4* o4 = reinterpret_cast<const float4*>(p.part_O + (c * cstride + row) * D);
+            const float2 ml = p.part_ml[c * mlstride + row];
+            const float4* o4 = reinterpret_cast<const float4*>(p.part_O + c * ostride + row * D);
             const float w = ml.y > 0.f ? ex2_mufu(ml.x - mstar) : 0.f;   // empty chunk contributes nothing
             L = fmaf(w, ml.y, L);
 #pragma unroll
@@ -198,6 +205,13 @@ merge_partials(MergeParams p) {
         }
     }
     if (sub != 0) return;
+    if (p.mode == kMergeTriple) {
+#pragma unroll
+        for (int i = 0; i < F4PL; ++i)
+            reinterpret_cast<float4*>(p.out_f32 + row * D)[li + LPC * i] = acc[i];
+        if (li == 0) p.out_ml[row] = make_float2(mstar, L);
+        return;
+    }
     const float inv = 1.f / L;
     const T* qf = reinterpret_cast<const T*>(p.q_fixed) + ((int64_t)h * p.M + m) * D;
 #pragma unroll

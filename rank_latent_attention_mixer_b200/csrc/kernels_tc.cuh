@@ -1160,5 +1160,83 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
+// ------------------------------------------------------------------ token-sharded stages
+//
+// The token-sharded (context-parallel) form: every rank runs the split passes
+// on its own tokens, reduces its chunks to one triple per latent row, and the
+// ranks' triples are merged after an all-gather (physicsnemo issue #2024,
+// section 2: latent-sized outputs and log-sum-exp statistics rebuild the
+// globally normalised attention; decoding stays local).
+
+// One split pass over this rank's tokens, reduced to one unnormalised triple
+// per latent row: O at triple[0, rows*D), (m, l) as float2 at triple + rows*D.
+// q is [H,M,D] (q_shared) or [B,H,M,D]; v == k reads each tile once (synthesis).
+template <typename E>
+int cp_split(const Problem& pr, const Buffers& bu, const void* q, bool q_shared, const void* kk, const void* vv,
+             float* triple, cudaStream_t st) {
+    const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
+    const CUtensorMapDataType ty = Elem<E>::kMapType;
+    const bool kv_same = kk == vv;
+    CUtensorMap mq, mk, mv;
+    bool ok = make_map(&mq, ty, q, M, H, q_shared ? 1 : B, D, contiguous_rows(M, H, D), kQTile) &&
+              make_map(&mk, ty, kk, N, H, B, D, pr.tok, kSplitKT) &&
+              make_map(&mv, ty, vv, N, H, B, D, pr.tok, kSplitKT);
+    if (!ok) return 3;
+    Params sp{};
+    sp.mode = kSplit;
+    sp.B = B; sp.H = H; sp.M = M; sp.N = N;
+    sp.kv_rows = N; sp.kv_tiles = (N + kSplitKT - 1) / kSplitKT;
+    sp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
+    sp.q_shared = q_shared ? 1 : 0; sp.k_shared = 0; sp.kv_same = kv_same ? 1 : 0;
+    sp.interleave = interleaved(M) ? 1 : 0;
+    sp.row_groups = row_groups(M);
+    sp.chunks = pr.chunks;
+    sp.chunk_tiles = pr.chunk_len / kSplitKT;
+    sp.items = BH * pr.chunks * sp.row_groups;
+    sp.scale_log2 = pr.scale_log2;
+    sp.part_O = bu.part_O;
+    sp.part_ml = bu.part_ml;
+    int rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, mq, mk, kv_same ? mk : mv, sp, st);
+    if (rc) return rc;
+    const int64_t rows = (int64_t)BH * M;
+    MergeParams mp{};
+    mp.part_O = bu.part_O; mp.part_ml = bu.part_ml; mp.chunks = pr.chunks * parts_per_chunk(M);
+    mp.B = B; mp.H = H; mp.M = M;
+    mp.mode = kMergeTriple;
+    mp.out_f32 = triple;
+    mp.out_ml = reinterpret_cast<float2*>(triple + rows * D);
+    launch_merge_d<E>(D, mp, rows, st);
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
+// Decode of this rank's tokens against the merged latents: keys q ([H,M,D]
+// when q_shared, else the [B,H,M,D] routing queries) and values z [B,H,M,D].
+template <typename E>
+int cp_decode(const Problem& pr, const void* q, bool q_shared, const void* z16, const void* kk, void* y,
+              cudaStream_t st) {
+    const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
+    const CUtensorMapDataType ty = Elem<E>::kMapType;
+    CUtensorMap mq, mk, mv;
+    bool ok = make_map(&mq, ty, kk, N, H, B, D, pr.tok, kQTile) &&
+              make_map(&mk, ty, q, M, H, q_shared ? 1 : B, D, contiguous_rows(M, H, D), kDecodeKT) &&
+              make_map(&mv, ty, z16, M, H, B, D, contiguous_rows(M, H, D), kDecodeKT);
+    if (!ok) return 3;
+    Params dp{};
+    dp.mode = kDecode;
+    dp.B = B; dp.H = H; dp.M = M; dp.N = N;
+    dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
+    dp.q_shared = 0; dp.k_shared = q_shared ? 1 : 0; dp.kv_same = 0;
+    dp.interleave = 0;
+    dp.q_groups = (N + kDecodeNW * kQTile - 1) / (kDecodeNW * kQTile);
+    dp.items = BH * dp.q_groups;
+    dp.scale_log2 = pr.scale_log2;
+    dp.y = y;
+    dp.y_row = pr.tok.row; dp.y_h = pr.tok.h; dp.y_b = pr.tok.b;
+    dp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
+    int rc = launch_attn_d<E, kDecodeNW, kDecodeKT>(D, mq, mk, mv, dp, st);
+    if (rc) return rc;
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
 }  // namespace tc
 }  // namespace flarepp

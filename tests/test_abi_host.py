@@ -124,3 +124,22 @@ def test_workspace_and_path_queries(lib):
 def test_flare_entry_checks(lib):
     assert lib.lib.flare_fwd(None, FAKE[4], FAKE[5], FAKE[6], 1, 2, 64, 16, 16, 1, None) == 1
     assert lib.lib.flare_fwd(FAKE[1], FAKE[4], FAKE[5], FAKE[6], 1, 2, 64, 16, 40, 1, None) == 2
+
+
+def test_token_sharded_entries_checked(lib):
+    assert lib.cp_triple_bytes(1, 2, 16, 16) == 1 * 2 * 16 * 18 * 4
+    assert lib.cp_latent_bytes(1, 2, 16, 16, lib.F32) == 2048
+    assert lib.cp_latent_bytes(1, 2, 16, 16, lib.BF16) == 2048 + 1024
+    assert lib.cp_triple_bytes(1, 2, 16, 48) == 0                       # D outside the supported set
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    merge = lib.lib.flarepp_cp_merge
+    merge.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, vp]
+    assert merge(FAKE[4], 0, None, None, FAKE[6], 1, 2, 16, 16, 1, None) == 1     # no ranks
+    assert merge(FAKE[4], 2, None, FAKE[2], FAKE[6], 1, 2, 16, 16, 1, None) == 1  # gate without q_fixed
+    part = lib.lib.flarepp_cp_partials
+    part.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, vp, vp]
+    assert part(FAKE[1], 2, FAKE[4], FAKE[5], FAKE[6], 1, 2, 64, 16, 16, 1, None, None) == 1   # q_shared not 0/1
+    assert part(FAKE[1], 1, FAKE[4], FAKE[5], None, 1, 2, 64, 16, 16, 1, None, None) == 1      # no triple
+    dec = lib.lib.flarepp_cp_decode
+    dec.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, vp, vp]
+    assert dec(FAKE[1], 1, FAKE[3], FAKE[4], FAKE[4], 1, 2, 64, 16, 16, 1, None, None) == 1   # y aliases k
