@@ -759,7 +759,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 if (lane == 0) mbar_arrive(&sfree[wg]);
 
                 const int valid = p.kv_rows - t * KT;             // key/value rows of this tile that exist
-                if (valid < KT) {                                 // ragged last tile only (warp-uniform)
+                if (__builtin_expect(valid < KT, 0)) {            // ragged last tile only (warp-uniform)
 #pragma unroll
                     for (int c = 0; c < LY::kChunks; ++c)
 #pragma unroll
@@ -782,7 +782,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const float m_new = fmaxf(m_run, mx * sl2 - Elem<E>::kPBias);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
-                if (resc) {
+                if (__builtin_expect(resc, 0)) {
                     factor = ex2_mufu(m_run - m_new);
                     m_run = m_new;
                 }
@@ -817,11 +817,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 if (!ok) break;
                 tc_fence_after();
-                if (pend) {
+                // P row -> TMEM (this thread's lane, KT/2 columns of packed pairs)
+#pragma unroll
+                for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
+                // Rare work on O, after P is out of the registers and before the
+                // value MMA of this job adds to O: the previous item's O row (first
+                // job of an item), or the O rescale of a grown running max.
+                if (__builtin_expect(pend, 0)) {
                     flush(pend_it, pend_jobs, pend_m, pend_l);
                     pend = false;
                 }
-                if (__any_sync(0xffffffffu, resc && njobs > 0)) {
+                if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0)) {
                     const float f = njobs > 0 ? factor : 1.f;
 #pragma unroll
                     for (int c = 0; c < D / 32 + (D % 32 ? 1 : 0); ++c) {
@@ -833,9 +839,6 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         tmem_st32(tO + c * 32, o);
                     }
                 }
-                // P row -> TMEM (this thread's lane, KT/2 columns of packed pairs)
-#pragma unroll
-                for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
