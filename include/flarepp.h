@@ -80,8 +80,8 @@ typedef enum flarepp_status {
 } flarepp_status_t;
 
 /* Kernel family.  AUTO picks the tcgen05 tensor-core kernels for 16-bit I/O
- * (bf16 or fp16) with D in {16,32,64} and the SIMT (FFMA) kernels otherwise
- * (all fp32 I/O: TF32 products would not meet fp32 accuracy). */
+ * (bf16 or fp16, every supported D) and the SIMT (FFMA) kernels for fp32 I/O
+ * (TF32 products would not meet fp32 accuracy). */
 typedef enum flarepp_path {
     FLAREPP_PATH_AUTO = 0,
     FLAREPP_PATH_SIMT = 1,

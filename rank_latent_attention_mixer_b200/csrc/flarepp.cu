@@ -94,7 +94,7 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
         pl->row_blocks = (s.M + kSimtThreads - 1) / kSimtThreads;
         units_per_bh = pl->row_blocks;
     } else {
-        tile = tc::kv_tile();
+        tile = tc::kv_tile(s.D);
         pl->row_blocks = tc::row_groups(s.M);
         units_per_bh = pl->row_blocks;
     }

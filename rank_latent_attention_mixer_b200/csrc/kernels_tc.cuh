@@ -378,10 +378,19 @@ struct Smem {
 
 template <int D, int NW, int KT>
 struct Layout {
-    // swizzle of a [rows x D] 16-bit tile whose rows are D*2 bytes
-    static constexpr uint32_t kType = D == 64 ? kLayoutSw128 : (D == 32 ? kLayoutSw64 : kLayoutSw32);
-    static constexpr uint32_t kRowBytes = D * 2;
+    // A [rows x D] 16-bit tile is stored as D/64 column blocks of [rows x 64]
+    // when D = 128 (a swizzle atom spans at most 128 bytes), else as one block;
+    // every block has rows of kRowBytes, swizzled by the same amount.
+    static constexpr int kBlocks = D > 64 ? D / 64 : 1;
+    static constexpr uint32_t kRowBytes = D > 64 ? 128 : D * 2;
+    static constexpr uint32_t kType = kRowBytes == 128 ? kLayoutSw128 : (kRowBytes == 64 ? kLayoutSw64 : kLayoutSw32);
     static constexpr uint32_t kSbo = 8 * kRowBytes;                  // 8-row group stride
+    static constexpr uint32_t kQBlockBytes = kQTile * kRowBytes;     // one column block of a query tile
+    static constexpr uint32_t kKVBlockBytes = KT * kRowBytes;        // one column block of a key/value tile
+    // byte offset of the K-step kk (16 columns) of a K-major tile with `block` bytes per column block
+    static __device__ __forceinline__ uint32_t kstep(int kk, uint32_t block) {
+        return (kk & 3) * 32 + (kk >> 2) * block;
+    }
     // TMEM: O accumulators at least 32 columns apart so that 32-column TMEM
     // loads/stores of one never touch another's
     static constexpr int kOStride = D < 32 ? 32 : D;
@@ -399,7 +408,7 @@ template <typename E, int D, int NW, int KT, int NST, int QS>
 __global__ void __launch_bounds__(Regs<NW>::kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const Params p) {
-    static_assert(D == 16 || D == 32 || D == 64, "tcgen05 path covers D in {16, 32, 64}");
+    static_assert(D == 16 || D == 32 || D == 64 || D == 128, "tcgen05 path covers D in {16, 32, 64, 128}");
     static_assert(KT == 64 || KT == 128, "key/value tiles of 64 or 128 rows");
     static_assert(NW >= 1 && NW <= 3, "the producer warpgroup holds one TMA warp and NW MMA warps");
     static_assert(NST >= 3, "at least three key/value stages");
@@ -488,10 +497,14 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 uint8_t* qdst = smem + SM::kQ + slot * NW * SM::kQTileBytes;
                 for (int qt = 0; qt < q_tiles; ++qt) {
                     const int qrow = it.qrow0 + qt * kQTile;
-                    if (p.mode == kDecode && p.tok_heads_inner)      // token queries, [B,N,H,D]
-                        tma_load_4d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, it.h, qrow, it.qb);
-                    else
-                        tma_load_4d(qdst + qt * SM::kQTileBytes, &map_q, &q_full[slot], 0, qrow, it.h, it.qb);
+#pragma unroll
+                    for (int cb = 0; cb < LY::kBlocks; ++cb) {
+                        uint8_t* dst = qdst + qt * SM::kQTileBytes + cb * LY::kQBlockBytes;
+                        if (p.mode == kDecode && p.tok_heads_inner)  // token queries, [B,N,H,D]
+                            tma_load_4d(dst, &map_q, &q_full[slot], cb * 64, it.h, qrow, it.qb);
+                        else
+                            tma_load_4d(dst, &map_q, &q_full[slot], cb * 64, qrow, it.h, it.qb);
+                    }
                 }
                 q_last_phase[slot] = (q_load / QS) & 1;
                 ++q_load;
@@ -512,10 +525,14 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     mbar_expect_tx(&kv_full[st], kv_bytes);
                     uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kKVTileBytes;
                     const bool hi = p.mode == kSplit && p.tok_heads_inner;   // token keys/values, [B,N,H,D]
-                    tma_load_4d(kdst, &map_k, &kv_full[st], 0, hi ? it.h : t * KT, hi ? t * KT : it.h, it.kb);
-                    if (!p.kv_same)
-                        tma_load_4d(kdst + SM::kKVTileBytes, &map_v, &kv_full[st], 0, hi ? it.h : t * KT,
-                                    hi ? t * KT : it.h, it.vb);
+#pragma unroll
+                    for (int cb = 0; cb < LY::kBlocks; ++cb) {
+                        tma_load_4d(kdst + cb * LY::kKVBlockBytes, &map_k, &kv_full[st], cb * 64,
+                                    hi ? it.h : t * KT, hi ? t * KT : it.h, it.kb);
+                        if (!p.kv_same)
+                            tma_load_4d(kdst + SM::kKVTileBytes + cb * LY::kKVBlockBytes, &map_v, &kv_full[st],
+                                        cb * 64, hi ? it.h : t * KT, hi ? t * KT : it.h, it.vb);
+                    }
                     kv_last_phase[st] = fill & 1;
                     ++kv_load;
                 }
@@ -619,8 +636,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const uint32_t d_tmem = tmem + w * KT;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = smem_desc(qaddr + kk * 32, 16, LY::kSbo, LY::kType);
-                    const uint64_t bd = smem_desc(kaddr + kk * 32, 16, LY::kSbo, LY::kType);
+                    const uint64_t ad = smem_desc(qaddr + LY::kstep(kk, LY::kQBlockBytes), 16, LY::kSbo, LY::kType);
+                    const uint64_t bd = smem_desc(kaddr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
                     umma_f16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sfull[w]);
@@ -644,7 +661,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     // A = P in TMEM: 16 key/value columns = 8 columns of packed pairs per step
                     // B = V tile [KT kv x D], D contiguous: MN-major; 16 kv rows per step
                     // (D fits one swizzle atom along MN, so the leading offset is never used)
-                    const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, SM::kKVTileBytes,
+                    // (D = 128: the two 64-column blocks are the MN atoms, kKVBlockBytes apart)
+                    const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, LY::kKVBlockBytes,
                                                   LY::kSbo, LY::kType);
                     umma_f16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
                 }
@@ -919,8 +937,8 @@ template <int D, int NW_, int KT_>
 struct Config {
     static constexpr int NW = NW_;
     static constexpr int KT = KT_;
-    static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 64 ? 4 : 6);
-    static constexpr int QS = 2;
+    static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 128 ? 4 : (D == 64 ? 4 : 6));
+    static constexpr int QS = D == 128 ? 1 : 2;
     using SM = Smem<D, NW, KT, NST, QS>;
     // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
     static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
@@ -930,13 +948,18 @@ constexpr int kDecodeNW = 3, kDecodeKT = 64;
 
 inline bool supported(bool io16, int D, int M) {
     (void)M;
-    return io16 && (D == 16 || D == 32 || D == 64);
+    return io16 && (D == 16 || D == 32 || D == 64 || D == 128);
 }
+
+// D = 128 keeps two warpgroups in both passes on 64-row tiles (TMEM: 2 x (64
+// score + 128 accumulator + 32 weight columns) = 448 of 512).
+inline int split_kt(int D) { return D == 128 ? 64 : kSplitKT; }
+inline int decode_nw(int D) { return D == 128 ? 2 : kDecodeNW; }
 
 // Split-pass plan.  With one 128-row tile holding all M latents, the two
 // warpgroups share it and take the key/value tiles round-robin (interleaved,
 // two partial triples per chunk); otherwise each takes its own 128 latents.
-inline int kv_tile() { return kSplitKT; }
+inline int kv_tile(int D) { return split_kt(D); }
 inline bool interleaved(int M) { return M <= kQTile; }
 inline int row_groups(int M) {
     return interleaved(M) ? (M + kQTile - 1) / kQTile : (M + kSplitNW * kQTile - 1) / (kSplitNW * kQTile);
@@ -997,11 +1020,12 @@ inline bool make_map(CUtensorMap* map, CUtensorMapDataType type, const void* bas
                                 (cuuint64_t)(heads_inner ? rows : H), (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)(heads_inner ? str.h : str.row) * 2,
                                    (cuuint64_t)(heads_inner ? str.row : str.h) * 2, (cuuint64_t)str.b * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)D, heads_inner ? 1u : (cuuint32_t)box_rows,
-                               heads_inner ? (cuuint32_t)box_rows : 1u, 1};
+    // a box holds one column block: all D columns, or 64 of them when D = 128
+    const cuuint32_t bx = D > 64 ? 64u : (cuuint32_t)D;
+    const cuuint32_t box[4] = {bx, heads_inner ? 1u : (cuuint32_t)box_rows, heads_inner ? (cuuint32_t)box_rows : 1u, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                          : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    const CUtensorMapSwizzle sw = bx == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (bx == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     return fn(map, type, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1056,6 +1080,20 @@ inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, co
     }
 }
 
+template <typename E>
+inline int launch_split(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const Params& prm, cudaStream_t st) {
+    if (D == 128) return launch_attn<E, 128, 2, 64>(mq, mk, mv, prm, st);
+    return launch_attn_d<E, kSplitNW, kSplitKT>(D, mq, mk, mv, prm, st);
+}
+
+template <typename E>
+inline int launch_decode(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const Params& prm, cudaStream_t st) {
+    if (D == 128) return launch_attn<E, 128, 2, 64>(mq, mk, mv, prm, st);
+    return launch_attn_d<E, kDecodeNW, kDecodeKT>(D, mq, mk, mv, prm, st);
+}
+
 template <typename E, int D>
 void launch_merge(const MergeParams& mp, int64_t rows, cudaStream_t st) {
     // the attention kernels run with the largest shared-memory carveout; the
@@ -1071,7 +1109,8 @@ inline void launch_merge_d(int D, const MergeParams& mp, int64_t rows, cudaStrea
     switch (D) {
         case 16: launch_merge<E, 16>(mp, rows, st); break;
         case 32: launch_merge<E, 32>(mp, rows, st); break;
-        default: launch_merge<E, 64>(mp, rows, st); break;
+        case 64: launch_merge<E, 64>(mp, rows, st); break;
+        default: launch_merge<E, 128>(mp, rows, st); break;
     }
 }
 
@@ -1093,15 +1132,15 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
               make_map(&m_q16_q, ty, bu.q16, M, H, B, D, latb, kQTile) &&
               make_map(&m_q16_kv, ty, bu.q16, M, H, B, D, latb, kDecodeKT) &&
               make_map(&m_z16, ty, bu.z16, M, H, B, D, latb, kDecodeKT) &&
-              make_map(&m_k_kv, ty, k, N, H, B, D, tok, kSplitKT) && make_map(&m_k_q, ty, k, N, H, B, D, tok, kQTile) &&
-              make_map(&m_v, ty, v, N, H, B, D, tok, kSplitKT);
+              make_map(&m_k_kv, ty, k, N, H, B, D, tok, split_kt(D)) && make_map(&m_k_q, ty, k, N, H, B, D, tok, kQTile) &&
+              make_map(&m_v, ty, v, N, H, B, D, tok, split_kt(D));
     if (gated)
         ok = ok && make_map(&m_q0, ty, q0, M, H, 1, D, lat1, kQTile) &&
-             make_map(&m_k0, ty, k0, N, H, B, D, tok, kSplitKT);
+             make_map(&m_k0, ty, k0, N, H, B, D, tok, split_kt(D));
     if (!ok) return 3;
 
-    const int kv_tiles = (N + kSplitKT - 1) / kSplitKT;
-    const int chunk_tiles = pr.chunk_len / kSplitKT;
+    const int kv_tiles = (N + split_kt(D) - 1) / split_kt(D);
+    const int chunk_tiles = pr.chunk_len / split_kt(D);
     Params sp{};
     sp.mode = kSplit;
     sp.B = B; sp.H = H; sp.M = M; sp.N = N;
@@ -1127,7 +1166,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     if (gated) {
         Params s1 = sp;
         s1.q_shared = 1; s1.k_shared = 0; s1.kv_same = 1;
-        rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, m_q0, m_k0, m_k0, s1, st);
+        rc = launch_split<E>(D, m_q0, m_k0, m_k0, s1, st);
         if (rc) return rc;
         mark(st);
         mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_16 = bu.q16; mp.user_out = q_out;
@@ -1137,7 +1176,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     }
     Params s2 = sp;
     s2.q_shared = gated ? 0 : 1; s2.k_shared = 0; s2.kv_same = 0;
-    rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, gated ? m_q16_q : m_qf_q, m_k_kv, m_v, s2, st);
+    rc = launch_split<E>(D, gated ? m_q16_q : m_qf_q, m_k_kv, m_v, s2, st);
     if (rc) return rc;
     mark(st);
     mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_16 = bu.z16; mp.user_out = z_out;
@@ -1151,13 +1190,13 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
     dp.q_shared = 0; dp.k_shared = gated ? 0 : 1; dp.kv_same = 0;
     dp.interleave = 0;
-    dp.q_groups = (N + kDecodeNW * kQTile - 1) / (kDecodeNW * kQTile);
+    dp.q_groups = (N + decode_nw(D) * kQTile - 1) / (decode_nw(D) * kQTile);
     dp.items = BH * dp.q_groups;
     dp.scale_log2 = pr.scale_log2;
     dp.y = y;
     dp.y_row = tok.row; dp.y_h = tok.h; dp.y_b = tok.b;
     dp.tok_heads_inner = tok.h < tok.row ? 1 : 0;
-    rc = launch_attn_d<E, kDecodeNW, kDecodeKT>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
+    rc = launch_decode<E>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
     if (rc) return rc;
     mark(st);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
@@ -1182,24 +1221,24 @@ int cp_split(const Problem& pr, const Buffers& bu, const void* q, bool q_shared,
     const bool kv_same = kk == vv;
     CUtensorMap mq, mk, mv;
     bool ok = make_map(&mq, ty, q, M, H, q_shared ? 1 : B, D, contiguous_rows(M, H, D), kQTile) &&
-              make_map(&mk, ty, kk, N, H, B, D, pr.tok, kSplitKT) &&
-              make_map(&mv, ty, vv, N, H, B, D, pr.tok, kSplitKT);
+              make_map(&mk, ty, kk, N, H, B, D, pr.tok, split_kt(D)) &&
+              make_map(&mv, ty, vv, N, H, B, D, pr.tok, split_kt(D));
     if (!ok) return 3;
     Params sp{};
     sp.mode = kSplit;
     sp.B = B; sp.H = H; sp.M = M; sp.N = N;
-    sp.kv_rows = N; sp.kv_tiles = (N + kSplitKT - 1) / kSplitKT;
+    sp.kv_rows = N; sp.kv_tiles = (N + split_kt(D) - 1) / split_kt(D);
     sp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
     sp.q_shared = q_shared ? 1 : 0; sp.k_shared = 0; sp.kv_same = kv_same ? 1 : 0;
     sp.interleave = interleaved(M) ? 1 : 0;
     sp.row_groups = row_groups(M);
     sp.chunks = pr.chunks;
-    sp.chunk_tiles = pr.chunk_len / kSplitKT;
+    sp.chunk_tiles = pr.chunk_len / split_kt(D);
     sp.items = BH * pr.chunks * sp.row_groups;
     sp.scale_log2 = pr.scale_log2;
     sp.part_O = bu.part_O;
     sp.part_ml = bu.part_ml;
-    int rc = launch_attn_d<E, kSplitNW, kSplitKT>(D, mq, mk, kv_same ? mk : mv, sp, st);
+    int rc = launch_split<E>(D, mq, mk, kv_same ? mk : mv, sp, st);
     if (rc) return rc;
     const int64_t rows = (int64_t)BH * M;
     MergeParams mp{};
@@ -1230,13 +1269,13 @@ int cp_decode(const Problem& pr, const void* q, bool q_shared, const void* z16, 
     dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
     dp.q_shared = 0; dp.k_shared = q_shared ? 1 : 0; dp.kv_same = 0;
     dp.interleave = 0;
-    dp.q_groups = (N + kDecodeNW * kQTile - 1) / (kDecodeNW * kQTile);
+    dp.q_groups = (N + decode_nw(D) * kQTile - 1) / (decode_nw(D) * kQTile);
     dp.items = BH * dp.q_groups;
     dp.scale_log2 = pr.scale_log2;
     dp.y = y;
     dp.y_row = pr.tok.row; dp.y_h = pr.tok.h; dp.y_b = pr.tok.b;
     dp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
-    int rc = launch_attn_d<E, kDecodeNW, kDecodeKT>(D, mq, mk, mv, dp, st);
+    int rc = launch_decode<E>(D, mq, mk, mv, dp, st);
     if (rc) return rc;
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }

@@ -87,6 +87,9 @@ WORKLOADS: Dict[str, Workload] = {
                  device_rng=True, note="scale1m_bf16 with fp16 I/O"),
         Workload("cloud40k_f16", 1, 8, 40000, 256, 32, "f16", 3, "clusters", False, False,
                  note="cloud40k_bf16 with fp16 I/O"),
+        # head dim 128 (outside the configs above): the widest supported D
+        Workload("scale256k_d128_bf16", 1, 8, 262144, 256, 128, "bf16", 5, "iid", True, True,
+                 device_rng=True, note="head dim 128, 256K tokens"),
     ]
 }
 ORDER = ["tiny_f32", "grid85_bf16", "grid129_peaky_bf16", "cloud40k_bf16", "scale1m_bf16"]

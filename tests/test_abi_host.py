@@ -115,9 +115,11 @@ def test_workspace_and_path_queries(lib):
     a = lib.workspace_bytes(1, 8, 100000, 64, 32, lib.BF16, force_chunks=1)
     b = lib.workspace_bytes(1, 8, 100000, 64, 32, lib.BF16, force_chunks=16)
     assert 0 < a < b
-    # fp16 I/O plans like bf16: the tcgen05 path for D in {16, 32, 64}, SIMT for D = 128
+    # 16-bit I/O plans the tcgen05 path for every supported D; fp32 the SIMT path
     assert lib.selected_path(1, 8, 100000, 64, 32, lib.F16) == lib.PATH_TCGEN05
-    assert lib.selected_path(1, 8, 100000, 64, 128, lib.F16) == lib.PATH_SIMT
+    assert lib.selected_path(1, 8, 100000, 64, 128, lib.F16) == lib.PATH_TCGEN05
+    assert lib.selected_path(1, 8, 100000, 64, 128, lib.BF16) == lib.PATH_TCGEN05
+    assert lib.selected_path(1, 8, 100000, 64, 128, lib.F32) == lib.PATH_SIMT
     assert lib.workspace_bytes(1, 8, 100000, 64, 32, lib.F16) == lib.workspace_bytes(1, 8, 100000, 64, 32, lib.BF16)
 
 

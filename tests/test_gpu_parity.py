@@ -90,6 +90,9 @@ EDGE = [
     (1, 1, 4097, 256, 32),
     (1, 2, 2000, 512, 64),
     (1, 1, 640, 100, 32),
+    (2, 4, 3001, 256, 128),
+    (1, 2, 1000, 64, 128),
+    (1, 1, 5000, 512, 128),
 ]
 
 
