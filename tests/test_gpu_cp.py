@@ -68,6 +68,7 @@ CASES = [
     ((1, 8, 5000, 256, 64), "f16", 0),
     ((2, 2, 1000, 64, 16), "f32", 0),
     ((1, 3, 2000, 100, 64), "bf16", 1),
+    ((1, 4, 2000, 256, 128), "f16", 0),
 ]
 
 

@@ -111,7 +111,7 @@ def test_edge_shapes(shape, dtype):
 @pytest.mark.parametrize("dtype,path", [("bf16", 0), ("f16", 0), ("f32", 0), ("bf16", 1)],
                          ids=["bf16-auto", "f16-auto", "f32", "bf16-simt"])
 @pytest.mark.parametrize("shape", [(2, 3, 1000, 64, 32), (1, 8, 3001, 256, 64), (2, 2, 300, 17, 16),
-                                   (1, 1, 777, 130, 64)], ids=lambda s: "x".join(map(str, s)))
+                                   (1, 1, 777, 130, 64), (1, 2, 900, 128, 128)], ids=lambda s: "x".join(map(str, s)))
 def test_bnhd_layout(shape, dtype, path):
     """k0, k, v, y in [B,N,H,D] (one token's heads adjacent) give exactly the
     [B,H,N,D] result: only the addressing differs."""
