@@ -101,12 +101,29 @@ def sdpa(Q, K, V, scale: float = 0.0, plant: int = 0) -> np.ndarray:
     return O
 
 
+NORM_EPS = 1e-6
+
+
+def rms_normalise(x, eps: float = NORM_EPS, plant: int = 0) -> np.ndarray:
+    """Head-wise normalisation of the synthesis seeds and keys/values
+    (physicsnemo issue #2024, FLARE++ list: "Normalizing the synthesis call"),
+    read as RMS over the head dimension without a learned scale:
+    x / sqrt(mean_d x^2 + eps), row by row, in fp64.
+    Planted mistakes (test use): 11 divides by the row's L2 norm instead."""
+    x = _f64(x)
+    if plant == 11:
+        return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
 def flarepp(q0, q_fixed, gate, k0, k, v, scale: float = 0.0, flare: bool = False,
-            plant: int = 0):
+            plant: int = 0, norm_synthesis: bool = False):
     """Full mixer in fp64.  Returns (y [B,H,N,D], q [B,H,M,D], z [B,H,M,D]).
 
     ``gate`` is sigmoid(g) per head ([H]); ``gate=None`` or ``flare=True`` is the
-    closed gate, i.e. FLARE with q = q_fixed.
+    closed gate, i.e. FLARE with q = q_fixed.  ``norm_synthesis`` applies
+    rms_normalise to the seeds q0 and the synthesis keys/values k0 first.
+    Planted mistakes (test use): 12 normalises the seeds but not k0.
     """
     q_fixed, k, v = _f64(q_fixed), _f64(k), _f64(v)
     B, H, N, D = k.shape
@@ -115,6 +132,11 @@ def flarepp(q0, q_fixed, gate, k0, k, v, scale: float = 0.0, flare: bool = False
     closed = flare or gate is None
     q0a = None if closed else _f64(q0)
     k0a = None if closed else _f64(k0)
+    if norm_synthesis and not closed:
+        q0a = np.ascontiguousarray(rms_normalise(q0a, plant=plant))
+        if plant != 12:
+            k0a = np.ascontiguousarray(rms_normalise(k0a, plant=plant))
+    plant = plant if plant <= 10 else 0          # 11, 12 live above, not in the C build
     ga = None if closed else _f64(gate).reshape(H)
     if not closed:
         assert q0a.shape == (H, M, D) and k0a.shape == (B, H, N, D)

@@ -234,4 +234,39 @@ def pin_head_slice_entry(plant):
     return bool(_close(ys, y[1, 1, toks]) and _close(qs, q[1, 1]) and _close(zs, z[1, 1]))
 
 
+def _unit_rows(seed, shape):
+    """Rows of +-1 entries: mean of squares exactly 1 (RMS 1) in any dimension."""
+    return np.where(_rng(seed).standard_normal(shape) < 0, -1.0, 1.0)
+
+
+def pin_norm_scale_invariance(plant):
+    """Normalised seeds and synthesis keys/values do not depend on the scale of
+    q0 and k0 (inputs far from the epsilon)."""
+    q0, qf, gate, k0, k, v = _inputs(21, 2, 2, 40, 6, 16)
+    q0, k0 = q0 * 100.0, k0 * 100.0
+    _, qa, _ = oracle.flarepp(q0, qf, gate, k0, k, v, plant=plant, norm_synthesis=True)
+    _, qb, _ = oracle.flarepp(q0 * 3.0, qf, gate, k0 * 11.0, k, v, plant=plant, norm_synthesis=True)
+    return _close(qa, qb, 1e-8)
+
+
+def pin_norm_identical_keys(plant):
+    """Every synthesis key equal to c*u with u of RMS 1: the values are the
+    normalised key u, so q = q_fixed + gate * u."""
+    q0, qf, gate, k0, k, v = _inputs(22, 2, 3, 17, 4, 16)
+    u = _unit_rows(23, (2, 3, 1, 16))
+    k0 = np.broadcast_to(1000.0 * u, k0.shape).copy()
+    _, q, _ = oracle.flarepp(q0, qf, gate, k0, k, v, plant=plant, norm_synthesis=True)
+    return _close(q, qf[None] + gate[None, :, None, None] * u, 1e-10)
+
+
+def pin_norm_of_unit_rows(plant):
+    """Seeds and keys whose rows already have RMS 1 pass the normalisation
+    unchanged up to the epsilon (a factor 1/sqrt(1 + 1e-6))."""
+    q0, qf, gate, k0, k, v = _inputs(24, 1, 2, 33, 5, 32)
+    q0, k0 = _unit_rows(25, q0.shape), _unit_rows(26, k0.shape)
+    ya, qa, za = oracle.flarepp(q0, qf, gate, k0, k, v, plant=plant, norm_synthesis=True)
+    yb, qb, zb = oracle.flarepp(q0, qf, gate, k0, k, v, plant=plant)
+    return _close(qa, qb, 1e-5) and _close(ya, yb, 1e-5)
+
+
 PINS = {name[4:]: fn for name, fn in sorted(globals().items()) if name.startswith("pin_") and callable(fn)}

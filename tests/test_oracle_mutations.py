@@ -7,13 +7,15 @@ The mistakes are compiled into separate builds of the oracle's C file
   3 synthesis reads k instead of k0             8 q_fixed indexed by batch, not head
   4 encode uses the keys as values              9 exponent sign flipped
   5 decode swaps latent keys and values        10 softmax normalisation dropped
+ 11 synthesis normalisation by the L2 norm     12 synthesis keys/values not normalised
+(11 and 12 are planted in the oracle's Python normalisation step.)
 """
 import pytest
 
 import oracle
 from oracle_pins import PINS  # noqa: E402
 
-PLANTS = [1, 2, 3, 4, 5, 7, 8, 9, 10]
+PLANTS = [1, 2, 3, 4, 5, 7, 8, 9, 10, 11, 12]
 
 
 @pytest.mark.parametrize("plant", PLANTS)
