@@ -53,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--path", choices=["auto", "simt", "tcgen05"], default="auto")
     p.add_argument("--flare", action="store_true", help="closed gate: the two-call FLARE form (flare_fwd)")
+    p.add_argument("--norm", action="store_true",
+                   help="RMS-normalise q0 and k0 rows inside the synthesis pass (norm_synthesis)")
     p.add_argument("--cp", action="store_true",
                    help="token-sharded form: one global problem, each rank holds N/world tokens (strong scaling)")
     p.add_argument("--layout", choices=["bhnd", "bnhd"], default="bhnd",
@@ -278,17 +280,18 @@ def run_ours(args):
     dtype_code = {"f32": fb.F32, "bf16": fb.BF16, "f16": fb.F16}[w.dtype]
     used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
     gated = not args.flare
-    ws = torch.empty(fb.workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, gated, path), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(fb.workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, gated, path, layout=args.layout,
+                                        norm_synthesis=args.norm), dtype=torch.uint8, device=dev)
     y = torch.empty_like(x["k"])
-    n_launch = fb.launches_per_call(gated)
-    stage_names = STAGES_GATED if gated else STAGES_FLARE
+    norm = args.norm and gated
+    n_launch = fb.launches_per_call(gated) + (1 if norm else 0)
+    stage_names = (["rms_norm(q0, k0)"] if norm else []) + (STAGES_GATED if gated else STAGES_FLARE)
     fits_l2 = 5 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
 
     def step(events=None):
         fb.mixer_fwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y, path=path,
-                     workspace=ws, stage_events=events, layout=args.layout)
+                     workspace=ws, stage_events=events, layout=args.layout, norm_synthesis=args.norm)
 
     for _ in range(args.warmup):
         step()
@@ -330,7 +333,8 @@ def run_ours(args):
     total_stage = sum(avg_stage)
     stages = {stage_names[j]: {"ms": round(avg_stage[j], 4), "share": round(avg_stage[j] / total_stage, 4)}
               for j in range(n_launch)}
-    split_ms = statistics.mean([avg_stage[0], avg_stage[2]]) if gated else avg_stage[0]
+    o = 1 if norm else 0                   # the normalisation launch comes first
+    split_ms = statistics.mean([avg_stage[o], avg_stage[o + 2]]) if gated else avg_stage[0]
     bhnmd = w.B * w.H * w.N * w.M * w.D
     flops_per_split_launch = 4.0 * bhnmd
     peaks, peak_src = load_peaks()
@@ -377,6 +381,7 @@ def run_ours(args):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
                    "gate": "open (FLARE++)" if gated else "closed (FLARE, flare_fwd)",
                    "layout": args.layout,
+                   "synthesis_norm": bool(args.norm),
                    "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)"),

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define FLAREPP_ABI_VERSION 2
+#define FLAREPP_ABI_VERSION 3
 
 typedef enum flarepp_dtype {
     FLAREPP_F32 = 0,
@@ -113,6 +113,15 @@ typedef struct flarepp_options {
                                   and [i] after the i-th launch, for i < n_stage_events; lets a
                                   caller time each kernel on the stream it runs on            */
     int layout;              /* flarepp_layout_t of k0, k, v, y; other values -> INVALID_ARG  */
+    int norm_synthesis;      /* 1: head-wise RMS normalisation of the synthesis seeds and
+                                keys/values, q0 and k0 rows -> x / sqrt(mean_d x^2 + 1e-6)
+                                (no learned scale; physicsnemo issue #2024, FLARE++ list,
+                                "Normalizing the synthesis call"): one extra launch writes
+                                normalised copies into the workspace (which grows by the
+                                sizes of q0 and k0) and the synthesis reads them.  In
+                                flarepp_cp_partials it applies to that call, which must then
+                                be the synthesis (q_shared = 1, v == k).  Ignored with the
+                                gate closed.  0: none.  Other values -> INVALID_ARG          */
 } flarepp_options_t;
 
 /* Kernel launches one forward call makes (gated = 0: closed gate / FLARE).

@@ -37,7 +37,8 @@ class Options(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("path", ctypes.c_int), ("force_chunks", ctypes.c_int),
                 ("n_stage_events", ctypes.c_int), ("q_out", ctypes.c_void_p), ("z_out", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("layout", ctypes.c_int)]
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("layout", ctypes.c_int),
+                ("norm_synthesis", ctypes.c_int)]
 
 
 def _load() -> ctypes.CDLL:
@@ -66,8 +67,8 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
-if lib.flarepp_abi_version() != 2:
-    raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs 2: rebuild it")
+if lib.flarepp_abi_version() != 3:
+    raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs 3: rebuild it")
 
 
 def status_string(status: int) -> str:
@@ -121,8 +122,9 @@ def launches_per_call(gated: bool = True) -> int:
     return int(lib.flarepp_launches_per_call(int(gated)))
 
 
-def workspace_bytes(B, H, N, M, D, dtype=BF16, gated=True, path=PATH_AUTO, force_chunks=0, layout="bhnd") -> int:
-    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout])
+def workspace_bytes(B, H, N, M, D, dtype=BF16, gated=True, path=PATH_AUTO, force_chunks=0, layout="bhnd",
+                    norm_synthesis=False) -> int:
+    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout], int(norm_synthesis))
     return int(lib.flarepp_workspace_bytes(B, H, N, M, D, dtype, int(gated), ctypes.byref(o)))
 
 
@@ -132,7 +134,7 @@ def selected_path(B, H, N, M, D, dtype=BF16) -> int:
 
 def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: int = PATH_AUTO,
               force_chunks: int = 0, return_qz: bool = False, workspace: Optional[torch.Tensor] = None,
-              stage_events=None, layout: str = "bhnd"):
+              stage_events=None, layout: str = "bhnd", norm_synthesis: bool = False):
     """FLARE++ mixer forward on the current CUDA stream.  ``gate=None`` is FLARE.
 
     q0, q_fixed [H,M,D]; gate fp32 [H] (sigmoid already applied); k0, k, v and y
@@ -140,7 +142,8 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
     written in place); all on the same CUDA device, contiguous, fp32, bf16 or
     fp16.  Returns y (and q, z fp32 [B,H,M,D] when ``return_qz``).
     ``stage_events``: torch.cuda.Event objects (created with enable_timing)
-    recorded before the first launch and after each launch on the current stream."""
+    recorded before the first launch and after each launch on the current stream.
+    ``norm_synthesis``: RMS-normalise the q0 and k0 rows inside the synthesis pass."""
     B, H, N, M, D = _shapes(q_fixed, k, layout)
     _contig(q0, q_fixed, gate, k0, k, v, y)
     dt = _dtype_code(k)
@@ -152,7 +155,7 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
         z_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
     if gate is not None and gate.dtype != torch.float32:
         raise TypeError("gate must be float32 [H]")
-    need = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks, layout)
+    need = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks, layout, norm_synthesis)
     if need == 0:
         ws_ptr, ws_len = None, 0
     else:
@@ -170,7 +173,7 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
         ev_arr = (ctypes.c_void_p * n_ev)(*handles)
     o = Options(float(scale), int(path), int(force_chunks), n_ev, _ptr(q_out), _ptr(z_out), ws_ptr, ws_len,
                 ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None,
-                LAYOUTS[layout])
+                LAYOUTS[layout], int(norm_synthesis))
     rc = lib.flarepp_mixer_fwd_ex(_ptr(q0) if gate is not None else None, _ptr(q_fixed), _ptr(gate),
                                   _ptr(k0) if gate is not None else None, _ptr(k), _ptr(v), _ptr(y),
                                   B, H, N, M, D, dt, ctypes.byref(o), _stream(k.device))
@@ -247,19 +250,21 @@ def cp_latent_bytes(B, H, M, D, dtype) -> int:
     return int(fn(B, H, M, D, dtype))
 
 
-def _cp_options(path, scale, force_chunks, layout, workspace=None):
+def _cp_options(path, scale, force_chunks, layout, workspace=None, norm=False):
     ws_ptr, ws_len = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
-    return Options(float(scale), int(path), int(force_chunks), 0, None, None, ws_ptr, ws_len, None, LAYOUTS[layout])
+    return Options(float(scale), int(path), int(force_chunks), 0, None, None, ws_ptr, ws_len, None, LAYOUTS[layout],
+                   int(norm))
 
 
 def cp_partials(q, q_shared: bool, k, v, triple, *, B, H, N, M, D, path=PATH_AUTO, scale=0.0, force_chunks=0,
-                layout="bhnd"):
-    """flarepp_cp_partials: this rank's split pass reduced to one triple per latent row."""
+                layout="bhnd", norm_synthesis=False):
+    """flarepp_cp_partials: this rank's split pass reduced to one triple per latent row
+    (``norm_synthesis``: RMS-normalise this pass's q and k rows first)."""
     fn = lib.flarepp_cp_partials
     vp, i = ctypes.c_void_p, ctypes.c_int
     fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, ctypes.POINTER(Options), vp]
     fn.restype = i
-    o = _cp_options(path, scale, force_chunks, layout)
+    o = _cp_options(path, scale, force_chunks, layout, norm=norm_synthesis)
     rc = fn(_ptr(q), int(q_shared), _ptr(k), _ptr(v), _ptr(triple), B, H, N, M, D, _dtype_code(k),
             ctypes.byref(o), _stream(k.device))
     _check(rc, "flarepp_cp_partials")

@@ -48,13 +48,14 @@ def _all_gather(t: torch.Tensor, group) -> torch.Tensor:
 
 def mixer_fwd_cp(q0, q_fixed, gate, k0, k, v, y=None, *, group=None, layout: str = "bhnd",
                  path: int = _b.PATH_AUTO, scale: float = 0.0, force_chunks: int = 0,
-                 return_qz: bool = False, _ops=None, _gather=None):
+                 return_qz: bool = False, norm_synthesis: bool = False, _ops=None, _gather=None):
     """FLARE++ mixer forward with the tokens sharded over the ranks of `group`.
 
     q0, q_fixed [H,M,D] and gate fp32 [H] (or None: FLARE) are the same on every
     rank; k0, k, v are this rank's tokens, [B,H,N_r,D] or [B,N_r,H,D]
     (``layout``).  Returns this rank's y (and the merged q, z as fp32
-    [B,H,M,D] when ``return_qz``; identical on every rank).
+    [B,H,M,D] when ``return_qz``; identical on every rank).  ``norm_synthesis``
+    RMS-normalises the q0 and k0 rows in the synthesis pass.
 
     ``_ops`` and ``_gather`` replace the library stages and the collective
     (tests of the orchestration on CPU ranks); the default is the CUDA library
@@ -73,7 +74,8 @@ def mixer_fwd_cp(q0, q_fixed, gate, k0, k, v, y=None, *, group=None, layout: str
     triple = torch.empty(ops.cp_triple_bytes(B, H, M, D) // 4, dtype=torch.float32, device=dev)
     lat_bytes = ops.cp_latent_bytes(B, H, M, D, dt)
     if gated:
-        ops.cp_partials(q0, True, k0, k0, triple, force_chunks=force_chunks, **common, **tok)
+        ops.cp_partials(q0, True, k0, k0, triple, force_chunks=force_chunks, norm_synthesis=norm_synthesis,
+                        **common, **tok)
         qs = torch.empty(lat_bytes, dtype=torch.uint8, device=dev)
         ops.cp_merge(gather(triple, group), ranks, q_fixed, gate, qs, dtype=dt, **common)
         ops.cp_partials(qs, False, k, v, triple, force_chunks=force_chunks, **common, **tok)

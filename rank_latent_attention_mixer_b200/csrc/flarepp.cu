@@ -46,8 +46,9 @@ struct Plan {
     int row_blocks;      // latent-row blocks per (b, h, chunk) (SIMT)
     float scale_log2;
     tc::RowStrides tok;  // element strides of the token tensors k0, k, v, y (flarepp_layout_t)
+    int norm_synthesis;  // RMS-normalise q0 and k0 rows in the synthesis pass
     // byte offsets into the workspace
-    size_t off_part_O, off_part_ml, off_q32, off_q16, off_z32, off_z16, total;
+    size_t off_part_O, off_part_ml, off_q32, off_q16, off_z32, off_z16, off_q0n, off_k0n, total;
 };
 
 int check_shape(const Shape& s) {
@@ -79,6 +80,8 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     if (o && o->n_stage_events > 0 && !o->stage_events) return FLAREPP_ERR_INVALID_ARG;
     if (o && o->force_chunks < 0) return FLAREPP_ERR_INVALID_ARG;
     const int layout = o ? o->layout : FLAREPP_LAYOUT_BHND;
+    if (o && o->norm_synthesis != 0 && o->norm_synthesis != 1) return FLAREPP_ERR_INVALID_ARG;
+    pl->norm_synthesis = o ? o->norm_synthesis : 0;
     if (layout != FLAREPP_LAYOUT_BHND && layout != FLAREPP_LAYOUT_BNHD) return FLAREPP_ERR_INVALID_ARG;
     pl->tok = layout == FLAREPP_LAYOUT_BNHD
                   ? tc::RowStrides{(int64_t)s.H * s.D, s.D, (int64_t)s.N * s.H * s.D}
@@ -124,6 +127,9 @@ int make_plan(const Shape& s, const flarepp_options_t* o, Plan* pl) {
     pl->off_q16 = off;     off = align_up(off + rows * s.D * sizeof(uint16_t));     // q in the 16-bit I/O dtype
     pl->off_z32 = off;     off = align_up(off + rows * s.D * sizeof(float));
     pl->off_z16 = off;     off = align_up(off + rows * s.D * sizeof(uint16_t));
+    // the normalised synthesis seeds and keys/values (norm_synthesis)
+    pl->off_q0n = off;     off = align_up(off + (pl->norm_synthesis ? s.lat_bytes() : 0));
+    pl->off_k0n = off;     off = align_up(off + (pl->norm_synthesis ? s.tok_bytes() : 0));
     pl->total = off;
     return FLAREPP_OK;
 }
@@ -265,6 +271,34 @@ int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, con
     return run_simt<__nv_bfloat16>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
 }
 
+// Head-wise RMS normalisation of the synthesis seeds (H*M rows) and
+// keys/values (B*H*N rows) into their workspace copies, one launch.
+constexpr float kNormEps = 1e-6f;
+
+template <typename T>
+void launch_rms_norm(const Shape& s, const void* q0, void* q0n, const void* k0, void* k0n, cudaStream_t st) {
+    const int64_t rows1 = (int64_t)s.H * s.M, rows2 = s.bh() * s.N;
+    const int rw = 32 / (s.D * (int)sizeof(T) / 16);                // rows per warp pass
+    const int64_t want = (rows1 + rows2 + 8 * rw - 1) / (8 * rw);
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)kNumSMs * 16);
+    const T* a = static_cast<const T*>(q0);
+    const T* b = static_cast<const T*>(k0);
+    T* oa = static_cast<T*>(q0n);
+    T* ob = static_cast<T*>(k0n);
+    switch (s.D) {
+        case 16: rms_normalise_rows<T, 16><<<grid, 256, 0, st>>>(a, oa, rows1, b, ob, rows2, kNormEps); break;
+        case 32: rms_normalise_rows<T, 32><<<grid, 256, 0, st>>>(a, oa, rows1, b, ob, rows2, kNormEps); break;
+        case 64: rms_normalise_rows<T, 64><<<grid, 256, 0, st>>>(a, oa, rows1, b, ob, rows2, kNormEps); break;
+        default: rms_normalise_rows<T, 128><<<grid, 256, 0, st>>>(a, oa, rows1, b, ob, rows2, kNormEps); break;
+    }
+}
+
+void rms_norm(const Shape& s, const void* q0, void* q0n, const void* k0, void* k0n, cudaStream_t st) {
+    if (s.dtype == FLAREPP_F32) launch_rms_norm<float>(s, q0, q0n, k0, k0n, st);
+    else if (s.dtype == FLAREPP_F16) launch_rms_norm<__half>(s, q0, q0n, k0, k0n, st);
+    else launch_rms_norm<__nv_bfloat16>(s, q0, q0n, k0, k0n, st);
+}
+
 int forward(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
             const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
             const flarepp_options_t* opts, void* stream) {
@@ -295,6 +329,13 @@ int forward(const void* q0, const void* q_fixed, const float* gate, const void* 
     if (opts && opts->n_stage_events > 0) {
         ev.ev = opts->stage_events;
         ev.n = opts->n_stage_events;
+    }
+    if (pl.norm_synthesis && gate) {
+        // the synthesis reads normalised copies (its own stage for the events)
+        ev.mark(st);
+        rms_norm(s, q0, ws + pl.off_q0n, k0, ws + pl.off_k0n, st);
+        q0 = ws + pl.off_q0n;
+        k0 = ws + pl.off_k0n;
     }
     rc = run(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
     if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
@@ -645,6 +686,15 @@ int cp_partials(const void* q, int q_shared, const void* k, const void* v, float
     StageScratch sc;
     rc = sc.acquire(pl, opts, st);
     if (rc) return rc;
+    if (pl.norm_synthesis) {
+        // normalised copies of this call's seeds and keys/values (the synthesis call)
+        if (!q_shared || k != v) {
+            return sc.release(FLAREPP_ERR_INVALID_ARG);
+        }
+        rms_norm(s, q, sc.ws + pl.off_q0n, k, sc.ws + pl.off_k0n, st);
+        q = sc.ws + pl.off_q0n;
+        k = v = sc.ws + pl.off_k0n;
+    }
     // a latent state's operand part: the I/O-dtype copy (tensor cores) or fp32 (SIMT)
     const void* q16 = q_shared ? q : static_cast<const char*>(q) + latent_16_offset(s);
     if (pl.path == FLAREPP_PATH_TCGEN05) {

@@ -120,6 +120,51 @@ split_partial_simt(SplitParams p) {
     }
 }
 
+// Head-wise RMS normalisation of rows of D elements (the synthesis seeds q0
+// and keys/values k0; physicsnemo issue #2024, FLARE++ list, "Normalizing the
+// synthesis call"): out = x / sqrt(mean_d x^2 + eps), computed in fp32 and
+// rounded to T.  Any tensor whose rows of D elements are contiguous in memory
+// -- [H,M,D], [B,H,N,D] or [B,N,H,D] -- is `rows` such rows back to back.
+// One 16-byte chunk per lane; a row's lanes combine their sums by shuffles.
+// HBM-bound: one read and one write of each tensor.  One launch serves two
+// tensors: rows [0, rows1) of x1 -> out1, then rows2 rows of x2 -> out2.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+rms_normalise_rows(const T* __restrict__ x1, T* __restrict__ out1, int64_t rows1, const T* __restrict__ x2,
+                   T* __restrict__ out2, int64_t rows2, float eps) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t rows = rows1 + rows2;
+    constexpr int E = 16 / sizeof(T);              // elements per chunk
+    constexpr int C = D / E;                       // chunks per row (<= 32)
+    constexpr int RW = 32 / C;                     // rows per warp pass
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int64_t r0 = first * RW; r0 < rows; r0 += warps * RW) {
+        const int64_t r = r0 + lane / C;
+        const bool in = r < rows;                  // every lane still takes part in the shuffles
+        const bool second = r >= rows1;
+        const T* src = second ? x2 + (r - rows1) * D : x1 + r * D;
+        T* dst = second ? out2 + (r - rows1) * D : out1 + r * D;
+        float v[E];
+        float ss = 0.f;
+        if (in) {
+            load_row_f32<T, E>(src + (lane % C) * E, v);
+#pragma unroll
+            for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
+        }
+#pragma unroll
+        for (int o = C / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (in) {
+            const float inv = rsqrtf(ss * (1.f / D) + eps);
+#pragma unroll
+            for (int e = 0; e < E; ++e) v[e] *= inv;
+            store_row<T, E>(dst + (lane % C) * E, v);
+        }
+    }
+}
+
 // Merge of the per-chunk triples of one latent row (one warp per row):
 // out = sum_c 2^(m_c - m*) O_c / sum_c 2^(m_c - m*) l_c with m* = max_c m_c.
 // Synthesis epilogue: q = q_fixed + gate[h] * out (FLARE.py README, FLARE++

@@ -42,7 +42,8 @@ class StandInOps:
     def _tok(t, layout):
         return t.double() if layout == "bhnd" else t.double().transpose(1, 2)
 
-    def cp_partials(self, q, q_shared, k, v, triple, *, B, H, N, M, D, path, scale, layout, force_chunks):
+    def cp_partials(self, q, q_shared, k, v, triple, *, B, H, N, M, D, path, scale, layout, force_chunks,
+                    norm_synthesis=False):
         Q = self._lat(q, q_shared, B, H, M, D)
         K, V = self._tok(k, layout), self._tok(v, layout)
         S = Q @ K.transpose(-1, -2) * (scale or 1.0 / math.sqrt(D))
