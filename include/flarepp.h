@@ -126,7 +126,8 @@ typedef struct flarepp_options {
 
 /* Kernel launches one forward call makes (gated = 0: closed gate / FLARE).
  * Launch order: gated -> split partial (synthesis), merge (q), split partial
- * (encode), merge (z), decode; closed gate -> the last three. */
+ * (encode), merge (z), decode; closed gate -> the last three.  A gated call
+ * with norm_synthesis makes one more, first: the normalisation of q0, k0. */
 int flarepp_launches_per_call(int gated);
 
 /* FLARE++ mixer forward (see the top of this file).  gate == NULL -> FLARE. */
