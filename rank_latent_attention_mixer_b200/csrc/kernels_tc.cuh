@@ -412,8 +412,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     static_assert(KT == 64 || KT == 128, "key/value tiles of 64 or 128 rows");
     static_assert(NW >= 1 && NW <= 3, "the producer warpgroup holds one TMA warp and NW MMA warps");
     static_assert(NST >= 3, "at least three key/value stages");
-    static_assert(NST % NW == 0, "interleaved mode splits the stages into one ring per warpgroup");
-    // Interleaved mode: warpgroup w owns stages [w R, w R + R) and consumes them in
+    // Interleaved mode (launch_attn refuses it unless NW divides NST): warpgroup w owns stages [w R, w R + R) and consumes them in
     // order, so no consumer can wait on a stage two fills ahead (a parity wait
     // cannot tell phase k+1 from phase k-1).  Shared mode: one ring of NST stages
     // that every warpgroup consumes in order.
@@ -933,12 +932,15 @@ struct Problem {
 // two warpgroups on 128-row key/value tiles that both consume (each tile read
 // from L2 once per 256 latents); the decode uses three warpgroups on 64-row
 // latent tiles (more softmax warps per SM sub-partition to hide latency).
-template <int D, int NW_, int KT_>
+template <int D, int NW_, int KT_, bool DECODE = false>
 struct Config {
     static constexpr int NW = NW_;
     static constexpr int KT = KT_;
-    static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 128 ? 4 : (D == 64 ? 4 : 6));
-    static constexpr int QS = D == 128 ? 1 : 2;
+    // D = 128 fits four key/value stages and one query slot (split passes:
+    // long items) or three stages and two slots (decode: an item is a few
+    // latent tiles, so the next item's query tiles load during the current one)
+    static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 128 ? (DECODE ? 3 : 4) : (D == 64 ? 4 : 6));
+    static constexpr int QS = D == 128 && !DECODE ? 1 : 2;
     using SM = Smem<D, NW, KT, NST, QS>;
     // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
     static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
@@ -1054,10 +1056,11 @@ inline int sm_count() {
     return n > 0 ? n : kNumSMs;
 }
 
-template <typename E, int D, int NW, int KT>
+template <typename E, int D, int NW, int KT, bool DECODE = false>
 int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& prm,
                 cudaStream_t st) {
-    using C = Config<D, NW, KT>;
+    using C = Config<D, NW, KT, DECODE>;
+    if (prm.interleave && C::NST % C::NW != 0) return 2;      // one stage ring per warpgroup needs NW | NST
     auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS>;
     static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
@@ -1090,7 +1093,7 @@ inline int launch_split(int D, const CUtensorMap& mq, const CUtensorMap& mk, con
 template <typename E>
 inline int launch_decode(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const Params& prm, cudaStream_t st) {
-    if (D == 128) return launch_attn<E, 128, 2, 64>(mq, mk, mv, prm, st);
+    if (D == 128) return launch_attn<E, 128, 2, 64, true>(mq, mk, mv, prm, st);
     return launch_attn_d<E, kDecodeNW, kDecodeKT>(D, mq, mk, mv, prm, st);
 }
 
