@@ -1,0 +1,83 @@
+"""fp64 CPU oracle for the gradients of the FLARE++ mixer.
+
+TEST INFRASTRUCTURE ONLY (same rules as the rest of ``oracle/``).
+
+The forward is the FLARE++ block of the FLARE.py README ("FLARE++" code
+block, three scaled-dot-product-attention calls):
+
+    q_dyn = SDPA(q0, k0, k0);  q = q_fixed + gate * q_dyn;  z = SDPA(q, k, v);  y = SDPA(k, q, z)
+
+and this module returns the gradients of a scalar loss L with dL/dy = dy with
+respect to q0, q_fixed, gate, k0, k and v, by the chain rule through each
+softmax attention O = softmax(s Q K^T) V (row-wise softmax over the keys):
+
+    dV = P^T dO,   dP = dO V^T,   dS = P * (dP - rowsum(P * dP)),
+    dQ = s dS K,   dK = s dS^T Q
+
+applied to the decode, the encode, the gate and the synthesis in that order
+(q0 and q_fixed are shared by the batch, so their gradients sum over b; k0 is
+both the keys and the values of the synthesis, so it collects both terms).
+Plain numpy in fp64 with explicit [M, N] matrices per (b, h): for small cases.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _f64
+
+
+def _softmax_rows(S):
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    return E / E.sum(axis=1, keepdims=True)
+
+
+def _sdpa_fwd(Q, K, V, s):
+    P = _softmax_rows(s * (Q @ K.T))
+    return P, P @ V
+
+
+def _sdpa_bwd(Q, K, V, P, dO, s):
+    """Gradients of O = softmax(s Q K^T) V with respect to Q, K and V."""
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - np.sum(P * dP, axis=1, keepdims=True))
+    return s * (dS @ K), s * (dS.T @ Q), dV
+
+
+def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
+    """Gradients of the gated mixer (gate open).  Returns a dict with
+    dq0, dq_fixed [H,M,D], dgate [H], dk0, dk, dv [B,H,N,D], and the forward's
+    y [B,H,N,D] (fp64)."""
+    q0, q_fixed, gate = _f64(q0), _f64(q_fixed), _f64(gate).reshape(-1)
+    k0, k, v, dy = _f64(k0), _f64(k), _f64(v), _f64(dy)
+    B, H, N, D = k.shape
+    M = q_fixed.shape[1]
+    s = scale if scale > 0 else 1.0 / np.sqrt(D)
+    g = {name: np.zeros_like(a) for name, a in
+         (("dq0", q0), ("dq_fixed", q_fixed), ("dgate", gate), ("dk0", k0), ("dk", k), ("dv", v))}
+    y = np.empty_like(k)
+    for b in range(B):
+        for h in range(H):
+            # forward, keeping the weights
+            P_syn, q_dyn = _sdpa_fwd(q0[h], k0[b, h], k0[b, h], s)
+            q = q_fixed[h] + gate[h] * q_dyn
+            P_enc, z = _sdpa_fwd(q, k[b, h], v[b, h], s)
+            P_dec, y[b, h] = _sdpa_fwd(k[b, h], q, z, s)
+            # decode: y = SDPA(k, q, z)
+            dk_a, dq_a, dz = _sdpa_bwd(k[b, h], q, z, P_dec, dy[b, h], s)
+            # encode: z = SDPA(q, k, v)
+            dq_b, dk_b, dv = _sdpa_bwd(q, k[b, h], v[b, h], P_enc, dz, s)
+            dq = dq_a + dq_b
+            # gate: q = q_fixed + gate * q_dyn
+            g["dq_fixed"][h] += dq
+            g["dgate"][h] += np.sum(dq * q_dyn)
+            dq_dyn = gate[h] * dq
+            # synthesis: q_dyn = SDPA(q0, k0, k0)
+            dq0, dk0_keys, dk0_values = _sdpa_bwd(q0[h], k0[b, h], k0[b, h], P_syn, dq_dyn, s)
+            g["dq0"][h] += dq0
+            g["dk0"][b, h] = dk0_keys + dk0_values
+            g["dk"][b, h] = dk_a + dk_b
+            g["dv"][b, h] = dv
+    g["y"] = y
+    return g
