@@ -59,6 +59,8 @@ def parse_args(argv=None):
                    help="token-sharded form: one global problem, each rank holds N/world tokens (strong scaling)")
     p.add_argument("--layout", choices=["bhnd", "bnhd"], default="bhnd",
                    help="memory layout of k0, k, v, y: [B,H,N,D] or [B,N,H,D] (read in place)")
+    p.add_argument("--backward", action="store_true",
+                   help="time the backward (flarepp_mixer_bwd: gradients of every input for a random dy)")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -622,10 +624,138 @@ def run_cp(args):
         print(json.dumps(out), flush=True)
 
 
+# --------------------------------------------------------------------------- backward arm
+
+BWD_STAGES_GATED = ["fwd split(synthesis)", "fwd merge(q)", "fwd split(encode)", "fwd merge(z)",
+                    "decode_rows", "decode_cols", "reduce(decode)", "token_cols(encode)", "latent_rows(encode)",
+                    "reduce(encode)", "token_cols(synthesis)", "latent_rows(synthesis)", "reduce(synthesis)",
+                    "reduce_batch"]
+BWD_STAGES_FLARE = ["fwd split(encode)", "fwd merge(z)", "decode_rows", "decode_cols", "reduce(decode)",
+                    "token_cols(encode)", "latent_rows(encode)", "reduce(encode)", "reduce_batch"]
+# FLOPs per (b, h, n, m, d) of each backward kernel as executed (2 per multiply-add):
+# decode rows recompute the decode softmax and y (4), then score, <dy, z> and dS q (6)
+BWD_KERNEL_FLOPS = {"decode_rows": 10, "decode_cols": 8, "token_cols": 8, "latent_rows": 6}
+
+
+def fp32_simt_peak_tflops(peaks):
+    """FP32 FMA peak of the SIMT pipes: 148 SMs x 128 lanes x 2 FLOP per clock
+    at the maximum SM clock."""
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_backward_bench(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from rank_latent_attention_mixer_b200 import binding as fb
+    from rank_latent_attention_mixer_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    w = w.with_shape(seed=rank_seed(w.seed, rank))
+    if args.tokens:
+        w = w.with_shape(N=args.tokens, name=f"{w.name}_n{args.tokens}")
+    x = W.make_inputs(w, device=str(dev))
+    dy = W.random_cotangent((w.B, w.H, w.N, w.D), w.dtype, seed=w.seed + 100, device=str(dev),
+                            device_rng=w.device_rng)
+    path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
+    dtype_code = {"f32": fb.F32, "bf16": fb.BF16, "f16": fb.F16}[w.dtype]
+    gated = not args.flare
+    ws = torch.empty(fb.bwd_workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, path), dtype=torch.uint8,
+                     device=dev)
+    out_t = {"dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
+             "dq_fixed": torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev)}
+    if gated:
+        out_t.update(dk0=torch.empty_like(x["k0"]), dq0=torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev),
+                     dgate=torch.empty((w.H,), dtype=torch.float32, device=dev))
+    n_launch = fb.bwd_launches(gated)
+    names = BWD_STAGES_GATED if gated else BWD_STAGES_FLARE
+    fits_l2 = 6 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
+
+    def step(events=None):
+        fb.mixer_bwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], dy, path=path,
+                     workspace=ws, stage_events=events, out=out_t)
+
+    for _ in range(args.warmup):
+        step()
+        if flush is not None:
+            flush.zero_()
+    torch.cuda.synchronize()
+    assert fb.check_device_status() == 0
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            step(evs[i])
+            if flush is not None:
+                flush.zero_()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if fb.check_device_status() != 0:
+        raise SystemExit("device status after the timed region")
+    local_ms = sum(evs[i][0].elapsed_time(evs[i][n_launch]) for i in range(K))
+    max_ms = reduce_max(local_ms, world, dev)
+    stage = [statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) for j in range(n_launch)]
+    total = sum(stage)
+    bhnmd = w.B * w.H * w.N * w.M * w.D
+    peaks, peak_src = load_peaks()
+    peak_alu = fp32_simt_peak_tflops(peaks)
+    kern = {}
+    for nm, ms in zip(names, stage):
+        base = nm.split("(")[0]
+        f = BWD_KERNEL_FLOPS.get(base)
+        kern[nm] = {"ms": round(ms, 4), "share": round(ms / total, 4)}
+        if f:
+            kern[nm]["tflops"] = round(f * bhnmd / (ms * 1e-3) / 1e12, 2)
+    # the dominant kernel's roofline: SIMT fp32 FMA arithmetic
+    top = max((nm for nm in names if BWD_KERNEL_FLOPS.get(nm.split("(")[0])), key=lambda nm: kern[nm]["ms"])
+    achieved = kern[top]["tflops"]
+    counts = W.algorithmic_counts(w, flare=not gated)
+    ms_step = max_ms / K
+    passes = 3 if gated else 2
+    out = {
+        "metric": "FLARE++ mixer bwd Mtokens/s on 1 B200 (gradients of every input)",
+        "value": round(aggregate_mtokens(counts["tokens"], world, K, max_ms), 4), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
+                   "gate": "open (FLARE++)" if gated else "closed (FLARE)", "forward_path": args.path,
+                   "l2": ("flushed between steps (512 MiB write)" if flush is not None
+                          else "inputs larger than L2 (back-to-back steps)")},
+        "algorithmic_tflops": round(10.0 * passes * bhnmd / (ms_step * 1e-3) / 1e12, 2),
+        "gpu_launches": K * n_launch,
+        "roofline": {"bound": "alu", "kernel": top, "achieved": achieved, "peak": round(peak_alu, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / peak_alu, 4), "traffic": None,
+                     "peak_kind": "FP32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"},
+        "stages": kern,
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.backward:
+        run_backward_bench(args)
     elif args.cp:
         run_cp(args)
     else:

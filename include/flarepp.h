@@ -1,5 +1,5 @@
 /*
- * flarepp.h -- C ABI of the B200 (sm_100a) FLARE++ token-mixer forward.
+ * flarepp.h -- C ABI of the B200 (sm_100a) FLARE++ token mixer: forward and backward.
  *
  * The operation (FLARE.py README, "FLARE++" code block, flarepp_multihead_mixer;
  * shapes from its docstring):
@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define FLAREPP_ABI_VERSION 3
+#define FLAREPP_ABI_VERSION 4
 
 typedef enum flarepp_dtype {
     FLAREPP_F32 = 0,
@@ -263,6 +263,53 @@ int flarepp_cp_merge(const float* gathered, int ranks, const void* q_fixed, cons
 int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const void* k, void* y,
                       int B, int H, int N, int M, int D, int dtype,
                       const flarepp_options_t* opts, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Backward: the gradients of a scalar loss L with respect to every input of
+ * the mixer, given dy = dL/dy.  By the chain rule through each softmax
+ * attention O = softmax(scale Q K^T) V of the FLARE++ block (FLARE.py
+ * README, "FLARE++" code block; the same algebra as FlashAttention's backward,
+ * applied to the decode, the encode, the gate q = q_fixed + gate * q_dyn and
+ * the synthesis in that order).  The forward is not saved: the call runs the
+ * forward's synthesis and encode passes again, on the forward's own kernel
+ * family, and recomputes the decode's per-token softmax inside the backward.
+ * The physicsnemo issue #2024 speaks of the encoder's custom backward; the
+ * pages state no formulas for it, so this is the plain chain rule.
+ *
+ * Arguments (same conventions, limits and checks as flarepp_mixer_fwd_ex):
+ *   q0, q_fixed, gate, k0, k, v   the forward's inputs (gate == NULL: FLARE,
+ *                                 then q0, k0, dq0, dgate, dk0 are ignored)
+ *   dy        [B,H,N,D] token layout, I/O dtype: the gradient of y
+ *   dq0, dq_fixed   DEVICE fp32 [H,M,D] (sums over the batch)
+ *   dgate     DEVICE fp32 [H]: dL/d(gate value), not of the logit
+ *   dk0, dk, dv     [B,H,N,D] token layout, I/O dtype
+ * No output may overlap an input or another output.  opts (may be NULL):
+ * scale, path (the kernel family of the recomputed forward passes; the
+ * backward's own kernels are SIMT fp32 for every dtype), force_chunks (the
+ * token chunks of both the recomputed passes and the backward's token sums),
+ * workspace / workspace_bytes (>= flarepp_mixer_bwd_workspace_bytes),
+ * stage_events (recorded before the first and after every launch), layout.
+ * norm_synthesis = 1 gives FLAREPP_ERR_UNSUPPORTED; q_out, z_out are ignored.
+ * Arithmetic is fp32 with fp32 accumulation of every sum; sums over tokens
+ * are taken per token chunk and added in a fixed order (deterministic); the
+ * 16-bit gradients are rounded once, at the end.  Asynchronous on `stream`. */
+int flarepp_mixer_bwd(const void* q0, const void* q_fixed, const float* gate,
+                      const void* k0, const void* k, const void* v, const void* dy,
+                      float* dq0, float* dq_fixed, float* dgate,
+                      void* dk0, void* dk, void* dv,
+                      int B, int H, int N, int M, int D, int dtype,
+                      const flarepp_options_t* opts, void* stream);
+
+/* Bytes of device scratch one backward call needs (the forward's scratch,
+ * the log-sum-exps, fp32 latent gradients, per-chunk partial sums and an
+ * fp32 [B,H,N,D] buffer for the decode's share of dk).  0 for arguments the
+ * backward would reject. */
+size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int dtype,
+                                         const flarepp_options_t* opts);
+
+/* Kernel launches one backward call makes: gated 14 (4 recomputed forward
+ * passes, 3 per attention, 1 batch reduce), closed gate 9. */
+int flarepp_mixer_bwd_launches(int gated);
 
 /* FLAREPP_ABI_VERSION of the loaded library. */
 int flarepp_abi_version(void);

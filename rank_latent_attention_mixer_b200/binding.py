@@ -23,7 +23,8 @@ STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
           4: "ERR_WORKSPACE", 5: "ERR_TIMEOUT"}
 EXPORTS = ["flarepp_mixer_fwd", "flare_fwd", "flarepp_mixer_fwd_ex", "flarepp_workspace_bytes",
            "flarepp_mixer_fwd_host", "flarepp_selected_path", "flarepp_check_device_status",
-           "flarepp_status_string", "flarepp_abi_version", "flarepp_launches_per_call"]
+           "flarepp_status_string", "flarepp_abi_version", "flarepp_launches_per_call",
+           "flarepp_mixer_bwd", "flarepp_mixer_bwd_workspace_bytes", "flarepp_mixer_bwd_launches"]
 
 
 class FlareppError(RuntimeError):
@@ -59,16 +60,22 @@ def _load() -> ctypes.CDLL:
     lib.flarepp_status_string.argtypes = [i]
     lib.flarepp_status_string.restype = ctypes.c_char_p
     lib.flarepp_launches_per_call.argtypes = [i]
+    lib.flarepp_mixer_bwd.argtypes = [vp] * 13 + [i] * 6 + [ctypes.POINTER(Options), vp]
+    lib.flarepp_mixer_bwd_workspace_bytes.argtypes = [i] * 6 + [ctypes.POINTER(Options)]
+    lib.flarepp_mixer_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.flarepp_mixer_bwd_launches.argtypes = [i]
     for name in ("flarepp_mixer_fwd", "flarepp_mixer_fwd_ex", "flarepp_mixer_fwd_host", "flare_fwd",
                  "flarepp_selected_path", "flarepp_check_device_status", "flarepp_abi_version",
-                 "flarepp_launches_per_call"):
+                 "flarepp_launches_per_call", "flarepp_mixer_bwd", "flarepp_mixer_bwd_launches"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
 
 lib = _load()
-if lib.flarepp_abi_version() != 3:
-    raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs 3: rebuild it")
+ABI_VERSION = 4
+if lib.flarepp_abi_version() != ABI_VERSION:
+    raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs {ABI_VERSION}: "
+                      "rebuild it")
 
 
 def status_string(status: int) -> str:
@@ -179,6 +186,68 @@ def mixer_fwd(q0, q_fixed, gate, k0, k, v, y=None, *, scale: float = 0.0, path: 
                                   B, H, N, M, D, dt, ctypes.byref(o), _stream(k.device))
     _check(rc, "flarepp_mixer_fwd_ex")
     return (y, q_out, z_out) if return_qz else y
+
+
+def _event_array(stage_events):
+    if not stage_events:
+        return None, 0
+    handles = []
+    for e in stage_events:
+        if e.cuda_event == 0:          # torch creates the CUDA event lazily
+            e.record()
+        handles.append(e.cuda_event)
+    return (ctypes.c_void_p * len(handles))(*handles), len(handles)
+
+
+def bwd_launches(gated: bool = True) -> int:
+    return int(lib.flarepp_mixer_bwd_launches(int(gated)))
+
+
+def bwd_workspace_bytes(B, H, N, M, D, dtype=BF16, path=PATH_AUTO, force_chunks=0, layout="bhnd") -> int:
+    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout], 0)
+    return int(lib.flarepp_mixer_bwd_workspace_bytes(B, H, N, M, D, dtype, ctypes.byref(o)))
+
+
+def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int = PATH_AUTO,
+              force_chunks: int = 0, layout: str = "bhnd", workspace: Optional[torch.Tensor] = None,
+              stage_events=None, out: Optional[dict] = None) -> dict:
+    """Gradients of the FLARE++ mixer (flarepp_mixer_bwd) for the upstream gradient dy of y.
+
+    Inputs as for ``mixer_fwd`` plus dy (the layout and dtype of k).  Returns a
+    dict with dk, dv (and dk0 when gated) in the I/O dtype and token layout,
+    dq_fixed (and dq0) fp32 [H,M,D], and dgate fp32 [H] (the gradient with
+    respect to the gate value, not its logit).  ``gate=None`` is FLARE.
+    ``out`` may supply preallocated gradient tensors under the same names."""
+    B, H, N, M, D = _shapes(q_fixed, k, layout)
+    _contig(q0, q_fixed, gate, k0, k, v, dy)
+    dt = _dtype_code(k)
+    gated = gate is not None
+    if gated and gate.dtype != torch.float32:
+        raise TypeError("gate must be float32 [H]")
+    g = dict(out or {})
+    dev = k.device
+    g.setdefault("dk", torch.empty_like(k))
+    g.setdefault("dv", torch.empty_like(v))
+    g.setdefault("dq_fixed", torch.empty((H, M, D), dtype=torch.float32, device=dev))
+    if gated:
+        g.setdefault("dk0", torch.empty_like(k0))
+        g.setdefault("dq0", torch.empty((H, M, D), dtype=torch.float32, device=dev))
+        g.setdefault("dgate", torch.empty((H,), dtype=torch.float32, device=dev))
+    need = bwd_workspace_bytes(B, H, N, M, D, dt, path, force_chunks, layout)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ev_arr, n_ev = _event_array(stage_events)
+    o = Options(float(scale), int(path), int(force_chunks), n_ev, None, None,
+                workspace.data_ptr() if need else None, workspace.numel() if need else 0,
+                ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None,
+                LAYOUTS[layout], 0)
+    rc = lib.flarepp_mixer_bwd(_ptr(q0) if gated else None, _ptr(q_fixed), _ptr(gate),
+                               _ptr(k0) if gated else None, _ptr(k), _ptr(v), _ptr(dy),
+                               _ptr(g.get("dq0")) if gated else None, _ptr(g["dq_fixed"]),
+                               _ptr(g.get("dgate")) if gated else None, _ptr(g.get("dk0")) if gated else None,
+                               _ptr(g["dk"]), _ptr(g["dv"]), B, H, N, M, D, dt, ctypes.byref(o), _stream(dev))
+    _check(rc, "flarepp_mixer_bwd")
+    return g
 
 
 def mixer_fwd_plain(q0, q_fixed, gate, k0, k, v, y):

@@ -17,6 +17,7 @@
 
 #include "../../include/flarepp.h"
 #include "common.cuh"
+#include "kernels_bwd.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 
@@ -171,7 +172,7 @@ int check_pointers(const Shape& s, const void* q0, const void* q_fixed, const fl
 template <typename T>
 int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, const float* gate,
              const void* k0, const void* k, const void* v, void* y, char* ws,
-             float* q_out, float* z_out, StageEvents& ev, cudaStream_t st) {
+             float* q_out, float* z_out, StageEvents& ev, cudaStream_t st, const FwdExtras& ex) {
     const bool gated = gate != nullptr;
     float* part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
     float2* part_ml = reinterpret_cast<float2*>(ws + pl.off_part_ml);
@@ -206,7 +207,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
             split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
             ev.mark(st);                                                                           \
             mp.mode = kMergeSynthesis; mp.out_f32 = q32; mp.out_16 = q16; mp.user_out = q_out;   \
-            mp.q_copy_out = nullptr;                                                               \
+            mp.q_copy_out = nullptr; mp.lse_out = ex.lse_syn; mp.pregate_out = ex.qdyn;           \
             merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                 \
             ev.mark(st);                                                                           \
             sp.Q = q32; sp.q_batch_heads = s.H; sp.K = k; sp.V = v;                                \
@@ -218,10 +219,11 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
             ev.mark(st);                                                                           \
         }                                                                                          \
         mp.mode = kMergeEncode; mp.out_f32 = z32; mp.out_16 = z16; mp.user_out = z_out;          \
-        mp.q_copy_out = gated ? nullptr : q_out;                                                   \
+        mp.q_copy_out = gated ? nullptr : q_out; mp.lse_out = ex.lse_enc; mp.pregate_out = nullptr; \
         merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                     \
         ev.mark(st);                                                                               \
-        if (gated) {                                                                               \
+        if (!ex.decode) {                                                                          \
+        } else if (gated) {                                                                        \
             dp.Qlat = q32; dp.q_batch_heads = s.H;                                                 \
             decode_simt<T, float, DD><<<dec_grid, kSimtThreads, 0, st>>>(dp);                      \
             ev.mark(st);                                                                           \
@@ -246,7 +248,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
 
 int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, const float* gate,
         const void* k0, const void* k, const void* v, void* y, char* ws,
-        float* q_out, float* z_out, StageEvents& ev, cudaStream_t st) {
+        float* q_out, float* z_out, StageEvents& ev, cudaStream_t st, const FwdExtras& ex = FwdExtras{}) {
     if (pl.path == FLAREPP_PATH_TCGEN05) {
         tc::Buffers bu{};
         bu.part_O = reinterpret_cast<float*>(ws + pl.off_part_O);
@@ -261,14 +263,14 @@ int run(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed, con
         pr.chunks = pl.chunks; pr.chunk_len = pl.chunk_len; pr.scale_log2 = pl.scale_log2;
         auto mark = [&ev](cudaStream_t t) { ev.mark(t); };
         if (s.dtype == FLAREPP_F16)
-            return tc::run<__half>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st);
-        return tc::run<__nv_bfloat16>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st);
+            return tc::run<__half>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st, ex);
+        return tc::run<__nv_bfloat16>(pr, bu, q0, q_fixed, gate, k0, k, v, y, q_out, z_out, mark, st, ex);
     }
     if (s.dtype == FLAREPP_F32)
-        return run_simt<float>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+        return run_simt<float>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st, ex);
     if (s.dtype == FLAREPP_F16)
-        return run_simt<__half>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
-    return run_simt<__nv_bfloat16>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+        return run_simt<__half>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st, ex);
+    return run_simt<__nv_bfloat16>(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st, ex);
 }
 
 // Head-wise RMS normalisation of the synthesis seeds (H*M rows) and
@@ -783,6 +785,266 @@ int cp_decode(const void* q, int q_shared, const void* z_state, const void* k, v
     return simt_cp_decode<__nv_bfloat16>(s, pl, q, q_shared, z32, k, y, st);
 }
 
+// ------------------------------------------------------------------ backward
+//
+// Gradients of the mixer with respect to all its inputs, for an upstream
+// gradient dy of y (the chain rule through each of the three attentions of the
+// FLARE.py README's FLARE++ block; kernels in kernels_bwd.cuh).  The forward's
+// synthesis and encode passes run again (split + merge, on the forward's own
+// kernel family) and keep their per-latent log-sum-exps and the synthesis
+// output before the gate; then
+//   decode rows     dk_dec, per-token log-sum-exp and <dy, y>
+//   decode cols     partials of dq_dec and dz over token chunks     -> reduce: dz, dq, <dz, z>
+//   encode cols     dk = dk_dec + dk_enc, dv
+//   encode rows     partials of dq_enc                              -> reduce: dq, dq_dyn, <dq_dyn, q_dyn>
+//   synthesis cols  dk0 (keys and values terms)
+//   synthesis rows  partials of dq0                                 -> reduce: dq0 per batch element
+//   batch reduce    dq_fixed, dq0, dgate (sums over the batch)
+// With the gate closed (FLARE) the synthesis stages are skipped and the batch
+// reduce gives dq_fixed only.
+struct BwdPlan {
+    Plan fwd;
+    int chunks, chunk_len, row_blocks;
+    int64_t tok_blocks;
+    size_t off_lse_syn, off_lse_enc, off_qdyn, off_lse_tok, off_delta_tok, off_dk_acc, off_part1, off_part2, off_dz,
+        off_dq, off_dqdyn, off_delta_enc, off_delta0, off_dq0b, total;
+};
+
+int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
+    int rc = make_plan(s, o, &bp->fwd);
+    if (rc) return rc;
+    if (bp->fwd.norm_synthesis) return FLAREPP_ERR_UNSUPPORTED;
+    const int G = s.D >= 64 ? s.D / 32 : 1;           // bwd::Lanes<D>::G
+    const int rows_per_cta = bwd::kThreads / G;
+    const int tile = 4096 / s.D;                       // bwd::Lanes<D>::TILE
+    bp->row_blocks = (s.M + rows_per_cta - 1) / rows_per_cta;
+    bp->tok_blocks = (s.N + (int64_t)rows_per_cta - 1) / rows_per_cta;
+    const int64_t tiles = (s.N + tile - 1) / tile;
+    int64_t chunks;
+    if (o && o->force_chunks > 0) {
+        chunks = std::min<int64_t>(o->force_chunks, tiles);
+    } else {
+        // about eight CTAs per SM over the latent-side grid, chunks of >= 1 tile
+        const int64_t target = 8 * kNumSMs, per = s.bh() * bp->row_blocks;
+        chunks = std::max<int64_t>(1, std::min<int64_t>((target + per - 1) / per, tiles));
+    }
+    const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
+    bp->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
+    bp->chunks = (int)((s.N + (int64_t)bp->chunk_len - 1) / bp->chunk_len);
+    const size_t lat = (size_t)s.bh() * s.M, latd = lat * s.D, tok = (size_t)s.bh() * s.N;
+    size_t off = bp->fwd.total;
+    bp->off_lse_syn = off;   off = align_up(off + lat * sizeof(float));
+    bp->off_lse_enc = off;   off = align_up(off + lat * sizeof(float));
+    bp->off_qdyn = off;      off = align_up(off + latd * sizeof(float));
+    bp->off_lse_tok = off;   off = align_up(off + tok * sizeof(float));
+    bp->off_delta_tok = off; off = align_up(off + tok * sizeof(float));
+    bp->off_dk_acc = off;    off = align_up(off + tok * s.D * sizeof(float));
+    bp->off_part1 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
+    bp->off_part2 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
+    bp->off_dz = off;        off = align_up(off + latd * sizeof(float));
+    bp->off_dq = off;        off = align_up(off + latd * sizeof(float));
+    bp->off_dqdyn = off;     off = align_up(off + latd * sizeof(float));
+    bp->off_delta_enc = off; off = align_up(off + lat * sizeof(float));
+    bp->off_delta0 = off;    off = align_up(off + lat * sizeof(float));
+    bp->off_dq0b = off;      off = align_up(off + latd * sizeof(float));
+    bp->total = off;
+    return FLAREPP_OK;
+}
+
+struct BwdArgs {
+    const void *q0, *q_fixed, *k0, *k, *v, *dy;
+    const float* gate;
+    float *dq0, *dq_fixed, *dgate;
+    void *dk0, *dk, *dv;
+};
+
+int check_bwd_pointers(const Shape& s, const BwdArgs& a) {
+    const bool gated = a.gate != nullptr;
+    if (!a.q_fixed || !a.k || !a.v || !a.dy || !a.dq_fixed || !a.dk || !a.dv) return FLAREPP_ERR_INVALID_ARG;
+    if (gated && (!a.q0 || !a.k0 || !a.dq0 || !a.dgate || !a.dk0)) return FLAREPP_ERR_INVALID_ARG;
+    const void* tensors[] = {a.q_fixed, a.k, a.v, a.dy, a.dq_fixed, a.dk, a.dv, gated ? a.q0 : nullptr,
+                             gated ? a.k0 : nullptr, gated ? a.dq0 : nullptr, gated ? a.dk0 : nullptr};
+    for (const void* t : tensors)
+        if (t && !aligned16(t)) return FLAREPP_ERR_INVALID_ARG;
+    if (gated && ((reinterpret_cast<uintptr_t>(a.gate) & 3u) || (reinterpret_cast<uintptr_t>(a.dgate) & 3u)))
+        return FLAREPP_ERR_INVALID_ARG;
+    const size_t tb = s.tok_bytes(), lb = s.lat_bytes(), l32 = (size_t)s.H * s.M * s.D * sizeof(float);
+    const size_t gb = (size_t)s.H * sizeof(float);
+    struct Span { const void* p; size_t n; };
+    const Span ins[] = {{a.q_fixed, lb}, {a.k, tb}, {a.v, tb}, {a.dy, tb}, {gated ? a.q0 : nullptr, lb},
+                        {gated ? a.k0 : nullptr, tb}, {gated ? a.gate : nullptr, gb}};
+    const Span outs[] = {{a.dq_fixed, l32}, {a.dk, tb}, {a.dv, tb}, {gated ? a.dq0 : nullptr, l32},
+                         {gated ? a.dgate : nullptr, gb}, {gated ? a.dk0 : nullptr, tb}};
+    for (const Span& o : outs) {
+        for (const Span& i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return FLAREPP_ERR_INVALID_ARG;
+        for (const Span& o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return FLAREPP_ERR_INVALID_ARG;
+    }
+    return FLAREPP_OK;
+}
+
+// Launches with programmatic stream serialization (every backward kernel calls
+// pdl_wait() before its first global access); keeps the first launch error.
+struct BwdLauncher {
+    cudaStream_t st;
+    cudaError_t err = cudaSuccess;
+    template <typename K, typename... Args>
+    void operator()(K kern, dim3 grid, dim3 block, Args... args) {
+        const cudaError_t e = tc::launch_pdl(kern, grid, block, 0, st, args...);
+        if (err == cudaSuccess) err = e;
+    }
+};
+
+// The backward launches for one I/O type T, one latent-operand type TQ of the
+// decode and encode (T, or fp32 when the forward's SIMT kernels ran the
+// encode from fp32 routing queries) and one head dim D.
+template <typename T, typename TQ, int D>
+cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, char* ws, const void* q_lat, int q_bh,
+                         StageEvents& ev, cudaStream_t st) {
+    const bool gated = a.gate != nullptr;
+    BwdLauncher launch_bwd_kernel{st};
+    const Plan& pl = bp.fwd;
+    using L = bwd::Lanes<D>;
+    bwd::Params p{};
+    p.B = s.B; p.H = s.H; p.N = s.N; p.M = s.M;
+    p.tok_row = pl.tok.row; p.tok_h = pl.tok.h; p.tok_b = pl.tok.b;
+    p.scale_log2 = pl.scale_log2;
+    p.scale = pl.scale_log2 / kLog2e;
+    p.chunks = bp.chunks; p.chunk_len = bp.chunk_len;
+    p.lse_tok = reinterpret_cast<float*>(ws + bp.off_lse_tok);
+    p.delta_tok = reinterpret_cast<float*>(ws + bp.off_delta_tok);
+    p.dk_acc = reinterpret_cast<float*>(ws + bp.off_dk_acc);
+    p.part1 = reinterpret_cast<float*>(ws + bp.off_part1);
+    p.part2 = reinterpret_cast<float*>(ws + bp.off_part2);
+    float* z32 = reinterpret_cast<float*>(ws + pl.off_z32);
+    float* dz = reinterpret_cast<float*>(ws + bp.off_dz);
+    float* dq = reinterpret_cast<float*>(ws + bp.off_dq);
+    float* dqdyn = reinterpret_cast<float*>(ws + bp.off_dqdyn);
+    float* qdyn = reinterpret_cast<float*>(ws + bp.off_qdyn);
+    float* delta_enc = reinterpret_cast<float*>(ws + bp.off_delta_enc);
+    float* delta0 = reinterpret_cast<float*>(ws + bp.off_delta0);
+    float* dq0b = reinterpret_cast<float*>(ws + bp.off_dq0b);
+    const dim3 tok_grid((unsigned)bp.tok_blocks, (unsigned)s.bh());
+    const dim3 lat_grid((unsigned)bp.chunks, (unsigned)s.bh(), (unsigned)bp.row_blocks);
+    const int64_t rows = s.bh() * s.M;
+    const dim3 red_grid((unsigned)((rows + 7) / 8));
+
+    // decode: y = SDPA(k, q, z)
+    p.Qlat = q_lat; p.q_batch_heads = q_bh; p.Zlat = z32;
+    p.Ktok = a.k; p.Vtok = nullptr; p.dYtok = a.dy;
+    launch_bwd_kernel(bwd::decode_rows<T, TQ, D>, tok_grid, dim3(bwd::kThreads), p);
+    ev.mark(st);
+    launch_bwd_kernel(bwd::decode_cols<T, TQ, D>, lat_grid, dim3(bwd::kThreads), p);
+    ev.mark(st);
+    bwd::ReduceParams rp{};
+    rp.part1 = p.part1; rp.part2 = p.part2; rp.chunks = bp.chunks;
+    rp.B = s.B; rp.H = s.H; rp.M = s.M; rp.scale = p.scale;
+    rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = dz; rp.dq = dq; rp.delta = delta_enc;
+    launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+    ev.mark(st);
+
+    // encode: z = SDPA(q, k, v)
+    p.dOlat = dz; p.lse_lat = reinterpret_cast<float*>(ws + bp.off_lse_enc); p.delta_lat = delta_enc;
+    p.Ktok = a.k; p.Vtok = a.v; p.dK = a.dk; p.dV = a.dv;
+    launch_bwd_kernel(bwd::token_cols<T, TQ, D>, tok_grid, dim3(bwd::kThreads), p);
+    ev.mark(st);
+    launch_bwd_kernel(bwd::latent_rows<T, TQ, D>, lat_grid, dim3(bwd::kThreads), p);
+    ev.mark(st);
+    rp.mode = bwd::kReduceEncode; rp.gate = a.gate; rp.qdyn = qdyn; rp.dqdyn = dqdyn; rp.delta = delta0;
+    launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+    ev.mark(st);
+
+    if (gated) {
+        // synthesis: q_dyn = SDPA(q0, k0, k0), output gradient dq_dyn = gate * dq
+        p.Qlat = a.q0; p.q_batch_heads = 0;
+        p.dOlat = dqdyn; p.lse_lat = reinterpret_cast<float*>(ws + bp.off_lse_syn); p.delta_lat = delta0;
+        p.Ktok = a.k0; p.Vtok = a.k0; p.dK = a.dk0; p.dV = nullptr;
+        launch_bwd_kernel(bwd::token_cols<T, T, D>, tok_grid, dim3(bwd::kThreads), p);
+        ev.mark(st);
+        launch_bwd_kernel(bwd::latent_rows<T, T, D>, lat_grid, dim3(bwd::kThreads), p);
+        ev.mark(st);
+        rp.mode = bwd::kReduceSynthesis; rp.dq0b = dq0b;
+        launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+        ev.mark(st);
+    }
+    bwd::BatchParams bt{};
+    bt.B = s.B; bt.H = s.H; bt.M = s.M;
+    bt.dq = dq; bt.dq_fixed = a.dq_fixed;
+    if (gated) { bt.dq0b = dq0b; bt.qdyn = qdyn; bt.dq0 = a.dq0; bt.dgate = a.dgate; }
+    launch_bwd_kernel(bwd::reduce_batch<D>, dim3((unsigned)s.H), dim3(256), bt);
+    ev.mark(st);
+    (void)L::G;
+    return launch_bwd_kernel.err;
+}
+
+template <typename T, typename TQ>
+cudaError_t run_backward_d(const Shape& s, const BwdPlan& bp, const BwdArgs& a, char* ws, const void* q_lat,
+                           int q_bh, StageEvents& ev, cudaStream_t st) {
+    switch (s.D) {
+        case 16: return run_backward<T, TQ, 16>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        case 32: return run_backward<T, TQ, 32>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        case 64: return run_backward<T, TQ, 64>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        default: return run_backward<T, TQ, 128>(s, bp, a, ws, q_lat, q_bh, ev, st);
+    }
+}
+
+int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
+             void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    BwdPlan bp{};
+    int rc = make_bwd_plan(s, opts, &bp);
+    if (rc) return rc;
+    rc = check_bwd_pointers(s, a);
+    if (rc) return rc;
+    const Plan& pl = bp.fwd;
+    const bool gated = a.gate != nullptr;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = nullptr;
+    bool owned = false;
+    if (opts && opts->workspace) {
+        if (opts->workspace_bytes < bp.total) return FLAREPP_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(opts->workspace) % kAlign) return FLAREPP_ERR_INVALID_ARG;
+        ws = static_cast<char*>(opts->workspace);
+    } else {
+        if (cudaMallocAsync(reinterpret_cast<void**>(&ws), bp.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return FLAREPP_ERR_WORKSPACE;
+        }
+        owned = true;
+    }
+    StageEvents ev;
+    if (opts && opts->n_stage_events > 0) {
+        ev.ev = opts->stage_events;
+        ev.n = opts->n_stage_events;
+    }
+    // the forward's synthesis and encode, keeping what the backward needs
+    FwdExtras ex;
+    ex.lse_syn = reinterpret_cast<float*>(ws + bp.off_lse_syn);
+    ex.lse_enc = reinterpret_cast<float*>(ws + bp.off_lse_enc);
+    ex.qdyn = reinterpret_cast<float*>(ws + bp.off_qdyn);
+    ex.decode = false;
+    rc = run(s, pl, a.q0, a.q_fixed, a.gate, a.k0, a.k, a.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
+    if (rc == FLAREPP_OK) {
+        // the routing queries the forward's encode read: q_fixed with the gate
+        // closed; else the I/O-dtype copy (tensor cores) or fp32 (SIMT)
+        const bool q_f32 = gated && (pl.path == FLAREPP_PATH_SIMT || dtype == FLAREPP_F32);
+        const void* q_lat = !gated ? a.q_fixed : q_f32 ? static_cast<const void*>(ws + pl.off_q32)
+                                                       : static_cast<const void*>(ws + pl.off_q16);
+        const int q_bh = gated ? s.H : 0;
+        cudaError_t e;
+        if (dtype == FLAREPP_F32) e = run_backward_d<float, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        else if (dtype == FLAREPP_F16 && q_f32) e = run_backward_d<__half, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        else if (dtype == FLAREPP_F16) e = run_backward_d<__half, __half>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        else if (q_f32) e = run_backward_d<__nv_bfloat16, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        else e = run_backward_d<__nv_bfloat16, __nv_bfloat16>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        if (cudaGetLastError() != cudaSuccess) e = cudaErrorLaunchFailure;
+        rc = e == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+    }
+    if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
+    return rc;
+}
+
 }  // namespace
 }  // namespace flarepp
 
@@ -901,6 +1163,26 @@ int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const vo
                       int M, int D, int dtype, const flarepp_options_t* opts, void* stream) {
     return cp_decode(q, q_shared, z_state, k, y, B, H, N, M, D, dtype, opts, stream);
 }
+
+int flarepp_mixer_bwd(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+                      const void* v, const void* dy, float* dq0, float* dq_fixed, float* dgate, void* dk0, void* dk,
+                      void* dv, int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
+                      void* stream) {
+    BwdArgs a{};
+    a.q0 = q0; a.q_fixed = q_fixed; a.gate = gate; a.k0 = k0; a.k = k; a.v = v; a.dy = dy;
+    a.dq0 = dq0; a.dq_fixed = dq_fixed; a.dgate = dgate; a.dk0 = dk0; a.dk = dk; a.dv = dv;
+    return backward(a, B, H, N, M, D, dtype, opts, stream);
+}
+
+size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int dtype,
+                                         const flarepp_options_t* opts) {
+    const Shape s{B, H, N, M, D, dtype};
+    BwdPlan bp{};
+    if (make_bwd_plan(s, opts, &bp)) return 0;
+    return bp.total;
+}
+
+int flarepp_mixer_bwd_launches(int gated) { return gated ? 4 + 10 : 2 + 7; }
 
 int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate, const void* k0,
                            const void* k, const void* v, void* y, int B, int H, int N, int M, int D,

@@ -174,6 +174,17 @@ rms_normalise_rows(const T* __restrict__ x1, T* __restrict__ out1, int64_t rows1
 // are merged again across ranks.
 enum MergeMode { kMergeSynthesis = 0, kMergeEncode = 1, kMergeTriple = 2 };
 
+// Optional extra outputs of a forward call, kept for its backward: the
+// log-sum-exp (log2 units, of the scaled scores) of every latent row of the
+// synthesis and encode softmaxes, the synthesis output before the gate, and
+// whether to run the decode at all (the backward recomputes it per token).
+struct FwdExtras {
+    float* lse_syn = nullptr;    // [B,H,M]
+    float* lse_enc = nullptr;    // [B,H,M]
+    float* qdyn = nullptr;       // [B,H,M,D] fp32
+    bool decode = true;
+};
+
 struct MergeParams {
     const float* part_O;        // part c's O row r at part_O + c*o_part_stride + r*D
     const float2* part_ml;      // part c's (m, l) of row r at part_ml[c*ml_part_stride + r]
@@ -189,6 +200,8 @@ struct MergeParams {
     void* out_16;               // [B,H,M,D] in the I/O dtype (16-bit I/O only; may be null)
     float* user_out;            // optional [B,H,M,D]
     float* q_copy_out;          // optional: closed gate, write q = q_fixed broadcast over b
+    float* lse_out;             // optional [B,H,M]: m* + log2(L), the row's log-sum-exp in log2 units
+    float* pregate_out;         // optional [B,H,M,D] (synthesis): the merged value before the gate
 };
 
 template <typename T, int D>
@@ -250,6 +263,7 @@ merge_partials(MergeParams p) {
         }
     }
     if (sub != 0) return;
+    if (p.lse_out && li == 0) p.lse_out[row] = mstar + log2f(L);
     if (p.mode == kMergeTriple) {
 #pragma unroll
         for (int i = 0; i < F4PL; ++i)
@@ -266,6 +280,7 @@ merge_partials(MergeParams p) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int d = d0 + e;
+            if (p.pregate_out) p.pregate_out[row * D + d] = val[e];
             if (p.mode == kMergeSynthesis) val[e] = fmaf(p.gate[h], val[e], to_f32<T>(qf[d]));
             p.out_f32[row * D + d] = val[e];
             if constexpr (sizeof(T) == 2) {

@@ -1122,7 +1122,7 @@ inline void launch_merge_d(int D, const MergeParams& mp, int64_t rows, cudaStrea
 template <typename E, typename Mark>
 int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixed, const float* gate,
         const void* k0, const void* k, const void* v, void* y, float* q_out, float* z_out, Mark&& mark,
-        cudaStream_t st) {
+        cudaStream_t st, const FwdExtras& ex = FwdExtras{}) {
     const bool gated = gate != nullptr;
     const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
     // query maps use 128-row boxes, key/value maps the pass's tile height; the
@@ -1173,7 +1173,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
         if (rc) return rc;
         mark(st);
         mp.mode = kMergeSynthesis; mp.out_f32 = bu.q32; mp.out_16 = bu.q16; mp.user_out = q_out;
-        mp.q_copy_out = nullptr;
+        mp.q_copy_out = nullptr; mp.lse_out = ex.lse_syn; mp.pregate_out = ex.qdyn;
         launch_merge_d<E>(D, mp, rows, st);
         mark(st);
     }
@@ -1183,9 +1183,10 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     if (rc) return rc;
     mark(st);
     mp.mode = kMergeEncode; mp.out_f32 = bu.z32; mp.out_16 = bu.z16; mp.user_out = z_out;
-    mp.q_copy_out = gated ? nullptr : q_out;
+    mp.q_copy_out = gated ? nullptr : q_out; mp.lse_out = ex.lse_enc; mp.pregate_out = nullptr;
     launch_merge_d<E>(D, mp, rows, st);
     mark(st);
+    if (!ex.decode) return cudaGetLastError() == cudaSuccess ? 0 : 3;
 
     Params dp{};
     dp.mode = kDecode;

@@ -171,6 +171,20 @@ def random_inputs(B: int, H: int, N: int, M: int, D: int, dtype: str = "bf16", s
     return make_inputs(w, device=device, gate_zero=gate_zero)
 
 
+def random_cotangent(shape, dtype: str = "bf16", seed: int = 0, device: str = "cpu",
+                     device_rng: bool = False) -> torch.Tensor:
+    """An upstream gradient dy for the backward: i.i.d. N(0, 1) of the given
+    shape, drawn in fp64 with ``torch.Generator('cpu')`` seeded with ``seed``
+    (or in fp32 on the device with ``device_rng``, for the 1M-token sizes) and
+    rounded to the I/O dtype."""
+    out_dtype = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[dtype]
+    gen_dev = "cuda" if device_rng else "cpu"
+    gen = torch.Generator(gen_dev)
+    gen.manual_seed(seed)
+    x = torch.randn(*shape, generator=gen, dtype=torch.float32 if device_rng else torch.float64, device=gen_dev)
+    return x.to(out_dtype).to(device).contiguous()
+
+
 def algorithmic_counts(w: Workload, flare: bool = False) -> Dict[str, float]:
     """Per-call algorithmic work: HBM bytes of the inputs read and the output
     written once, tensor-core FLOPs of the score and value contractions, and
@@ -192,5 +206,5 @@ def describe(w: Workload) -> str:
             f"recipe={w.recipe} rms(q0)={w.rms_q0} rms(k0)={w.rms_k0}")
 
 
-__all__ = ["Workload", "WORKLOADS", "ORDER", "make_inputs", "random_inputs",
+__all__ = ["Workload", "WORKLOADS", "ORDER", "make_inputs", "random_inputs", "random_cotangent",
            "algorithmic_counts", "describe"]

@@ -41,7 +41,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.lib.flarepp_abi_version() == 3
+    assert lib.lib.flarepp_abi_version() == 4
+    assert lib.bwd_launches(True) == 14 and lib.bwd_launches(False) == 9
     assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
     for code in range(6):
         assert lib.status_string(code) not in ("", "unknown status")
@@ -145,3 +146,52 @@ def test_token_sharded_entries_checked(lib):
     dec = lib.lib.flarepp_cp_decode
     dec.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, i, vp, vp]
     assert dec(FAKE[1], 1, FAKE[3], FAKE[4], FAKE[4], 1, 2, 64, 16, 16, 1, None, None) == 1   # y aliases k
+
+
+def _bwd(lib, ptrs, B=1, H=2, N=64, M=16, D=16, dtype=1, opts=None):
+    return lib.lib.flarepp_mixer_bwd(*ptrs, B, H, N, M, D, dtype, opts, None)
+
+
+# q0, q_fixed, gate, k0, k, v, dy | dq0, dq_fixed, dgate, dk0, dk, dv (16-byte aligned, never dereferenced)
+BWD = [0x100000 * (i + 1) for i in range(13)]
+
+
+def test_backward_entry_checks(lib):
+    for i in (1, 4, 5, 6, 8, 11, 12):      # always required
+        p = list(BWD)
+        p[i] = None
+        assert _bwd(lib, p) == 1, i
+    for i in (0, 3, 7, 9, 10):             # required with the gate open
+        p = list(BWD)
+        p[i] = None
+        assert _bwd(lib, p) == 1, i
+    p = list(BWD)
+    p[2] = None                            # closed gate: q0, k0, dq0, dgate, dk0 not needed, but no GPU here:
+    for i in (0, 3, 7, 9, 10):             # the call gets past the checks and fails on the allocation
+        p[i] = None
+    assert _bwd(lib, p) in (3, 4)
+    p = list(BWD)
+    p[11] = p[4] + 32                      # dk overlaps k
+    assert _bwd(lib, p) == 1
+    p = list(BWD)
+    p[12] = p[11]                          # dv aliases dk
+    assert _bwd(lib, p) == 1
+    p = list(BWD)
+    p[6] = p[6] + 8                        # dy misaligned
+    assert _bwd(lib, p) == 1
+    assert _bwd(lib, BWD, D=48) == 2
+    assert _bwd(lib, BWD, B=0) == 1
+    o = lib.Options(0.0, 0, 0, 0, None, None, None, 0, None, 0, 1)   # synthesis normalisation: not in the backward
+    assert _bwd(lib, BWD, opts=ctypes.byref(o)) == 2
+    o = lib.Options(0.0, 0, 0, 0, None, None, 0x1000, 16, None)      # workspace too small
+    assert _bwd(lib, BWD, opts=ctypes.byref(o)) == 4
+
+
+def test_backward_workspace_query(lib):
+    a = lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16)
+    assert a > lib.workspace_bytes(1, 2, 1000, 64, 32, lib.BF16)
+    assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 48, lib.BF16) == 0
+    # the fp32 buffer of the decode's share of dk dominates: B*H*N*D*4 bytes
+    big = lib.bwd_workspace_bytes(1, 8, 1 << 20, 512, 64, lib.BF16)
+    assert big > 8 * (1 << 20) * 64 * 4
+    assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16, force_chunks=1) < a

@@ -1,0 +1,148 @@
+"""Backward of the mixer (flarepp_mixer_bwd) against the fp64 gradient oracle
+(oracle/backward.py, itself pinned by central differences of the forward
+oracle), through the C ABI on seeded inputs.
+
+Covers every I/O dtype and head dim, ragged token and latent counts (several
+shared-memory stages on both sides, tails), both forward kernel families for
+the recomputed passes, the closed gate (FLARE), the scale option, both token
+layouts, forced token-chunk counts, and determinism."""
+import numpy as np
+import pytest
+import torch
+
+from oracle.backward import flarepp_backward
+from parity import assert_grad_parity, to64
+from rank_latent_attention_mixer_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+GRADS = ("dq0", "dq_fixed", "dgate", "dk0", "dk", "dv")
+FLARE_GRADS = ("dq_fixed", "dk", "dv")
+
+
+def binding():
+    from rank_latent_attention_mixer_b200 import binding as b
+    return b
+
+
+def inputs(B, H, N, M, D, dt, seed):
+    x = W.random_inputs(B, H, N, M, D, dtype=dt, seed=seed)
+    dy = W.random_cotangent((B, H, N, D), dt, seed=seed + 100)
+    return x, dy
+
+
+def oracle_grads(x, dy, gate=None, scale=0.0):
+    g = x["gate"] if gate is None else gate
+    return flarepp_backward(to64(x["q0"]), to64(x["q_fixed"]), to64(g), to64(x["k0"]), to64(x["k"]),
+                            to64(x["v"]), to64(dy), scale=scale)
+
+
+def gpu_grads(x, dy, flare=False, **kw):
+    b = binding()
+    d = {k: v.to(DEV) for k, v in x.items()}
+    g = b.mixer_bwd(d["q0"], d["q_fixed"], None if flare else d["gate"], d["k0"], d["k"], d["v"], dy.to(DEV), **kw)
+    torch.cuda.synchronize()
+    assert b.check_device_status() == 0
+    return g
+
+
+CASES = [
+    # (B, H, N, M, D, dtype, path): ragged N and M, several latent stages (M > 4096/D), every D
+    ((1, 2, 1000, 48, 16, "f32"), 0),
+    ((2, 1, 530, 70, 128, "f32"), 0),
+    ((1, 2, 777, 300, 32, "f32"), 0),
+    ((2, 2, 1500, 128, 64, "bf16"), 0),
+    ((1, 2, 700, 64, 32, "bf16"), 0),
+    ((1, 3, 1100, 200, 16, "bf16"), 0),
+    ((1, 2, 650, 96, 128, "bf16"), 0),
+    ((1, 2, 700, 96, 32, "f16"), 0),
+    ((1, 2, 900, 80, 64, "bf16"), 1),     # the recomputed forward on the SIMT kernels (fp32 routing queries)
+    ((1, 2, 600, 40, 64, "f16"), 1),
+]
+
+
+@pytest.mark.parametrize("case,path", CASES, ids=[f"{'x'.join(map(str, c[:5]))}-{c[5]}-p{p}" for c, p in CASES])
+def test_backward_parity(case, path):
+    B, H, N, M, D, dt = case
+    x, dy = inputs(B, H, N, M, D, dt, seed=sum(case[:5]))
+    ref = oracle_grads(x, dy)
+    g = gpu_grads(x, dy, path=path)
+    for name in GRADS:
+        m = assert_grad_parity(g[name], ref[name], dt, name)
+        print(case, path, name, {k: m[k] for k in ("rel_l2", "max_abs_rel_to_max") if k in m})
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_closed_gate_is_flare_backward(dt):
+    """gate == NULL gives FLARE's gradients; they equal the gated mixer's at gate 0."""
+    x, dy = inputs(2, 2, 900, 64, 32, dt, seed=5)
+    ref = oracle_grads(x, dy, gate=np.zeros(2))
+    g = gpu_grads(x, dy, flare=True)
+    assert set(g) == set(FLARE_GRADS)
+    for name in FLARE_GRADS:
+        assert_grad_parity(g[name], ref[name], dt, name)
+    gz = gpu_grads({**x, "gate": torch.zeros_like(x["gate"])}, dy)
+    for name in FLARE_GRADS:
+        assert torch.equal(g[name], gz[name]), f"{name}: closed gate and zero gate differ"
+    assert torch.count_nonzero(gz["dq0"]) == 0 and torch.count_nonzero(gz["dk0"]) == 0
+    assert_grad_parity(gz["dgate"], ref["dgate"], dt, "dgate")
+
+
+def test_scale_option():
+    x, dy = inputs(1, 2, 640, 40, 32, "f32", seed=11)
+    ref = oracle_grads(x, dy, scale=1.0)
+    g = gpu_grads(x, dy, scale=1.0)
+    for name in GRADS:
+        assert_grad_parity(g[name], ref[name], "f32", name)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_token_layout_bnhd_identical(dt):
+    x, dy = inputs(2, 3, 500, 50, 32, dt, seed=13)
+    g = gpu_grads(x, dy)
+    xt = {k: (v.transpose(1, 2).contiguous() if v.dim() == 4 else v) for k, v in x.items()}
+    gt = gpu_grads(xt, dy.transpose(1, 2).contiguous(), layout="bnhd")
+    for name in GRADS:
+        a = gt[name].transpose(1, 2) if gt[name].dim() == 4 else gt[name]
+        assert torch.equal(a, g[name]), f"{name}: [B,N,H,D] layout differs from [B,H,N,D]"
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_chunk_invariance_and_determinism(dt):
+    """The token sums split into chunks are exact up to rounding; repeated calls are bitwise equal."""
+    x, dy = inputs(1, 2, 3000, 64, 64, dt, seed=17)
+    ref = oracle_grads(x, dy)
+    g_def = gpu_grads(x, dy)
+    g_again = gpu_grads(x, dy)
+    for name in GRADS:
+        assert torch.equal(g_def[name], g_again[name]), f"{name}: not deterministic"
+    for chunks in (1, 2, 7):
+        g = gpu_grads(x, dy, force_chunks=chunks)
+        for name in GRADS:
+            assert_grad_parity(g[name], ref[name], dt, f"{name} (chunks={chunks})")
+            diff = (g[name].double() - g_def[name].double()).abs().max().item()
+            scale = g_def[name].double().abs().max().item()
+            assert diff <= (1e-5 if dt == "f32" else 1e-2) * scale, (name, chunks, diff, scale)
+
+
+def test_single_token_and_single_latent():
+    """N = 1: every softmax over tokens has one term (its gradients through P vanish);
+    M = 1: the decode weight is 1, so dk gets no decode term."""
+    for (N, M) in ((1, 8), (37, 1)):
+        x, dy = inputs(1, 2, N, M, 16, "f32", seed=N + M)
+        ref = oracle_grads(x, dy)
+        g = gpu_grads(x, dy)
+        for name in GRADS:
+            assert_grad_parity(g[name], ref[name], "f32", f"{name} N={N} M={M}")
+
+
+def test_caller_workspace():
+    b = binding()
+    x, dy = inputs(1, 2, 300, 32, 32, "bf16", seed=3)
+    need = b.bwd_workspace_bytes(1, 2, 300, 32, 32, b.BF16)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    g1 = gpu_grads(x, dy, workspace=ws)
+    g2 = gpu_grads(x, dy)
+    for name in GRADS:
+        assert torch.equal(g1[name], g2[name])
