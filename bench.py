@@ -632,9 +632,19 @@ BWD_STAGES_GATED = ["fwd split(synthesis)", "fwd merge(q)", "fwd split(encode)",
                     "reduce_batch"]
 BWD_STAGES_FLARE = ["fwd split(encode)", "fwd merge(z)", "decode_rows", "decode_cols", "reduce(decode)",
                     "token_cols(encode)", "latent_rows(encode)", "reduce(encode)", "reduce_batch"]
+BWD_TC_STAGES_GATED = ["fwd split(synthesis)", "fwd merge(q)", "fwd split(encode)", "fwd merge(z)",
+                       "fwd decode(stats)", "tc_latent(decode)", "tc_token(decode)", "reduce(decode)",
+                       "tc_token(encode)", "tc_latent(encode)", "reduce(encode)", "tc_token(synthesis)",
+                       "tc_latent(synthesis)", "reduce(synthesis)", "reduce_batch"]
+BWD_TC_STAGES_FLARE = ["fwd split(encode)", "fwd merge(z)", "fwd decode(stats)", "tc_latent(decode)",
+                       "tc_token(decode)", "reduce(decode)", "tc_token(encode)", "tc_latent(encode)",
+                       "reduce(encode)", "reduce_batch"]
 # FLOPs per (b, h, n, m, d) of each backward kernel as executed (2 per multiply-add):
 # decode rows recompute the decode softmax and y (4), then score, <dy, z> and dS q (6)
 BWD_KERNEL_FLOPS = {"decode_rows": 10, "decode_cols": 8, "token_cols": 8, "latent_rows": 6}
+# tensor-core kernel: S and dP (4), acc1 (2), acc2 (2 where present)
+BWD_TC_FLOPS = {"tc_latent(decode)": 8, "tc_token(decode)": 6, "tc_token(encode)": 8, "tc_latent(encode)": 6,
+                "tc_token(synthesis)": 8, "tc_latent(synthesis)": 6}
 
 
 def fp32_simt_peak_tflops(peaks):
@@ -675,8 +685,12 @@ def run_backward_bench(args):
     if gated:
         out_t.update(dk0=torch.empty_like(x["k0"]), dq0=torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev),
                      dgate=torch.empty((w.H,), dtype=torch.float32, device=dev))
-    n_launch = fb.bwd_launches(gated)
-    names = BWD_STAGES_GATED if gated else BWD_STAGES_FLARE
+    used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
+    n_launch = fb.bwd_launches(gated, used_path)
+    if used_path == fb.PATH_TCGEN05:
+        names = BWD_TC_STAGES_GATED if gated else BWD_TC_STAGES_FLARE
+    else:
+        names = BWD_STAGES_GATED if gated else BWD_STAGES_FLARE
     fits_l2 = 6 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
 
@@ -714,15 +728,21 @@ def run_backward_bench(args):
     peaks, peak_src = load_peaks()
     peak_alu = fp32_simt_peak_tflops(peaks)
     kern = {}
+    tc_path = used_path == fb.PATH_TCGEN05
+
+    def flops_of(nm):
+        return BWD_TC_FLOPS.get(nm) if tc_path else BWD_KERNEL_FLOPS.get(nm.split("(")[0])
+
     for nm, ms in zip(names, stage):
-        base = nm.split("(")[0]
-        f = BWD_KERNEL_FLOPS.get(base)
+        f = flops_of(nm)
         kern[nm] = {"ms": round(ms, 4), "share": round(ms / total, 4)}
         if f:
             kern[nm]["tflops"] = round(f * bhnmd / (ms * 1e-3) / 1e12, 2)
-    # the dominant kernel's roofline: SIMT fp32 FMA arithmetic
-    top = max((nm for nm in names if BWD_KERNEL_FLOPS.get(nm.split("(")[0])), key=lambda nm: kern[nm]["ms"])
+    # the dominant backward kernel's roofline: the tensor pipe (tcgen05 kernel) or
+    # SIMT fp32 FMA arithmetic
+    top = max((nm for nm in names if flops_of(nm)), key=lambda nm: kern[nm]["ms"])
     achieved = kern[top]["tflops"]
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     counts = W.algorithmic_counts(w, flare=not gated)
     ms_step = max_ms / K
     passes = 3 if gated else 2
@@ -732,14 +752,18 @@ def run_backward_bench(args):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
-                   "gate": "open (FLARE++)" if gated else "closed (FLARE)", "forward_path": args.path,
+                   "gate": "open (FLARE++)" if gated else "closed (FLARE)",
+                   "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)")},
         "algorithmic_tflops": round(10.0 * passes * bhnmd / (ms_step * 1e-3) / 1e12, 2),
         "gpu_launches": K * n_launch,
-        "roofline": {"bound": "alu", "kernel": top, "achieved": achieved, "peak": round(peak_alu, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / peak_alu, 4), "traffic": None,
-                     "peak_kind": "FP32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"},
+        "roofline": ({"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                      "frac": round(achieved / peak_t, 4), "traffic": None,
+                      "peak_kind": f"{peak_src} bf16 sustained"} if tc_path else
+                     {"bound": "alu", "kernel": top, "achieved": achieved, "peak": round(peak_alu, 1),
+                      "unit": "TFLOP/s", "frac": round(achieved / peak_alu, 4), "traffic": None,
+                      "peak_kind": "FP32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}),
         "stages": kern,
         "clocks": sampler.summary(),
     }

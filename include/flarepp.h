@@ -284,15 +284,17 @@ int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const vo
  *   dgate     DEVICE fp32 [H]: dL/d(gate value), not of the logit
  *   dk0, dk, dv     [B,H,N,D] token layout, I/O dtype
  * No output may overlap an input or another output.  opts (may be NULL):
- * scale, path (the kernel family of the recomputed forward passes; the
- * backward's own kernels are SIMT fp32 for every dtype), force_chunks (the
- * token chunks of both the recomputed passes and the backward's token sums),
+ * scale, path (the kernel family: with 16-bit I/O the tcgen05 forward and the
+ * tcgen05 backward kernel, whose score and gradient products take bf16/fp16
+ * operands -- P and dS rounded to the I/O type -- with fp32 accumulation;
+ * with fp32 I/O, or path = SIMT, fp32 SIMT kernels throughout), force_chunks
+ * (the token chunks of both the recomputed passes and the backward's token sums),
  * workspace / workspace_bytes (>= flarepp_mixer_bwd_workspace_bytes),
  * stage_events (recorded before the first and after every launch), layout.
  * norm_synthesis = 1 gives FLAREPP_ERR_UNSUPPORTED; q_out, z_out are ignored.
- * Arithmetic is fp32 with fp32 accumulation of every sum; sums over tokens
- * are taken per token chunk and added in a fixed order (deterministic); the
- * 16-bit gradients are rounded once, at the end.  Asynchronous on `stream`. */
+ * Sums over tokens are taken per token chunk and added in a fixed order
+ * (deterministic); the 16-bit gradients are rounded once, at the end.
+ * Asynchronous on `stream`. */
 int flarepp_mixer_bwd(const void* q0, const void* q_fixed, const float* gate,
                       const void* k0, const void* k, const void* v, const void* dy,
                       float* dq0, float* dq_fixed, float* dgate,
@@ -307,9 +309,12 @@ int flarepp_mixer_bwd(const void* q0, const void* q_fixed, const float* gate,
 size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int dtype,
                                          const flarepp_options_t* opts);
 
-/* Kernel launches one backward call makes: gated 14 (4 recomputed forward
- * passes, 3 per attention, 1 batch reduce), closed gate 9. */
-int flarepp_mixer_bwd_launches(int gated);
+/* Kernel launches one backward call makes, for the kernel family `path`
+ * (flarepp_path_t, as flarepp_selected_path reports it) of its recomputed
+ * forward: SIMT, gated 14 (4 recomputed forward passes, 3 per attention, 1
+ * batch reduce), closed gate 9; TCGEN05, gated 15 (the forward's decode runs
+ * too, for the per-token statistics), closed gate 10. */
+int flarepp_mixer_bwd_launches(int gated, int path);
 
 /* FLAREPP_ABI_VERSION of the loaded library. */
 int flarepp_abi_version(void);

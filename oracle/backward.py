@@ -47,8 +47,8 @@ def _sdpa_bwd(Q, K, V, P, dO, s):
 
 def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
     """Gradients of the gated mixer (gate open).  Returns a dict with
-    dq0, dq_fixed [H,M,D], dgate [H], dk0, dk, dv [B,H,N,D], and the forward's
-    y [B,H,N,D] (fp64)."""
+    dq0, dq_fixed [H,M,D], dgate [H], dk0, dk, dv [B,H,N,D], the forward's
+    y [B,H,N,D], and the intermediates q_dyn and dq = dL/dq [B,H,M,D] (fp64)."""
     q0, q_fixed, gate = _f64(q0), _f64(q_fixed), _f64(gate).reshape(-1)
     k0, k, v, dy = _f64(k0), _f64(k), _f64(v), _f64(dy)
     B, H, N, D = k.shape
@@ -57,6 +57,8 @@ def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
     g = {name: np.zeros_like(a) for name, a in
          (("dq0", q0), ("dq_fixed", q_fixed), ("dgate", gate), ("dk0", k0), ("dk", k), ("dv", v))}
     y = np.empty_like(k)
+    q_dyn_all = np.empty((B, H, M, D))
+    dq_all = np.empty((B, H, M, D))
     for b in range(B):
         for h in range(H):
             # forward, keeping the weights
@@ -69,6 +71,7 @@ def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
             # encode: z = SDPA(q, k, v)
             dq_b, dk_b, dv = _sdpa_bwd(q, k[b, h], v[b, h], P_enc, dz, s)
             dq = dq_a + dq_b
+            q_dyn_all[b, h], dq_all[b, h] = q_dyn, dq
             # gate: q = q_fixed + gate * q_dyn
             g["dq_fixed"][h] += dq
             g["dgate"][h] += np.sum(dq * q_dyn)
@@ -80,4 +83,5 @@ def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
             g["dk"][b, h] = dk_a + dk_b
             g["dv"][b, h] = dv
     g["y"] = y
+    g["q_dyn"], g["dq"] = q_dyn_all, dq_all
     return g

@@ -63,7 +63,7 @@ def _load() -> ctypes.CDLL:
     lib.flarepp_mixer_bwd.argtypes = [vp] * 13 + [i] * 6 + [ctypes.POINTER(Options), vp]
     lib.flarepp_mixer_bwd_workspace_bytes.argtypes = [i] * 6 + [ctypes.POINTER(Options)]
     lib.flarepp_mixer_bwd_workspace_bytes.restype = ctypes.c_size_t
-    lib.flarepp_mixer_bwd_launches.argtypes = [i]
+    lib.flarepp_mixer_bwd_launches.argtypes = [i, i]
     for name in ("flarepp_mixer_fwd", "flarepp_mixer_fwd_ex", "flarepp_mixer_fwd_host", "flare_fwd",
                  "flarepp_selected_path", "flarepp_check_device_status", "flarepp_abi_version",
                  "flarepp_launches_per_call", "flarepp_mixer_bwd", "flarepp_mixer_bwd_launches"):
@@ -199,8 +199,9 @@ def _event_array(stage_events):
     return (ctypes.c_void_p * len(handles))(*handles), len(handles)
 
 
-def bwd_launches(gated: bool = True) -> int:
-    return int(lib.flarepp_mixer_bwd_launches(int(gated)))
+def bwd_launches(gated: bool = True, path: int = PATH_SIMT) -> int:
+    """Launches of one backward call whose forward runs on kernel family ``path`` (SIMT or TCGEN05)."""
+    return int(lib.flarepp_mixer_bwd_launches(int(gated), int(path)))
 
 
 def bwd_workspace_bytes(B, H, N, M, D, dtype=BF16, path=PATH_AUTO, force_chunks=0, layout="bhnd") -> int:

@@ -18,6 +18,7 @@
 #include "../../include/flarepp.h"
 #include "common.cuh"
 #include "kernels_bwd.cuh"
+#include "kernels_bwd_tc.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 
@@ -802,13 +803,30 @@ int cp_decode(const void* q, int q_shared, const void* z_state, const void* k, v
 //   batch reduce    dq_fixed, dq0, dgate (sums over the batch)
 // With the gate closed (FLARE) the synthesis stages are skipped and the batch
 // reduce gives dq_fixed only.
+//
+// On the tensor-core path (16-bit I/O with the tcgen05 forward) the forward's
+// decode runs too, writing per token the log-sum-exp and <dy, y> instead of y,
+// and every token-sum and latent-sum step is one launch of bwd_tc::bwd_kernel
+// (kernels_bwd_tc.cuh); the reduces also write 16-bit copies of dz and dq_dyn
+// (tensor-core operands) and the padded (log-sum-exp, Delta) pairs of the next
+// pass.
 struct BwdPlan {
     Plan fwd;
+    bool tc;                     // tensor-core backward
     int chunks, chunk_len, row_blocks;
     int64_t tok_blocks;
+    int64_t n_pad, m_pad;        // strides of the padded statistics (multiples of the column tile)
     size_t off_lse_syn, off_lse_enc, off_qdyn, off_lse_tok, off_delta_tok, off_dk_acc, off_part1, off_part2, off_dz,
-        off_dq, off_dqdyn, off_delta_enc, off_delta0, off_dq0b, total;
+        off_dq, off_dqdyn, off_delta_enc, off_delta0, off_dq0b, off_stats_tok, off_stats_enc, off_stats_syn,
+        off_dz16, off_dqdyn16, total;
 };
+
+int tc_bwd_chunks(const Shape& s, int force) {
+    const int tiles = (s.N + bwd_tc::kKT - 1) / bwd_tc::kKT;
+    const int chunks = force > 0 ? std::min(force, tiles) : bwd_tc::plan_chunks(s.B, s.H, s.M, s.N, s.D);
+    const int per = (tiles + chunks - 1) / chunks;
+    return (tiles + per - 1) / per;
+}
 
 int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     int rc = make_plan(s, o, &bp->fwd);
@@ -820,24 +838,40 @@ int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     bp->row_blocks = (s.M + rows_per_cta - 1) / rows_per_cta;
     bp->tok_blocks = (s.N + (int64_t)rows_per_cta - 1) / rows_per_cta;
     const int64_t tiles = (s.N + tile - 1) / tile;
-    int64_t chunks;
-    if (o && o->force_chunks > 0) {
-        chunks = std::min<int64_t>(o->force_chunks, tiles);
+    bp->tc = bp->fwd.path == FLAREPP_PATH_TCGEN05;
+    const int force = o ? o->force_chunks : 0;
+    if (bp->tc) {
+        bp->chunks = tc_bwd_chunks(s, force);
+        bp->chunk_len = 0;
     } else {
-        // about eight CTAs per SM over the latent-side grid, chunks of >= 1 tile
-        const int64_t target = 8 * kNumSMs, per = s.bh() * bp->row_blocks;
-        chunks = std::max<int64_t>(1, std::min<int64_t>((target + per - 1) / per, tiles));
+        int64_t chunks;
+        if (force > 0) {
+            chunks = std::min<int64_t>(force, tiles);
+        } else {
+            // about eight CTAs per SM over the latent-side grid, chunks of >= 1 tile
+            const int64_t target = 8 * kNumSMs, per = s.bh() * bp->row_blocks;
+            chunks = std::max<int64_t>(1, std::min<int64_t>((target + per - 1) / per, tiles));
+        }
+        const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
+        bp->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
+        bp->chunks = (int)((s.N + (int64_t)bp->chunk_len - 1) / bp->chunk_len);
     }
-    const int64_t tiles_per_chunk = (tiles + chunks - 1) / chunks;
-    bp->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
-    bp->chunks = (int)((s.N + (int64_t)bp->chunk_len - 1) / bp->chunk_len);
+    const int64_t kt = bwd_tc::kKT;
+    bp->n_pad = (s.N + kt - 1) / kt * kt;
+    bp->m_pad = (s.M + kt - 1) / kt * kt;
     const size_t lat = (size_t)s.bh() * s.M, latd = lat * s.D, tok = (size_t)s.bh() * s.N;
+    const size_t tc_on = bp->tc ? 1 : 0, simt_on = 1 - tc_on;
     size_t off = bp->fwd.total;
     bp->off_lse_syn = off;   off = align_up(off + lat * sizeof(float));
     bp->off_lse_enc = off;   off = align_up(off + lat * sizeof(float));
     bp->off_qdyn = off;      off = align_up(off + latd * sizeof(float));
-    bp->off_lse_tok = off;   off = align_up(off + tok * sizeof(float));
-    bp->off_delta_tok = off; off = align_up(off + tok * sizeof(float));
+    bp->off_lse_tok = off;   off = align_up(off + simt_on * tok * sizeof(float));
+    bp->off_delta_tok = off; off = align_up(off + simt_on * tok * sizeof(float));
+    bp->off_stats_tok = off; off = align_up(off + tc_on * (size_t)s.bh() * bp->n_pad * sizeof(float2));
+    bp->off_stats_enc = off; off = align_up(off + tc_on * (size_t)s.bh() * bp->m_pad * sizeof(float2));
+    bp->off_stats_syn = off; off = align_up(off + tc_on * (size_t)s.bh() * bp->m_pad * sizeof(float2));
+    bp->off_dz16 = off;      off = align_up(off + tc_on * latd * sizeof(uint16_t));
+    bp->off_dqdyn16 = off;   off = align_up(off + tc_on * latd * sizeof(uint16_t));
     bp->off_dk_acc = off;    off = align_up(off + tok * s.D * sizeof(float));
     bp->off_part1 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
     bp->off_part2 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
@@ -941,7 +975,7 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
     rp.part1 = p.part1; rp.part2 = p.part2; rp.chunks = bp.chunks;
     rp.B = s.B; rp.H = s.H; rp.M = s.M; rp.scale = p.scale;
     rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = dz; rp.dq = dq; rp.delta = delta_enc;
-    launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+    launch_bwd_kernel(bwd::reduce_partials<float, D>, red_grid, dim3(256), rp);
     ev.mark(st);
 
     // encode: z = SDPA(q, k, v)
@@ -952,7 +986,7 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
     launch_bwd_kernel(bwd::latent_rows<T, TQ, D>, lat_grid, dim3(bwd::kThreads), p);
     ev.mark(st);
     rp.mode = bwd::kReduceEncode; rp.gate = a.gate; rp.qdyn = qdyn; rp.dqdyn = dqdyn; rp.delta = delta0;
-    launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+    launch_bwd_kernel(bwd::reduce_partials<float, D>, red_grid, dim3(256), rp);
     ev.mark(st);
 
     if (gated) {
@@ -965,7 +999,7 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
         launch_bwd_kernel(bwd::latent_rows<T, T, D>, lat_grid, dim3(bwd::kThreads), p);
         ev.mark(st);
         rp.mode = bwd::kReduceSynthesis; rp.dq0b = dq0b;
-        launch_bwd_kernel(bwd::reduce_partials<D>, red_grid, dim3(256), rp);
+        launch_bwd_kernel(bwd::reduce_partials<float, D>, red_grid, dim3(256), rp);
         ev.mark(st);
     }
     bwd::BatchParams bt{};
@@ -976,6 +1010,115 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
     ev.mark(st);
     (void)L::G;
     return launch_bwd_kernel.err;
+}
+
+// The tensor-core backward after the recomputed forward (which has left q, z,
+// their 16-bit copies, the log-sum-exps, q_dyn and the per-token statistics
+// in the workspace).
+template <typename E, int D>
+cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a, char* ws, StageEvents& ev,
+                            cudaStream_t st) {
+    using bwd_tc::Operand;
+    const bool gated = a.gate != nullptr;
+    const Plan& pl = bp.fwd;
+    const float scale = pl.scale_log2 / kLog2e;
+    cudaError_t err = cudaSuccess;
+    auto note = [&](int rc) {
+        if (rc && err == cudaSuccess) err = cudaErrorLaunchFailure;
+        ev.mark(st);
+    };
+    float2* stats_tok = reinterpret_cast<float2*>(ws + bp.off_stats_tok);
+    float2* stats_enc = reinterpret_cast<float2*>(ws + bp.off_stats_enc);
+    float2* stats_syn = reinterpret_cast<float2*>(ws + bp.off_stats_syn);
+    float* part1 = reinterpret_cast<float*>(ws + bp.off_part1);
+    float* part2 = reinterpret_cast<float*>(ws + bp.off_part2);
+    float* dk_acc = reinterpret_cast<float*>(ws + bp.off_dk_acc);
+    const Operand q_lat = gated ? Operand{ws + pl.off_q16, false, false} : Operand{a.q_fixed, false, true};
+    const Operand z_lat{ws + pl.off_z16, false, false};
+    const Operand dz_lat{ws + bp.off_dz16, false, false};
+    const Operand dqdyn_lat{ws + bp.off_dqdyn16, false, false};
+    const Operand q0{a.q0, false, true};
+    const Operand k{a.k, true, false}, v{a.v, true, false}, dy{a.dy, true, false}, k0{a.k0, true, false};
+
+    bwd_tc::Launch base{};
+    base.B = s.B; base.H = s.H; base.N = s.N; base.M = s.M; base.D = s.D;
+    base.tok = pl.tok;
+    base.scale_log2 = pl.scale_log2;
+    base.scale = scale;
+    base.chunks = bp.chunks;
+    auto latent_rows = [&](Operand A, Operand C, Operand Bc, Operand Ec, bool acc2, bool col_stats,
+                           const float2* stats, int64_t stride) {
+        bwd_tc::Launch L = base;
+        L.a = A; L.c = C; L.b = Bc; L.e = Ec;
+        L.rows_tok = false; L.has_acc2 = acc2; L.stats_per_col = col_stats;
+        L.stats = stats; L.stats_stride = stride;
+        L.epi = bwd_tc::kEpiPartials; L.part1 = part1; L.part2 = part2;
+        note(bwd_tc::launch_bwd_d<E>(L, st));
+    };
+    auto token_rows = [&](Operand A, Operand C, Operand Bc, Operand Ec, bool acc2, bool col_stats,
+                          const float2* stats, int64_t stride, int epi, void* out1, void* out2) {
+        bwd_tc::Launch L = base;
+        L.a = A; L.c = C; L.b = Bc; L.e = Ec;
+        L.rows_tok = true; L.has_acc2 = acc2; L.stats_per_col = col_stats;
+        L.stats = stats; L.stats_stride = stride;
+        L.epi = epi; L.f32 = dk_acc; L.out1 = out1; L.out2 = out2;
+        note(bwd_tc::launch_bwd_d<E>(L, st));
+    };
+    BwdLauncher launch{st};
+    const int64_t rows = s.bh() * s.M;
+    const dim3 red_grid((unsigned)((rows + 7) / 8));
+    bwd::ReduceParams rp{};
+    rp.part1 = part1; rp.part2 = part2; rp.chunks = bp.chunks;
+    rp.B = s.B; rp.H = s.H; rp.M = s.M; rp.scale = scale;
+    rp.stats_stride = bp.m_pad;
+    float* z32 = reinterpret_cast<float*>(ws + pl.off_z32);
+    float* dq = reinterpret_cast<float*>(ws + bp.off_dq);
+    float* qdyn = reinterpret_cast<float*>(ws + bp.off_qdyn);
+    float* dq0b = reinterpret_cast<float*>(ws + bp.off_dq0b);
+
+    // decode y = SDPA(k, q, z): latent side (dq_dec, dz partials), token side (dk_dec)
+    latent_rows(q_lat, z_lat, k, dy, true, true, stats_tok, bp.n_pad);
+    token_rows(k, dy, q_lat, z_lat, false, false, stats_tok, bp.n_pad, bwd_tc::kEpiTokF32, nullptr, nullptr);
+    rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = reinterpret_cast<float*>(ws + bp.off_dz); rp.dq = dq;
+    rp.delta = reinterpret_cast<float*>(ws + bp.off_delta_enc);
+    rp.out16 = ws + bp.off_dz16; rp.stats_out = stats_enc; rp.lse_in = reinterpret_cast<float*>(ws + bp.off_lse_enc);
+    launch(bwd::reduce_partials<E, D>, red_grid, dim3(256), rp);
+    ev.mark(st);
+    // encode z = SDPA(q, k, v): token side (dk = dk_dec + dk_enc, dv), latent side (dq_enc partials)
+    token_rows(k, v, q_lat, dz_lat, true, true, stats_enc, bp.m_pad, bwd_tc::kEpiTokDkDv, a.dk, a.dv);
+    latent_rows(q_lat, dz_lat, k, v, false, false, stats_enc, bp.m_pad);
+    rp.mode = bwd::kReduceEncode; rp.gate = a.gate; rp.qdyn = qdyn;
+    rp.dqdyn = reinterpret_cast<float*>(ws + bp.off_dqdyn); rp.delta = reinterpret_cast<float*>(ws + bp.off_delta0);
+    rp.out16 = ws + bp.off_dqdyn16; rp.stats_out = gated ? stats_syn : nullptr;
+    rp.lse_in = reinterpret_cast<float*>(ws + bp.off_lse_syn);
+    launch(bwd::reduce_partials<E, D>, red_grid, dim3(256), rp);
+    ev.mark(st);
+    if (gated) {
+        // synthesis q_dyn = SDPA(q0, k0, k0) with output gradient dq_dyn = gate dq
+        token_rows(k0, k0, q0, dqdyn_lat, true, true, stats_syn, bp.m_pad, bwd_tc::kEpiTokDk0, a.dk0, nullptr);
+        latent_rows(q0, dqdyn_lat, k0, k0, false, false, stats_syn, bp.m_pad);
+        rp.mode = bwd::kReduceSynthesis; rp.dq0b = dq0b; rp.out16 = nullptr; rp.stats_out = nullptr;
+        launch(bwd::reduce_partials<E, D>, red_grid, dim3(256), rp);
+        ev.mark(st);
+    }
+    bwd::BatchParams bt{};
+    bt.B = s.B; bt.H = s.H; bt.M = s.M;
+    bt.dq = dq; bt.dq_fixed = a.dq_fixed;
+    if (gated) { bt.dq0b = dq0b; bt.qdyn = qdyn; bt.dq0 = a.dq0; bt.dgate = a.dgate; }
+    launch(bwd::reduce_batch<D>, dim3((unsigned)s.H), dim3(256), bt);
+    ev.mark(st);
+    return err != cudaSuccess ? err : launch.err;
+}
+
+template <typename E>
+cudaError_t run_backward_tc_d(const Shape& s, const BwdPlan& bp, const BwdArgs& a, char* ws, StageEvents& ev,
+                              cudaStream_t st) {
+    switch (s.D) {
+        case 16: return run_backward_tc<E, 16>(s, bp, a, ws, ev, st);
+        case 32: return run_backward_tc<E, 32>(s, bp, a, ws, ev, st);
+        case 64: return run_backward_tc<E, 64>(s, bp, a, ws, ev, st);
+        default: return run_backward_tc<E, 128>(s, bp, a, ws, ev, st);
+    }
 }
 
 template <typename T, typename TQ>
@@ -1023,9 +1166,19 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
     ex.lse_syn = reinterpret_cast<float*>(ws + bp.off_lse_syn);
     ex.lse_enc = reinterpret_cast<float*>(ws + bp.off_lse_enc);
     ex.qdyn = reinterpret_cast<float*>(ws + bp.off_qdyn);
-    ex.decode = false;
+    ex.decode = bp.tc;      // the tensor-core path takes the per-token statistics from the forward's decode
+    if (bp.tc) {
+        ex.tok_stats = reinterpret_cast<float2*>(ws + bp.off_stats_tok);
+        ex.tok_stats_stride = bp.n_pad;
+        ex.dy = a.dy;
+    }
     rc = run(s, pl, a.q0, a.q_fixed, a.gate, a.k0, a.k, a.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
-    if (rc == FLAREPP_OK) {
+    if (rc == FLAREPP_OK && bp.tc) {
+        cudaError_t e;
+        if (dtype == FLAREPP_F16) e = run_backward_tc_d<__half>(s, bp, a, ws, ev, st);
+        else e = run_backward_tc_d<__nv_bfloat16>(s, bp, a, ws, ev, st);
+        rc = (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+    } else if (rc == FLAREPP_OK) {
         // the routing queries the forward's encode read: q_fixed with the gate
         // closed; else the I/O-dtype copy (tensor cores) or fp32 (SIMT)
         const bool q_f32 = gated && (pl.path == FLAREPP_PATH_SIMT || dtype == FLAREPP_F32);
@@ -1182,7 +1335,10 @@ size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int 
     return bp.total;
 }
 
-int flarepp_mixer_bwd_launches(int gated) { return gated ? 4 + 10 : 2 + 7; }
+int flarepp_mixer_bwd_launches(int gated, int path) {
+    if (path == FLAREPP_PATH_TCGEN05) return gated ? 5 + 10 : 3 + 7;
+    return gated ? 4 + 10 : 2 + 7;
+}
 
 int flarepp_mixer_fwd_host(const void* q0, const void* q_fixed, const float* gate, const void* k0,
                            const void* k, const void* v, void* y, int B, int H, int N, int M, int D,

@@ -433,9 +433,16 @@ struct ReduceParams {
     const float* qdyn;      // encode (gated): q_dyn [B,H,M,D]
     float* dqdyn;           // encode (gated): out
     float* dq0b;            // synthesis: out [B,H,M,D]
+    // tensor-core backward only (else NULL): the 16-bit copy of dz (decode) or dq_dyn
+    // (encode), and the next pass's (log-sum-exp, Delta) per latent row at
+    // stats_out[(b*H + h)*stats_stride + m], the log-sum-exp read from lse_in[row]
+    void* out16;
+    float2* stats_out;
+    int64_t stats_stride;
+    const float* lse_in;
 };
 
-template <int D>
+template <typename T, int D>
 __global__ void __launch_bounds__(256)
 reduce_partials(ReduceParams p) {
     constexpr int PL = D >= 32 ? D / 32 : 1;    // dims per lane
@@ -466,6 +473,9 @@ reduce_partials(ReduceParams p) {
             if (!lane_on) continue;
             const int64_t idx = row * D + lane + 32 * i;
             p.dz[idx] = s2[i];
+            if constexpr (sizeof(T) == 2) {
+                if (p.out16) static_cast<T*>(p.out16)[idx] = from_f32<T>(s2[i]);
+            }
             p.dq[idx] = p.scale * s1[i];
             dsum = fmaf(s2[i], p.z[idx], dsum);
         }
@@ -481,6 +491,9 @@ reduce_partials(ReduceParams p) {
             if (p.gate) {
                 const float dd = gh * dq;
                 p.dqdyn[idx] = dd;
+                if constexpr (sizeof(T) == 2) {
+                    if (p.out16) static_cast<T*>(p.out16)[idx] = from_f32<T>(dd);
+                }
                 dsum = fmaf(dd, p.qdyn[idx], dsum);
             }
         }
@@ -493,7 +506,11 @@ reduce_partials(ReduceParams p) {
     if (p.mode == kReduceDecode || (p.mode == kReduceEncode && p.gate)) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-        if (lane == 0) p.delta[row] = dsum;
+        if (lane == 0) {
+            p.delta[row] = dsum;
+            if (p.stats_out)
+                p.stats_out[(row / p.M) * p.stats_stride + row % p.M] = make_float2(p.lse_in[row], dsum);
+        }
     }
 }
 

@@ -183,6 +183,11 @@ struct FwdExtras {
     float* lse_enc = nullptr;    // [B,H,M]
     float* qdyn = nullptr;       // [B,H,M,D] fp32
     bool decode = true;
+    // tcgen05 decode only: per token (log-sum-exp, <dy, y>) at [(b*H + h)*stride + n];
+    // y may then be NULL (not written)
+    float2* tok_stats = nullptr;
+    int64_t tok_stats_stride = 0;
+    const void* dy = nullptr;
 };
 
 struct MergeParams {

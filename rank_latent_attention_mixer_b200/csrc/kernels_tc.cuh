@@ -320,8 +320,12 @@ struct Params {
     float* part_O;        // split: [parts][B*H][M][D]
     float2* part_ml;      // split: [parts][B*H][M]
     int tok_heads_inner;  // the token tensor's map is ordered (D, H, rows, B): [B,N,H,D] layout
-    void* y;              // decode: token rows in E, addressed by the strides below
+    void* y;              // decode: token rows in E, addressed by the strides below (NULL: not written)
     int64_t y_row, y_h, y_b;   // decode: element strides of y between tokens, heads, batch elements
+    float2* tok_stats;    // decode, optional: per token (log-sum-exp in log2 units, <dy, y>) at
+                          // tok_stats[(b*H + h)*tok_stats_stride + n] (kept for the backward)
+    int64_t tok_stats_stride;
+    const void* dy;       // decode with tok_stats: the gradient of y, in E with y's strides
 };
 
 struct Item {
@@ -730,16 +734,37 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const int n = it.qrow0 + wg * kQTile + row;
                 if (n < p.N && o) {
                     const float inv = 1.f / l;
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + (int64_t)(it.bh / p.H) * p.y_b +
-                                                          (int64_t)it.h * p.y_h + (int64_t)n * p.y_row);
+                    const int64_t off = (int64_t)(it.bh / p.H) * p.y_b + (int64_t)it.h * p.y_h + (int64_t)n * p.y_row;
+                    if (p.y) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + off);
 #pragma unroll
-                    for (int i = 0; i < D / 8; ++i) {
-                        const int c = i / 4, j = (i % 4) * 8;
-                        dst[i] = make_uint4(
-                            pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                        for (int i = 0; i < D / 8; ++i) {
+                            const int c = i / 4, j = (i % 4) * 8;
+                            dst[i] = make_uint4(
+                                pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
+                                pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
+                                pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
+                                pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                        }
+                    }
+                    if (__builtin_expect(p.tok_stats != nullptr, 0)) {
+                        // the backward's per-token statistics: the softmax's log-sum-exp
+                        // (log2 units, against the same running max as l) and <dy, y>
+                        const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
+                        float dsum = 0.f;
+#pragma unroll
+                        for (int i = 0; i < D / 8; ++i) {
+                            const uint4 v = g4[i];
+                            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                            const int c = i / 4, j = (i % 4) * 8;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 g2 = unpack2<E>(w4[e]);
+                                dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
+                                dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
+                            }
+                        }
+                        p.tok_stats[(int64_t)it.bh * p.tok_stats_stride + n] = make_float2(m + log2f(l), dsum * inv);
                     }
                 }
             }
@@ -1200,6 +1225,9 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     dp.y = y;
     dp.y_row = tok.row; dp.y_h = tok.h; dp.y_b = tok.b;
     dp.tok_heads_inner = tok.h < tok.row ? 1 : 0;
+    dp.tok_stats = ex.tok_stats;
+    dp.tok_stats_stride = ex.tok_stats_stride;
+    dp.dy = ex.dy;
     rc = launch_decode<E>(D, m_k_q, gated ? m_q16_kv : m_qf_kv, m_z16, dp, st);
     if (rc) return rc;
     mark(st);

@@ -14,12 +14,19 @@ zero-mean values, so single entries cancel to near zero and fp32 rounding of
 the accumulation order alone gives them relative errors far above 1e-4.  The
 elementwise figure (floored at 1e-3 * rms) is still reported.
 
-Gradients (the backward) are held to the same numbers taken relative to the
-gradient tensor's own size, since their scale follows the upstream gradient
-and the sizes of the sums they come from, not the unit scale of y:
+Gradients (the backward) are held to bounds taken relative to the gradient
+tensor's own size, since their scale follows the upstream gradient and the
+sizes of the sums they come from, not the unit scale of y:
   fp32 : max |g - o| <= 1e-4 * max |o|
-  bf16 : rel L2 <= 1e-2  and  max |g - o| <= 2e-2 * max |o|
-  fp16 : rel L2 <= 2.5e-3 and max |g - o| <= 5e-3 * max |o|
+  bf16 : rel L2 <= 1e-2   and  max |g - o| <= 3e-2 * max |o|
+  fp16 : rel L2 <= 2.5e-3 and  max |g - o| <= 7.5e-3 * max |o|
+The elementwise bound is wider than y's because 16-bit I/O rounds the routing
+queries q to the I/O type where they feed the tensor cores (the forward's
+convention), and the latent gradients are sums over all tokens of terms
+P (dP - Delta) k that cancel: on a D = 16, M = 200 case an emulation of that
+one rounding alone moves max |dq_fixed - o| / max |o| to 1.7e-2 (all the
+backward's bf16 roundings together: 2.1e-2), against 1.3e-3 for each of the
+others (P, dS, dz, z).  fp16 keeps the factor 1/4 of the forward bounds.
 """
 import numpy as np
 import torch
@@ -29,6 +36,8 @@ BF16_REL_L2 = 1e-2
 BF16_MAX_ABS = 2e-2
 F16_REL_L2 = 2.5e-3
 F16_MAX_ABS = 5e-3
+GRAD_BF16_MAX = 3e-2
+GRAD_F16_MAX = 7.5e-3
 
 
 def to64(t):
@@ -84,8 +93,24 @@ def assert_grad_parity(g, o, dtype: str, what: str, zero_atol: float = 1e-5):
         assert m["max_abs_rel_to_max"] <= FP32_MAX_REL, f"{what}: fp32 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     elif dtype == "f16":
         assert m["rel_l2"] <= F16_REL_L2, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} ({m})"
-        assert m["max_abs_rel_to_max"] <= F16_MAX_ABS, f"{what}: fp16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
+        assert m["max_abs_rel_to_max"] <= GRAD_F16_MAX, f"{what}: fp16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     else:
         assert m["rel_l2"] <= BF16_REL_L2, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} ({m})"
-        assert m["max_abs_rel_to_max"] <= BF16_MAX_ABS, f"{what}: bf16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
+        assert m["max_abs_rel_to_max"] <= GRAD_BF16_MAX, f"{what}: bf16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     return m
+
+
+def assert_dgate_parity(g, ref: dict, dtype: str, zero_atol: float = 0.0):
+    """dgate[h] = sum over (b, m, d) of dq * q_dyn is a dot product whose terms
+    cancel, so its error is bounded through dq's by Cauchy-Schwarz:
+    |err_h| <= ||err(dq)_h|| ||q_dyn_h|| <= tol ||dq_h|| ||q_dyn_h||, with tol
+    the rel-L2 bound of the dtype (fp32: 1e-4).  Where the mathematics makes
+    dq exactly zero (one token) the bound is the absolute zero_atol."""
+    g = to64(g)
+    o = to64(ref["dgate"])
+    dq, qd = to64(ref["dq"]), to64(ref["q_dyn"])
+    tol = {"f32": FP32_MAX_REL, "f16": F16_REL_L2}.get(dtype, BF16_REL_L2)
+    assert np.all(np.isfinite(g)), "dgate: non-finite values"
+    for h in range(o.shape[0]):
+        bound = max(tol * np.linalg.norm(dq[:, h]) * np.linalg.norm(qd[:, h]), zero_atol)
+        assert abs(g[h] - o[h]) <= bound, f"dgate[{h}]: |{g[h]:.6e} - {o[h]:.6e}| > {bound:.3e}"

@@ -43,6 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_abi_version_and_status_strings(lib):
     assert lib.lib.flarepp_abi_version() == 4
     assert lib.bwd_launches(True) == 14 and lib.bwd_launches(False) == 9
+    assert lib.bwd_launches(True, lib.PATH_TCGEN05) == 15 and lib.bwd_launches(False, lib.PATH_TCGEN05) == 10
     assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
     for code in range(6):
         assert lib.status_string(code) not in ("", "unknown status")
