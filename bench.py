@@ -633,17 +633,17 @@ BWD_STAGES_GATED = ["fwd split(synthesis)", "fwd merge(q)", "fwd split(encode)",
 BWD_STAGES_FLARE = ["fwd split(encode)", "fwd merge(z)", "decode_rows", "decode_cols", "reduce(decode)",
                     "token_cols(encode)", "latent_rows(encode)", "reduce(encode)", "reduce_batch"]
 BWD_TC_STAGES_GATED = ["fwd split(synthesis)", "fwd merge(q)", "fwd split(encode)", "fwd merge(z)",
-                       "fwd decode(stats)", "tc_latent(decode)", "tc_token(decode)", "reduce(decode)",
-                       "tc_token(encode)", "tc_latent(encode)", "reduce(encode)", "tc_token(synthesis)",
-                       "tc_latent(synthesis)", "reduce(synthesis)", "reduce_batch"]
+                       "fwd decode(stats)", "tc_latent(decode)", "reduce(decode)", "tc_token(decode+encode)",
+                       "tc_latent(encode)", "reduce(encode)", "tc_token(synthesis)", "tc_latent(synthesis)",
+                       "reduce(synthesis)", "reduce_batch"]
 BWD_TC_STAGES_FLARE = ["fwd split(encode)", "fwd merge(z)", "fwd decode(stats)", "tc_latent(decode)",
-                       "tc_token(decode)", "reduce(decode)", "tc_token(encode)", "tc_latent(encode)",
-                       "reduce(encode)", "reduce_batch"]
+                       "reduce(decode)", "tc_token(decode+encode)", "tc_latent(encode)", "reduce(encode)",
+                       "reduce_batch"]
 # FLOPs per (b, h, n, m, d) of each backward kernel as executed (2 per multiply-add):
 # decode rows recompute the decode softmax and y (4), then score, <dy, z> and dS q (6)
 BWD_KERNEL_FLOPS = {"decode_rows": 10, "decode_cols": 8, "token_cols": 8, "latent_rows": 6}
-# tensor-core kernel: S and dP (4), acc1 (2), acc2 (2 where present)
-BWD_TC_FLOPS = {"tc_latent(decode)": 8, "tc_token(decode)": 6, "tc_token(encode)": 8, "tc_latent(encode)": 6,
+# tensor-core kernel: S and dP (4; the fused token side has two dP: 6), acc1 (2), acc2 (2 where present)
+BWD_TC_FLOPS = {"tc_latent(decode)": 8, "tc_token(decode+encode)": 10, "tc_latent(encode)": 6,
                 "tc_token(synthesis)": 8, "tc_latent(synthesis)": 6}
 
 

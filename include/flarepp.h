@@ -312,8 +312,9 @@ size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int 
 /* Kernel launches one backward call makes, for the kernel family `path`
  * (flarepp_path_t, as flarepp_selected_path reports it) of its recomputed
  * forward: SIMT, gated 14 (4 recomputed forward passes, 3 per attention, 1
- * batch reduce), closed gate 9; TCGEN05, gated 15 (the forward's decode runs
- * too, for the per-token statistics), closed gate 10. */
+ * batch reduce), closed gate 9; TCGEN05, also gated 14 and closed gate 9 (the
+ * forward's decode runs too, for the per-token statistics, and the token
+ * sides of the decode and the encode are one launch). */
 int flarepp_mixer_bwd_launches(int gated, int path);
 
 /* FLAREPP_ABI_VERSION of the loaded library. */

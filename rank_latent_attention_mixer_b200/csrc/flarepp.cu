@@ -807,9 +807,9 @@ int cp_decode(const void* q, int q_shared, const void* z_state, const void* k, v
 // On the tensor-core path (16-bit I/O with the tcgen05 forward) the forward's
 // decode runs too, writing per token the log-sum-exp and <dy, y> instead of y,
 // and every token-sum and latent-sum step is one launch of bwd_tc::bwd_kernel
-// (kernels_bwd_tc.cuh); the reduces also write 16-bit copies of dz and dq_dyn
-// (tensor-core operands) and the padded (log-sum-exp, Delta) pairs of the next
-// pass.
+// (kernels_bwd_tc.cuh), the token sides of the decode and the encode fused in
+// one; the reduces also write 16-bit copies of dz and dq_dyn (tensor-core
+// operands) and the padded (log-sum-exp, Delta) pairs of the next pass.
 struct BwdPlan {
     Plan fwd;
     bool tc;                     // tensor-core backward
@@ -872,7 +872,7 @@ int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     bp->off_stats_syn = off; off = align_up(off + tc_on * (size_t)s.bh() * bp->m_pad * sizeof(float2));
     bp->off_dz16 = off;      off = align_up(off + tc_on * latd * sizeof(uint16_t));
     bp->off_dqdyn16 = off;   off = align_up(off + tc_on * latd * sizeof(uint16_t));
-    bp->off_dk_acc = off;    off = align_up(off + tok * s.D * sizeof(float));
+    bp->off_dk_acc = off;    off = align_up(off + simt_on * tok * s.D * sizeof(float));
     bp->off_part1 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
     bp->off_part2 = off;     off = align_up(off + (size_t)bp->chunks * latd * sizeof(float));
     bp->off_dz = off;        off = align_up(off + latd * sizeof(float));
@@ -1032,7 +1032,6 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
     float2* stats_syn = reinterpret_cast<float2*>(ws + bp.off_stats_syn);
     float* part1 = reinterpret_cast<float*>(ws + bp.off_part1);
     float* part2 = reinterpret_cast<float*>(ws + bp.off_part2);
-    float* dk_acc = reinterpret_cast<float*>(ws + bp.off_dk_acc);
     const Operand q_lat = gated ? Operand{ws + pl.off_q16, false, false} : Operand{a.q_fixed, false, true};
     const Operand z_lat{ws + pl.off_z16, false, false};
     const Operand dz_lat{ws + bp.off_dz16, false, false};
@@ -1061,7 +1060,7 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
         L.a = A; L.c = C; L.b = Bc; L.e = Ec;
         L.rows_tok = true; L.has_acc2 = acc2; L.stats_per_col = col_stats;
         L.stats = stats; L.stats_stride = stride;
-        L.epi = epi; L.f32 = dk_acc; L.out1 = out1; L.out2 = out2;
+        L.epi = epi; L.f32 = nullptr; L.out1 = out1; L.out2 = out2;
         note(bwd_tc::launch_bwd_d<E>(L, st));
     };
     BwdLauncher launch{st};
@@ -1076,16 +1075,25 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
     float* qdyn = reinterpret_cast<float*>(ws + bp.off_qdyn);
     float* dq0b = reinterpret_cast<float*>(ws + bp.off_dq0b);
 
-    // decode y = SDPA(k, q, z): latent side (dq_dec, dz partials), token side (dk_dec)
+    // decode y = SDPA(k, q, z): latent side (dq_dec, dz partials)
     latent_rows(q_lat, z_lat, k, dy, true, true, stats_tok, bp.n_pad);
-    token_rows(k, dy, q_lat, z_lat, false, false, stats_tok, bp.n_pad, bwd_tc::kEpiTokF32, nullptr, nullptr);
     rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = reinterpret_cast<float*>(ws + bp.off_dz); rp.dq = dq;
     rp.delta = reinterpret_cast<float*>(ws + bp.off_delta_enc);
     rp.out16 = ws + bp.off_dz16; rp.stats_out = stats_enc; rp.lse_in = reinterpret_cast<float*>(ws + bp.off_lse_enc);
     launch(bwd::reduce_partials<E, D>, red_grid, dim3(256), rp);
     ev.mark(st);
-    // encode z = SDPA(q, k, v): token side (dk = dk_dec + dk_enc, dv), latent side (dq_enc partials)
-    token_rows(k, v, q_lat, dz_lat, true, true, stats_enc, bp.m_pad, bwd_tc::kEpiTokDkDv, a.dk, a.dv);
+    // the token sides of the decode and the encode in one launch (they share S = k q^T
+    // and the product with q): dk = dk_dec + dk_enc and dv
+    {
+        bwd_tc::Launch L = base;
+        L.a = k; L.c = dy; L.c2 = v; L.b = q_lat; L.e = z_lat; L.e2 = dz_lat;
+        L.dual = true; L.rows_tok = true; L.has_acc2 = true; L.stats_per_col = false;
+        L.stats = stats_tok; L.stats_stride = bp.n_pad;      // the decode's softmax: per token
+        L.stats2 = stats_enc; L.stats2_stride = bp.m_pad;    // the encode's: per latent
+        L.epi = bwd_tc::kEpiTokDkDv; L.f32 = nullptr; L.out1 = a.dk; L.out2 = a.dv;
+        note(bwd_tc::launch_bwd_d<E>(L, st));
+    }
+    // encode z = SDPA(q, k, v): latent side (dq_enc partials)
     latent_rows(q_lat, dz_lat, k, v, false, false, stats_enc, bp.m_pad);
     rp.mode = bwd::kReduceEncode; rp.gate = a.gate; rp.qdyn = qdyn;
     rp.dqdyn = reinterpret_cast<float*>(ws + bp.off_dqdyn); rp.delta = reinterpret_cast<float*>(ws + bp.off_delta0);
@@ -1336,7 +1344,7 @@ size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int 
 }
 
 int flarepp_mixer_bwd_launches(int gated, int path) {
-    if (path == FLAREPP_PATH_TCGEN05) return gated ? 5 + 10 : 3 + 7;
+    if (path == FLAREPP_PATH_TCGEN05) return gated ? 5 + 9 : 3 + 6;
     return gated ? 4 + 10 : 2 + 7;
 }
 

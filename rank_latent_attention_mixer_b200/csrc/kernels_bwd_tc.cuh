@@ -22,6 +22,11 @@
 //     latent side
 // (the synthesis has A = C = k0 on the token side and B = E = k0 on the latent
 // side; its dk0 is scale acc1 + acc2).
+// The decode's and the encode's token sides share the score S = k q^T and the
+// product with q, so one "dual" launch serves both: a third row tile C2 = v
+// and column tile E2 = dz give dPe = v dz^T, the weights Pd (row statistics)
+// and Pe (column statistics) come from the same S, and
+//     acc1 += (dSd + dSe) q  = dk / scale,     acc2 += Pe dz = dv.
 //
 // Per CTA (persistent, one per SM): NW softmax warpgroups, each with its own
 // 128 rows, sharing every column tile, and one producer warpgroup:
@@ -46,7 +51,15 @@ using tc::kQTile;
 
 constexpr int kKT = 32;        // column tile rows (one 32-column TMEM load per job)
 constexpr int kNST = 4;        // column stages
-constexpr int kQS = 2;         // row slots
+
+// Tiles per row slot and per column stage, and row slots: the dual form holds
+// three of each and one row slot (shared memory), the others two and two.
+template <bool DUAL>
+struct Shape {
+    static constexpr int RT = DUAL ? 3 : 2;
+    static constexpr int CT = DUAL ? 3 : 2;
+    static constexpr int QS = DUAL ? 1 : 2;
+};
 
 enum Epilogue {
     kEpiPartials = 0,   // latent rows: acc1 (and acc2) -> fp32 partials [chunk][B*H][rows][D]
@@ -67,14 +80,16 @@ struct Params {
     int a_shared, c_shared, b_shared, e_shared;   // [H,rows,D] tensors shared over the batch
     int c_same_a, e_same_b;     // C is A / E is B: one load serves both
     int has_acc2;
-    int stats_per_col;          // lse, Delta per column (else per row)
+    int stats_per_col;          // lse, Delta per column (else per row); dual: per row
     const float2* stats;        // [B*H][stats_stride] (lse in log2 units, Delta)
     int64_t stats_stride;       // a multiple of KT (column statistics are bulk-copied per tile)
+    const float2* stats2;       // dual: the column statistics of the second softmax
+    int64_t stats2_stride;
     float scale_log2, scale;
     int epi;                    // Epilogue
     float* part1;
     float* part2;
-    float* f32;                 // kEpiTokF32: out; kEpiTokDkDv: the decode's share of dk, in
+    float* f32;                 // kEpiTokF32: out; kEpiTokDkDv: the decode's share of dk, in (or NULL)
     void* out1;                 // token outputs in E: dK (or dK0)
     void* out2;                 // dV
     int64_t tok_row, tok_h, tok_b;   // element strides of the token outputs
@@ -99,16 +114,17 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item) {
     return it;
 }
 
-template <int D, int NW>
+template <int D, int NW, bool DUAL>
 struct Smem {
+    using SH = Shape<DUAL>;
     static constexpr int kRowTile = kQTile * D * 2;
     static constexpr int kColTile = kKT * D * 2;
-    static constexpr int kRow = 0;                                  // [QS][NW][A, C]
-    static constexpr int kCol = kRow + kQS * NW * 2 * kRowTile;     // [NST][B, E]
-    static constexpr int kStats = kCol + kNST * 2 * kColTile;       // [NST][KT] float2
+    static constexpr int kRow = 0;                                      // [QS][NW][A, C (, C2)]
+    static constexpr int kCol = kRow + SH::QS * NW * SH::RT * kRowTile;  // [NST][B, E (, E2)]
+    static constexpr int kStats = kCol + kNST * SH::CT * kColTile;      // [NST][KT] float2
     static constexpr int kBar = kStats + kNST * kKT * 8;
     // row_full[QS], row_empty[QS], col_full[NST], col_empty[NST], sfull, sfree, pfull, pfree, drain [NW]
-    static constexpr int kNumBars = 2 * kQS + 2 * kNST + 5 * NW;
+    static constexpr int kNumBars = 2 * SH::QS + 2 * kNST + 5 * NW;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kLaunchBytes = kBytes + 1024;
@@ -116,12 +132,13 @@ struct Smem {
     static constexpr int kSmemLaunch = kLaunchBytes > 118784 ? kLaunchBytes : 118784;
 };
 
-template <int D, int NW>
+template <int D, int NW, bool DUAL>
 struct Tmem {
     static constexpr int OS = D < 32 ? 32 : D;
     static constexpr int kS = 0;
     static constexpr int kDP = NW * kKT;
-    static constexpr int kA1 = 2 * NW * kKT;
+    static constexpr int kDP2 = 2 * NW * kKT;                  // dual only
+    static constexpr int kA1 = (DUAL ? 3 : 2) * NW * kKT;
     static constexpr int kA2 = kA1 + NW * OS;
     static constexpr int kP = kA2 + NW * OS;
     static constexpr int kDS = kP + NW * (kKT / 2);
@@ -146,14 +163,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-template <typename E, int D, int NW>
+template <typename E, int D, int NW, bool DUAL>
 __global__ void __launch_bounds__((NW + 1) * 128, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_c,
-           const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_e, const Params p) {
+           const __grid_constant__ CUtensorMap map_c2, const __grid_constant__ CUtensorMap map_b,
+           const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_e2, const Params p) {
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dims 16, 32, 64, 128");
-    using SM = Smem<D, NW>;
-    using TM = Tmem<D, NW>;
+    using SM = Smem<D, NW, DUAL>;
+    using TM = Tmem<D, NW, DUAL>;
+    using SH = Shape<DUAL>;
     using LY = tc::Layout<D, NW, kKT>;
+    constexpr int kQS = SH::QS;
     constexpr int kTmaWarp = 4 * NW;
     constexpr int kMmaWarp0 = 4 * NW + 1;
 
@@ -194,6 +214,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
         tc::prefetch_tensormap(&map_c);
         tc::prefetch_tensormap(&map_b);
         tc::prefetch_tensormap(&map_e);
+        if (DUAL) {
+            tc::prefetch_tensormap(&map_c2);
+            tc::prefetch_tensormap(&map_e2);
+        }
     }
     if (warp == kMmaWarp0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -214,8 +238,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             int col_last[kNST], row_last[kQS];
             for (int i = 0; i < kNST; ++i) col_last[i] = -1;
             for (int i = 0; i < kQS; ++i) row_last[i] = -1;
-            const uint32_t row_bytes = NW * (p.c_same_a ? 1 : 2) * SM::kRowTile;
-            const uint32_t col_bytes = (p.e_same_b ? 1 : 2) * SM::kColTile + (p.stats_per_col ? kKT * 8 : 0);
+            const bool col_stats = DUAL || p.stats_per_col;
+            const uint32_t row_bytes = NW * ((p.c_same_a ? 1 : 2) + (DUAL ? 1 : 0)) * SM::kRowTile;
+            const uint32_t col_bytes =
+                ((p.e_same_b ? 1 : 2) + (DUAL ? 1 : 0)) * SM::kColTile + (col_stats ? kKT * 8 : 0);
+            const float2* cstats = DUAL ? p.stats2 : p.stats;
+            const int64_t cstride = DUAL ? p.stats2_stride : p.stats_stride;
             bool ok = true;
             // coordinates of a tile of `rows` starting at row r of (b, h): token maps may be
             // ordered (D, H, rows, B); latent maps are always (D, rows, H, B)
@@ -229,16 +257,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 ok = tc::mbar_wait(&row_empty[slot], ((ic / kQS) & 1) ^ 1, abort_flag);
                 if (!ok) break;
                 tc::mbar_expect_tx(&row_full[slot], row_bytes);
-                uint8_t* rdst = smem + SM::kRow + slot * NW * 2 * SM::kRowTile;
+                uint8_t* rdst = smem + SM::kRow + slot * NW * SH::RT * SM::kRowTile;
                 for (int w = 0; w < NW; ++w) {
                     const int r = it.row0 + w * kQTile;
+                    uint8_t* wdst = rdst + w * SH::RT * SM::kRowTile;
 #pragma unroll
                     for (int cb = 0; cb < LY::kBlocks; ++cb) {
-                        load(rdst + (2 * w) * SM::kRowTile + cb * LY::kQBlockBytes, &map_a, &row_full[slot],
-                             p.row_tok, cb, r, it.h, p.a_shared ? 0 : it.b);
+                        load(wdst + cb * LY::kQBlockBytes, &map_a, &row_full[slot], p.row_tok, cb, r, it.h,
+                             p.a_shared ? 0 : it.b);
                         if (!p.c_same_a)
-                            load(rdst + (2 * w + 1) * SM::kRowTile + cb * LY::kQBlockBytes, &map_c, &row_full[slot],
-                                 p.row_tok, cb, r, it.h, p.c_shared ? 0 : it.b);
+                            load(wdst + SM::kRowTile + cb * LY::kQBlockBytes, &map_c, &row_full[slot], p.row_tok,
+                                 cb, r, it.h, p.c_shared ? 0 : it.b);
+                        if (DUAL)   // C2: the second output-gradient operand (same batch as the tokens)
+                            load(wdst + 2 * SM::kRowTile + cb * LY::kQBlockBytes, &map_c2, &row_full[slot],
+                                 p.row_tok, cb, r, it.h, it.b);
                     }
                 }
                 row_last[slot] = (ic / kQS) & 1;
@@ -248,7 +280,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     ok = tc::mbar_wait(&col_empty[st], ((g / kNST) & 1) ^ 1, abort_flag);
                     if (!ok) break;
                     tc::mbar_expect_tx(&col_full[st], col_bytes);
-                    uint8_t* cdst = smem + SM::kCol + st * 2 * SM::kColTile;
+                    uint8_t* cdst = smem + SM::kCol + st * SH::CT * SM::kColTile;
 #pragma unroll
                     for (int cb = 0; cb < LY::kBlocks; ++cb) {
                         load(cdst + cb * LY::kKVBlockBytes, &map_b, &col_full[st], p.col_tok, cb, t * kKT, it.h,
@@ -256,10 +288,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                         if (!p.e_same_b)
                             load(cdst + SM::kColTile + cb * LY::kKVBlockBytes, &map_e, &col_full[st], p.col_tok, cb,
                                  t * kKT, it.h, p.e_shared ? 0 : it.b);
+                        if (DUAL)   // E2: the second output gradient's column tile (per batch)
+                            load(cdst + 2 * SM::kColTile + cb * LY::kKVBlockBytes, &map_e2, &col_full[st], p.col_tok,
+                                 cb, t * kKT, it.h, it.b);
                     }
-                    if (p.stats_per_col)
-                        bulk_load(smem + SM::kStats + st * kKT * 8, p.stats + it.bh * p.stats_stride + t * kKT,
-                                  kKT * 8, &col_full[st]);
+                    if (col_stats)
+                        bulk_load(smem + SM::kStats + st * kKT * 8, cstats + it.bh * cstride + t * kKT, kKT * 8,
+                                  &col_full[st]);
                     col_last[st] = (g / kNST) & 1;
                     ++g;
                 }
@@ -321,10 +356,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 if (!tc::mbar_wait(&col_full[st], (j.g / kNST) & 1, abort_flag)) return false;
                 if (!tc::mbar_wait(&sfree[w], (s_issued & 1) ^ 1, abort_flag)) return false;
                 tc::tc_fence_after();
-                const uint8_t* rbase = smem + SM::kRow + slot * NW * 2 * SM::kRowTile + 2 * w * SM::kRowTile;
+                const uint8_t* rbase = smem + SM::kRow + (slot * NW + w) * SH::RT * SM::kRowTile;
                 const uint32_t aaddr = tc::smem_u32(rbase);
                 const uint32_t caddr = tc::smem_u32(p.c_same_a ? rbase : rbase + SM::kRowTile);
-                const uint8_t* cbase = smem + SM::kCol + st * 2 * SM::kColTile;
+                const uint8_t* cbase = smem + SM::kCol + st * SH::CT * SM::kColTile;
                 const uint32_t baddr = tc::smem_u32(cbase);
                 const uint32_t eaddr = tc::smem_u32(p.e_same_b ? cbase : cbase + SM::kColTile);
 #pragma unroll
@@ -339,6 +374,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     const uint64_t ed = tc::smem_desc(eaddr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
                     tc::umma_f16(tmem + TM::kDP + w * kKT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
                 }
+                if constexpr (DUAL) {
+                    const uint32_t c2addr = tc::smem_u32(rbase + 2 * SM::kRowTile);
+                    const uint32_t e2addr = tc::smem_u32(cbase + 2 * SM::kColTile);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t cd =
+                            tc::smem_desc(c2addr + LY::kstep(kk, LY::kQBlockBytes), 16, LY::kSbo, LY::kType);
+                        const uint64_t ed =
+                            tc::smem_desc(e2addr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
+                        tc::umma_f16(tmem + TM::kDP2 + w * kKT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                }
                 tc::umma_commit(&sfull[w]);
                 ++s_issued;
                 // the last score MMAs of the item release this warpgroup's share of the row slot
@@ -349,9 +396,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 if (!tc::mbar_wait(&pfull[w], a_issued & 1, abort_flag)) return false;
                 tc::tc_fence_after();
                 const int st = j.g % kNST;
-                const uint8_t* cbase = smem + SM::kCol + st * 2 * SM::kColTile;
+                const uint8_t* cbase = smem + SM::kCol + st * SH::CT * SM::kColTile;
                 const uint32_t baddr = tc::smem_u32(cbase);
-                const uint32_t eaddr = tc::smem_u32(p.e_same_b ? cbase : cbase + SM::kColTile);
+                // acc2's B operand: E, or E2 in the dual form (acc2 = Pe E2)
+                const uint32_t eaddr = tc::smem_u32(DUAL ? cbase + 2 * SM::kColTile
+                                                         : (p.e_same_b ? cbase : cbase + SM::kColTile));
                 const bool first = j.t == j.info.t_begin;
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk) {
@@ -406,6 +455,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + TM::kS + wg * kKT;
         const uint32_t tDP = tmem + lane_base + TM::kDP + wg * kKT;
+        const uint32_t tDP2 = tmem + lane_base + TM::kDP2 + wg * kKT;
         const uint32_t tA1 = tmem + lane_base + TM::kA1 + wg * TM::OS;
         const uint32_t tA2 = tmem + lane_base + TM::kA2 + wg * TM::OS;
         const uint32_t tP = tmem + lane_base + TM::kP + wg * (kKT / 2);
@@ -418,7 +468,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             const int r = it.row0 + wg * kQTile + row;
             const bool rvalid = r < p.row_count;
             float lse_r = 0.f, del_r = 0.f;
-            if (!p.stats_per_col && rvalid) {
+            if ((DUAL || !p.stats_per_col) && rvalid) {
                 const float2 sv = p.stats[it.bh * p.stats_stride + r];
                 lse_r = sv.x;
                 del_r = sv.y;
@@ -427,9 +477,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 if (!tc::mbar_wait(&sfull[wg], sfull_waits & 1, abort_flag)) { ok = false; break; }
                 ++sfull_waits;
                 tc::tc_fence_after();
-                uint32_t sr[32], dr[32];
+                uint32_t sr[32], dr[32], dr2[DUAL ? 32 : 1];
                 tc::tmem_ld32(tS, sr);
                 tc::tmem_ld32(tDP, dr);
+                if constexpr (DUAL) tc::tmem_ld32(tDP2, dr2);
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 __syncwarp();
@@ -437,7 +488,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
 
                 const int st = g % kNST;
                 const float2* cs = sstats + st * kKT;
-                if (p.stats_per_col) {
+                if (DUAL || p.stats_per_col) {
                     // the stage's statistics: acquire the TMA writes (the phase has completed)
                     if (!tc::mbar_wait(&col_full[st], (g / kNST) & 1, abort_flag)) { ok = false; break; }
                 }
@@ -449,17 +500,29 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int c = 2 * j + e;
-                        float lse = lse_r, del = del_r;
-                        if (p.stats_per_col) {
-                            const float2 sv = cs[c];
-                            lse = sv.x;
-                            del = sv.y;
-                        }
                         const bool on = rvalid && c < valid;
-                        const float x = fmaf(__uint_as_float(sr[c]), sl2, -lse);
-                        const float pw = on ? ex2_mufu(x) : 0.f;
-                        pv[e] = pw;
-                        dv[e] = on ? pw * (__uint_as_float(dr[c]) - del) : 0.f;
+                        const float sc = __uint_as_float(sr[c]);
+                        if constexpr (DUAL) {
+                            // Pd from the row statistics (first softmax), Pe from the column
+                            // statistics (second); dS = dSd + dSe, the weights stored are Pe
+                            const float2 sv = cs[c];
+                            const float pd = on ? ex2_mufu(fmaf(sc, sl2, -lse_r)) : 0.f;
+                            const float pe = on ? ex2_mufu(fmaf(sc, sl2, -sv.x)) : 0.f;
+                            pv[e] = pe;
+                            dv[e] = on ? fmaf(pd, __uint_as_float(dr[c]) - del_r, pe * (__uint_as_float(dr2[c]) - sv.y))
+                                       : 0.f;
+                        } else {
+                            float lse = lse_r, del = del_r;
+                            if (p.stats_per_col) {
+                                const float2 sv = cs[c];
+                                lse = sv.x;
+                                del = sv.y;
+                            }
+                            const float x = fmaf(sc, sl2, -lse);
+                            const float pw = on ? ex2_mufu(x) : 0.f;
+                            pv[e] = pw;
+                            dv[e] = on ? pw * (__uint_as_float(dr[c]) - del) : 0.f;
+                        }
                     }
                     pk[j] = pack2<E>(pv[0], pv[1]);
                     dk[j] = pack2<E>(dv[0], dv[1]);
@@ -521,15 +584,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
                     float v1[CW];
                     if (p.epi == kEpiTokDkDv) {
-                        const float4* prev =
-                            reinterpret_cast<const float4*>(p.f32 + ((int64_t)it.bh * p.row_count + r) * D + c0);
+                        if (p.f32) {
+                            const float4* prev =
+                                reinterpret_cast<const float4*>(p.f32 + ((int64_t)it.bh * p.row_count + r) * D + c0);
 #pragma unroll
-                        for (int i = 0; i < CW / 4; ++i) {
-                            const float4 q4 = prev[i];
-                            v1[4 * i] = fmaf(p.scale, __uint_as_float(a1[4 * i]), q4.x);
-                            v1[4 * i + 1] = fmaf(p.scale, __uint_as_float(a1[4 * i + 1]), q4.y);
-                            v1[4 * i + 2] = fmaf(p.scale, __uint_as_float(a1[4 * i + 2]), q4.z);
-                            v1[4 * i + 3] = fmaf(p.scale, __uint_as_float(a1[4 * i + 3]), q4.w);
+                            for (int i = 0; i < CW / 4; ++i) {
+                                const float4 q4 = prev[i];
+                                v1[4 * i] = fmaf(p.scale, __uint_as_float(a1[4 * i]), q4.x);
+                                v1[4 * i + 1] = fmaf(p.scale, __uint_as_float(a1[4 * i + 1]), q4.y);
+                                v1[4 * i + 2] = fmaf(p.scale, __uint_as_float(a1[4 * i + 2]), q4.z);
+                                v1[4 * i + 3] = fmaf(p.scale, __uint_as_float(a1[4 * i + 3]), q4.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < CW; ++i) v1[i] = p.scale * __uint_as_float(a1[i]);
                         }
                         float v2[CW];
 #pragma unroll
@@ -571,6 +639,10 @@ struct Launch {
     int B, H, N, M, D;
     tc::RowStrides tok;
     Operand a, c, b, e;
+    bool dual;                 // the fused decode + encode token side (c2, e2, stats2 used)
+    Operand c2, e2;
+    const float2* stats2;
+    int64_t stats2_stride;
     bool rows_tok;             // rows are tokens (N rows), else latents (M rows)
     bool has_acc2, stats_per_col;
     const float2* stats;
@@ -595,10 +667,10 @@ inline int plan_chunks(int B, int H, int M, int N, int D) {
     return (int)tc::choose_chunks(units, tiles, kNumSMs, 1);
 }
 
-template <typename E, int D>
+template <typename E, int D, bool DUAL>
 int launch_bwd(const Launch& L, cudaStream_t st) {
     constexpr int NW = nw_for(D);
-    using SM = Smem<D, NW>;
+    using SM = Smem<D, NW, DUAL>;
     static_assert(SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     const CUtensorMapDataType ty = tc::Elem<E>::kMapType;
     const tc::RowStrides lat = tc::contiguous_rows(L.M, L.H, D);
@@ -606,8 +678,14 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
         if (o.tok) return tc::make_map(m, ty, o.ptr, L.N, L.H, L.B, D, L.tok, box);
         return tc::make_map(m, ty, o.ptr, L.M, L.H, o.shared ? 1 : L.B, D, lat, box);
     };
-    CUtensorMap ma, mc, mb, me;
+    CUtensorMap ma, mc, mb, me, mc2, me2;
     if (!map(&ma, L.a, kQTile) || !map(&mc, L.c, kQTile) || !map(&mb, L.b, kKT) || !map(&me, L.e, kKT)) return 3;
+    if (DUAL) {
+        if (!map(&mc2, L.c2, kQTile) || !map(&me2, L.e2, kKT)) return 3;
+    } else {
+        mc2 = mc;
+        me2 = me;
+    }
     Params p{};
     p.B = L.B; p.H = L.H;
     p.row_count = L.rows_tok ? L.N : L.M;
@@ -629,29 +707,36 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
     p.stats_per_col = L.stats_per_col ? 1 : 0;
     p.stats = L.stats;
     p.stats_stride = L.stats_stride;
+    p.stats2 = L.stats2;
+    p.stats2_stride = L.stats2_stride;
     p.scale_log2 = L.scale_log2;
     p.scale = L.scale;
     p.epi = L.epi;
     p.part1 = L.part1; p.part2 = L.part2; p.f32 = L.f32;
     p.out1 = L.out1; p.out2 = L.out2;
     p.tok_row = L.tok.row; p.tok_h = L.tok.h; p.tok_b = L.tok.b;
-    auto kern = bwd_kernel<E, D, NW>;
+    auto kern = bwd_kernel<E, D, NW, DUAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = p.items < tc::sm_count() ? p.items : tc::sm_count();
-    return tc::launch_pdl(kern, dim3(grid), dim3((NW + 1) * 128), SM::kSmemLaunch, st, ma, mc, mb, me, p) ==
-                   cudaSuccess
+    return tc::launch_pdl(kern, dim3(grid), dim3((NW + 1) * 128), SM::kSmemLaunch, st, ma, mc, mc2, mb, me, me2,
+                          p) == cudaSuccess
                ? 0
                : 3;
+}
+
+template <typename E, int D>
+int launch_bwd_dual(const Launch& L, cudaStream_t st) {
+    return L.dual ? launch_bwd<E, D, true>(L, st) : launch_bwd<E, D, false>(L, st);
 }
 
 template <typename E>
 int launch_bwd_d(const Launch& L, cudaStream_t st) {
     switch (L.D) {
-        case 16: return launch_bwd<E, 16>(L, st);
-        case 32: return launch_bwd<E, 32>(L, st);
-        case 64: return launch_bwd<E, 64>(L, st);
-        case 128: return launch_bwd<E, 128>(L, st);
+        case 16: return launch_bwd_dual<E, 16>(L, st);
+        case 32: return launch_bwd_dual<E, 32>(L, st);
+        case 64: return launch_bwd_dual<E, 64>(L, st);
+        case 128: return launch_bwd_dual<E, 128>(L, st);
         default: return 2;
     }
 }

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_abi_version_and_status_strings(lib):
     assert lib.lib.flarepp_abi_version() == 4
     assert lib.bwd_launches(True) == 14 and lib.bwd_launches(False) == 9
-    assert lib.bwd_launches(True, lib.PATH_TCGEN05) == 15 and lib.bwd_launches(False, lib.PATH_TCGEN05) == 10
+    assert lib.bwd_launches(True, lib.PATH_TCGEN05) == 14 and lib.bwd_launches(False, lib.PATH_TCGEN05) == 9
     assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
     for code in range(6):
         assert lib.status_string(code) not in ("", "unknown status")
@@ -192,7 +192,9 @@ def test_backward_workspace_query(lib):
     a = lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16)
     assert a > lib.workspace_bytes(1, 2, 1000, 64, 32, lib.BF16)
     assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 48, lib.BF16) == 0
-    # the fp32 buffer of the decode's share of dk dominates: B*H*N*D*4 bytes
-    big = lib.bwd_workspace_bytes(1, 8, 1 << 20, 512, 64, lib.BF16)
+    # SIMT: the fp32 buffer of the decode's share of dk dominates (B*H*N*D*4 bytes);
+    # tensor cores: per-token statistics only (the token sides are fused)
+    big = lib.bwd_workspace_bytes(1, 8, 1 << 20, 512, 64, lib.BF16, path=lib.PATH_SIMT)
     assert big > 8 * (1 << 20) * 64 * 4
+    assert lib.bwd_workspace_bytes(1, 8, 1 << 20, 512, 64, lib.BF16) < 8 * (1 << 20) * 64 * 2
     assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16, force_chunks=1) < a
