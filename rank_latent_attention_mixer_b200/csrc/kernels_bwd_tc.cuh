@@ -230,8 +230,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
     const uint32_t tmem = *tmem_slot;
     pdl_wait();
     pdl_launch_dependents();
+    // Registers: with two softmax warpgroups the launch gives 168 per thread; the
+    // producer warpgroup gives back down to 56 and the softmax warpgroups rise to
+    // 224 (2 x 128 x 224 + 128 x 56 = 384 x 168).  The build refuses a library whose
+    // launch allocation for this kernel is not exactly 168, since a larger `inc`
+    // than the pool holds would wait forever.
+    static_assert(NW != 2 || tc::Regs<2>::kSoftmax == 224, "register split of the backward kernel");
 
-    if (warp == kTmaWarp) {
+    if (warp >= 4 * NW) {
+      if constexpr (NW == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(tc::kProducerRegs));
+      if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
             uint32_t ic = 0, g = 0;
@@ -312,7 +320,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     }
             }
         }
-    } else if (warp >= kMmaWarp0) {
+      } else {
         // ---------------------------------------------------------- MMA issuers
         if (lane == 0 && warp < kMmaWarp0 + NW) {
             const int w = warp - kMmaWarp0;
@@ -447,7 +455,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             while (!tc::mbar_try_wait(&drain[w], 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
             }
         }
+      }
     } else {
+        if constexpr (NW == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(tc::Regs<2>::kSoftmax));
         // ---------------------------------------------------------- softmax warpgroups
         const int wg = warp >> 2;
         const int wq = warp & 3;
@@ -467,6 +477,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             const Item it = decode_item<NW>(p, item);
             const int r = it.row0 + wg * kQTile + row;
             const bool rvalid = r < p.row_count;
+            const bool warp_rows_valid = it.row0 + wg * kQTile + wq * 32 + 31 < p.row_count;
             float lse_r = 0.f, del_r = 0.f;
             if ((DUAL || !p.stats_per_col) && rvalid) {
                 const float2 sv = p.stats[it.bh * p.stats_stride + r];
@@ -494,6 +505,41 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 }
                 const int valid = p.col_count - t * kKT;     // columns of this tile that exist
                 uint32_t pk[16], dk[16];
+                if (__builtin_expect(valid >= kKT && warp_rows_valid, 1)) {
+                    // every row of the warp and every column of the tile exists (warp-uniform):
+                    // no masking, column pairs in packed fp32 arithmetic
+                    const float2 sl2v = make_float2(sl2, sl2);
+                    const float2 nlr = make_float2(-lse_r, -lse_r), ndr = make_float2(-del_r, -del_r);
+                    const float4* cs4 = reinterpret_cast<const float4*>(cs);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float2 s2 = make_float2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+                        const float2 d2 = make_float2(__uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1]));
+                        float2 pw, ds;
+                        if constexpr (DUAL) {
+                            const float4 sv = cs4[j];                    // (lse, Delta) of columns 2j, 2j+1
+                            const float2 xd = __ffma2_rn(s2, sl2v, nlr);
+                            const float2 xe = __ffma2_rn(s2, sl2v, make_float2(-sv.x, -sv.z));
+                            const float2 pd = make_float2(ex2_mufu(xd.x), ex2_mufu(xd.y));
+                            pw = make_float2(ex2_mufu(xe.x), ex2_mufu(xe.y));
+                            const float2 e2 = make_float2(__uint_as_float(dr2[2 * j]), __uint_as_float(dr2[2 * j + 1]));
+                            const float2 ge = __fmul2_rn(pw, __fadd2_rn(e2, make_float2(-sv.y, -sv.w)));
+                            ds = __ffma2_rn(pd, __fadd2_rn(d2, ndr), ge);
+                        } else {
+                            float2 nl = nlr, nd = ndr;
+                            if (p.stats_per_col) {
+                                const float4 sv = cs4[j];
+                                nl = make_float2(-sv.x, -sv.z);
+                                nd = make_float2(-sv.y, -sv.w);
+                            }
+                            const float2 x = __ffma2_rn(s2, sl2v, nl);
+                            pw = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
+                            ds = __fmul2_rn(pw, __fadd2_rn(d2, nd));
+                        }
+                        pk[j] = pack2<E>(pw.x, pw.y);
+                        dk[j] = pack2<E>(ds.x, ds.y);
+                    }
+                } else {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     float pv[2], dv[2];
@@ -526,6 +572,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     }
                     pk[j] = pack2<E>(pv[0], pv[1]);
                     dk[j] = pack2<E>(dv[0], dv[1]);
+                }
                 }
                 // the previous job's accumulating MMAs must be done before P and dS are overwritten
                 while (pfree_waits < jobs_done) {
