@@ -678,25 +678,28 @@ def run_backward_bench(args):
     path = {"auto": fb.PATH_AUTO, "simt": fb.PATH_SIMT, "tcgen05": fb.PATH_TCGEN05}[args.path]
     dtype_code = {"f32": fb.F32, "bf16": fb.BF16, "f16": fb.F16}[w.dtype]
     gated = not args.flare
-    ws = torch.empty(fb.bwd_workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, path), dtype=torch.uint8,
-                     device=dev)
+    norm = args.norm and gated
+    ws = torch.empty(fb.bwd_workspace_bytes(w.B, w.H, w.N, w.M, w.D, dtype_code, path, norm_synthesis=norm),
+                     dtype=torch.uint8, device=dev)
     out_t = {"dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
              "dq_fixed": torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev)}
     if gated:
         out_t.update(dk0=torch.empty_like(x["k0"]), dq0=torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev),
                      dgate=torch.empty((w.H,), dtype=torch.float32, device=dev))
     used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
-    n_launch = fb.bwd_launches(gated, used_path)
+    n_launch = fb.bwd_launches(gated, used_path) + (3 if norm else 0)
     if used_path == fb.PATH_TCGEN05:
         names = BWD_TC_STAGES_GATED if gated else BWD_TC_STAGES_FLARE
     else:
         names = BWD_STAGES_GATED if gated else BWD_STAGES_FLARE
+    if norm:
+        names = ["rms_norm(q0, k0)"] + names + ["rms_bwd(k0)", "rms_bwd(q0)"]
     fits_l2 = 6 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
 
     def step(events=None):
         fb.mixer_bwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], dy, path=path,
-                     workspace=ws, stage_events=events, out=out_t)
+                     workspace=ws, stage_events=events, out=out_t, norm_synthesis=norm)
 
     for _ in range(args.warmup):
         step()
@@ -752,7 +755,7 @@ def run_backward_bench(args):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
-                   "gate": "open (FLARE++)" if gated else "closed (FLARE)",
+                   "gate": "open (FLARE++)" if gated else "closed (FLARE)", "synthesis_norm": norm,
                    "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)")},

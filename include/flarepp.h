@@ -290,8 +290,11 @@ int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const vo
  * with fp32 I/O, or path = SIMT, fp32 SIMT kernels throughout), force_chunks
  * (the token chunks of both the recomputed passes and the backward's token sums),
  * workspace / workspace_bytes (>= flarepp_mixer_bwd_workspace_bytes),
- * stage_events (recorded before the first and after every launch), layout.
- * norm_synthesis = 1 gives FLAREPP_ERR_UNSUPPORTED; q_out, z_out are ignored.
+ * stage_events (recorded before the first and after every launch), layout,
+ * norm_synthesis (the synthesis reads RMS-normalised q0 and k0 rows as in the
+ * forward, and dq0, dk0 are taken through that step: dx = r (g - xh <g, xh>/D)
+ * per row, xh = x r, r = (mean x^2 + 1e-6)^(-1/2); three more launches).
+ * q_out, z_out are ignored.
  * Sums over tokens are taken per token chunk and added in a fixed order
  * (deterministic); the 16-bit gradients are rounded once, at the end.
  * Asynchronous on `stream`. */
@@ -314,7 +317,9 @@ size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int 
  * forward: SIMT, gated 14 (4 recomputed forward passes, 3 per attention, 1
  * batch reduce), closed gate 9; TCGEN05, also gated 14 and closed gate 9 (the
  * forward's decode runs too, for the per-token statistics, and the token
- * sides of the decode and the encode are one launch). */
+ * sides of the decode and the encode are one launch).  A gated call with
+ * norm_synthesis makes three more: the normalisation of q0, k0 first, and the
+ * gradients of k0 and q0 through it last. */
 int flarepp_mixer_bwd_launches(int gated, int path);
 
 /* FLAREPP_ABI_VERSION of the loaded library. */

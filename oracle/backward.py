@@ -23,7 +23,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import _f64
+from . import NORM_EPS, _f64
 
 
 def _softmax_rows(S):
@@ -45,12 +45,29 @@ def _sdpa_bwd(Q, K, V, P, dO, s):
     return s * (dS @ K), s * (dS.T @ Q), dV
 
 
-def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
+def _rms_backward(x, g, eps=NORM_EPS):
+    """Gradient through the row-wise RMS normalisation xh = x r,
+    r = (mean_d x^2 + eps)^(-1/2), for the gradient g of xh: by the chain rule
+    (dr/dx_j = -r^3 x_j / D) dx = r (g - xh <g, xh> / D), row by row."""
+    D = x.shape[-1]
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    xh = x * r
+    return r * (g - xh * np.sum(g * xh, axis=-1, keepdims=True) / D)
+
+
+def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0, norm_synthesis: bool = False):
     """Gradients of the gated mixer (gate open).  Returns a dict with
     dq0, dq_fixed [H,M,D], dgate [H], dk0, dk, dv [B,H,N,D], the forward's
-    y [B,H,N,D], and the intermediates q_dyn and dq = dL/dq [B,H,M,D] (fp64)."""
+    y [B,H,N,D], and the intermediates q_dyn and dq = dL/dq [B,H,M,D] (fp64).
+    ``norm_synthesis``: the synthesis reads RMS-normalised q0 and k0 rows
+    (physicsnemo issue #2024, "Normalizing the synthesis call"; the reading of
+    ``rms_normalise``), and dq0, dk0 are taken through that step."""
     q0, q_fixed, gate = _f64(q0), _f64(q_fixed), _f64(gate).reshape(-1)
     k0, k, v, dy = _f64(k0), _f64(k), _f64(v), _f64(dy)
+    if norm_synthesis:
+        q0_raw, k0_raw = q0, k0
+        q0 = q0_raw / np.sqrt(np.mean(q0_raw * q0_raw, axis=-1, keepdims=True) + NORM_EPS)
+        k0 = k0_raw / np.sqrt(np.mean(k0_raw * k0_raw, axis=-1, keepdims=True) + NORM_EPS)
     B, H, N, D = k.shape
     M = q_fixed.shape[1]
     s = scale if scale > 0 else 1.0 / np.sqrt(D)
@@ -82,6 +99,9 @@ def flarepp_backward(q0, q_fixed, gate, k0, k, v, dy, scale: float = 0.0):
             g["dk0"][b, h] = dk0_keys + dk0_values
             g["dk"][b, h] = dk_a + dk_b
             g["dv"][b, h] = dv
+    if norm_synthesis:
+        g["dq0"] = _rms_backward(q0_raw, g["dq0"])
+        g["dk0"] = _rms_backward(k0_raw, g["dk0"])
     g["y"] = y
     g["q_dyn"], g["dq"] = q_dyn_all, dq_all
     return g

@@ -204,21 +204,24 @@ def bwd_launches(gated: bool = True, path: int = PATH_SIMT) -> int:
     return int(lib.flarepp_mixer_bwd_launches(int(gated), int(path)))
 
 
-def bwd_workspace_bytes(B, H, N, M, D, dtype=BF16, path=PATH_AUTO, force_chunks=0, layout="bhnd") -> int:
-    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout], 0)
+def bwd_workspace_bytes(B, H, N, M, D, dtype=BF16, path=PATH_AUTO, force_chunks=0, layout="bhnd",
+                        norm_synthesis=False) -> int:
+    o = Options(0.0, path, force_chunks, 0, None, None, None, 0, None, LAYOUTS[layout], int(norm_synthesis))
     return int(lib.flarepp_mixer_bwd_workspace_bytes(B, H, N, M, D, dtype, ctypes.byref(o)))
 
 
 def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int = PATH_AUTO,
               force_chunks: int = 0, layout: str = "bhnd", workspace: Optional[torch.Tensor] = None,
-              stage_events=None, out: Optional[dict] = None) -> dict:
+              stage_events=None, out: Optional[dict] = None, norm_synthesis: bool = False) -> dict:
     """Gradients of the FLARE++ mixer (flarepp_mixer_bwd) for the upstream gradient dy of y.
 
     Inputs as for ``mixer_fwd`` plus dy (the layout and dtype of k).  Returns a
     dict with dk, dv (and dk0 when gated) in the I/O dtype and token layout,
     dq_fixed (and dq0) fp32 [H,M,D], and dgate fp32 [H] (the gradient with
     respect to the gate value, not its logit).  ``gate=None`` is FLARE.
-    ``out`` may supply preallocated gradient tensors under the same names."""
+    ``out`` may supply preallocated gradient tensors under the same names.
+    ``norm_synthesis``: the synthesis reads RMS-normalised q0, k0 rows, as in
+    ``mixer_fwd``, and dq0, dk0 are taken through that step."""
     B, H, N, M, D = _shapes(q_fixed, k, layout)
     _contig(q0, q_fixed, gate, k0, k, v, dy)
     dt = _dtype_code(k)
@@ -234,14 +237,14 @@ def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int 
         g.setdefault("dk0", torch.empty_like(k0))
         g.setdefault("dq0", torch.empty((H, M, D), dtype=torch.float32, device=dev))
         g.setdefault("dgate", torch.empty((H,), dtype=torch.float32, device=dev))
-    need = bwd_workspace_bytes(B, H, N, M, D, dt, path, force_chunks, layout)
+    need = bwd_workspace_bytes(B, H, N, M, D, dt, path, force_chunks, layout, norm_synthesis)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ev_arr, n_ev = _event_array(stage_events)
     o = Options(float(scale), int(path), int(force_chunks), n_ev, None, None,
                 workspace.data_ptr() if need else None, workspace.numel() if need else 0,
                 ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None,
-                LAYOUTS[layout], 0)
+                LAYOUTS[layout], int(norm_synthesis))
     rc = lib.flarepp_mixer_bwd(_ptr(q0) if gated else None, _ptr(q_fixed), _ptr(gate),
                                _ptr(k0) if gated else None, _ptr(k), _ptr(v), _ptr(dy),
                                _ptr(g.get("dq0")) if gated else None, _ptr(g["dq_fixed"]),

@@ -831,7 +831,6 @@ int tc_bwd_chunks(const Shape& s, int force) {
 int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     int rc = make_plan(s, o, &bp->fwd);
     if (rc) return rc;
-    if (bp->fwd.norm_synthesis) return FLAREPP_ERR_UNSUPPORTED;
     const int G = s.D >= 64 ? s.D / 32 : 1;           // bwd::Lanes<D>::G
     const int rows_per_cta = bwd::kThreads / G;
     const int tile = 4096 / s.D;                       // bwd::Lanes<D>::TILE
@@ -1140,6 +1139,32 @@ cudaError_t run_backward_d(const Shape& s, const BwdPlan& bp, const BwdArgs& a, 
     }
 }
 
+// Gradient through the synthesis normalisation (norm_synthesis): dk0 (I/O
+// dtype, token rows) and dq0 (fp32 [H,M,D]) were taken with respect to the
+// normalised rows; map them to the raw q0, k0 rows in place.
+template <typename T, int D>
+void launch_rms_backward(const Shape& s, const BwdArgs& a, StageEvents& ev, cudaStream_t st) {
+    const int64_t rows_k = s.bh() * s.N, rows_q = (int64_t)s.H * s.M;
+    const int rw = 32 / (D * (int)sizeof(T) / 16);                  // rows per warp pass
+    const int64_t want = (rows_k + 8 * rw - 1) / (8 * rw);
+    bwd::rms_backward_rows_coop<T, D><<<(unsigned)std::min<int64_t>(want, (int64_t)kNumSMs * 16), 256, 0, st>>>(
+        static_cast<const T*>(a.k0), static_cast<T*>(a.dk0), rows_k, kNormEps);
+    ev.mark(st);
+    bwd::rms_backward_rows<T, float, D><<<(unsigned)((rows_q + 255) / 256), 256, 0, st>>>(
+        static_cast<const T*>(a.q0), a.dq0, rows_q, kNormEps);
+    ev.mark(st);
+}
+
+template <typename T>
+void rms_backward(const Shape& s, const BwdArgs& a, StageEvents& ev, cudaStream_t st) {
+    switch (s.D) {
+        case 16: launch_rms_backward<T, 16>(s, a, ev, st); break;
+        case 32: launch_rms_backward<T, 32>(s, a, ev, st); break;
+        case 64: launch_rms_backward<T, 64>(s, a, ev, st); break;
+        default: launch_rms_backward<T, 128>(s, a, ev, st); break;
+    }
+}
+
 int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
              void* stream) {
     const Shape s{B, H, N, M, D, dtype};
@@ -1180,11 +1205,21 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
         ex.tok_stats_stride = bp.n_pad;
         ex.dy = a.dy;
     }
-    rc = run(s, pl, a.q0, a.q_fixed, a.gate, a.k0, a.k, a.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
+    // with norm_synthesis the synthesis (forward and backward) reads normalised
+    // copies of q0 and k0, and dq0, dk0 are mapped back through the step at the end
+    const bool norm = pl.norm_synthesis && gated;
+    BwdArgs an = a;
+    if (norm) {
+        ev.mark(st);
+        rms_norm(s, a.q0, ws + pl.off_q0n, a.k0, ws + pl.off_k0n, st);
+        an.q0 = ws + pl.off_q0n;
+        an.k0 = ws + pl.off_k0n;
+    }
+    rc = run(s, pl, an.q0, an.q_fixed, an.gate, an.k0, an.k, an.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
     if (rc == FLAREPP_OK && bp.tc) {
         cudaError_t e;
-        if (dtype == FLAREPP_F16) e = run_backward_tc_d<__half>(s, bp, a, ws, ev, st);
-        else e = run_backward_tc_d<__nv_bfloat16>(s, bp, a, ws, ev, st);
+        if (dtype == FLAREPP_F16) e = run_backward_tc_d<__half>(s, bp, an, ws, ev, st);
+        else e = run_backward_tc_d<__nv_bfloat16>(s, bp, an, ws, ev, st);
         rc = (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? FLAREPP_OK : FLAREPP_ERR_CUDA;
     } else if (rc == FLAREPP_OK) {
         // the routing queries the forward's encode read: q_fixed with the gate
@@ -1194,13 +1229,19 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
                                                        : static_cast<const void*>(ws + pl.off_q16);
         const int q_bh = gated ? s.H : 0;
         cudaError_t e;
-        if (dtype == FLAREPP_F32) e = run_backward_d<float, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
-        else if (dtype == FLAREPP_F16 && q_f32) e = run_backward_d<__half, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
-        else if (dtype == FLAREPP_F16) e = run_backward_d<__half, __half>(s, bp, a, ws, q_lat, q_bh, ev, st);
-        else if (q_f32) e = run_backward_d<__nv_bfloat16, float>(s, bp, a, ws, q_lat, q_bh, ev, st);
-        else e = run_backward_d<__nv_bfloat16, __nv_bfloat16>(s, bp, a, ws, q_lat, q_bh, ev, st);
+        if (dtype == FLAREPP_F32) e = run_backward_d<float, float>(s, bp, an, ws, q_lat, q_bh, ev, st);
+        else if (dtype == FLAREPP_F16 && q_f32) e = run_backward_d<__half, float>(s, bp, an, ws, q_lat, q_bh, ev, st);
+        else if (dtype == FLAREPP_F16) e = run_backward_d<__half, __half>(s, bp, an, ws, q_lat, q_bh, ev, st);
+        else if (q_f32) e = run_backward_d<__nv_bfloat16, float>(s, bp, an, ws, q_lat, q_bh, ev, st);
+        else e = run_backward_d<__nv_bfloat16, __nv_bfloat16>(s, bp, an, ws, q_lat, q_bh, ev, st);
         if (cudaGetLastError() != cudaSuccess) e = cudaErrorLaunchFailure;
         rc = e == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+    }
+    if (rc == FLAREPP_OK && norm) {
+        if (dtype == FLAREPP_F32) rms_backward<float>(s, a, ev, st);
+        else if (dtype == FLAREPP_F16) rms_backward<__half>(s, a, ev, st);
+        else rms_backward<__nv_bfloat16>(s, a, ev, st);
+        rc = cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
     }
     if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
     return rc;

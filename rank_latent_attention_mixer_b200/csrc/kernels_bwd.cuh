@@ -514,6 +514,93 @@ reduce_partials(ReduceParams p) {
     }
 }
 
+// Gradient through the head-wise RMS normalisation of the synthesis seeds and
+// keys/values (physicsnemo issue #2024, FLARE++ list, "Normalizing the
+// synthesis call"; read as xh = x r, r = (mean_d x^2 + eps)^(-1/2)): for each
+// row x and the gradient g of its normalised form, dx = r (g - xh <g, xh> / D)
+// (chain rule, dr/dx_j = -r^3 x_j / D), written over g.  One thread per row,
+// 32 dimensions at a time in two passes (sums, then the update); HBM-bound:
+// x read once (twice from cache), g read and written.
+template <typename TX, typename TG, int D>
+__global__ void __launch_bounds__(256)
+rms_backward_rows(const TX* __restrict__ x, TG* __restrict__ g, int64_t rows, float eps) {
+    constexpr int C = D < 32 ? D : 32;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const TX* xr = x + r * D;
+    TG* gr = g + r * D;
+    float ss = 0.f, gx = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += C) {
+        float xv[C], gv[C];
+        load_row_f32<TX, C>(xr + c0, xv);
+        load_row_f32<TG, C>(gr + c0, gv);
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            ss = fmaf(xv[i], xv[i], ss);
+            gx = fmaf(gv[i], xv[i], gx);
+        }
+    }
+    const float rs = rsqrtf(ss * (1.f / D) + eps);
+    const float coef = rs * rs * gx * (1.f / D);        // <g, xh> / D divided by r: xh_i = x_i r
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += C) {
+        float xv[C], gv[C];
+        load_row_f32<TX, C>(xr + c0, xv);
+        load_row_f32<TG, C>(gr + c0, gv);
+#pragma unroll
+        for (int i = 0; i < C; ++i) gv[i] = rs * fmaf(-xv[i], coef, gv[i]);
+        store_row<TG, C>(gr + c0, gv);
+    }
+}
+
+// The same step when x and g have one type (the token rows: k0 and dk0): one
+// 16-byte chunk per lane, the lanes of a row combining their sums by shuffles,
+// so every warp access is coalesced (one read of x, one read and one write of
+// g).  A grid-stride loop over rows.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+rms_backward_rows_coop(const T* __restrict__ x, T* __restrict__ g, int64_t rows, float eps) {
+    pdl_wait();
+    pdl_launch_dependents();
+    constexpr int E = 16 / sizeof(T);              // elements per chunk
+    constexpr int C = D / E;                       // chunks per row (<= 32)
+    constexpr int RW = 32 / C;                     // rows per warp pass
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int64_t r0 = first * RW; r0 < rows; r0 += warps * RW) {
+        const int64_t r = r0 + lane / C;
+        const bool in = r < rows;                  // every lane still takes part in the shuffles
+        const int64_t off = r * D + (lane % C) * E;
+        float xv[E], gv[E];
+        float ss = 0.f, gx = 0.f;
+        if (in) {
+            load_row_f32<T, E>(x + off, xv);
+            load_row_f32<T, E>(g + off, gv);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                ss = fmaf(xv[e], xv[e], ss);
+                gx = fmaf(gv[e], xv[e], gx);
+            }
+        }
+#pragma unroll
+        for (int o = C / 2; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            gx += __shfl_xor_sync(0xffffffffu, gx, o);
+        }
+        if (in) {
+            const float rs = rsqrtf(ss * (1.f / D) + eps);
+            const float coef = rs * rs * gx * (1.f / D);
+#pragma unroll
+            for (int e = 0; e < E; ++e) gv[e] = rs * fmaf(-xv[e], coef, gv[e]);
+            store_row<T, E>(g + off, gv);
+        }
+    }
+}
+
 // Gradients of the batch-shared inputs, one CTA per head: dq_fixed[h] =
 // sum_b dq[b,h], dq0[h] = sum_b dq0_b[b,h] and dgate[h] = sum_{b,m} <dq, q_dyn>
 // (q = q_fixed + gate q_dyn).  Deterministic: fixed summation order.

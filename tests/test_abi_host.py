@@ -182,8 +182,11 @@ def test_backward_entry_checks(lib):
     assert _bwd(lib, p) == 1
     assert _bwd(lib, BWD, D=48) == 2
     assert _bwd(lib, BWD, B=0) == 1
-    o = lib.Options(0.0, 0, 0, 0, None, None, None, 0, None, 0, 1)   # synthesis normalisation: not in the backward
-    assert _bwd(lib, BWD, opts=ctypes.byref(o)) == 2
+    o = lib.Options(0.0, 0, 0, 0, None, None, None, 0, None, 0, 2)   # norm_synthesis must be 0 or 1
+    assert _bwd(lib, BWD, opts=ctypes.byref(o)) == 1
+    # norm_synthesis: the workspace grows by the normalised copies of q0 and k0
+    assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16, norm_synthesis=True) > \
+        lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16)
     o = lib.Options(0.0, 0, 0, 0, None, None, 0x1000, 16, None)      # workspace too small
     assert _bwd(lib, BWD, opts=ctypes.byref(o)) == 4
 

@@ -32,10 +32,10 @@ def inputs(B, H, N, M, D, dt, seed):
     return x, dy
 
 
-def oracle_grads(x, dy, gate=None, scale=0.0):
+def oracle_grads(x, dy, gate=None, scale=0.0, norm=False):
     g = x["gate"] if gate is None else gate
     return flarepp_backward(to64(x["q0"]), to64(x["q_fixed"]), to64(g), to64(x["k0"]), to64(x["k"]),
-                            to64(x["v"]), to64(dy), scale=scale)
+                            to64(x["v"]), to64(dy), scale=scale, norm_synthesis=norm)
 
 
 def gpu_grads(x, dy, flare=False, **kw):
@@ -152,3 +152,20 @@ def test_caller_workspace():
     g2 = gpu_grads(x, dy)
     for name in GRADS + ("dgate",):
         assert torch.equal(g1[name], g2[name])
+
+
+@pytest.mark.parametrize("dt,path", [("f32", 0), ("bf16", 0), ("f16", 0), ("bf16", 1)])
+def test_normalised_synthesis_backward(dt, path):
+    """norm_synthesis: the synthesis reads RMS-normalised q0, k0 rows and dq0, dk0
+    go through that step; rows scaled far from RMS 1 so the step matters."""
+    x, dy = inputs(1, 2, 900, 80, 32, dt, seed=23)
+    x["q0"] = (x["q0"].double() * 3.0).to(x["q0"].dtype)
+    x["k0"] = (x["k0"].double() * 0.4).to(x["k0"].dtype)
+    ref = oracle_grads(x, dy, norm=True)
+    g = gpu_grads(x, dy, path=path, norm_synthesis=True)
+    for name in GRADS:
+        assert_grad_parity(g[name], ref[name], dt, name)
+    assert_dgate_parity(g["dgate"], ref, dt)
+    # and it differs from the gradient without the step
+    plain = oracle_grads(x, dy)
+    assert np.max(np.abs(plain["dk0"] - ref["dk0"])) > 10 * np.max(np.abs(to64(g["dk0"]) - ref["dk0"]))

@@ -16,8 +16,9 @@ def _inputs(seed, B, H, N, M, D):
                 v=r.standard_normal((B, H, N, D))), r.standard_normal((B, H, N, D))
 
 
-def _loss(x, dy):
-    y, _, _ = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+def _loss(x, dy, norm=False):
+    q0, k0 = (oracle.rms_normalise(x["q0"]), oracle.rms_normalise(x["k0"])) if norm else (x["q0"], x["k0"])
+    y, _, _ = oracle.flarepp(q0, x["q_fixed"], x["gate"], k0, x["k"], x["v"])
     return float(np.sum(y * dy))
 
 
@@ -47,3 +48,31 @@ def test_zero_gate_cuts_the_synthesis():
     g = flarepp_backward(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], dy)
     assert np.all(g["dq0"] == 0) and np.all(g["dk0"] == 0)
     assert np.any(g["dgate"] != 0)        # the gate's own gradient is not zero
+
+
+@pytest.mark.parametrize("scale_rows", [1.0, 3.7])
+def test_normalised_synthesis_gradients_match_central_differences(scale_rows):
+    """With the synthesis reading RMS-normalised q0 and k0 rows, dq0 and dk0 go
+    through the normalisation: central differences of the forward oracle with
+    the same step.  Rows far from RMS 1 make the step matter."""
+    B, H, N, M, D = 1, 2, 19, 6, 16
+    x, dy = _inputs(11, B, H, N, M, D)
+    x["q0"] = x["q0"] * scale_rows
+    x["k0"] = x["k0"] * scale_rows
+    g = flarepp_backward(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], dy, norm_synthesis=True)
+    r = np.random.default_rng(5)
+    h = 1e-5
+    for name, grad in (("q0", "dq0"), ("k0", "dk0"), ("q_fixed", "dq_fixed"), ("gate", "dgate"), ("k", "dk")):
+        for _ in range(3):
+            e = r.standard_normal(x[name].shape)
+            xp = dict(x); xp[name] = x[name] + h * e
+            xm = dict(x); xm[name] = x[name] - h * e
+            fd = (_loss(xp, dy, True) - _loss(xm, dy, True)) / (2 * h)
+            an = float(np.sum(g[grad] * e))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
+    # the normalisation is invariant to each row's scale up to eps, so dq0 and dk0
+    # are orthogonal to their rows up to eps / (mean x^2 + eps) ~ 1e-6 (a radial
+    # change does almost nothing)
+    for gx, xx in ((g["dq0"], x["q0"]), (g["dk0"], x["k0"])):
+        radial = np.abs(np.sum(gx * xx, axis=-1))
+        assert np.all(radial <= 1e-5 * np.linalg.norm(gx, axis=-1) * np.linalg.norm(xx, axis=-1))
