@@ -61,6 +61,9 @@ def parse_args(argv=None):
                    help="memory layout of k0, k, v, y: [B,H,N,D] or [B,N,H,D] (read in place)")
     p.add_argument("--backward", action="store_true",
                    help="time the backward (flarepp_mixer_bwd: gradients of every input for a random dy)")
+    p.add_argument("--saved-state", action="store_true",
+                   help="with --backward: time the backward from a training forward's saved state "
+                        "(flarepp_mixer_bwd_ctx; the forward runs once, untimed)")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -687,19 +690,31 @@ def run_backward_bench(args):
         out_t.update(dk0=torch.empty_like(x["k0"]), dq0=torch.empty((w.H, w.M, w.D), dtype=torch.float32, device=dev),
                      dgate=torch.empty((w.H,), dtype=torch.float32, device=dev))
     used_path = path or fb.selected_path(w.B, w.H, w.N, w.M, w.D, dtype_code)
-    n_launch = fb.bwd_launches(gated, used_path) + (3 if norm else 0)
     if used_path == fb.PATH_TCGEN05:
         names = BWD_TC_STAGES_GATED if gated else BWD_TC_STAGES_FLARE
     else:
         names = BWD_STAGES_GATED if gated else BWD_STAGES_FLARE
+    extra_kernels = 0
+    saved = None
+    if args.saved_state:
+        # the recomputed forward passes are replaced by the saved state
+        names = [nm for nm in names if not nm.startswith("fwd ")]
+        if used_path == fb.PATH_TCGEN05:
+            names = ["round(q, z)", "token <dy, y>"] + names
+            extra_kernels = 1                      # the rounding stage is two launches
+        y_fwd, ctx = fb.mixer_fwd_train(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"],
+                                        x["v"], path=path, norm_synthesis=norm)
+        saved = (y_fwd, ctx)
     if norm:
         names = ["rms_norm(q0, k0)"] + names + ["rms_bwd(k0)", "rms_bwd(q0)"]
+    n_launch = len(names)
     fits_l2 = 6 * x["k"].numel() * x["k"].element_size() < L2_BYTES * 4
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev) if fits_l2 else None
 
     def step(events=None):
         fb.mixer_bwd(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], dy, path=path,
-                     workspace=ws, stage_events=events, out=out_t, norm_synthesis=norm)
+                     workspace=ws, stage_events=events, out=out_t, norm_synthesis=norm,
+                     ctx=saved[1] if saved else None, y=saved[0] if saved else None)
 
     for _ in range(args.warmup):
         step()
@@ -756,11 +771,12 @@ def run_backward_bench(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
                    "gate": "open (FLARE++)" if gated else "closed (FLARE)", "synthesis_norm": norm,
+                   "saved_state": bool(args.saved_state),
                    "kernel_path": {1: "simt", 2: "tcgen05"}.get(used_path, used_path),
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)")},
         "algorithmic_tflops": round(10.0 * passes * bhnmd / (ms_step * 1e-3) / 1e12, 2),
-        "gpu_launches": K * n_launch,
+        "gpu_launches": K * (n_launch + extra_kernels),
         "roofline": ({"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                       "frac": round(achieved / peak_t, 4), "traffic": None,
                       "peak_kind": f"{peak_src} bf16 sustained"} if tc_path else

@@ -322,6 +322,39 @@ size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int 
  * gradients of k0 and q0 through it last. */
 int flarepp_mixer_bwd_launches(int gated, int path);
 
+/* ---------------------------------------------------------------------------
+ * Training step with saved forward state.  (A convenience of this library for
+ * a forward followed by its backward; the pages have no counterpart.)
+ * flarepp_mixer_fwd_train is flarepp_mixer_fwd_ex (same arguments, checks and
+ * result y, bitwise) that also writes into the caller-owned DEVICE buffer ctx
+ * (256-byte aligned, >= flarepp_train_context_bytes) what the backward would
+ * otherwise recompute: q and z (fp32 [B,H,M,D]), the synthesis output before
+ * the gate, the per-latent log-sum-exps of the synthesis and the encode, and
+ * (tcgen05 path) the decode's per-token log-sum-exp -- latent-sized except the
+ * last, B*H*N*8 bytes.  opts->q_out and opts->z_out are ignored (the context
+ * holds q and z).  ctx must not overlap any tensor argument.
+ * flarepp_mixer_bwd_ctx is flarepp_mixer_bwd given that context and the
+ * forward's output y (token layout, I/O dtype): it skips the recomputed
+ * forward passes (on the tcgen05 path it rounds q and z to the I/O dtype for
+ * the tensor cores and takes <dy, y> per token from y).  The inputs, shape,
+ * dtype and options must be those of the forward call that filled ctx;
+ * nothing checks this.  Results equal flarepp_mixer_bwd's up to rounding (the
+ * per-token <dy, y> uses the rounded y).  Launches: the backward's minus the
+ * recomputed forward passes, plus two (q/z rounding, <dy, y>) on the tcgen05
+ * path.  Errors: ctx NULL or misaligned, y NULL -> FLAREPP_ERR_INVALID_ARG;
+ * ctx_bytes too small -> FLAREPP_ERR_WORKSPACE. */
+size_t flarepp_train_context_bytes(int B, int H, int N, int M, int D, int dtype);
+int flarepp_mixer_fwd_train(const void* q0, const void* q_fixed, const float* gate,
+                            const void* k0, const void* k, const void* v, void* y,
+                            int B, int H, int N, int M, int D, int dtype,
+                            const flarepp_options_t* opts, void* ctx, size_t ctx_bytes, void* stream);
+int flarepp_mixer_bwd_ctx(const void* q0, const void* q_fixed, const float* gate,
+                          const void* k0, const void* k, const void* v, const void* y, const void* dy,
+                          float* dq0, float* dq_fixed, float* dgate,
+                          void* dk0, void* dk, void* dv,
+                          int B, int H, int N, int M, int D, int dtype,
+                          const flarepp_options_t* opts, const void* ctx, size_t ctx_bytes, void* stream);
+
 /* FLAREPP_ABI_VERSION of the loaded library. */
 int flarepp_abi_version(void);
 

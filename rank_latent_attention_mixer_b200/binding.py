@@ -24,7 +24,8 @@ STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
 EXPORTS = ["flarepp_mixer_fwd", "flare_fwd", "flarepp_mixer_fwd_ex", "flarepp_workspace_bytes",
            "flarepp_mixer_fwd_host", "flarepp_selected_path", "flarepp_check_device_status",
            "flarepp_status_string", "flarepp_abi_version", "flarepp_launches_per_call",
-           "flarepp_mixer_bwd", "flarepp_mixer_bwd_workspace_bytes", "flarepp_mixer_bwd_launches"]
+           "flarepp_mixer_bwd", "flarepp_mixer_bwd_workspace_bytes", "flarepp_mixer_bwd_launches",
+           "flarepp_train_context_bytes", "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx"]
 
 
 class FlareppError(RuntimeError):
@@ -64,9 +65,14 @@ def _load() -> ctypes.CDLL:
     lib.flarepp_mixer_bwd_workspace_bytes.argtypes = [i] * 6 + [ctypes.POINTER(Options)]
     lib.flarepp_mixer_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.flarepp_mixer_bwd_launches.argtypes = [i, i]
+    lib.flarepp_train_context_bytes.argtypes = [i] * 6
+    lib.flarepp_train_context_bytes.restype = ctypes.c_size_t
+    lib.flarepp_mixer_fwd_train.argtypes = sig + [ctypes.POINTER(Options), vp, ctypes.c_size_t, vp]
+    lib.flarepp_mixer_bwd_ctx.argtypes = [vp] * 14 + [i] * 6 + [ctypes.POINTER(Options), vp, ctypes.c_size_t, vp]
     for name in ("flarepp_mixer_fwd", "flarepp_mixer_fwd_ex", "flarepp_mixer_fwd_host", "flare_fwd",
                  "flarepp_selected_path", "flarepp_check_device_status", "flarepp_abi_version",
-                 "flarepp_launches_per_call", "flarepp_mixer_bwd", "flarepp_mixer_bwd_launches"):
+                 "flarepp_launches_per_call", "flarepp_mixer_bwd", "flarepp_mixer_bwd_launches",
+                 "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -210,9 +216,40 @@ def bwd_workspace_bytes(B, H, N, M, D, dtype=BF16, path=PATH_AUTO, force_chunks=
     return int(lib.flarepp_mixer_bwd_workspace_bytes(B, H, N, M, D, dtype, ctypes.byref(o)))
 
 
+def train_context_bytes(B, H, N, M, D, dtype=BF16) -> int:
+    return int(lib.flarepp_train_context_bytes(B, H, N, M, D, dtype))
+
+
+def mixer_fwd_train(q0, q_fixed, gate, k0, k, v, y=None, *, ctx: Optional[torch.Tensor] = None, scale: float = 0.0,
+                    path: int = PATH_AUTO, force_chunks: int = 0, layout: str = "bhnd", norm_synthesis: bool = False,
+                    workspace: Optional[torch.Tensor] = None):
+    """flarepp_mixer_fwd_train: the forward, also saving the state its backward
+    needs into ``ctx`` (a uint8 device tensor, allocated if None).  Returns (y, ctx)."""
+    B, H, N, M, D = _shapes(q_fixed, k, layout)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    dt = _dtype_code(k)
+    if y is None:
+        y = torch.empty_like(k)
+    need = train_context_bytes(B, H, N, M, D, dt)
+    if ctx is None or ctx.numel() < need:
+        ctx = torch.empty(need, dtype=torch.uint8, device=k.device)
+    wneed = workspace_bytes(B, H, N, M, D, dt, gate is not None, path, force_chunks, layout, norm_synthesis)
+    if workspace is None or workspace.numel() < wneed:
+        workspace = torch.empty(max(wneed, 1), dtype=torch.uint8, device=k.device)
+    o = Options(float(scale), int(path), int(force_chunks), 0, None, None, workspace.data_ptr(), workspace.numel(),
+                None, LAYOUTS[layout], int(norm_synthesis))
+    rc = lib.flarepp_mixer_fwd_train(_ptr(q0) if gate is not None else None, _ptr(q_fixed), _ptr(gate),
+                                     _ptr(k0) if gate is not None else None, _ptr(k), _ptr(v), _ptr(y),
+                                     B, H, N, M, D, dt, ctypes.byref(o), ctx.data_ptr(), ctx.numel(),
+                                     _stream(k.device))
+    _check(rc, "flarepp_mixer_fwd_train")
+    return y, ctx
+
+
 def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int = PATH_AUTO,
               force_chunks: int = 0, layout: str = "bhnd", workspace: Optional[torch.Tensor] = None,
-              stage_events=None, out: Optional[dict] = None, norm_synthesis: bool = False) -> dict:
+              stage_events=None, out: Optional[dict] = None, norm_synthesis: bool = False,
+              ctx: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None) -> dict:
     """Gradients of the FLARE++ mixer (flarepp_mixer_bwd) for the upstream gradient dy of y.
 
     Inputs as for ``mixer_fwd`` plus dy (the layout and dtype of k).  Returns a
@@ -221,7 +258,9 @@ def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int 
     respect to the gate value, not its logit).  ``gate=None`` is FLARE.
     ``out`` may supply preallocated gradient tensors under the same names.
     ``norm_synthesis``: the synthesis reads RMS-normalised q0, k0 rows, as in
-    ``mixer_fwd``, and dq0, dk0 are taken through that step."""
+    ``mixer_fwd``, and dq0, dk0 are taken through that step.
+    ``ctx``, ``y``: the context and output of ``mixer_fwd_train`` on the same
+    inputs and options (flarepp_mixer_bwd_ctx: no recomputed forward passes)."""
     B, H, N, M, D = _shapes(q_fixed, k, layout)
     _contig(q0, q_fixed, gate, k0, k, v, dy)
     dt = _dtype_code(k)
@@ -245,11 +284,17 @@ def mixer_bwd(q0, q_fixed, gate, k0, k, v, dy, *, scale: float = 0.0, path: int 
                 workspace.data_ptr() if need else None, workspace.numel() if need else 0,
                 ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p)) if ev_arr is not None else None,
                 LAYOUTS[layout], int(norm_synthesis))
-    rc = lib.flarepp_mixer_bwd(_ptr(q0) if gated else None, _ptr(q_fixed), _ptr(gate),
-                               _ptr(k0) if gated else None, _ptr(k), _ptr(v), _ptr(dy),
-                               _ptr(g.get("dq0")) if gated else None, _ptr(g["dq_fixed"]),
-                               _ptr(g.get("dgate")) if gated else None, _ptr(g.get("dk0")) if gated else None,
-                               _ptr(g["dk"]), _ptr(g["dv"]), B, H, N, M, D, dt, ctypes.byref(o), _stream(dev))
+    grads = (_ptr(g.get("dq0")) if gated else None, _ptr(g["dq_fixed"]), _ptr(g.get("dgate")) if gated else None,
+             _ptr(g.get("dk0")) if gated else None, _ptr(g["dk"]), _ptr(g["dv"]))
+    ins = (_ptr(q0) if gated else None, _ptr(q_fixed), _ptr(gate), _ptr(k0) if gated else None, _ptr(k), _ptr(v))
+    if ctx is not None:
+        if y is None:
+            raise ValueError("the context backward needs the forward's output y")
+        rc = lib.flarepp_mixer_bwd_ctx(*ins, _ptr(y), _ptr(dy), *grads, B, H, N, M, D, dt, ctypes.byref(o),
+                                       ctx.data_ptr(), ctx.numel(), _stream(dev))
+        _check(rc, "flarepp_mixer_bwd_ctx")
+        return g
+    rc = lib.flarepp_mixer_bwd(*ins, _ptr(dy), *grads, B, H, N, M, D, dt, ctypes.byref(o), _stream(dev))
     _check(rc, "flarepp_mixer_bwd")
     return g
 

@@ -304,7 +304,7 @@ void rms_norm(const Shape& s, const void* q0, void* q0n, const void* k0, void* k
 
 int forward(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
             const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
-            const flarepp_options_t* opts, void* stream) {
+            const flarepp_options_t* opts, void* stream, const FwdExtras& ex = FwdExtras{}) {
     const Shape s{B, H, N, M, D, dtype};
     Plan pl{};
     int rc = make_plan(s, opts, &pl);
@@ -340,7 +340,7 @@ int forward(const void* q0, const void* q_fixed, const float* gate, const void* 
         q0 = ws + pl.off_q0n;
         k0 = ws + pl.off_k0n;
     }
-    rc = run(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st);
+    rc = run(s, pl, q0, q_fixed, gate, k0, k, v, y, ws, q_out, z_out, ev, st, ex);
     if (owned && cudaFreeAsync(ws, st) != cudaSuccess && rc == FLAREPP_OK) rc = FLAREPP_ERR_CUDA;
     return rc;
 }
@@ -1139,6 +1139,124 @@ cudaError_t run_backward_d(const Shape& s, const BwdPlan& bp, const BwdArgs& a, 
     }
 }
 
+// ------------------------------------------------------------------ saved forward state
+//
+// A training step runs the forward and then the backward.  The training forward
+// keeps, in a caller-owned context, what the backward would otherwise recompute:
+// the routing queries q and the latents z (fp32), the synthesis output before the
+// gate, the per-latent log-sum-exps of the synthesis and the encode, and (tensor-
+// core path) the decode's per-token log-sum-exp.  The backward given the context
+// skips the recomputed forward passes: it rebuilds the 16-bit operand copies of q
+// and z by rounding, and takes <dy, y> per token from the forward's output y.
+struct Context {
+    size_t q32, z32, qdyn, lse_syn, lse_enc, tok, total;
+};
+
+Context context_layout(const Shape& s) {
+    const size_t lat = (size_t)s.bh() * s.M, latd = lat * s.D;
+    const int64_t kt = bwd_tc::kKT, n_pad = (s.N + kt - 1) / kt * kt;
+    Context c{};
+    size_t off = 0;
+    c.q32 = off;     off = align_up(off + latd * sizeof(float));
+    c.z32 = off;     off = align_up(off + latd * sizeof(float));
+    c.qdyn = off;    off = align_up(off + latd * sizeof(float));
+    c.lse_syn = off; off = align_up(off + lat * sizeof(float));
+    c.lse_enc = off; off = align_up(off + lat * sizeof(float));
+    c.tok = off;     off = align_up(off + (size_t)s.bh() * n_pad * sizeof(float2));
+    c.total = off;
+    return c;
+}
+
+int check_context(const Shape& s, const void* ctx, size_t ctx_bytes) {
+    if (!ctx) return FLAREPP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ctx) % kAlign) return FLAREPP_ERR_INVALID_ARG;
+    if (ctx_bytes < context_layout(s).total) return FLAREPP_ERR_WORKSPACE;
+    return FLAREPP_OK;
+}
+
+int forward_train(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+                  const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
+                  const flarepp_options_t* opts, void* ctx, size_t ctx_bytes, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    int rc = check_shape(s);
+    if (rc) return rc;
+    rc = check_context(s, ctx, ctx_bytes);
+    if (rc) return rc;
+    const Context c = context_layout(s);
+    char* base = static_cast<char*>(ctx);
+    const size_t tb = s.tok_bytes();
+    if (overlaps(ctx, c.total, y, tb) || overlaps(ctx, c.total, k, tb) || overlaps(ctx, c.total, v, tb) ||
+        overlaps(ctx, c.total, q_fixed, s.lat_bytes()) || (gate && overlaps(ctx, c.total, k0, tb)))
+        return FLAREPP_ERR_INVALID_ARG;
+    flarepp_options_t o = opts ? *opts : flarepp_options_t{};
+    o.q_out = reinterpret_cast<float*>(base + c.q32);
+    o.z_out = reinterpret_cast<float*>(base + c.z32);
+    Plan pl{};
+    rc = make_plan(s, &o, &pl);
+    if (rc) return rc;
+    FwdExtras ex;
+    ex.lse_syn = reinterpret_cast<float*>(base + c.lse_syn);
+    ex.lse_enc = reinterpret_cast<float*>(base + c.lse_enc);
+    ex.qdyn = reinterpret_cast<float*>(base + c.qdyn);
+    if (pl.path == FLAREPP_PATH_TCGEN05) {
+        const int64_t kt = bwd_tc::kKT;
+        ex.tok_stats = reinterpret_cast<float2*>(base + c.tok);
+        ex.tok_stats_stride = (s.N + kt - 1) / kt * kt;
+    }
+    return forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, &o, stream, ex);
+}
+
+// Fills the backward's workspace regions from a saved context: the plain copies
+// (cudaMemcpyAsync), the 16-bit operand copies of q and z (tensor-core path),
+// and <dy, y> per token.
+template <typename E, int D>
+int restore_context(const Shape& s, const BwdPlan& bp, const BwdArgs& a, const void* y, const char* ctx, char* ws,
+                    StageEvents& ev, cudaStream_t st) {
+    const Plan& pl = bp.fwd;
+    const Context c = context_layout(s);
+    const size_t lat = (size_t)s.bh() * s.M, latd = lat * s.D;
+    ev.mark(st);        // before the first launch, as the recomputed forward does
+    bool ok = cudaMemcpyAsync(ws + pl.off_q32, ctx + c.q32, latd * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess &&
+              cudaMemcpyAsync(ws + pl.off_z32, ctx + c.z32, latd * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess &&
+              cudaMemcpyAsync(ws + bp.off_lse_enc, ctx + c.lse_enc, lat * 4, cudaMemcpyDeviceToDevice, st) ==
+                  cudaSuccess;
+    if (ok && a.gate)
+        ok = cudaMemcpyAsync(ws + bp.off_qdyn, ctx + c.qdyn, latd * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess &&
+             cudaMemcpyAsync(ws + bp.off_lse_syn, ctx + c.lse_syn, lat * 4, cudaMemcpyDeviceToDevice, st) ==
+                 cudaSuccess;
+    if (!ok) return FLAREPP_ERR_CUDA;
+    if (bp.tc) {
+        ok = cudaMemcpyAsync(ws + bp.off_stats_tok, ctx + c.tok, (size_t)s.bh() * bp.n_pad * sizeof(float2),
+                             cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+        if (!ok) return FLAREPP_ERR_CUDA;
+        const unsigned rgrid = (unsigned)std::min<int64_t>((int64_t)((latd / 8 + 255) / 256), (int64_t)kNumSMs * 8);
+        bwd::round_to_io<E><<<rgrid, 256, 0, st>>>(reinterpret_cast<const float*>(ctx + c.q32),
+                                                   reinterpret_cast<E*>(ws + pl.off_q16), (int64_t)latd);
+        bwd::round_to_io<E><<<rgrid, 256, 0, st>>>(reinterpret_cast<const float*>(ctx + c.z32),
+                                                   reinterpret_cast<E*>(ws + pl.off_z16), (int64_t)latd);
+        ev.mark(st);
+        const int64_t rows = s.bh() * s.N;
+        const int rw = 32 / (D * 2 / 16);
+        const int64_t want = (rows + 8 * rw - 1) / (8 * rw);
+        bwd::token_delta<E, D><<<(unsigned)std::min<int64_t>(want, (int64_t)kNumSMs * 16), 256, 0, st>>>(
+            reinterpret_cast<float2*>(ws + bp.off_stats_tok), bp.n_pad, static_cast<const E*>(a.dy),
+            static_cast<const E*>(y), s.H, s.N, rows, pl.tok.row, pl.tok.h, pl.tok.b);
+        ev.mark(st);
+    }
+    return cudaGetLastError() == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
+template <typename E>
+int restore_context_d(const Shape& s, const BwdPlan& bp, const BwdArgs& a, const void* y, const char* ctx, char* ws,
+                      StageEvents& ev, cudaStream_t st) {
+    switch (s.D) {
+        case 16: return restore_context<E, 16>(s, bp, a, y, ctx, ws, ev, st);
+        case 32: return restore_context<E, 32>(s, bp, a, y, ctx, ws, ev, st);
+        case 64: return restore_context<E, 64>(s, bp, a, y, ctx, ws, ev, st);
+        default: return restore_context<E, 128>(s, bp, a, y, ctx, ws, ev, st);
+    }
+}
+
 // Gradient through the synthesis normalisation (norm_synthesis): dk0 (I/O
 // dtype, token rows) and dq0 (fp32 [H,M,D]) were taken with respect to the
 // normalised rows; map them to the raw q0, k0 rows in place.
@@ -1166,7 +1284,7 @@ void rms_backward(const Shape& s, const BwdArgs& a, StageEvents& ev, cudaStream_
 }
 
 int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
-             void* stream) {
+             void* stream, const void* ctx = nullptr, size_t ctx_bytes = 0, const void* y = nullptr) {
     const Shape s{B, H, N, M, D, dtype};
     BwdPlan bp{};
     int rc = make_bwd_plan(s, opts, &bp);
@@ -1175,6 +1293,11 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
     if (rc) return rc;
     const Plan& pl = bp.fwd;
     const bool gated = a.gate != nullptr;
+    if (ctx) {
+        rc = check_context(s, ctx, ctx_bytes);
+        if (rc) return rc;
+        if (!y || !aligned16(y)) return FLAREPP_ERR_INVALID_ARG;
+    }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char* ws = nullptr;
     bool owned = false;
@@ -1215,7 +1338,15 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
         an.q0 = ws + pl.off_q0n;
         an.k0 = ws + pl.off_k0n;
     }
-    rc = run(s, pl, an.q0, an.q_fixed, an.gate, an.k0, an.k, an.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
+    if (ctx) {
+        // the training forward's saved state replaces the recomputed passes
+        const char* c = static_cast<const char*>(ctx);
+        if (dtype == FLAREPP_F16) rc = restore_context_d<__half>(s, bp, an, y, c, ws, ev, st);
+        else if (dtype == FLAREPP_BF16) rc = restore_context_d<__nv_bfloat16>(s, bp, an, y, c, ws, ev, st);
+        else rc = restore_context_d<float>(s, bp, an, y, c, ws, ev, st);
+    } else {
+        rc = run(s, pl, an.q0, an.q_fixed, an.gate, an.k0, an.k, an.v, nullptr, ws, nullptr, nullptr, ev, st, ex);
+    }
     if (rc == FLAREPP_OK && bp.tc) {
         cudaError_t e;
         if (dtype == FLAREPP_F16) e = run_backward_tc_d<__half>(s, bp, an, ws, ev, st);
@@ -1374,6 +1505,29 @@ int flarepp_mixer_bwd(const void* q0, const void* q_fixed, const float* gate, co
     a.q0 = q0; a.q_fixed = q_fixed; a.gate = gate; a.k0 = k0; a.k = k; a.v = v; a.dy = dy;
     a.dq0 = dq0; a.dq_fixed = dq_fixed; a.dgate = dgate; a.dk0 = dk0; a.dk = dk; a.dv = dv;
     return backward(a, B, H, N, M, D, dtype, opts, stream);
+}
+
+size_t flarepp_train_context_bytes(int B, int H, int N, int M, int D, int dtype) {
+    const Shape s{B, H, N, M, D, dtype};
+    if (check_shape(s)) return 0;
+    return context_layout(s).total;
+}
+
+int flarepp_mixer_fwd_train(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+                            const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
+                            const flarepp_options_t* opts, void* ctx, size_t ctx_bytes, void* stream) {
+    return forward_train(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, opts, ctx, ctx_bytes, stream);
+}
+
+int flarepp_mixer_bwd_ctx(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
+                          const void* v, const void* y, const void* dy, float* dq0, float* dq_fixed, float* dgate,
+                          void* dk0, void* dk, void* dv, int B, int H, int N, int M, int D, int dtype,
+                          const flarepp_options_t* opts, const void* ctx, size_t ctx_bytes, void* stream) {
+    BwdArgs a{};
+    a.q0 = q0; a.q_fixed = q_fixed; a.gate = gate; a.k0 = k0; a.k = k; a.v = v; a.dy = dy;
+    a.dq0 = dq0; a.dq_fixed = dq_fixed; a.dgate = dgate; a.dk0 = dk0; a.dk = dk; a.dv = dv;
+    if (!ctx) return FLAREPP_ERR_INVALID_ARG;
+    return backward(a, B, H, N, M, D, dtype, opts, stream, ctx, ctx_bytes, y);
 }
 
 size_t flarepp_mixer_bwd_workspace_bytes(int B, int H, int N, int M, int D, int dtype,

@@ -601,6 +601,61 @@ rms_backward_rows_coop(const T* __restrict__ x, T* __restrict__ g, int64_t rows,
     }
 }
 
+// fp32 rows -> the 16-bit I/O type (round to nearest even): the tensor-core
+// operands q and z rebuilt from a saved forward state, the same rounding the
+// forward's merge applies.  n is a multiple of 8 (whole rows of D >= 16).
+template <typename E>
+__global__ void __launch_bounds__(256)
+round_to_io(const float* __restrict__ in, E* __restrict__ out, int64_t n) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x * 8;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += stride) {
+        float v[8];
+        load_row_f32<float, 8>(in + i, v);
+        store_row<E, 8>(out + i, v);
+    }
+}
+
+// Per token, <dy_n, y_n> into the second member of the backward's per-token
+// statistics (the first, the decode's log-sum-exp, came from the forward):
+// tok_stats[(b*H + h)*stride + n].y.  y and dy in the I/O type E, token rows
+// addressed by their strides; one 16-byte chunk per lane, the lanes of a row
+// combining by shuffles (coalesced; HBM-bound: one read of dy and of y).
+template <typename E, int D>
+__global__ void __launch_bounds__(256)
+token_delta(float2* __restrict__ tok_stats, int64_t stride, const E* __restrict__ dy, const E* __restrict__ y,
+            int H, int N, int64_t rows, int64_t tok_row, int64_t tok_h, int64_t tok_b) {
+    pdl_wait();
+    pdl_launch_dependents();
+    constexpr int EL = 16 / sizeof(E);             // elements per chunk
+    constexpr int C = D / EL;                      // chunks per row (<= 32)
+    constexpr int RW = 32 / C;                     // rows per warp pass
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    for (int64_t r0 = first * RW; r0 < rows; r0 += warps * RW) {
+        const int64_t r = r0 + lane / C;           // row = (b*H + h)*N + n
+        const bool in = r < rows;
+        float sum = 0.f;
+        int64_t bh = 0, n = 0;
+        if (in) {
+            bh = r / N;
+            n = r - bh * N;
+            const int64_t b = bh / H, h = bh - b * H;
+            const int64_t off = b * tok_b + h * tok_h + n * tok_row + (lane % C) * EL;
+            float gv[EL], yv[EL];
+            load_row_f32<E, EL>(dy + off, gv);
+            load_row_f32<E, EL>(y + off, yv);
+#pragma unroll
+            for (int e = 0; e < EL; ++e) sum = fmaf(gv[e], yv[e], sum);
+        }
+#pragma unroll
+        for (int o = C / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (in && lane % C == 0) tok_stats[bh * stride + n].y = sum;
+    }
+}
+
 // Gradients of the batch-shared inputs, one CTA per head: dq_fixed[h] =
 // sum_b dq[b,h], dq0[h] = sum_b dq0_b[b,h] and dgate[h] = sum_{b,m} <dq, q_dyn>
 // (q = q_fixed + gate q_dyn).  Deterministic: fixed summation order.

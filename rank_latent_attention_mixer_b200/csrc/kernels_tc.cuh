@@ -750,18 +750,21 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     if (__builtin_expect(p.tok_stats != nullptr, 0)) {
                         // the backward's per-token statistics: the softmax's log-sum-exp
                         // (log2 units, against the same running max as l) and <dy, y>
-                        const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
+                        // (0 when no dy is given: a forward that saves its state)
                         float dsum = 0.f;
+                        if (p.dy) {
+                            const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
 #pragma unroll
-                        for (int i = 0; i < D / 8; ++i) {
-                            const uint4 v = g4[i];
-                            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                            const int c = i / 4, j = (i % 4) * 8;
+                            for (int i = 0; i < D / 8; ++i) {
+                                const uint4 v = g4[i];
+                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                                const int c = i / 4, j = (i % 4) * 8;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 g2 = unpack2<E>(w4[e]);
-                                dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
-                                dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 g2 = unpack2<E>(w4[e]);
+                                    dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
+                                    dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
+                                }
                             }
                         }
                         p.tok_stats[(int64_t)it.bh * p.tok_stats_stride + n] = make_float2(m + log2f(l), dsum * inv);

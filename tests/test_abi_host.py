@@ -201,3 +201,21 @@ def test_backward_workspace_query(lib):
     assert big > 8 * (1 << 20) * 64 * 4
     assert lib.bwd_workspace_bytes(1, 8, 1 << 20, 512, 64, lib.BF16) < 8 * (1 << 20) * 64 * 2
     assert lib.bwd_workspace_bytes(1, 2, 1000, 64, 32, lib.BF16, force_chunks=1) < a
+
+
+def test_training_context_entries_checked(lib):
+    assert lib.train_context_bytes(1, 2, 1000, 64, 32, lib.BF16) > 0
+    assert lib.train_context_bytes(1, 2, 1000, 64, 48, lib.BF16) == 0
+    # the per-token log-sum-exps dominate at many tokens: B*H*N*8 bytes
+    assert lib.train_context_bytes(1, 8, 1 << 20, 512, 64, lib.BF16) >= 8 * (1 << 20) * 8
+    fwd = lib.lib.flarepp_mixer_fwd_train
+    args = FAKE + [1, 2, 64, 16, 16, 1, None]
+    assert fwd(*args, None, 1 << 20, None) == 1                  # no context
+    assert fwd(*args, 0x900010, 1 << 20, None) == 1              # misaligned context
+    assert fwd(*args, 0x900000, 16, None) == 4                   # context too small
+    bwd = lib.lib.flarepp_mixer_bwd_ctx
+    p = BWD[:6] + [0xe00000] + BWD[6:]                           # ... y, dy, grads
+    assert bwd(*p, 1, 2, 64, 16, 16, 1, None, None, 1 << 20, None) == 1     # no context
+    p2 = list(p)
+    p2[6] = None                                                  # no y
+    assert bwd(*p2, 1, 2, 64, 16, 16, 1, None, 0x900000, 1 << 20, None) == 1

@@ -169,3 +169,48 @@ def test_normalised_synthesis_backward(dt, path):
     # and it differs from the gradient without the step
     plain = oracle_grads(x, dy)
     assert np.max(np.abs(plain["dk0"] - ref["dk0"])) > 10 * np.max(np.abs(to64(g["dk0"]) - ref["dk0"]))
+
+
+@pytest.mark.parametrize("dt,path,flare,norm", [("bf16", 0, False, False), ("f32", 0, False, False),
+                                               ("f16", 0, False, True), ("bf16", 0, True, False),
+                                               ("bf16", 1, False, False), ("bf16", 0, False, True)])
+def test_training_step_with_saved_state(dt, path, flare, norm):
+    """mixer_fwd_train returns the forward's y bitwise and a context; the
+    backward from that context (no recomputed forward) matches the oracle and
+    the recomputing backward."""
+    b = binding()
+    x, dy = inputs(2, 2, 1100, 96, 64, dt, seed=29)
+    d = {k: v.to(DEV) for k, v in x.items()}
+    gate = None if flare else d["gate"]
+    y_plain = b.mixer_fwd(d["q0"], d["q_fixed"], gate, d["k0"], d["k"], d["v"], path=path, norm_synthesis=norm)
+    y, ctx = b.mixer_fwd_train(d["q0"], d["q_fixed"], gate, d["k0"], d["k"], d["v"], path=path,
+                               norm_synthesis=norm)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_plain), "the training forward must return the forward's y"
+    g = b.mixer_bwd(d["q0"], d["q_fixed"], gate, d["k0"], d["k"], d["v"], dy.to(DEV), path=path,
+                    norm_synthesis=norm, ctx=ctx, y=y)
+    g_re = b.mixer_bwd(d["q0"], d["q_fixed"], gate, d["k0"], d["k"], d["v"], dy.to(DEV), path=path,
+                       norm_synthesis=norm)
+    torch.cuda.synchronize()
+    assert b.check_device_status() == 0
+    ref = oracle_grads(x, dy, gate=np.zeros(2) if flare else None, norm=norm)
+    names = FLARE_GRADS if flare else GRADS
+    for name in names:
+        assert_grad_parity(g[name], ref[name], dt, name + " (saved state)")
+        if dt == "f32" or path == 1:
+            # the SIMT backward takes nothing from y: the two must agree to rounding of the sums
+            assert torch.allclose(g[name].double(), g_re[name].double(), rtol=0,
+                                  atol=1e-5 * float(g_re[name].double().abs().max()))
+    if not flare:
+        assert_dgate_parity(g["dgate"], ref, dt)
+
+
+def test_saved_state_argument_errors():
+    b = binding()
+    x, dy = inputs(1, 2, 300, 32, 32, "bf16", seed=31)
+    d = {k: v.to(DEV) for k, v in x.items()}
+    y, ctx = b.mixer_fwd_train(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"])
+    with pytest.raises(b.FlareppError):                     # context too small
+        b.mixer_bwd(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"], dy.to(DEV), ctx=ctx[:64], y=y)
+    with pytest.raises(ValueError):                          # no y
+        b.mixer_bwd(d["q0"], d["q_fixed"], d["gate"], d["k0"], d["k"], d["v"], dy.to(DEV), ctx=ctx)
