@@ -564,9 +564,18 @@ def run_cp(args):
 
     ops = TimedOps()
 
+    if args.backward:
+        dy = W.random_cotangent((w.B, w.H, w.N, w.D), w.dtype, seed=w.seed + 100, device=str(dev),
+                                device_rng=w.device_rng)[:, :, lo:hi]
+        dy = (dy.transpose(1, 2) if args.layout == "bnhd" else dy).contiguous()
+
     def step():
-        cp.mixer_fwd_cp(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y,
-                        layout=args.layout, path=path, _ops=ops)
+        if args.backward:
+            cp.mixer_bwd_cp(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], dy,
+                            layout=args.layout, path=path, _ops=ops)
+        else:
+            cp.mixer_fwd_cp(x["q0"], x["q_fixed"], x["gate"] if gated else None, x["k0"], x["k"], x["v"], y,
+                            layout=args.layout, path=path, _ops=ops)
 
     for _ in range(args.warmup):
         step()
@@ -603,7 +612,8 @@ def run_cp(args):
     flops_split = 4.0 * w.B * w.H * n_local * w.M * w.D
     achieved = flops_split / (split_ms * 1e-3) / 1e12
     out = {
-        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": ("FLARE++ mixer bwd Mtokens/s (token-sharded)" if args.backward else METRIC),
+        "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(max_ms / K, 4), "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "io_dtype": w.dtype,
@@ -613,7 +623,11 @@ def run_cp(args):
                    "l2": ("flushed between steps (512 MiB write)" if flush is not None
                           else "inputs larger than L2 (back-to-back steps)")},
         "tflops": round(counts["flops"] / (max_ms / K * 1e-3) / 1e12, 2),
-        "gpu_launches": K * ((5 if gated else 3) + (2 if gated else 1)),
+        # forward: split + triple merge per sharded pass, merges, decode (+1 normalisation);
+        # backward: the recomputed sharded passes and merges, then stages 1-4 (3, 4, 4 and 2
+        # launches gated; 3, 4, 1, 1 closed)
+        "gpu_launches": K * (((6 if gated else 3) + (13 if gated else 9)) if args.backward
+                             else ((5 if gated else 3) + (2 if gated else 1))),
         "roofline": {"bound": "tensor", "kernel": "split_partial (+ local triple reduction)",
                      "achieved": round(achieved, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_t, 4), "traffic": None,
@@ -797,10 +811,10 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
-    elif args.backward:
-        run_backward_bench(args)
     elif args.cp:
         run_cp(args)
+    elif args.backward:
+        run_backward_bench(args)
     else:
         run_ours(args)
 

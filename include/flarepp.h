@@ -264,6 +264,14 @@ int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const vo
                       int B, int H, int N, int M, int D, int dtype,
                       const flarepp_options_t* opts, void* stream);
 
+/* Log-sum-exp merge as flarepp_cp_merge that also writes, for the backward,
+ * lse_out: fp32 [B,H,M], each latent row's log-sum-exp over all ranks' tokens
+ * (log2 units, of the scores times scale*log2(e)), and (gate != NULL)
+ * pregate_out: fp32 [B,H,M,D], the merged value before the gate.  Either may
+ * be NULL; neither may overlap the state or the gathered triples. */
+int flarepp_cp_merge_ex(const float* gathered, int ranks, const void* q_fixed, const float* gate, void* state,
+                        float* lse_out, float* pregate_out, int B, int H, int M, int D, int dtype, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Backward: the gradients of a scalar loss L with respect to every input of
  * the mixer, given dy = dL/dy.  By the chain rule through each softmax
@@ -354,6 +362,48 @@ int flarepp_mixer_bwd_ctx(const void* q0, const void* q_fixed, const float* gate
                           void* dk0, void* dk, void* dv,
                           int B, int H, int N, int M, int D, int dtype,
                           const flarepp_options_t* opts, const void* ctx, size_t ctx_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Token-sharded backward (physicsnemo issue #2024, section 2: the distributed
+ * encoder and its backward).  Every sum over tokens in the backward is a sum
+ * of per-rank sums, every sum over latents is local; so each rank runs the
+ * backward's steps on its own tokens in four stages, and after stages 1, 2
+ * and 3 the caller sums one fp32 region of every rank's state over the ranks,
+ * in place (an all-reduce, e.g. NCCL), before the next stage:
+ *   stage 1: per-token decode statistics; the decode's latent side -> region 0
+ *   stage 2: dz, the token sides of decode and encode (dk, dv of this rank's
+ *            tokens), the encode's latent side                  -> region 1
+ *   stage 3: dq, dq_dyn; the synthesis' token side (dk0), its latent side
+ *                                                               -> region 2
+ *   stage 4: dq_fixed, dq0, dgate (the same on every rank).
+ * Arguments: the latent inputs and gate as for flarepp_mixer_bwd; q_state and
+ * z_state: the merged states of the forward's token-sharded passes
+ * (flarepp_cp_merge; q_state is ignored with the gate closed); lse_syn,
+ * lse_enc, qdyn: from flarepp_cp_merge_ex of the synthesis and the encode
+ * merges (lse_syn and qdyn ignored with the gate closed); k0, k, v, dy and
+ * dk0, dk, dv: this rank's N tokens in the layout of opts; dq0, dq_fixed,
+ * dgate as for flarepp_mixer_bwd.  Pass the same arguments to every stage and
+ * the same sizes, dtype and options on every rank.  state: DEVICE, 256-byte
+ * aligned, flarepp_cp_bwd_layout().bytes, kept by the caller across the four
+ * stages.  opts: as for flarepp_mixer_bwd (q_out, z_out must be NULL).
+ * Errors and asynchrony as for flarepp_mixer_bwd; stage outside 1..4 ->
+ * FLAREPP_ERR_INVALID_ARG. */
+typedef struct flarepp_cp_bwd_layout {
+    size_t bytes;               /* the per-rank state */
+    size_t reduce_offset[3];    /* byte offset in the state of the region stage 1, 2, 3 leaves to sum */
+    size_t reduce_bytes[3];     /* its size (fp32 values) */
+} flarepp_cp_bwd_layout_t;
+
+int flarepp_cp_bwd_layout(int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
+                          flarepp_cp_bwd_layout_t* out);
+
+int flarepp_cp_bwd_stage(int stage, const void* q0, const void* q_fixed, const float* gate,
+                         const void* q_state, const void* z_state,
+                         const float* lse_syn, const float* lse_enc, const float* qdyn,
+                         const void* k0, const void* k, const void* v, const void* dy,
+                         float* dq0, float* dq_fixed, float* dgate, void* dk0, void* dk, void* dv,
+                         void* state, int B, int H, int N, int M, int D, int dtype,
+                         const flarepp_options_t* opts, void* stream);
 
 /* FLAREPP_ABI_VERSION of the loaded library. */
 int flarepp_abi_version(void);

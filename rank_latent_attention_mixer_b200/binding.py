@@ -389,16 +389,65 @@ def cp_partials(q, q_shared: bool, k, v, triple, *, B, H, N, M, D, path=PATH_AUT
     return triple
 
 
-def cp_merge(gathered, ranks: int, q_fixed, gate, state, *, B, H, M, D, dtype):
-    """flarepp_cp_merge: log-sum-exp merge of the gathered triples into a latent state."""
-    fn = lib.flarepp_cp_merge
+def cp_merge(gathered, ranks: int, q_fixed, gate, state, *, B, H, M, D, dtype, lse_out=None, pregate_out=None):
+    """flarepp_cp_merge: log-sum-exp merge of the gathered triples into a latent state
+    (flarepp_cp_merge_ex when ``lse_out`` [B,H,M] or ``pregate_out`` [B,H,M,D], fp32, are given)."""
     vp, i = ctypes.c_void_p, ctypes.c_int
-    fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, vp]
+    if lse_out is None and pregate_out is None:
+        fn = lib.flarepp_cp_merge
+        fn.argtypes = [vp, i, vp, vp, vp, i, i, i, i, i, vp]
+        fn.restype = i
+        rc = fn(_ptr(gathered), int(ranks), _ptr(q_fixed), _ptr(gate), _ptr(state), B, H, M, D, dtype,
+                _stream(gathered.device))
+        _check(rc, "flarepp_cp_merge")
+        return state
+    fn = lib.flarepp_cp_merge_ex
+    fn.argtypes = [vp, i, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     fn.restype = i
-    rc = fn(_ptr(gathered), int(ranks), _ptr(q_fixed), _ptr(gate), _ptr(state), B, H, M, D, dtype,
-            _stream(gathered.device))
-    _check(rc, "flarepp_cp_merge")
+    rc = fn(_ptr(gathered), int(ranks), _ptr(q_fixed), _ptr(gate), _ptr(state), _ptr(lse_out), _ptr(pregate_out),
+            B, H, M, D, dtype, _stream(gathered.device))
+    _check(rc, "flarepp_cp_merge_ex")
     return state
+
+
+class CpBwdLayout(ctypes.Structure):
+    """flarepp_cp_bwd_layout_t."""
+    _fields_ = [("bytes", ctypes.c_size_t), ("reduce_offset", ctypes.c_size_t * 3),
+                ("reduce_bytes", ctypes.c_size_t * 3)]
+
+
+def cp_bwd_layout(B, H, N, M, D, dtype, *, path=PATH_AUTO, scale=0.0, force_chunks=0, layout="bhnd",
+                  norm_synthesis=False) -> CpBwdLayout:
+    """flarepp_cp_bwd_layout: the per-rank state of the token-sharded backward and the
+    regions to sum over the ranks after stages 1, 2, 3."""
+    fn = lib.flarepp_cp_bwd_layout
+    i = ctypes.c_int
+    fn.argtypes = [i] * 6 + [ctypes.POINTER(Options), ctypes.POINTER(CpBwdLayout)]
+    fn.restype = i
+    out = CpBwdLayout()
+    o = _cp_options(path, scale, force_chunks, layout, norm=norm_synthesis)
+    _check(fn(B, H, N, M, D, dtype, ctypes.byref(o), ctypes.byref(out)), "flarepp_cp_bwd_layout")
+    return out
+
+
+def cp_bwd_stage(stage: int, q0, q_fixed, gate, q_state, z_state, lse_syn, lse_enc, qdyn, k0, k, v, dy, grads: dict,
+                 state, *, B, H, N, M, D, path=PATH_AUTO, scale=0.0, force_chunks=0, layout="bhnd",
+                 norm_synthesis=False):
+    """flarepp_cp_bwd_stage: one stage of the token-sharded backward on this rank's tokens."""
+    fn = lib.flarepp_cp_bwd_stage
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [i] + [vp] * 19 + [i] * 6 + [ctypes.POINTER(Options), vp]
+    fn.restype = i
+    o = _cp_options(path, scale, force_chunks, layout, norm=norm_synthesis)
+    gated = gate is not None
+    rc = fn(int(stage), _ptr(q0) if gated else None, _ptr(q_fixed), _ptr(gate), _ptr(q_state) if gated else None,
+            _ptr(z_state), _ptr(lse_syn) if gated else None, _ptr(lse_enc), _ptr(qdyn) if gated else None,
+            _ptr(k0) if gated else None, _ptr(k), _ptr(v), _ptr(dy),
+            _ptr(grads.get("dq0")) if gated else None, _ptr(grads["dq_fixed"]),
+            _ptr(grads.get("dgate")) if gated else None, _ptr(grads.get("dk0")) if gated else None,
+            _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(state), B, H, N, M, D, _dtype_code(k), ctypes.byref(o),
+            _stream(k.device))
+    _check(rc, f"flarepp_cp_bwd_stage({stage})")
 
 
 def cp_decode(q, q_shared: bool, z_state, k, y, *, B, H, N, M, D, path=PATH_AUTO, scale=0.0, layout="bhnd"):

@@ -717,7 +717,7 @@ int cp_partials(const void* q, int q_shared, const void* k, const void* v, float
 }
 
 int cp_merge(const float* gathered, int G, const void* q_fixed, const float* gate, void* state, int B, int H, int M,
-             int D, int dtype, void* stream) {
+             int D, int dtype, void* stream, float* lse_out = nullptr, float* pregate_out = nullptr) {
     const Shape s{B, H, 1, M, D, dtype};
     int rc = check_shape(s);
     if (rc) return rc;
@@ -740,6 +740,13 @@ int cp_merge(const float* gathered, int G, const void* q_fixed, const float* gat
     mp.q_fixed = q_fixed; mp.gate = gate;
     mp.out_f32 = static_cast<float*>(state);
     mp.out_16 = dtype == FLAREPP_F32 ? nullptr : static_cast<char*>(state) + latent_16_offset(s);
+    mp.lse_out = lse_out;
+    mp.pregate_out = gate ? pregate_out : nullptr;
+    if ((lse_out && (overlaps(lse_out, rows * 4, state, latent_state_bytes(s)) ||
+                     overlaps(lse_out, rows * 4, gathered, gb))) ||
+        (mp.pregate_out && (overlaps(pregate_out, rows * D * 4, state, latent_state_bytes(s)) ||
+                            overlaps(pregate_out, rows * D * 4, gathered, gb))))
+        return FLAREPP_ERR_INVALID_ARG;
     const dim3 grid((unsigned)((rows + 7) / 8));
 #define FLAREPP_CP_MERGE(T)                                                                        \
     switch (D) {                                                                                   \
@@ -1378,6 +1385,293 @@ int backward(const BwdArgs& a, int B, int H, int N, int M, int D, int dtype, con
     return rc;
 }
 
+// ------------------------------------------------------------------ token-sharded backward
+//
+// The backward with the N tokens split across ranks (physicsnemo issue #2024,
+// section 2: the distributed encoder and its backward).  Every sum over
+// tokens in the backward is a sum of per-rank partial sums; every sum over
+// latents stays local.  So each rank runs the single-GPU steps on its tokens,
+// and where the single-GPU backward reduces token-chunk partials, a rank
+// reduces its own chunks into a latent-sized fp32 region of its state that the
+// caller sums over the ranks (an all-reduce) before the next stage:
+//   stage 1  decode: per-token statistics, latent side        -> region 1 = (dq_dec, dz)
+//   stage 2  dz, <dz, z>; token sides of decode + encode (dk, dv); latent side of the encode
+//                                                             -> region 2 = dq_enc
+//   stage 3  dq = dq_dec + dq_enc, dq_dyn = gate dq; token side of the synthesis (dk0);
+//            latent side of the synthesis                     -> region 3 = dq0 per batch element
+//   stage 4  batch reduce: dq_fixed, dq0, dgate (identical on every rank)
+// The forward's merged latent states (flarepp_cp_merge) provide q and z, and
+// flarepp_cp_merge_ex the per-latent log-sum-exps and the pre-gate q_dyn.
+struct CpLayout {
+    size_t r1, r2, r3, ws, total;
+};
+
+CpLayout cp_layout(const Shape& s, const BwdPlan& bp) {
+    const size_t latd = (size_t)s.bh() * s.M * s.D * sizeof(float);
+    CpLayout L{};
+    size_t off = 0;
+    L.r1 = off; off = align_up(off + 2 * latd);        // dq_dec, dz
+    L.r2 = off; off = align_up(off + latd);            // dq_enc
+    L.r3 = off; off = align_up(off + latd);            // dq0 per batch element
+    L.ws = off; off = align_up(off + bp.total);        // the backward's workspace
+    L.total = off;
+    return L;
+}
+
+struct CpBwdArgs {
+    BwdArgs a;
+    const void* q_state;     // gated: the routing-query state (fp32 rows, then the I/O-dtype copy)
+    const void* z_state;     // the latent state
+    const float *lse_syn, *lse_enc, *qdyn;
+};
+
+template <typename T, int D>
+cudaError_t cp_stage(int stage, const Shape& s, const BwdPlan& bp, const CpBwdArgs& c, char* state,
+                     StageEvents& ev, cudaStream_t st) {
+    const BwdArgs& a = c.a;
+    const bool gated = a.gate != nullptr;
+    const Plan& pl = bp.fwd;
+    const bool tcp = bp.tc;
+    const CpLayout L = cp_layout(s, bp);
+    char* ws = state + L.ws;
+    const int64_t latd = s.bh() * s.M * s.D;
+    float* r1q = reinterpret_cast<float*>(state + L.r1);
+    float* r1z = r1q + latd;
+    float* r2 = reinterpret_cast<float*>(state + L.r2);
+    float* r3 = reinterpret_cast<float*>(state + L.r3);
+    const float scale = pl.scale_log2 / kLog2e;
+    const size_t o16 = latent_16_offset(s);
+    const float* z32 = static_cast<const float*>(c.z_state);
+    const char* z16 = static_cast<const char*>(c.z_state) + o16;
+    float* dz = reinterpret_cast<float*>(ws + bp.off_dz);
+    float* dq = reinterpret_cast<float*>(ws + bp.off_dq);
+    float* dqdyn = reinterpret_cast<float*>(ws + bp.off_dqdyn);
+    float* delta_enc = reinterpret_cast<float*>(ws + bp.off_delta_enc);
+    float* delta0 = reinterpret_cast<float*>(ws + bp.off_delta0);
+    float* dq0b = reinterpret_cast<float*>(ws + bp.off_dq0b);
+    float* part1 = reinterpret_cast<float*>(ws + bp.off_part1);
+    float* part2 = reinterpret_cast<float*>(ws + bp.off_part2);
+    float2* stats_tok = reinterpret_cast<float2*>(ws + bp.off_stats_tok);
+    float2* stats_enc = reinterpret_cast<float2*>(ws + bp.off_stats_enc);
+    float2* stats_syn = reinterpret_cast<float2*>(ws + bp.off_stats_syn);
+    // the synthesis reads normalised copies of q0, k0 with norm_synthesis
+    const bool norm = pl.norm_synthesis && gated;
+    const void* q0s = norm ? static_cast<const void*>(ws + pl.off_q0n) : a.q0;
+    const void* k0s = norm ? static_cast<const void*>(ws + pl.off_k0n) : a.k0;
+
+    BwdLauncher launch{st};
+    const dim3 red_grid((unsigned)((s.bh() * s.M + 7) / 8));
+    bwd::ReduceParams rp{};
+    rp.B = s.B; rp.H = s.H; rp.M = s.M;
+    auto reduce = [&](const bwd::ReduceParams& r) {
+        launch(bwd::reduce_partials<T, D>, red_grid, dim3(256), r);
+        ev.mark(st);
+    };
+    cudaError_t err = cudaSuccess;
+    auto note = [&](int rc) {
+        if (rc && err == cudaSuccess) err = cudaErrorLaunchFailure;
+        ev.mark(st);
+    };
+
+    // ---- the kernel families' steps (the tensor-core path for 16-bit I/O with the
+    // tcgen05 forward, else SIMT), with the same operands as the single-GPU backward
+    using bwd_tc::Operand;
+    bwd_tc::Launch base{};
+    base.B = s.B; base.H = s.H; base.N = s.N; base.M = s.M; base.D = s.D;
+    base.tok = pl.tok; base.scale_log2 = pl.scale_log2; base.scale = scale; base.chunks = bp.chunks;
+    const Operand q_lat = gated ? Operand{static_cast<const char*>(c.q_state) + o16, false, false}
+                                : Operand{a.q_fixed, false, true};
+    const Operand z_lat{z16, false, false};
+    const Operand k{a.k, true, false}, v{a.v, true, false}, dyo{a.dy, true, false}, k0o{k0s, true, false};
+    const Operand q0o{q0s, false, true};
+    const Operand dz_lat{ws + bp.off_dz16, false, false}, dqdyn_lat{ws + bp.off_dqdyn16, false, false};
+    // the tensor-core launches exist for the 16-bit I/O types only
+    constexpr bool kTc = sizeof(T) == 2;
+    auto tc_launch = [&](const bwd_tc::Launch& Lc) {
+        if constexpr (kTc) note(bwd_tc::launch_bwd_d<T>(Lc, st));
+    };
+    auto tc_latent = [&](Operand A, Operand C, Operand Bc, Operand Ec, bool acc2, bool col, const float2* stt,
+                         int64_t stride) {
+        bwd_tc::Launch Lc = base;
+        Lc.a = A; Lc.c = C; Lc.b = Bc; Lc.e = Ec; Lc.rows_tok = false; Lc.has_acc2 = acc2; Lc.stats_per_col = col;
+        Lc.stats = stt; Lc.stats_stride = stride; Lc.epi = bwd_tc::kEpiPartials; Lc.part1 = part1; Lc.part2 = part2;
+        tc_launch(Lc);
+    };
+    // SIMT operands: fp32 routing queries (the SIMT forward's) when gated
+    bwd::Params sp{};
+    sp.B = s.B; sp.H = s.H; sp.N = s.N; sp.M = s.M;
+    sp.tok_row = pl.tok.row; sp.tok_h = pl.tok.h; sp.tok_b = pl.tok.b;
+    sp.scale_log2 = pl.scale_log2; sp.scale = scale; sp.chunks = bp.chunks; sp.chunk_len = bp.chunk_len;
+    sp.lse_tok = reinterpret_cast<float*>(ws + bp.off_lse_tok);
+    sp.delta_tok = reinterpret_cast<float*>(ws + bp.off_delta_tok);
+    sp.dk_acc = reinterpret_cast<float*>(ws + bp.off_dk_acc);
+    sp.part1 = part1; sp.part2 = part2;
+    sp.Zlat = z32;
+    const void* q_simt = gated ? c.q_state : a.q_fixed;
+    const int q_bh = gated ? s.H : 0;
+    const dim3 tok_grid((unsigned)bp.tok_blocks, (unsigned)s.bh());
+    const dim3 lat_grid((unsigned)bp.chunks, (unsigned)s.bh(), (unsigned)bp.row_blocks);
+    constexpr int kT = bwd::kThreads;
+
+    if (stage == 1) {
+        // decode y = SDPA(k, q, z) over this rank's tokens; the latent side's
+        // chunk partials reduced into region 1
+        if (kTc && tcp) {
+            if constexpr (kTc)
+                note(tc::cp_decode<T>(tc_problem(s, pl), q_lat.ptr, !gated, z16, a.k, nullptr, st, stats_tok,
+                                      bp.n_pad, a.dy));
+            tc_latent(q_lat, z_lat, k, dyo, true, true, stats_tok, bp.n_pad);
+        } else {
+            sp.Qlat = q_simt; sp.q_batch_heads = q_bh; sp.Ktok = a.k; sp.dYtok = a.dy;
+            if (gated) {
+                launch(bwd::decode_rows<T, float, D>, tok_grid, dim3(kT), sp); ev.mark(st);
+                launch(bwd::decode_cols<T, float, D>, lat_grid, dim3(kT), sp); ev.mark(st);
+            } else {
+                launch(bwd::decode_rows<T, T, D>, tok_grid, dim3(kT), sp); ev.mark(st);
+                launch(bwd::decode_cols<T, T, D>, lat_grid, dim3(kT), sp); ev.mark(st);
+            }
+        }
+        rp.part1 = part1; rp.part2 = part2; rp.chunks = bp.chunks; rp.scale = scale;
+        rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = r1z; rp.dq = r1q; rp.delta = delta_enc;
+        reduce(rp);
+    } else if (stage == 2) {
+        // region 1 holds the summed (dq_dec, dz): dz, <dz, z> and the encode's statistics
+        rp.part1 = r1q; rp.part2 = r1z; rp.chunks = 1; rp.scale = 1.f;
+        rp.mode = bwd::kReduceDecode; rp.z = z32; rp.dz = dz; rp.dq = dq; rp.delta = delta_enc;
+        if (tcp) { rp.out16 = ws + bp.off_dz16; rp.stats_out = stats_enc; rp.stats_stride = bp.m_pad; rp.lse_in = c.lse_enc; }
+        reduce(rp);
+        if (tcp) {
+            bwd_tc::Launch Lc = base;
+            Lc.a = k; Lc.c = dyo; Lc.c2 = v; Lc.b = q_lat; Lc.e = z_lat; Lc.e2 = dz_lat;
+            Lc.dual = true; Lc.rows_tok = true; Lc.has_acc2 = true; Lc.stats_per_col = false;
+            Lc.stats = stats_tok; Lc.stats_stride = bp.n_pad; Lc.stats2 = stats_enc; Lc.stats2_stride = bp.m_pad;
+            Lc.epi = bwd_tc::kEpiTokDkDv; Lc.f32 = nullptr; Lc.out1 = a.dk; Lc.out2 = a.dv;
+            tc_launch(Lc);
+            tc_latent(q_lat, dz_lat, k, v, false, false, stats_enc, bp.m_pad);
+        } else {
+            sp.Qlat = q_simt; sp.q_batch_heads = q_bh; sp.dOlat = dz; sp.lse_lat = c.lse_enc; sp.delta_lat = delta_enc;
+            sp.Ktok = a.k; sp.Vtok = a.v; sp.dK = a.dk; sp.dV = a.dv;
+            if (gated) {
+                launch(bwd::token_cols<T, float, D>, tok_grid, dim3(kT), sp); ev.mark(st);
+                launch(bwd::latent_rows<T, float, D>, lat_grid, dim3(kT), sp); ev.mark(st);
+            } else {
+                launch(bwd::token_cols<T, T, D>, tok_grid, dim3(kT), sp); ev.mark(st);
+                launch(bwd::latent_rows<T, T, D>, lat_grid, dim3(kT), sp); ev.mark(st);
+            }
+        }
+        bwd::ReduceParams r = rp;
+        r.part1 = part1; r.chunks = bp.chunks; r.scale = scale; r.mode = bwd::kReduceSynthesis; r.dq0b = r2;
+        r.out16 = nullptr; r.stats_out = nullptr;
+        reduce(r);
+    } else if (stage == 3) {
+        // region 2 holds the summed dq_enc: dq, dq_dyn and the synthesis' statistics
+        rp.part1 = r2; rp.chunks = 1; rp.scale = 1.f; rp.mode = bwd::kReduceEncode; rp.dq = dq;
+        rp.gate = a.gate; rp.qdyn = c.qdyn; rp.dqdyn = dqdyn; rp.delta = delta0;
+        if (tcp && gated) {
+            rp.out16 = ws + bp.off_dqdyn16; rp.stats_out = stats_syn; rp.stats_stride = bp.m_pad; rp.lse_in = c.lse_syn;
+        }
+        reduce(rp);
+        if (gated) {
+            if (norm) {
+                ev.mark(st);
+                rms_norm(s, a.q0, ws + pl.off_q0n, a.k0, ws + pl.off_k0n, st);
+                ev.mark(st);
+            }
+            if (tcp) {
+                bwd_tc::Launch Lc = base;
+                Lc.a = k0o; Lc.c = k0o; Lc.b = q0o; Lc.e = dqdyn_lat; Lc.rows_tok = true; Lc.has_acc2 = true;
+                Lc.stats_per_col = true; Lc.stats = stats_syn; Lc.stats_stride = bp.m_pad;
+                Lc.epi = bwd_tc::kEpiTokDk0; Lc.f32 = nullptr; Lc.out1 = a.dk0; Lc.out2 = nullptr;
+                tc_launch(Lc);
+                tc_latent(q0o, dqdyn_lat, k0o, k0o, false, false, stats_syn, bp.m_pad);
+            } else {
+                sp.Qlat = q0s; sp.q_batch_heads = 0; sp.dOlat = dqdyn; sp.lse_lat = c.lse_syn; sp.delta_lat = delta0;
+                sp.Ktok = k0s; sp.Vtok = k0s; sp.dK = a.dk0; sp.dV = nullptr;
+                launch(bwd::token_cols<T, T, D>, tok_grid, dim3(kT), sp); ev.mark(st);
+                launch(bwd::latent_rows<T, T, D>, lat_grid, dim3(kT), sp); ev.mark(st);
+            }
+            bwd::ReduceParams r{};
+            r.B = s.B; r.H = s.H; r.M = s.M; r.part1 = part1; r.chunks = bp.chunks; r.scale = scale;
+            r.mode = bwd::kReduceSynthesis; r.dq0b = r3;
+            reduce(r);
+            if (norm) {
+                // dk0 (this rank's tokens) through the normalisation
+                const int64_t rows_k = s.bh() * s.N;
+                const int rw = 32 / (D * (int)sizeof(T) / 16);
+                const int64_t want = (rows_k + 8 * rw - 1) / (8 * rw);
+                bwd::rms_backward_rows_coop<T, D><<<(unsigned)std::min<int64_t>(want, (int64_t)kNumSMs * 16), 256, 0,
+                                                   st>>>(static_cast<const T*>(a.k0), static_cast<T*>(a.dk0), rows_k,
+                                                         kNormEps);
+                ev.mark(st);
+            }
+        }
+    } else {
+        // region 3 holds the summed dq0 per batch element: the batch-shared gradients
+        if (gated) {
+            rp.part1 = r3; rp.chunks = 1; rp.scale = 1.f; rp.mode = bwd::kReduceSynthesis; rp.dq0b = dq0b;
+            reduce(rp);
+        }
+        bwd::BatchParams bt{};
+        bt.B = s.B; bt.H = s.H; bt.M = s.M;
+        bt.dq = dq; bt.dq_fixed = a.dq_fixed;
+        if (gated) { bt.dq0b = dq0b; bt.qdyn = c.qdyn; bt.dq0 = a.dq0; bt.dgate = a.dgate; }
+        launch(bwd::reduce_batch<D>, dim3((unsigned)s.H), dim3(256), bt);
+        ev.mark(st);
+        if (norm) {
+            const int64_t rows_q = (int64_t)s.H * s.M;
+            bwd::rms_backward_rows<T, float, D><<<(unsigned)((rows_q + 255) / 256), 256, 0, st>>>(
+                static_cast<const T*>(a.q0), a.dq0, rows_q, kNormEps);
+            ev.mark(st);
+        }
+    }
+    if (err == cudaSuccess) err = launch.err;
+    if (err == cudaSuccess && cudaGetLastError() != cudaSuccess) err = cudaErrorLaunchFailure;
+    return err;
+}
+
+template <typename T>
+cudaError_t cp_stage_d(int stage, const Shape& s, const BwdPlan& bp, const CpBwdArgs& c, char* state,
+                       StageEvents& ev, cudaStream_t st) {
+    switch (s.D) {
+        case 16: return cp_stage<T, 16>(stage, s, bp, c, state, ev, st);
+        case 32: return cp_stage<T, 32>(stage, s, bp, c, state, ev, st);
+        case 64: return cp_stage<T, 64>(stage, s, bp, c, state, ev, st);
+        default: return cp_stage<T, 128>(stage, s, bp, c, state, ev, st);
+    }
+}
+
+int cp_bwd_stage(int stage, const CpBwdArgs& c, void* state, int B, int H, int N, int M, int D, int dtype,
+                 const flarepp_options_t* opts, void* stream) {
+    const Shape s{B, H, N, M, D, dtype};
+    BwdPlan bp{};
+    int rc = make_bwd_plan(s, opts, &bp);
+    if (rc) return rc;
+    if (stage < 1 || stage > 4) return FLAREPP_ERR_INVALID_ARG;
+    rc = check_bwd_pointers(s, c.a);
+    if (rc) return rc;
+    const bool gated = c.a.gate != nullptr;
+    if (!state || reinterpret_cast<uintptr_t>(state) % kAlign || !c.z_state || !c.lse_enc ||
+        (gated && (!c.q_state || !c.lse_syn || !c.qdyn)))
+        return FLAREPP_ERR_INVALID_ARG;
+    if (!aligned16(c.z_state) || (gated && !aligned16(c.q_state))) return FLAREPP_ERR_INVALID_ARG;
+    // the CP stages take the recomputed forward's state from flarepp_cp_merge(_ex):
+    // its latent inputs must keep the layout the forward's merge wrote
+    if (opts && (opts->q_out || opts->z_out)) return FLAREPP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    StageEvents ev;
+    if (opts && opts->n_stage_events > 0) {
+        ev.ev = opts->stage_events;
+        ev.n = opts->n_stage_events;
+    }
+    ev.mark(st);
+    char* base = static_cast<char*>(state);
+    cudaError_t e;
+    if (dtype == FLAREPP_F32) e = cp_stage_d<float>(stage, s, bp, c, base, ev, st);
+    else if (dtype == FLAREPP_F16) e = cp_stage_d<__half>(stage, s, bp, c, base, ev, st);
+    else e = cp_stage_d<__nv_bfloat16>(stage, s, bp, c, base, ev, st);
+    return e == cudaSuccess ? FLAREPP_OK : FLAREPP_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace flarepp
 
@@ -1490,6 +1784,39 @@ int flarepp_cp_partials(const void* q, int q_shared, const void* k, const void* 
 int flarepp_cp_merge(const float* gathered, int ranks, const void* q_fixed, const float* gate, void* state, int B,
                      int H, int M, int D, int dtype, void* stream) {
     return cp_merge(gathered, ranks, q_fixed, gate, state, B, H, M, D, dtype, stream);
+}
+
+int flarepp_cp_merge_ex(const float* gathered, int ranks, const void* q_fixed, const float* gate, void* state,
+                        float* lse_out, float* pregate_out, int B, int H, int M, int D, int dtype, void* stream) {
+    return cp_merge(gathered, ranks, q_fixed, gate, state, B, H, M, D, dtype, stream, lse_out, pregate_out);
+}
+
+int flarepp_cp_bwd_layout(int B, int H, int N, int M, int D, int dtype, const flarepp_options_t* opts,
+                          flarepp_cp_bwd_layout_t* out) {
+    const Shape s{B, H, N, M, D, dtype};
+    BwdPlan bp{};
+    int rc = make_bwd_plan(s, opts, &bp);
+    if (rc) return rc;
+    if (!out) return FLAREPP_ERR_INVALID_ARG;
+    const CpLayout L = cp_layout(s, bp);
+    const size_t latd = (size_t)s.bh() * M * D * sizeof(float);
+    out->bytes = L.total;
+    out->reduce_offset[0] = L.r1; out->reduce_bytes[0] = 2 * latd;
+    out->reduce_offset[1] = L.r2; out->reduce_bytes[1] = latd;
+    out->reduce_offset[2] = L.r3; out->reduce_bytes[2] = latd;
+    return FLAREPP_OK;
+}
+
+int flarepp_cp_bwd_stage(int stage, const void* q0, const void* q_fixed, const float* gate, const void* q_state,
+                         const void* z_state, const float* lse_syn, const float* lse_enc, const float* qdyn,
+                         const void* k0, const void* k, const void* v, const void* dy, float* dq0, float* dq_fixed,
+                         float* dgate, void* dk0, void* dk, void* dv, void* state, int B, int H, int N, int M, int D,
+                         int dtype, const flarepp_options_t* opts, void* stream) {
+    CpBwdArgs c{};
+    c.a.q0 = q0; c.a.q_fixed = q_fixed; c.a.gate = gate; c.a.k0 = k0; c.a.k = k; c.a.v = v; c.a.dy = dy;
+    c.a.dq0 = dq0; c.a.dq_fixed = dq_fixed; c.a.dgate = dgate; c.a.dk0 = dk0; c.a.dk = dk; c.a.dv = dv;
+    c.q_state = q_state; c.z_state = z_state; c.lse_syn = lse_syn; c.lse_enc = lse_enc; c.qdyn = qdyn;
+    return cp_bwd_stage(stage, c, state, B, H, N, M, D, dtype, opts, stream);
 }
 
 int flarepp_cp_decode(const void* q, int q_shared, const void* z_state, const void* k, void* y, int B, int H, int N,

@@ -1290,7 +1290,7 @@ int cp_split(const Problem& pr, const Buffers& bu, const void* q, bool q_shared,
 // when q_shared, else the [B,H,M,D] routing queries) and values z [B,H,M,D].
 template <typename E>
 int cp_decode(const Problem& pr, const void* q, bool q_shared, const void* z16, const void* kk, void* y,
-              cudaStream_t st) {
+              cudaStream_t st, float2* tok_stats = nullptr, int64_t tok_stats_stride = 0, const void* dy = nullptr) {
     const int B = pr.B, H = pr.H, N = pr.N, M = pr.M, D = pr.D, BH = B * H;
     const CUtensorMapDataType ty = Elem<E>::kMapType;
     CUtensorMap mq, mk, mv;
@@ -1310,6 +1310,9 @@ int cp_decode(const Problem& pr, const void* q, bool q_shared, const void* z16, 
     dp.y = y;
     dp.y_row = pr.tok.row; dp.y_h = pr.tok.h; dp.y_b = pr.tok.b;
     dp.tok_heads_inner = pr.tok.h < pr.tok.row ? 1 : 0;
+    dp.tok_stats = tok_stats;
+    dp.tok_stats_stride = tok_stats_stride;
+    dp.dy = dy;
     int rc = launch_decode<E>(D, mq, mk, mv, dp, st);
     if (rc) return rc;
     return cudaGetLastError() == cudaSuccess ? 0 : 3;

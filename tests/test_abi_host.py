@@ -219,3 +219,25 @@ def test_training_context_entries_checked(lib):
     p2 = list(p)
     p2[6] = None                                                  # no y
     assert bwd(*p2, 1, 2, 64, 16, 16, 1, None, 0x900000, 1 << 20, None) == 1
+
+
+def test_sharded_backward_entries_checked(lib):
+    lay = lib.cp_bwd_layout(1, 2, 64, 16, 16, lib.BF16)
+    assert lay.bytes > 0
+    latd = 1 * 2 * 16 * 16 * 4
+    assert list(lay.reduce_bytes) == [2 * latd, latd, latd]
+    assert lay.reduce_offset[0] % 256 == 0 and lay.reduce_offset[1] >= lay.reduce_offset[0] + 2 * latd
+    with pytest.raises(lib.FlareppError):
+        lib.cp_bwd_layout(1, 2, 64, 16, 48, lib.BF16)
+    fn = lib.lib.flarepp_cp_bwd_stage
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [i] + [vp] * 19 + [i] * 6 + [vp, vp]
+    ptrs = [0x100000 * (j + 1) for j in range(19)]
+    assert fn(0, *ptrs, 1, 2, 64, 16, 16, 1, None, None) == 1        # stage outside 1..4
+    assert fn(5, *ptrs, 1, 2, 64, 16, 16, 1, None, None) == 1
+    p = list(ptrs)
+    p[18] = 0x100010                                                  # state misaligned
+    assert fn(1, *p, 1, 2, 64, 16, 16, 1, None, None) == 1
+    p = list(ptrs)
+    p[4] = None                                                       # no z state
+    assert fn(1, *p, 1, 2, 64, 16, 16, 1, None, None) == 1
