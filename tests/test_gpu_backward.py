@@ -59,6 +59,9 @@ CASES = [
     ((1, 2, 700, 96, 32, "f16"), 0),
     ((1, 2, 900, 80, 64, "bf16"), 1),     # the recomputed forward on the SIMT kernels (fp32 routing queries)
     ((1, 2, 600, 40, 64, "f16"), 1),
+    ((2, 1, 520, 150, 128, "f16"), 0),    # fp16 on the tensor cores at the widest and narrowest head dims
+    ((1, 2, 999, 33, 16, "f16"), 0),
+    ((1, 1, 4100, 512, 64, "bf16"), 0),   # M = 512: both latent row groups, many token tiles
 ]
 
 
