@@ -945,7 +945,6 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
     const bool gated = a.gate != nullptr;
     BwdLauncher launch_bwd_kernel{st};
     const Plan& pl = bp.fwd;
-    using L = bwd::Lanes<D>;
     bwd::Params p{};
     p.B = s.B; p.H = s.H; p.N = s.N; p.M = s.M;
     p.tok_row = pl.tok.row; p.tok_h = pl.tok.h; p.tok_b = pl.tok.b;
@@ -1014,7 +1013,6 @@ cudaError_t run_backward(const Shape& s, const BwdPlan& bp, const BwdArgs& a, ch
     if (gated) { bt.dq0b = dq0b; bt.qdyn = qdyn; bt.dq0 = a.dq0; bt.dgate = a.dgate; }
     launch_bwd_kernel(bwd::reduce_batch<D>, dim3((unsigned)s.H), dim3(256), bt);
     ev.mark(st);
-    (void)L::G;
     return launch_bwd_kernel.err;
 }
 
@@ -1066,7 +1064,7 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
         L.a = A; L.c = C; L.b = Bc; L.e = Ec;
         L.rows_tok = true; L.has_acc2 = acc2; L.stats_per_col = col_stats;
         L.stats = stats; L.stats_stride = stride;
-        L.epi = epi; L.f32 = nullptr; L.out1 = out1; L.out2 = out2;
+        L.epi = epi; L.out1 = out1; L.out2 = out2;
         note(bwd_tc::launch_bwd_d<E>(L, st));
     };
     BwdLauncher launch{st};
@@ -1096,7 +1094,7 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
         L.dual = true; L.rows_tok = true; L.has_acc2 = true; L.stats_per_col = false;
         L.stats = stats_tok; L.stats_stride = bp.n_pad;      // the decode's softmax: per token
         L.stats2 = stats_enc; L.stats2_stride = bp.m_pad;    // the encode's: per latent
-        L.epi = bwd_tc::kEpiTokDkDv; L.f32 = nullptr; L.out1 = a.dk; L.out2 = a.dv;
+        L.epi = bwd_tc::kEpiTokDkDv; L.out1 = a.dk; L.out2 = a.dv;
         note(bwd_tc::launch_bwd_d<E>(L, st));
     }
     // encode z = SDPA(q, k, v): latent side (dq_enc partials)
@@ -1545,7 +1543,7 @@ cudaError_t cp_stage(int stage, const Shape& s, const BwdPlan& bp, const CpBwdAr
             Lc.a = k; Lc.c = dyo; Lc.c2 = v; Lc.b = q_lat; Lc.e = z_lat; Lc.e2 = dz_lat;
             Lc.dual = true; Lc.rows_tok = true; Lc.has_acc2 = true; Lc.stats_per_col = false;
             Lc.stats = stats_tok; Lc.stats_stride = bp.n_pad; Lc.stats2 = stats_enc; Lc.stats2_stride = bp.m_pad;
-            Lc.epi = bwd_tc::kEpiTokDkDv; Lc.f32 = nullptr; Lc.out1 = a.dk; Lc.out2 = a.dv;
+            Lc.epi = bwd_tc::kEpiTokDkDv; Lc.out1 = a.dk; Lc.out2 = a.dv;
             tc_launch(Lc);
             tc_latent(q_lat, dz_lat, k, v, false, false, stats_enc, bp.m_pad);
         } else {
@@ -1581,7 +1579,7 @@ cudaError_t cp_stage(int stage, const Shape& s, const BwdPlan& bp, const CpBwdAr
                 bwd_tc::Launch Lc = base;
                 Lc.a = k0o; Lc.c = k0o; Lc.b = q0o; Lc.e = dqdyn_lat; Lc.rows_tok = true; Lc.has_acc2 = true;
                 Lc.stats_per_col = true; Lc.stats = stats_syn; Lc.stats_stride = bp.m_pad;
-                Lc.epi = bwd_tc::kEpiTokDk0; Lc.f32 = nullptr; Lc.out1 = a.dk0; Lc.out2 = nullptr;
+                Lc.epi = bwd_tc::kEpiTokDk0; Lc.out1 = a.dk0; Lc.out2 = nullptr;
                 tc_launch(Lc);
                 tc_latent(q0o, dqdyn_lat, k0o, k0o, false, false, stats_syn, bp.m_pad);
             } else {

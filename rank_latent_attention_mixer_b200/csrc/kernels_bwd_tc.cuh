@@ -63,9 +63,8 @@ struct Shape {
 
 enum Epilogue {
     kEpiPartials = 0,   // latent rows: acc1 (and acc2) -> fp32 partials [chunk][B*H][rows][D]
-    kEpiTokF32 = 1,     // token rows: scale acc1 -> fp32 [B*H][N][D]              (decode's dk)
-    kEpiTokDkDv = 2,    // token rows: dK = scale acc1 + f32 in, dV = acc2, in E   (encode)
-    kEpiTokDk0 = 3      // token rows: dK0 = scale acc1 + acc2, in E               (synthesis)
+    kEpiTokDkDv = 2,    // token rows: dK = scale acc1, dV = acc2, in E   (decode + encode)
+    kEpiTokDk0 = 3      // token rows: dK0 = scale acc1 + acc2, in E      (synthesis)
 };
 
 struct Params {
@@ -89,7 +88,6 @@ struct Params {
     int epi;                    // Epilogue
     float* part1;
     float* part2;
-    float* f32;                 // kEpiTokF32: out; kEpiTokDkDv: the decode's share of dk, in (or NULL)
     void* out1;                 // token outputs in E: dK (or dK0)
     void* out2;                 // dV
     int64_t tok_row, tok_h, tok_b;   // element strides of the token outputs
@@ -620,32 +618,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                             d2[i] = make_float4(__uint_as_float(a2[4 * i]), __uint_as_float(a2[4 * i + 1]),
                                                 __uint_as_float(a2[4 * i + 2]), __uint_as_float(a2[4 * i + 3]));
                     }
-                } else if (p.epi == kEpiTokF32) {
-                    float4* d1 = reinterpret_cast<float4*>(p.f32 + ((int64_t)it.bh * p.row_count + r) * D + c0);
-#pragma unroll
-                    for (int i = 0; i < CW / 4; ++i)
-                        d1[i] = make_float4(p.scale * __uint_as_float(a1[4 * i]), p.scale * __uint_as_float(a1[4 * i + 1]),
-                                            p.scale * __uint_as_float(a1[4 * i + 2]),
-                                            p.scale * __uint_as_float(a1[4 * i + 3]));
                 } else {
                     const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
                     float v1[CW];
                     if (p.epi == kEpiTokDkDv) {
-                        if (p.f32) {
-                            const float4* prev =
-                                reinterpret_cast<const float4*>(p.f32 + ((int64_t)it.bh * p.row_count + r) * D + c0);
 #pragma unroll
-                            for (int i = 0; i < CW / 4; ++i) {
-                                const float4 q4 = prev[i];
-                                v1[4 * i] = fmaf(p.scale, __uint_as_float(a1[4 * i]), q4.x);
-                                v1[4 * i + 1] = fmaf(p.scale, __uint_as_float(a1[4 * i + 1]), q4.y);
-                                v1[4 * i + 2] = fmaf(p.scale, __uint_as_float(a1[4 * i + 2]), q4.z);
-                                v1[4 * i + 3] = fmaf(p.scale, __uint_as_float(a1[4 * i + 3]), q4.w);
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < CW; ++i) v1[i] = p.scale * __uint_as_float(a1[i]);
-                        }
+                        for (int i = 0; i < CW; ++i) v1[i] = p.scale * __uint_as_float(a1[i]);
                         float v2[CW];
 #pragma unroll
                         for (int i = 0; i < CW; ++i) v2[i] = __uint_as_float(a2[i]);
@@ -697,7 +675,7 @@ struct Launch {
     float scale_log2, scale;
     int epi;
     int chunks;                // latent rows: column chunks (0 = planned)
-    float *part1, *part2, *f32;
+    float *part1, *part2;
     void *out1, *out2;
 };
 
@@ -759,7 +737,7 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
     p.scale_log2 = L.scale_log2;
     p.scale = L.scale;
     p.epi = L.epi;
-    p.part1 = L.part1; p.part2 = L.part2; p.f32 = L.f32;
+    p.part1 = L.part1; p.part2 = L.part2;
     p.out1 = L.out1; p.out2 = L.out2;
     p.tok_row = L.tok.row; p.tok_h = L.tok.h; p.tok_b = L.tok.b;
     auto kern = bwd_kernel<E, D, NW, DUAL>;
