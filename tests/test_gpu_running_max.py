@@ -1,12 +1,13 @@
 """Scores that rise from one key/value tile to the next.
 
 The online softmax of the tcgen05 kernels keeps a running row maximum and only
-rescales when a tile's maximum exceeds it by more than 8 log2 units.  These
+rescales when a tile's maximum exceeds it by more than 8 log2 units (fp16 I/O
+takes the weights against the maximum minus 7, so they stay below 2^15).  These
 inputs make later tiles exceed it by a few units, by 8 to 120 units and by far
 more (where exponentials against the old maximum would overflow fp32), in the
-synthesis, encode and decode passes; the result is compared with the fp64
-oracle.  The softmax is the one of scaled dot-product attention (FLARE++ mixer,
-encode/decode equations).
+synthesis, encode and decode passes, with bf16 and fp16 I/O; the result is
+compared with the fp64 oracle.  The softmax is the one of scaled dot-product
+attention (FLARE++ mixer, encode/decode equations).
 """
 import math
 
@@ -22,7 +23,7 @@ KT = 128          # key/value tile of the split passes
 DEC_KT = 64       # latent tile of the decode pass
 
 
-def structured(kind, B, H, N, M, D, seed):
+def structured(kind, B, H, N, M, D, seed, dtype="bf16"):
     """Latents q0 = q_fixed ~ (1 + m/16) * ones, tokens k0 = k ~ b(n) * ones/8,
     small noise, so that a score is about (1 + m/16) * b(n) * sqrt(D)/8 and
     rises along n (split passes) and along m (decode)."""
@@ -34,12 +35,13 @@ def structured(kind, B, H, N, M, D, seed):
         b = torch.where(n < 3 * KT, torch.zeros_like(n), torch.full_like(n, 70.0))
     lat = (1.0 + torch.arange(M, dtype=torch.float64) / 16.0)[:, None].expand(M, D)
     noise = lambda *s: 0.05 * torch.randn(*s, generator=g, dtype=torch.float64)
-    q0 = (lat[None] + noise(H, M, D)).to(torch.bfloat16)
-    q_fixed = (lat[None] + noise(H, M, D)).to(torch.bfloat16)
+    io = torch.float16 if dtype == "f16" else torch.bfloat16
+    q0 = (lat[None] + noise(H, M, D)).to(io)
+    q_fixed = (lat[None] + noise(H, M, D)).to(io)
     tok = (b[:, None] / 8.0).expand(N, D)
-    k0 = (tok[None, None] + noise(B, H, N, D)).to(torch.bfloat16)
-    k = (tok[None, None] + noise(B, H, N, D)).to(torch.bfloat16)
-    v = torch.randn(B, H, N, D, generator=g, dtype=torch.float64).to(torch.bfloat16)
+    k0 = (tok[None, None] + noise(B, H, N, D)).to(io)
+    k = (tok[None, None] + noise(B, H, N, D)).to(io)
+    v = torch.randn(B, H, N, D, generator=g, dtype=torch.float64).to(io)
     gate = torch.full((H,), 0.5, dtype=torch.float32)
     return dict(q0=q0, q_fixed=q_fixed, gate=gate, k0=k0, k=k, v=v)
 
@@ -60,11 +62,12 @@ def lags(q, keys, tile, stride):
     return torch.cat(out)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("kind", ["ramp", "jump"])
 @pytest.mark.parametrize("M", [128, 256])
-def test_lagging_running_max(kind, M):
+def test_lagging_running_max(kind, M, dtype):
     B, H, N, D = 1, 2, 1000, 64
-    x = structured(kind, B, H, N, M, D, seed=M + len(kind))
+    x = structured(kind, B, H, N, M, D, seed=M + len(kind), dtype=dtype)
     # the inputs reach every case of the check in the synthesis pass (one
     # chunk: an item spans all tiles; M <= 128 gives the warpgroups every
     # other tile)
@@ -86,7 +89,7 @@ def test_lagging_running_max(kind, M):
                                     d["v"], return_qz=True, path=2, force_chunks=fc)
             torch.cuda.synchronize()
             assert bnd.check_device_status() == 0
-            tag = f"{kind} M={M} flare={flare} chunks={fc}"
-            assert_parity(z, z_ref, "bf16", "z " + tag)
-            assert_parity(q, q_ref, "bf16", "q " + tag)
-            assert_parity(y, y_ref, "bf16", "y " + tag)
+            tag = f"{kind} M={M} flare={flare} chunks={fc} {dtype}"
+            assert_parity(z, z_ref, dtype, "z " + tag)
+            assert_parity(q, q_ref, dtype, "q " + tag)
+            assert_parity(y, y_ref, dtype, "y " + tag)
