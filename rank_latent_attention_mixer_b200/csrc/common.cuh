@@ -71,7 +71,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // 2^x on the MUFU unit (PTX ex2.approx, flush-to-zero).
 __device__ __forceinline__ float ex2_mufu(float x) {
     float y;
-    asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 

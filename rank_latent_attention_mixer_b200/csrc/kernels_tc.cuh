@@ -277,8 +277,13 @@ __device__ __forceinline__ float2 ex2_fma_pair(float2 x) {
 }
 
 // Share of the exponentials that run on the FMA pipe instead of the MUFU unit:
-// this many column pairs out of every 64 (scaled to the tile width).
+// this many column pairs out of every 64, spread evenly along the row (pair i
+// when (i * share) mod 64 falls in the top `share` residues), so that each
+// stretch of the row keeps both pipes busy.
 constexpr int kFmaExpPairsPer64 = 16;
+__host__ __device__ constexpr bool fma_exp_pair(int i) {
+    return (i * kFmaExpPairsPer64) % 64 >= 64 - kFmaExpPairsPer64;
+}
 
 // max(a, b, c) in one instruction (three-input max.f32)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -403,7 +408,6 @@ struct Layout {
     static_assert(kPCol + NW * (KT / 2) <= 512, "TMEM plan exceeds 512 columns");
     static constexpr int kChunks = KT / 32;                          // 32-column score chunks per row
     static constexpr int kPairs = KT / 2;                            // column pairs per row
-    static constexpr int kFmaPairs = kFmaExpPairsPer64 * kPairs / 64;
 };
 
 // ------------------------------------------------------------------ the kernel
@@ -843,7 +847,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     for (int j = 0; j < 16; ++j) {
                         const float2 sv = make_float2(__uint_as_float(sr[c][2 * j]), __uint_as_float(sr[c][2 * j + 1]));
                         const float2 xv = __ffma2_rn(sv, sl2v, negm);
-                        const float2 pv = (c * 16 + j >= LY::kPairs - LY::kFmaPairs)
+                        const float2 pv = fma_exp_pair(c * 16 + j)
                                               ? ex2_fma_pair(xv)
                                               : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
