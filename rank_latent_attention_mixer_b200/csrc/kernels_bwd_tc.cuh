@@ -471,6 +471,60 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
         const float sl2 = p.scale_log2;
         uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0, g = 0;
         bool ok = true;
+        // An item's accumulators -> its outputs (every accumulating MMA of the
+        // item has completed).  The fused token side (DUAL: items of 16 jobs)
+        // defers it into the next item's first job: the item's last
+        // accumulation finishes in the shadow of the next exponentials, and
+        // the accumulators are read after that job's P and dS stores, before
+        // its pfull releases the MMA that resets them.  The other forms (items
+        // of hundreds of jobs, or a single softmax per job) ran faster with it
+        // at the end of the item.
+        auto epilogue = [&](const Item& it, int r, bool rvalid) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                constexpr int CW = D < 32 ? D : 32;        // valid columns of a 32-column load
+                uint32_t a1[32], a2[32];
+                tc::tmem_ld32(tA1 + c0, a1);
+                if (p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
+                tc::tmem_wait_ld();
+                if (!rvalid) continue;
+                if (p.epi == kEpiPartials) {
+                    const int64_t ridx = ((int64_t)it.chunk * p.B * p.H + it.bh) * p.row_count + r;
+                    float4* d1 = reinterpret_cast<float4*>(p.part1 + ridx * D + c0);
+#pragma unroll
+                    for (int i = 0; i < CW / 4; ++i)
+                        d1[i] = make_float4(__uint_as_float(a1[4 * i]), __uint_as_float(a1[4 * i + 1]),
+                                            __uint_as_float(a1[4 * i + 2]), __uint_as_float(a1[4 * i + 3]));
+                    if (p.has_acc2) {
+                        float4* d2 = reinterpret_cast<float4*>(p.part2 + ridx * D + c0);
+#pragma unroll
+                        for (int i = 0; i < CW / 4; ++i)
+                            d2[i] = make_float4(__uint_as_float(a2[4 * i]), __uint_as_float(a2[4 * i + 1]),
+                                                __uint_as_float(a2[4 * i + 2]), __uint_as_float(a2[4 * i + 3]));
+                    }
+                } else {
+                    const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
+                    float v1[CW];
+                    if (p.epi == kEpiTokDkDv) {
+#pragma unroll
+                        for (int i = 0; i < CW; ++i) v1[i] = p.scale * __uint_as_float(a1[i]);
+                        float v2[CW];
+#pragma unroll
+                        for (int i = 0; i < CW; ++i) v2[i] = __uint_as_float(a2[i]);
+                        store_row<E, CW>(static_cast<E*>(p.out2) + off, v2);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < CW; ++i)
+                            v1[i] = fmaf(p.scale, __uint_as_float(a1[i]), __uint_as_float(a2[i]));
+                    }
+                    store_row<E, CW>(static_cast<E*>(p.out1) + off, v1);
+                }
+            }
+        };
+        bool pend = false;
+        Item pend_it{};
+        int pend_r = 0;
+        bool pend_rvalid = false;
         for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
             const Item it = decode_item<NW>(p, item);
             const int r = it.row0 + wg * kQTile + row;
@@ -581,6 +635,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 tc::tc_fence_after();
                 tmem_st16(tP, pk);
                 tmem_st16(tDS, dk);
+                if constexpr (DUAL) {
+                    if (pend) {
+                        epilogue(pend_it, pend_r, pend_rvalid);
+                        pend = false;
+                    }
+                }
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
@@ -589,55 +649,34 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             }
             if (!ok) break;
 
-            // ---------------- end of the item: the accumulators -> outputs
+            // ---------------- end of the item
+            if constexpr (DUAL) {
+                pend = true;         // its epilogue waits for the next item's first job
+                pend_it = it;
+                pend_r = r;
+                pend_rvalid = rvalid;
+            } else {
+                while (pfree_waits < jobs_done) {
+                    if (!tc::mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                    ++pfree_waits;
+                }
+                if (!ok) break;
+                tc::tc_fence_after();
+                epilogue(it, r, rvalid);
+                // the accumulators are read before the next item's first job is released to the MMA
+                tc::tc_fence_before();
+            }
+        }
+        if (ok && pend) {
+            // the last item's epilogue, once its last accumulating MMA has completed
             while (pfree_waits < jobs_done) {
                 if (!tc::mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
                 ++pfree_waits;
             }
-            if (!ok) break;
-            tc::tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                constexpr int CW = D < 32 ? D : 32;        // valid columns of a 32-column load
-                uint32_t a1[32], a2[32];
-                tc::tmem_ld32(tA1 + c0, a1);
-                if (p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
-                tc::tmem_wait_ld();
-                if (!rvalid) continue;
-                if (p.epi == kEpiPartials) {
-                    const int64_t ridx = ((int64_t)it.chunk * p.B * p.H + it.bh) * p.row_count + r;
-                    float4* d1 = reinterpret_cast<float4*>(p.part1 + ridx * D + c0);
-#pragma unroll
-                    for (int i = 0; i < CW / 4; ++i)
-                        d1[i] = make_float4(__uint_as_float(a1[4 * i]), __uint_as_float(a1[4 * i + 1]),
-                                            __uint_as_float(a1[4 * i + 2]), __uint_as_float(a1[4 * i + 3]));
-                    if (p.has_acc2) {
-                        float4* d2 = reinterpret_cast<float4*>(p.part2 + ridx * D + c0);
-#pragma unroll
-                        for (int i = 0; i < CW / 4; ++i)
-                            d2[i] = make_float4(__uint_as_float(a2[4 * i]), __uint_as_float(a2[4 * i + 1]),
-                                                __uint_as_float(a2[4 * i + 2]), __uint_as_float(a2[4 * i + 3]));
-                    }
-                } else {
-                    const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
-                    float v1[CW];
-                    if (p.epi == kEpiTokDkDv) {
-#pragma unroll
-                        for (int i = 0; i < CW; ++i) v1[i] = p.scale * __uint_as_float(a1[i]);
-                        float v2[CW];
-#pragma unroll
-                        for (int i = 0; i < CW; ++i) v2[i] = __uint_as_float(a2[i]);
-                        store_row<E, CW>(static_cast<E*>(p.out2) + off, v2);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < CW; ++i)
-                            v1[i] = fmaf(p.scale, __uint_as_float(a1[i]), __uint_as_float(a2[i]));
-                    }
-                    store_row<E, CW>(static_cast<E*>(p.out1) + off, v1);
-                }
+            if (ok) {
+                tc::tc_fence_after();
+                epilogue(pend_it, pend_r, pend_rvalid);
             }
-            // the accumulators are read before the next item's first job is released to the MMA
-            tc::tc_fence_before();
         }
     }
 

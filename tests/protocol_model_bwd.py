@@ -66,6 +66,7 @@ def simulate(p, blk, grid, seed, writes):
     P_job = [None] * NW                 # job whose P, dS the warpgroup's TMEM buffer holds
     P_readers = [0] * NW                # accumulating MMAs still reading P/dS
     acc_item = [None] * NW              # item the accumulators belong to
+    acc_done = [{} for _ in range(NW)]  # item -> its accumulating MMAs completed
     epilogue_done = [set() for _ in range(NW)]
 
     def producer():
@@ -144,8 +145,9 @@ def simulate(p, blk, grid, seed, writes):
                 acc_item[w] = item
             P_readers[w] += 1
 
-            def done(w=w, st=st):
+            def done(w=w, st=st, item=item):
                 P_readers[w] -= 1
+                acc_done[w][item] = acc_done[w].get(item, 0) + 1
                 bars[f"pfree{w}"].arrive()
                 bars[f"col_empty{st}"].arrive()
             commit(done)
@@ -166,6 +168,20 @@ def simulate(p, blk, grid, seed, writes):
 
     def softmax(wg):
         sfull_waits = pfree_waits = jobs_done = 0
+        pend = None                      # the finished item whose epilogue is deferred
+
+        def epilogue(item, it):
+            assert acc_item[wg] == item, ("epilogue reads another item's accumulators", acc_item[wg], item)
+            assert P_readers[wg] == 0, ("epilogue while an accumulating MMA still runs", wg)
+            assert acc_done[wg].get(item, 0) == it["t_end"] - it["t_begin"], \
+                ("epilogue before the item's last accumulation", acc_done[wg].get(item, 0))
+            epilogue_done[wg].add(item)
+            for row in range(QT):
+                r = it["row0"] + wg * QT + row
+                if r < p["row_count"]:
+                    key = (it["chunk"], it["bh"], r)
+                    writes[key] = writes.get(key, 0) + 1
+
         for item, it, t, ic, g, first, last in jobs():
             yield ("wait", f"sfull{wg}", sfull_waits & 1)
             sfull_waits += 1
@@ -182,20 +198,30 @@ def simulate(p, blk, grid, seed, writes):
                 pfree_waits += 1
             assert P_readers[wg] == 0, ("P/dS overwritten while an accumulating MMA reads it", wg)
             P_job[wg] = (item, t)
+            if pend is not None and not p.get("no_deferred_wait"):
+                # the previous item's accumulators, read before this job's
+                # accumulating MMA (released by pfull) overwrites them
+                epilogue(*pend)
+                pend = None
             for _ in range(4):
                 bars[f"pfull{wg}"].arrive()
             jobs_done += 1
             if last:
-                while pfree_waits < jobs_done:
-                    yield ("wait", f"pfree{wg}", pfree_waits & 1)
-                    pfree_waits += 1
-                assert acc_item[wg] == item
-                epilogue_done[wg].add(item)
-                for row in range(QT):
-                    r = it["row0"] + wg * QT + row
-                    if r < p["row_count"]:
-                        key = (it["chunk"], it["bh"], r)
-                        writes[key] = writes.get(key, 0) + 1
+                if p.get("no_deferred_wait"):
+                    # planted: the epilogue without waiting for the item's last accumulating MMA
+                    epilogue(item, it)
+                elif p["deferred"]:
+                    pend = (item, it)
+                else:
+                    while pfree_waits < jobs_done:
+                        yield ("wait", f"pfree{wg}", pfree_waits & 1)
+                        pfree_waits += 1
+                    epilogue(item, it)
+        if pend is not None:
+            while pfree_waits < jobs_done:
+                yield ("wait", f"pfree{wg}", pfree_waits & 1)
+                pfree_waits += 1
+            epilogue(*pend)
 
     roles = [producer()] + [mma(w) for w in range(NW)] + [softmax(w) for w in range(NW)]
     state = [None] * len(roles)
@@ -242,7 +268,8 @@ def choose_chunks(units, tiles, sms=148):
     return best_c
 
 
-def check(B, H, N, M, D, side, col_stats, grid=148, seed=0, force_chunks=0, dual=False, skip_pfree_wait=False):
+def check(B, H, N, M, D, side, col_stats, grid=148, seed=0, force_chunks=0, dual=False, skip_pfree_wait=False,
+          no_deferred_wait=False):
     """side: "latent" (rows = M latents, columns = a chunk of the N tokens) or
     "token" (rows = N tokens, columns = all M latents); col_stats: the
     statistics come with the column tiles (else they belong to the rows)."""
@@ -260,7 +287,8 @@ def check(B, H, N, M, D, side, col_stats, grid=148, seed=0, force_chunks=0, dual
     p = dict(NW=NW, NST=4, QS=1 if dual else 2, row_groups=rg, chunks=chunks, chunk_tiles=tpc,
              col_tiles=col_tiles, items=BH * chunks * rg, row_count=rows,
              row_tiles=3 if dual else 2, col_tiles_per_stage=3 if dual else 2,
-             col_stats=dual or col_stats, skip_pfree_wait=skip_pfree_wait)
+             col_stats=dual or col_stats, skip_pfree_wait=skip_pfree_wait, no_deferred_wait=no_deferred_wait,
+             deferred=dual)
     g = min(grid, p["items"])
     writes = {}
     for blk in range(g):

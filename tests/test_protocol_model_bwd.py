@@ -37,3 +37,12 @@ def test_model_catches_a_missing_pfree_wait():
     the race the pfree barrier prevents; the model must see it."""
     with pytest.raises(AssertionError, match="P/dS overwritten"):
         check(1, 2, 3000, 64, 64, side="latent", col_stats=True, grid=23, skip_pfree_wait=True)
+
+
+def test_model_catches_an_epilogue_before_the_last_accumulation():
+    # planted: the item's epilogue reads the accumulators as soon as its last
+    # P/dS is released, without waiting for that accumulating MMA
+    with pytest.raises(AssertionError, match="last accumulation|still runs"):
+        for seed in range(20):
+            check(1, 2, 3000, 512, 64, side="token", col_stats=False, grid=7, seed=seed, dual=True,
+                  no_deferred_wait=True)
