@@ -828,13 +828,6 @@ struct BwdPlan {
         off_dz16, off_dqdyn16, total;
 };
 
-int tc_bwd_chunks(const Shape& s, int force) {
-    const int tiles = (s.N + bwd_tc::kKT - 1) / bwd_tc::kKT;
-    const int chunks = force > 0 ? std::min(force, tiles) : bwd_tc::plan_chunks(s.B, s.H, s.M, s.N, s.D);
-    const int per = (tiles + chunks - 1) / chunks;
-    return (tiles + per - 1) / per;
-}
-
 int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     int rc = make_plan(s, o, &bp->fwd);
     if (rc) return rc;
@@ -847,8 +840,9 @@ int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
     bp->tc = bp->fwd.path == FLAREPP_PATH_TCGEN05;
     const int force = o ? o->force_chunks : 0;
     if (bp->tc) {
-        bp->chunks = tc_bwd_chunks(s, force);
-        bp->chunk_len = 0;
+        // the latent-row passes split the tokens in chunks of a multiple of 64
+        bp->chunk_len = bwd_tc::plan_chunk_len(s.B, s.H, s.M, s.N, s.D, force);
+        bp->chunks = bwd_tc::chunks_of(s.N, bp->chunk_len);
     } else {
         int64_t chunks;
         if (force > 0) {
@@ -1048,7 +1042,7 @@ cudaError_t run_backward_tc(const Shape& s, const BwdPlan& bp, const BwdArgs& a,
     base.tok = pl.tok;
     base.scale_log2 = pl.scale_log2;
     base.scale = scale;
-    base.chunks = bp.chunks;
+    base.chunk_len = bp.chunk_len;
     auto latent_rows = [&](Operand A, Operand C, Operand Bc, Operand Ec, bool acc2, bool col_stats,
                            const float2* stats, int64_t stride) {
         bwd_tc::Launch L = base;
@@ -1476,7 +1470,7 @@ cudaError_t cp_stage(int stage, const Shape& s, const BwdPlan& bp, const CpBwdAr
     using bwd_tc::Operand;
     bwd_tc::Launch base{};
     base.B = s.B; base.H = s.H; base.N = s.N; base.M = s.M; base.D = s.D;
-    base.tok = pl.tok; base.scale_log2 = pl.scale_log2; base.scale = scale; base.chunks = bp.chunks;
+    base.tok = pl.tok; base.scale_log2 = pl.scale_log2; base.scale = scale; base.chunk_len = bp.chunk_len;
     const Operand q_lat = gated ? Operand{static_cast<const char*>(c.q_state) + o16, false, false}
                                 : Operand{a.q_fixed, false, true};
     const Operand z_lat{z16, false, false};

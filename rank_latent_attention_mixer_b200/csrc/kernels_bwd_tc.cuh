@@ -49,7 +49,8 @@ namespace bwd_tc {
 
 using tc::kQTile;
 
-constexpr int kKT = 32;        // column tile rows (one 32-column TMEM load per job)
+constexpr int kKT = 32;        // column tile rows of a job (one 32-column TMEM load per half)
+constexpr int kKTWide = 64;    // latent-row passes with one accumulator: 64-column jobs
 constexpr int kNST = 4;        // column stages
 
 // Tiles per row slot and per column stage, and row slots: the dual form holds
@@ -112,15 +113,15 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item) {
     return it;
 }
 
-template <int D, int NW, bool DUAL>
+template <int D, int NW, bool DUAL, int KT>
 struct Smem {
     using SH = Shape<DUAL>;
     static constexpr int kRowTile = kQTile * D * 2;
-    static constexpr int kColTile = kKT * D * 2;
+    static constexpr int kColTile = KT * D * 2;
     static constexpr int kRow = 0;                                      // [QS][NW][A, C (, C2)]
     static constexpr int kCol = kRow + SH::QS * NW * SH::RT * kRowTile;  // [NST][B, E (, E2)]
     static constexpr int kStats = kCol + kNST * SH::CT * kColTile;      // [NST][KT] float2
-    static constexpr int kBar = kStats + kNST * kKT * 8;
+    static constexpr int kBar = kStats + kNST * KT * 8;
     // row_full[QS], row_empty[QS], col_full[NST], col_empty[NST], sfull, sfree, pfull, pfree, drain [NW]
     static constexpr int kNumBars = 2 * SH::QS + 2 * kNST + 5 * NW;
     static constexpr int kMisc = kBar + kNumBars * 8;
@@ -130,18 +131,21 @@ struct Smem {
     static constexpr int kSmemLaunch = kLaunchBytes > 118784 ? kLaunchBytes : 118784;
 };
 
-template <int D, int NW, bool DUAL>
+// TMEM columns of the plan: S, dP (, dP2) of KT columns, acc1 (, acc2: ACC2)
+// of max(D, 32), P and dS as packed pairs of KT/2, per warpgroup.
+template <int D, int NW, bool DUAL, int KT, bool ACC2>
 struct Tmem {
     static constexpr int OS = D < 32 ? 32 : D;
     static constexpr int kS = 0;
-    static constexpr int kDP = NW * kKT;
-    static constexpr int kDP2 = 2 * NW * kKT;                  // dual only
-    static constexpr int kA1 = (DUAL ? 3 : 2) * NW * kKT;
-    static constexpr int kA2 = kA1 + NW * OS;
-    static constexpr int kP = kA2 + NW * OS;
-    static constexpr int kDS = kP + NW * (kKT / 2);
-    static constexpr int kTotal = kDS + NW * (kKT / 2);
+    static constexpr int kDP = NW * KT;
+    static constexpr int kDP2 = 2 * NW * KT;                   // dual only
+    static constexpr int kA1 = (DUAL ? 3 : 2) * NW * KT;
+    static constexpr int kA2 = kA1 + NW * OS;                  // ACC2 only
+    static constexpr int kP = kA2 + (ACC2 ? NW * OS : 0);
+    static constexpr int kDS = kP + NW * (KT / 2);
+    static constexpr int kTotal = kDS + NW * (KT / 2);
     static_assert(kTotal <= 512, "TMEM plan exceeds 512 columns");
+    static_assert(ACC2 || !DUAL, "the dual form accumulates two products");
 };
 
 // 16 consecutive TMEM columns of this thread's lane <- 16 registers.
@@ -161,16 +165,18 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-template <typename E, int D, int NW, bool DUAL>
+template <typename E, int D, int NW, bool DUAL, int KT, bool ACC2>
 __global__ void __launch_bounds__((NW + 1) * 128, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_c,
            const __grid_constant__ CUtensorMap map_c2, const __grid_constant__ CUtensorMap map_b,
            const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_e2, const Params p) {
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dims 16, 32, 64, 128");
-    using SM = Smem<D, NW, DUAL>;
-    using TM = Tmem<D, NW, DUAL>;
+    static_assert(KT == 32 || KT == 64, "jobs of one or two 32-column halves");
+    using SM = Smem<D, NW, DUAL, KT>;
+    using TM = Tmem<D, NW, DUAL, KT, ACC2>;
     using SH = Shape<DUAL>;
-    using LY = tc::Layout<D, NW, kKT>;
+    using LY = tc::Layout<D, NW, KT>;
+    constexpr int kHalves = KT / 32;
     constexpr int kQS = SH::QS;
     constexpr int kTmaWarp = 4 * NW;
     constexpr int kMmaWarp0 = 4 * NW + 1;
@@ -247,7 +253,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
             const bool col_stats = DUAL || p.stats_per_col;
             const uint32_t row_bytes = NW * ((p.c_same_a ? 1 : 2) + (DUAL ? 1 : 0)) * SM::kRowTile;
             const uint32_t col_bytes =
-                ((p.e_same_b ? 1 : 2) + (DUAL ? 1 : 0)) * SM::kColTile + (col_stats ? kKT * 8 : 0);
+                ((p.e_same_b ? 1 : 2) + (DUAL ? 1 : 0)) * SM::kColTile + (col_stats ? KT * 8 : 0);
             const float2* cstats = DUAL ? p.stats2 : p.stats;
             const int64_t cstride = DUAL ? p.stats2_stride : p.stats_stride;
             bool ok = true;
@@ -289,17 +295,17 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     uint8_t* cdst = smem + SM::kCol + st * SH::CT * SM::kColTile;
 #pragma unroll
                     for (int cb = 0; cb < LY::kBlocks; ++cb) {
-                        load(cdst + cb * LY::kKVBlockBytes, &map_b, &col_full[st], p.col_tok, cb, t * kKT, it.h,
+                        load(cdst + cb * LY::kKVBlockBytes, &map_b, &col_full[st], p.col_tok, cb, t * KT, it.h,
                              p.b_shared ? 0 : it.b);
                         if (!p.e_same_b)
                             load(cdst + SM::kColTile + cb * LY::kKVBlockBytes, &map_e, &col_full[st], p.col_tok, cb,
-                                 t * kKT, it.h, p.e_shared ? 0 : it.b);
+                                 t * KT, it.h, p.e_shared ? 0 : it.b);
                         if (DUAL)   // E2: the second output gradient's column tile (per batch)
                             load(cdst + 2 * SM::kColTile + cb * LY::kKVBlockBytes, &map_e2, &col_full[st], p.col_tok,
-                                 cb, t * kKT, it.h, it.b);
+                                 cb, t * KT, it.h, it.b);
                     }
                     if (col_stats)
-                        bulk_load(smem + SM::kStats + st * kKT * 8, cstats + it.bh * cstride + t * kKT, kKT * 8,
+                        bulk_load(smem + SM::kStats + st * KT * 8, cstats + it.bh * cstride + t * KT, KT * 8,
                                   &col_full[st]);
                     col_last[st] = (g / kNST) & 1;
                     ++g;
@@ -322,7 +328,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
         // ---------------------------------------------------------- MMA issuers
         if (lane == 0 && warp < kMmaWarp0 + NW) {
             const int w = warp - kMmaWarp0;
-            constexpr uint32_t idesc_s = tc::make_idesc(kQTile, kKT, false, tc::Elem<E>::kFmt);  // [128 x KT]
+            constexpr uint32_t idesc_s = tc::make_idesc(kQTile, KT, false, tc::Elem<E>::kFmt);  // [128 x KT]
             constexpr uint32_t idesc_a = tc::make_idesc(kQTile, D, true, tc::Elem<E>::kFmt);     // [128 x D], B MN-major
             // The job stream of this CTA: every column tile of every item, in order.
             struct Job {
@@ -372,13 +378,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad = tc::smem_desc(aaddr + LY::kstep(kk, LY::kQBlockBytes), 16, LY::kSbo, LY::kType);
                     const uint64_t bd = tc::smem_desc(baddr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
-                    tc::umma_f16(tmem + TM::kS + w * kKT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    tc::umma_f16(tmem + TM::kS + w * KT, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t cd = tc::smem_desc(caddr + LY::kstep(kk, LY::kQBlockBytes), 16, LY::kSbo, LY::kType);
                     const uint64_t ed = tc::smem_desc(eaddr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
-                    tc::umma_f16(tmem + TM::kDP + w * kKT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
+                    tc::umma_f16(tmem + TM::kDP + w * KT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 if constexpr (DUAL) {
                     const uint32_t c2addr = tc::smem_u32(rbase + 2 * SM::kRowTile);
@@ -389,7 +395,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                             tc::smem_desc(c2addr + LY::kstep(kk, LY::kQBlockBytes), 16, LY::kSbo, LY::kType);
                         const uint64_t ed =
                             tc::smem_desc(e2addr + LY::kstep(kk, LY::kKVBlockBytes), 16, LY::kSbo, LY::kType);
-                        tc::umma_f16(tmem + TM::kDP2 + w * kKT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
+                        tc::umma_f16(tmem + TM::kDP2 + w * KT, cd, ed, idesc_s, kk > 0 ? 1u : 0u);
                     }
                 }
                 tc::umma_commit(&sfull[w]);
@@ -409,20 +415,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                                                          : (p.e_same_b ? cbase : cbase + SM::kColTile));
                 const bool first = j.t == j.info.t_begin;
 #pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk) {
+                for (int kk = 0; kk < KT / 16; ++kk) {
                     // A = dS (or P) in TMEM: 16 columns of the tile = 8 packed TMEM columns per step;
                     // B = the column tile [KT x D], D contiguous: MN-major, 16 rows per step
                     const uint64_t bd = tc::smem_desc(baddr + kk * 16 * LY::kRowBytes, LY::kKVBlockBytes, LY::kSbo,
                                                       LY::kType);
-                    tc::umma_f16_tmem_a(tmem + TM::kA1 + w * TM::OS, tmem + TM::kDS + w * (kKT / 2) + kk * 8, bd,
+                    tc::umma_f16_tmem_a(tmem + TM::kA1 + w * TM::OS, tmem + TM::kDS + w * (KT / 2) + kk * 8, bd,
                                         idesc_a, (first && kk == 0) ? 0u : 1u);
                 }
-                if (p.has_acc2) {
+                if (ACC2 && p.has_acc2) {
 #pragma unroll
-                    for (int kk = 0; kk < kKT / 16; ++kk) {
+                    for (int kk = 0; kk < KT / 16; ++kk) {
                         const uint64_t ed = tc::smem_desc(eaddr + kk * 16 * LY::kRowBytes, LY::kKVBlockBytes,
                                                           LY::kSbo, LY::kType);
-                        tc::umma_f16_tmem_a(tmem + TM::kA2 + w * TM::OS, tmem + TM::kP + w * (kKT / 2) + kk * 8, ed,
+                        tc::umma_f16_tmem_a(tmem + TM::kA2 + w * TM::OS, tmem + TM::kP + w * (KT / 2) + kk * 8, ed,
                                             idesc_a, (first && kk == 0) ? 0u : 1u);
                     }
                 }
@@ -461,13 +467,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_base + TM::kS + wg * kKT;
-        const uint32_t tDP = tmem + lane_base + TM::kDP + wg * kKT;
-        const uint32_t tDP2 = tmem + lane_base + TM::kDP2 + wg * kKT;
+        const uint32_t tS = tmem + lane_base + TM::kS + wg * KT;
+        const uint32_t tDP = tmem + lane_base + TM::kDP + wg * KT;
+        const uint32_t tDP2 = tmem + lane_base + TM::kDP2 + wg * KT;
         const uint32_t tA1 = tmem + lane_base + TM::kA1 + wg * TM::OS;
         const uint32_t tA2 = tmem + lane_base + TM::kA2 + wg * TM::OS;
-        const uint32_t tP = tmem + lane_base + TM::kP + wg * (kKT / 2);
-        const uint32_t tDS = tmem + lane_base + TM::kDS + wg * (kKT / 2);
+        const uint32_t tP = tmem + lane_base + TM::kP + wg * (KT / 2);
+        const uint32_t tDS = tmem + lane_base + TM::kDS + wg * (KT / 2);
         const float sl2 = p.scale_log2;
         uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0, g = 0;
         bool ok = true;
@@ -485,7 +491,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 constexpr int CW = D < 32 ? D : 32;        // valid columns of a 32-column load
                 uint32_t a1[32], a2[32];
                 tc::tmem_ld32(tA1 + c0, a1);
-                if (p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
+                if (ACC2 && p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
                 tc::tmem_wait_ld();
                 if (!rvalid) continue;
                 if (p.epi == kEpiPartials) {
@@ -495,14 +501,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     for (int i = 0; i < CW / 4; ++i)
                         d1[i] = make_float4(__uint_as_float(a1[4 * i]), __uint_as_float(a1[4 * i + 1]),
                                             __uint_as_float(a1[4 * i + 2]), __uint_as_float(a1[4 * i + 3]));
-                    if (p.has_acc2) {
+                    if (ACC2 && p.has_acc2) {
                         float4* d2 = reinterpret_cast<float4*>(p.part2 + ridx * D + c0);
 #pragma unroll
                         for (int i = 0; i < CW / 4; ++i)
                             d2[i] = make_float4(__uint_as_float(a2[4 * i]), __uint_as_float(a2[4 * i + 1]),
                                                 __uint_as_float(a2[4 * i + 2]), __uint_as_float(a2[4 * i + 3]));
                     }
-                } else {
+                } else if constexpr (ACC2) {
                     const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
                     float v1[CW];
                     if (p.epi == kEpiTokDkDv) {
@@ -540,101 +546,110 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 if (!tc::mbar_wait(&sfull[wg], sfull_waits & 1, abort_flag)) { ok = false; break; }
                 ++sfull_waits;
                 tc::tc_fence_after();
-                uint32_t sr[32], dr[32], dr2[DUAL ? 32 : 1];
-                tc::tmem_ld32(tS, sr);
-                tc::tmem_ld32(tDP, dr);
-                if constexpr (DUAL) tc::tmem_ld32(tDP2, dr2);
+                uint32_t sr[kHalves][32], dr[kHalves][32], dr2[DUAL ? kHalves : 1][DUAL ? 32 : 1];
+#pragma unroll
+                for (int h = 0; h < kHalves; ++h) {
+                    tc::tmem_ld32(tS + 32 * h, sr[h]);
+                    tc::tmem_ld32(tDP + 32 * h, dr[h]);
+                    if constexpr (DUAL) tc::tmem_ld32(tDP2 + 32 * h, dr2[h]);
+                }
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sfree[wg]);
 
                 const int st = g % kNST;
-                const float2* cs = sstats + st * kKT;
                 if (DUAL || p.stats_per_col) {
                     // the stage's statistics: acquire the TMA writes (the phase has completed)
                     if (!tc::mbar_wait(&col_full[st], (g / kNST) & 1, abort_flag)) { ok = false; break; }
                 }
-                const int valid = p.col_count - t * kKT;     // columns of this tile that exist
-                uint32_t pk[16], dk[16];
-                if (__builtin_expect(valid >= kKT && warp_rows_valid, 1)) {
-                    // every row of the warp and every column of the tile exists (warp-uniform):
-                    // no masking, column pairs in packed fp32 arithmetic
-                    const float2 sl2v = make_float2(sl2, sl2);
-                    const float2 nlr = make_float2(-lse_r, -lse_r), ndr = make_float2(-del_r, -del_r);
-                    const float4* cs4 = reinterpret_cast<const float4*>(cs);
+#pragma unroll
+                for (int h = 0; h < kHalves; ++h) {
+                    const float2* cs = sstats + st * KT + 32 * h;
+                    const int valid = p.col_count - t * KT - 32 * h;     // columns of this half that exist
+                    uint32_t pk[16], dk[16];
+                    if (__builtin_expect(valid >= 32 && warp_rows_valid, 1)) {
+                        // every row of the warp and every column of the tile exists (warp-uniform):
+                        // no masking, column pairs in packed fp32 arithmetic
+                        const float2 sl2v = make_float2(sl2, sl2);
+                        const float2 nlr = make_float2(-lse_r, -lse_r), ndr = make_float2(-del_r, -del_r);
+                        const float4* cs4 = reinterpret_cast<const float4*>(cs);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float2 s2 = make_float2(__uint_as_float(sr[h][2 * j]), __uint_as_float(sr[h][2 * j + 1]));
+                            const float2 d2 = make_float2(__uint_as_float(dr[h][2 * j]), __uint_as_float(dr[h][2 * j + 1]));
+                            float2 pw, ds;
+                            if constexpr (DUAL) {
+                                const float4 sv = cs4[j];                    // (lse, Delta) of columns 2j, 2j+1
+                                const float2 xd = __ffma2_rn(s2, sl2v, nlr);
+                                const float2 xe = __ffma2_rn(s2, sl2v, make_float2(-sv.x, -sv.z));
+                                const float2 pd = make_float2(ex2_mufu(xd.x), ex2_mufu(xd.y));
+                                pw = make_float2(ex2_mufu(xe.x), ex2_mufu(xe.y));
+                                const float2 e2 = make_float2(__uint_as_float(dr2[h][2 * j]), __uint_as_float(dr2[h][2 * j + 1]));
+                                const float2 ge = __fmul2_rn(pw, __fadd2_rn(e2, make_float2(-sv.y, -sv.w)));
+                                ds = __ffma2_rn(pd, __fadd2_rn(d2, ndr), ge);
+                            } else {
+                                float2 nl = nlr, nd = ndr;
+                                if (p.stats_per_col) {
+                                    const float4 sv = cs4[j];
+                                    nl = make_float2(-sv.x, -sv.z);
+                                    nd = make_float2(-sv.y, -sv.w);
+                                }
+                                const float2 x = __ffma2_rn(s2, sl2v, nl);
+                                pw = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
+                                ds = __fmul2_rn(pw, __fadd2_rn(d2, nd));
+                            }
+                            pk[j] = pack2<E>(pw.x, pw.y);
+                            dk[j] = pack2<E>(ds.x, ds.y);
+                        }
+                    } else {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const float2 s2 = make_float2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
-                        const float2 d2 = make_float2(__uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1]));
-                        float2 pw, ds;
-                        if constexpr (DUAL) {
-                            const float4 sv = cs4[j];                    // (lse, Delta) of columns 2j, 2j+1
-                            const float2 xd = __ffma2_rn(s2, sl2v, nlr);
-                            const float2 xe = __ffma2_rn(s2, sl2v, make_float2(-sv.x, -sv.z));
-                            const float2 pd = make_float2(ex2_mufu(xd.x), ex2_mufu(xd.y));
-                            pw = make_float2(ex2_mufu(xe.x), ex2_mufu(xe.y));
-                            const float2 e2 = make_float2(__uint_as_float(dr2[2 * j]), __uint_as_float(dr2[2 * j + 1]));
-                            const float2 ge = __fmul2_rn(pw, __fadd2_rn(e2, make_float2(-sv.y, -sv.w)));
-                            ds = __ffma2_rn(pd, __fadd2_rn(d2, ndr), ge);
-                        } else {
-                            float2 nl = nlr, nd = ndr;
-                            if (p.stats_per_col) {
-                                const float4 sv = cs4[j];
-                                nl = make_float2(-sv.x, -sv.z);
-                                nd = make_float2(-sv.y, -sv.w);
-                            }
-                            const float2 x = __ffma2_rn(s2, sl2v, nl);
-                            pw = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
-                            ds = __fmul2_rn(pw, __fadd2_rn(d2, nd));
-                        }
-                        pk[j] = pack2<E>(pw.x, pw.y);
-                        dk[j] = pack2<E>(ds.x, ds.y);
-                    }
-                } else {
+                        float pv[2], dv[2];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float pv[2], dv[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int c = 2 * j + e;
-                        const bool on = rvalid && c < valid;
-                        const float sc = __uint_as_float(sr[c]);
-                        if constexpr (DUAL) {
-                            // Pd from the row statistics (first softmax), Pe from the column
-                            // statistics (second); dS = dSd + dSe, the weights stored are Pe
-                            const float2 sv = cs[c];
-                            const float pd = on ? ex2_mufu(fmaf(sc, sl2, -lse_r)) : 0.f;
-                            const float pe = on ? ex2_mufu(fmaf(sc, sl2, -sv.x)) : 0.f;
-                            pv[e] = pe;
-                            dv[e] = on ? fmaf(pd, __uint_as_float(dr[c]) - del_r, pe * (__uint_as_float(dr2[c]) - sv.y))
-                                       : 0.f;
-                        } else {
-                            float lse = lse_r, del = del_r;
-                            if (p.stats_per_col) {
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = 2 * j + e;
+                            const bool on = rvalid && c < valid;
+                            const float sc = __uint_as_float(sr[h][c]);
+                            if constexpr (DUAL) {
+                                // Pd from the row statistics (first softmax), Pe from the column
+                                // statistics (second); dS = dSd + dSe, the weights stored are Pe
                                 const float2 sv = cs[c];
-                                lse = sv.x;
-                                del = sv.y;
+                                const float pd = on ? ex2_mufu(fmaf(sc, sl2, -lse_r)) : 0.f;
+                                const float pe = on ? ex2_mufu(fmaf(sc, sl2, -sv.x)) : 0.f;
+                                pv[e] = pe;
+                                dv[e] = on ? fmaf(pd, __uint_as_float(dr[h][c]) - del_r, pe * (__uint_as_float(dr2[h][c]) - sv.y))
+                                           : 0.f;
+                            } else {
+                                float lse = lse_r, del = del_r;
+                                if (p.stats_per_col) {
+                                    const float2 sv = cs[c];
+                                    lse = sv.x;
+                                    del = sv.y;
+                                }
+                                const float x = fmaf(sc, sl2, -lse);
+                                const float pw = on ? ex2_mufu(x) : 0.f;
+                                pv[e] = pw;
+                                dv[e] = on ? pw * (__uint_as_float(dr[h][c]) - del) : 0.f;
                             }
-                            const float x = fmaf(sc, sl2, -lse);
-                            const float pw = on ? ex2_mufu(x) : 0.f;
-                            pv[e] = pw;
-                            dv[e] = on ? pw * (__uint_as_float(dr[c]) - del) : 0.f;
                         }
+                        pk[j] = pack2<E>(pv[0], pv[1]);
+                        dk[j] = pack2<E>(dv[0], dv[1]);
                     }
-                    pk[j] = pack2<E>(pv[0], pv[1]);
-                    dk[j] = pack2<E>(dv[0], dv[1]);
-                }
-                }
-                // the previous job's accumulating MMAs must be done before P and dS are overwritten
-                while (pfree_waits < jobs_done) {
-                    if (!tc::mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
-                    ++pfree_waits;
+                    }
+                    if (h == 0) {
+                        // the previous job's accumulating MMAs must be done before P and dS are overwritten
+                        while (pfree_waits < jobs_done) {
+                            if (!tc::mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                            ++pfree_waits;
+                        }
+                        if (!ok) break;
+                        tc::tc_fence_after();
+                    }
+                    tmem_st16(tP + 16 * h, pk);
+                    tmem_st16(tDS + 16 * h, dk);
                 }
                 if (!ok) break;
-                tc::tc_fence_after();
-                tmem_st16(tP, pk);
-                tmem_st16(tDS, dk);
                 if constexpr (DUAL) {
                     if (pend) {
                         epilogue(pend_it, pend_r, pend_rvalid);
@@ -713,7 +728,7 @@ struct Launch {
     int64_t stats_stride;
     float scale_log2, scale;
     int epi;
-    int chunks;                // latent rows: column chunks (0 = planned)
+    int chunk_len;             // latent rows: tokens per column chunk, a multiple of kKTWide (0 = planned)
     float *part1, *part2;
     void *out1, *out2;
 };
@@ -722,19 +737,27 @@ struct Launch {
 // one for D = 128.
 constexpr int nw_for(int D) { return D == 128 ? 1 : 2; }
 
-// Column chunks of a latent-row pass: the forward split pass's cost model
-// (waves x (fixed work + jobs per item)).
-inline int plan_chunks(int B, int H, int M, int N, int D) {
+// Tokens per column chunk of the latent-row passes: the forward split pass's
+// cost model (waves x (fixed work + jobs per item)) over 64-token tiles, or
+// `force` chunks.  A multiple of kKTWide, so that every latent-row pass,
+// whatever its job width, splits the tokens at the same places and writes
+// the same partial slots.
+inline int plan_chunk_len(int B, int H, int M, int N, int D, int force) {
     const int NW = nw_for(D);
     const int64_t units = (int64_t)B * H * ((M + NW * kQTile - 1) / (NW * kQTile));
-    const int64_t tiles = (N + kKT - 1) / kKT;
-    return (int)tc::choose_chunks(units, tiles, kNumSMs, 1);
+    const int64_t tiles = (N + kKTWide - 1) / kKTWide;
+    const int64_t chunks = force > 0 ? std::min<int64_t>(force, tiles) : tc::choose_chunks(units, tiles, kNumSMs, 1);
+    const int64_t per = (tiles + chunks - 1) / chunks;
+    return (int)(per * kKTWide);
 }
 
-template <typename E, int D, bool DUAL>
-int launch_bwd(const Launch& L, cudaStream_t st) {
+// Column chunks of a latent-row pass with `chunk_len` tokens per chunk.
+inline int chunks_of(int N, int chunk_len) { return (int)(((int64_t)N + chunk_len - 1) / chunk_len); }
+
+template <typename E, int D, bool DUAL, int KT, bool ACC2>
+int launch_bwd_kt(const Launch& L, cudaStream_t st) {
     constexpr int NW = nw_for(D);
-    using SM = Smem<D, NW, DUAL>;
+    using SM = Smem<D, NW, DUAL, KT>;
     static_assert(SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     const CUtensorMapDataType ty = tc::Elem<E>::kMapType;
     const tc::RowStrides lat = tc::contiguous_rows(L.M, L.H, D);
@@ -743,9 +766,9 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
         return tc::make_map(m, ty, o.ptr, L.M, L.H, o.shared ? 1 : L.B, D, lat, box);
     };
     CUtensorMap ma, mc, mb, me, mc2, me2;
-    if (!map(&ma, L.a, kQTile) || !map(&mc, L.c, kQTile) || !map(&mb, L.b, kKT) || !map(&me, L.e, kKT)) return 3;
+    if (!map(&ma, L.a, kQTile) || !map(&mc, L.c, kQTile) || !map(&mb, L.b, KT) || !map(&me, L.e, KT)) return 3;
     if (DUAL) {
-        if (!map(&mc2, L.c2, kQTile) || !map(&me2, L.e2, kKT)) return 3;
+        if (!map(&mc2, L.c2, kQTile) || !map(&me2, L.e2, KT)) return 3;
     } else {
         mc2 = mc;
         me2 = me;
@@ -754,11 +777,15 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
     p.B = L.B; p.H = L.H;
     p.row_count = L.rows_tok ? L.N : L.M;
     p.col_count = L.rows_tok ? L.M : L.N;
-    p.col_tiles = (p.col_count + kKT - 1) / kKT;
+    p.col_tiles = (p.col_count + KT - 1) / KT;
     p.row_groups = (p.row_count + NW * kQTile - 1) / (NW * kQTile);
-    int chunks = 1;
-    if (!L.rows_tok) chunks = L.chunks > 0 ? std::min(L.chunks, p.col_tiles) : plan_chunks(L.B, L.H, L.M, L.N, D);
-    p.chunk_tiles = (p.col_tiles + chunks - 1) / chunks;
+    if (L.rows_tok) {
+        p.chunk_tiles = p.col_tiles;          // an item holds all the latents
+    } else {
+        const int len = L.chunk_len > 0 ? L.chunk_len : plan_chunk_len(L.B, L.H, L.M, L.N, D, 0);
+        if (len % kKTWide != 0) return 2;
+        p.chunk_tiles = len / KT;
+    }
     p.chunks = (p.col_tiles + p.chunk_tiles - 1) / p.chunk_tiles;
     p.items = L.B * L.H * p.chunks * p.row_groups;
     p.row_tok = L.rows_tok ? 1 : 0;
@@ -779,7 +806,8 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
     p.part1 = L.part1; p.part2 = L.part2;
     p.out1 = L.out1; p.out2 = L.out2;
     p.tok_row = L.tok.row; p.tok_h = L.tok.h; p.tok_b = L.tok.b;
-    auto kern = bwd_kernel<E, D, NW, DUAL>;
+    if (!ACC2 && L.has_acc2) return 2;
+    auto kern = bwd_kernel<E, D, NW, DUAL, KT, ACC2>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = p.items < tc::sm_count() ? p.items : tc::sm_count();
@@ -787,6 +815,18 @@ int launch_bwd(const Launch& L, cudaStream_t st) {
                           p) == cudaSuccess
                ? 0
                : 3;
+}
+
+// Job width: a latent-row pass with one accumulator and row statistics
+// takes 64-column jobs with two warpgroups (TMEM: 2 x (64 S + 64 dP + 64
+// acc1 + 32 P + 32 dS) = 512; the per-job synchronisation is spread over
+// twice the columns); every other pass takes 32-column jobs.
+template <typename E, int D, bool DUAL>
+int launch_bwd(const Launch& L, cudaStream_t st) {
+    if constexpr (!DUAL && nw_for(D) == 2) {
+        if (!L.rows_tok && !L.has_acc2 && !L.stats_per_col) return launch_bwd_kt<E, D, false, kKTWide, false>(L, st);
+    }
+    return launch_bwd_kt<E, D, DUAL, kKT, true>(L, st);
 }
 
 template <typename E, int D>
@@ -807,10 +847,7 @@ int launch_bwd_d(const Launch& L, cudaStream_t st) {
 
 // Number of partial-sum slots a latent-row pass writes (its column chunks).
 inline int partial_chunks(const Launch& L) {
-    const int tiles = (L.N + kKT - 1) / kKT;
-    const int chunks = L.chunks > 0 ? std::min(L.chunks, tiles) : plan_chunks(L.B, L.H, L.M, L.N, L.D);
-    const int per = (tiles + chunks - 1) / chunks;
-    return (tiles + per - 1) / per;
+    return chunks_of(L.N, L.chunk_len > 0 ? L.chunk_len : plan_chunk_len(L.B, L.H, L.M, L.N, L.D, 0));
 }
 
 }  // namespace bwd_tc

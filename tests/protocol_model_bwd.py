@@ -26,6 +26,7 @@ from protocol_model import Bar
 
 QT = 128      # rows per warpgroup tile
 KT = 32       # columns per job
+KT_WIDE = 64  # columns per job of a latent pass with one accumulator and row statistics
 
 
 def decode_item(p, item):
@@ -276,14 +277,22 @@ def check(B, H, N, M, D, side, col_stats, grid=148, seed=0, force_chunks=0, dual
     BH = B * H
     NW = 1 if D == 128 else 2
     rows, cols = (M, N) if side == "latent" else (N, M)
-    col_tiles = -(-cols // KT)
     rg = -(-rows // (NW * QT))
     if side == "latent":
-        chunks = min(force_chunks or choose_chunks(BH * rg, col_tiles), col_tiles)
+        # tokens per chunk: a multiple of the wide tile, planned over wide tiles;
+        # a latent pass with row statistics and two warpgroups takes wide jobs
+        wide = -(-cols // KT_WIDE)
+        c = min(force_chunks or choose_chunks(BH * rg, wide), wide)
+        chunk_len = -(-wide // c) * KT_WIDE
+        kt = KT_WIDE if (NW == 2 and not col_stats and not dual) else KT
+        col_tiles = -(-cols // kt)
+        tpc = chunk_len // kt
+        chunks = -(-col_tiles // tpc)
+        assert chunks == -(-cols // chunk_len)          # the partial slots the reduction reads
     else:
+        col_tiles = -(-cols // KT)
+        tpc = col_tiles
         chunks = 1
-    tpc = -(-col_tiles // chunks)
-    chunks = -(-col_tiles // tpc)
     p = dict(NW=NW, NST=4, QS=1 if dual else 2, row_groups=rg, chunks=chunks, chunk_tiles=tpc,
              col_tiles=col_tiles, items=BH * chunks * rg, row_count=rows,
              row_tiles=3 if dual else 2, col_tiles_per_stage=3 if dual else 2,
