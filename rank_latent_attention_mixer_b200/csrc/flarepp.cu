@@ -856,9 +856,10 @@ int make_bwd_plan(const Shape& s, const flarepp_options_t* o, BwdPlan* bp) {
         bp->chunk_len = (int)std::min<int64_t>(tiles_per_chunk * tile, INT32_MAX);
         bp->chunks = (int)((s.N + (int64_t)bp->chunk_len - 1) / bp->chunk_len);
     }
-    const int64_t kt = bwd_tc::kKT;
+    // per-token statistics are read in 32-column tiles, per-latent ones in up to 64
+    const int64_t kt = bwd_tc::kKT, ktw = bwd_tc::kKTWide;
     bp->n_pad = (s.N + kt - 1) / kt * kt;
-    bp->m_pad = (s.M + kt - 1) / kt * kt;
+    bp->m_pad = (s.M + ktw - 1) / ktw * ktw;
     const size_t lat = (size_t)s.bh() * s.M, latd = lat * s.D, tok = (size_t)s.bh() * s.N;
     const size_t tc_on = bp->tc ? 1 : 0, simt_on = 1 - tc_on;
     size_t off = bp->fwd.total;

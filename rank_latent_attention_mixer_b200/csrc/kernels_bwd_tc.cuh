@@ -50,7 +50,13 @@ namespace bwd_tc {
 using tc::kQTile;
 
 constexpr int kKT = 32;        // column tile rows of a job (one 32-column TMEM load per half)
-constexpr int kKTWide = 64;    // latent-row passes with one accumulator: 64-column jobs
+constexpr int kKTWide = 64;    // passes with one accumulator: 64-column jobs
+
+// How a job's accumulating products map to TMEM accumulators: one product
+// (acc1 = dS B); two products into two accumulators (acc1 = dS B, acc2 =
+// P E); two products into acc1 (acc1 = scale dS B + P E, dS scaled before it
+// is packed: the synthesis token side, whose two products are one gradient).
+enum AccForm { kAccOne = 0, kAccTwo = 1, kAccMerged = 2 };
 constexpr int kNST = 4;        // column stages
 
 // Tiles per row slot and per column stage, and row slots: the dual form holds
@@ -131,21 +137,21 @@ struct Smem {
     static constexpr int kSmemLaunch = kLaunchBytes > 118784 ? kLaunchBytes : 118784;
 };
 
-// TMEM columns of the plan: S, dP (, dP2) of KT columns, acc1 (, acc2: ACC2)
-// of max(D, 32), P and dS as packed pairs of KT/2, per warpgroup.
-template <int D, int NW, bool DUAL, int KT, bool ACC2>
+// TMEM columns of the plan: S, dP (, dP2) of KT columns, acc1 (, acc2 with
+// kAccTwo) of max(D, 32), P and dS as packed pairs of KT/2, per warpgroup.
+template <int D, int NW, bool DUAL, int KT, int ACC>
 struct Tmem {
     static constexpr int OS = D < 32 ? 32 : D;
     static constexpr int kS = 0;
     static constexpr int kDP = NW * KT;
     static constexpr int kDP2 = 2 * NW * KT;                   // dual only
     static constexpr int kA1 = (DUAL ? 3 : 2) * NW * KT;
-    static constexpr int kA2 = kA1 + NW * OS;                  // ACC2 only
-    static constexpr int kP = kA2 + (ACC2 ? NW * OS : 0);
+    static constexpr int kA2 = kA1 + NW * OS;                  // kAccTwo only
+    static constexpr int kP = kA2 + (ACC == kAccTwo ? NW * OS : 0);
     static constexpr int kDS = kP + NW * (KT / 2);
     static constexpr int kTotal = kDS + NW * (KT / 2);
     static_assert(kTotal <= 512, "TMEM plan exceeds 512 columns");
-    static_assert(ACC2 || !DUAL, "the dual form accumulates two products");
+    static_assert(ACC == kAccTwo || !DUAL, "the dual form accumulates two gradients");
 };
 
 // 16 consecutive TMEM columns of this thread's lane <- 16 registers.
@@ -165,7 +171,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-template <typename E, int D, int NW, bool DUAL, int KT, bool ACC2>
+template <typename E, int D, int NW, bool DUAL, int KT, int ACC>
 __global__ void __launch_bounds__((NW + 1) * 128, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_c,
            const __grid_constant__ CUtensorMap map_c2, const __grid_constant__ CUtensorMap map_b,
@@ -173,7 +179,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dims 16, 32, 64, 128");
     static_assert(KT == 32 || KT == 64, "jobs of one or two 32-column halves");
     using SM = Smem<D, NW, DUAL, KT>;
-    using TM = Tmem<D, NW, DUAL, KT, ACC2>;
+    using TM = Tmem<D, NW, DUAL, KT, ACC>;
     using SH = Shape<DUAL>;
     using LY = tc::Layout<D, NW, KT>;
     constexpr int kHalves = KT / 32;
@@ -423,13 +429,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     tc::umma_f16_tmem_a(tmem + TM::kA1 + w * TM::OS, tmem + TM::kDS + w * (KT / 2) + kk * 8, bd,
                                         idesc_a, (first && kk == 0) ? 0u : 1u);
                 }
-                if (ACC2 && p.has_acc2) {
+                if (ACC == kAccMerged || (ACC == kAccTwo && p.has_acc2)) {
+                    // the second product: into acc2, or added to acc1 (kAccMerged)
+                    const uint32_t acc = ACC == kAccMerged ? TM::kA1 : TM::kA2;
 #pragma unroll
                     for (int kk = 0; kk < KT / 16; ++kk) {
                         const uint64_t ed = tc::smem_desc(eaddr + kk * 16 * LY::kRowBytes, LY::kKVBlockBytes,
                                                           LY::kSbo, LY::kType);
-                        tc::umma_f16_tmem_a(tmem + TM::kA2 + w * TM::OS, tmem + TM::kP + w * (KT / 2) + kk * 8, ed,
-                                            idesc_a, (first && kk == 0) ? 0u : 1u);
+                        tc::umma_f16_tmem_a(tmem + acc + w * TM::OS, tmem + TM::kP + w * (KT / 2) + kk * 8, ed,
+                                            idesc_a, (ACC == kAccTwo && first && kk == 0) ? 0u : 1u);
                     }
                 }
                 tc::umma_commit(&pfree[w]);
@@ -491,7 +499,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 constexpr int CW = D < 32 ? D : 32;        // valid columns of a 32-column load
                 uint32_t a1[32], a2[32];
                 tc::tmem_ld32(tA1 + c0, a1);
-                if (ACC2 && p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
+                if (ACC == kAccTwo && p.has_acc2) tc::tmem_ld32(tA2 + c0, a2);
                 tc::tmem_wait_ld();
                 if (!rvalid) continue;
                 if (p.epi == kEpiPartials) {
@@ -501,14 +509,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                     for (int i = 0; i < CW / 4; ++i)
                         d1[i] = make_float4(__uint_as_float(a1[4 * i]), __uint_as_float(a1[4 * i + 1]),
                                             __uint_as_float(a1[4 * i + 2]), __uint_as_float(a1[4 * i + 3]));
-                    if (ACC2 && p.has_acc2) {
+                    if (ACC == kAccTwo && p.has_acc2) {
                         float4* d2 = reinterpret_cast<float4*>(p.part2 + ridx * D + c0);
 #pragma unroll
                         for (int i = 0; i < CW / 4; ++i)
                             d2[i] = make_float4(__uint_as_float(a2[4 * i]), __uint_as_float(a2[4 * i + 1]),
                                                 __uint_as_float(a2[4 * i + 2]), __uint_as_float(a2[4 * i + 3]));
                     }
-                } else if constexpr (ACC2) {
+                } else if constexpr (ACC != kAccOne) {
                     const int64_t off = (int64_t)it.b * p.tok_b + (int64_t)it.h * p.tok_h + (int64_t)r * p.tok_row + c0;
                     float v1[CW];
                     if (p.epi == kEpiTokDkDv) {
@@ -518,6 +526,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
 #pragma unroll
                         for (int i = 0; i < CW; ++i) v2[i] = __uint_as_float(a2[i]);
                         store_row<E, CW>(static_cast<E*>(p.out2) + off, v2);
+                    } else if constexpr (ACC == kAccMerged) {
+#pragma unroll
+                        for (int i = 0; i < CW; ++i) v1[i] = __uint_as_float(a1[i]);      // scale dS B + P E
                     } else {
 #pragma unroll
                         for (int i = 0; i < CW; ++i)
@@ -598,6 +609,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                                 const float2 x = __ffma2_rn(s2, sl2v, nl);
                                 pw = make_float2(ex2_mufu(x.x), ex2_mufu(x.y));
                                 ds = __fmul2_rn(pw, __fadd2_rn(d2, nd));
+                                if constexpr (ACC == kAccMerged) ds = __fmul2_rn(ds, make_float2(p.scale, p.scale));
                             }
                             pk[j] = pack2<E>(pw.x, pw.y);
                             dk[j] = pack2<E>(ds.x, ds.y);
@@ -631,6 +643,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                                 const float pw = on ? ex2_mufu(x) : 0.f;
                                 pv[e] = pw;
                                 dv[e] = on ? pw * (__uint_as_float(dr[h][c]) - del) : 0.f;
+                                if constexpr (ACC == kAccMerged) dv[e] *= p.scale;
                             }
                         }
                         pk[j] = pack2<E>(pv[0], pv[1]);
@@ -754,7 +767,7 @@ inline int plan_chunk_len(int B, int H, int M, int N, int D, int force) {
 // Column chunks of a latent-row pass with `chunk_len` tokens per chunk.
 inline int chunks_of(int N, int chunk_len) { return (int)(((int64_t)N + chunk_len - 1) / chunk_len); }
 
-template <typename E, int D, bool DUAL, int KT, bool ACC2>
+template <typename E, int D, bool DUAL, int KT, int ACC>
 int launch_bwd_kt(const Launch& L, cudaStream_t st) {
     constexpr int NW = nw_for(D);
     using SM = Smem<D, NW, DUAL, KT>;
@@ -806,8 +819,9 @@ int launch_bwd_kt(const Launch& L, cudaStream_t st) {
     p.part1 = L.part1; p.part2 = L.part2;
     p.out1 = L.out1; p.out2 = L.out2;
     p.tok_row = L.tok.row; p.tok_h = L.tok.h; p.tok_b = L.tok.b;
-    if (!ACC2 && L.has_acc2) return 2;
-    auto kern = bwd_kernel<E, D, NW, DUAL, KT, ACC2>;
+    if (ACC == kAccOne && L.has_acc2) return 2;
+    if (ACC == kAccMerged && (!L.has_acc2 || L.epi != kEpiTokDk0)) return 2;
+    auto kern = bwd_kernel<E, D, NW, DUAL, KT, ACC>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = p.items < tc::sm_count() ? p.items : tc::sm_count();
@@ -817,16 +831,21 @@ int launch_bwd_kt(const Launch& L, cudaStream_t st) {
                : 3;
 }
 
-// Job width: a latent-row pass with one accumulator and row statistics
-// takes 64-column jobs with two warpgroups (TMEM: 2 x (64 S + 64 dP + 64
-// acc1 + 32 P + 32 dS) = 512; the per-job synchronisation is spread over
-// twice the columns); every other pass takes 32-column jobs.
+// Job width: with two warpgroups, a pass with one accumulator takes
+// 64-column jobs (TMEM: 2 x (64 S + 64 dP + 64 acc1 + 32 P + 32 dS) = 512;
+// the per-job synchronisation is spread over twice the columns): the latent
+// sides of the encode and the synthesis (one product, row statistics) and the
+// synthesis token side (two products merged into acc1).  The decode's latent
+// side and the fused token side keep two accumulators and 32-column jobs.
 template <typename E, int D, bool DUAL>
 int launch_bwd(const Launch& L, cudaStream_t st) {
     if constexpr (!DUAL && nw_for(D) == 2) {
-        if (!L.rows_tok && !L.has_acc2 && !L.stats_per_col) return launch_bwd_kt<E, D, false, kKTWide, false>(L, st);
+        if (!L.rows_tok && !L.has_acc2 && !L.stats_per_col)
+            return launch_bwd_kt<E, D, false, kKTWide, kAccOne>(L, st);
+        if (L.rows_tok && L.has_acc2 && L.epi == kEpiTokDk0)
+            return launch_bwd_kt<E, D, false, kKTWide, kAccMerged>(L, st);
     }
-    return launch_bwd_kt<E, D, DUAL, kKT, true>(L, st);
+    return launch_bwd_kt<E, D, DUAL, kKT, kAccTwo>(L, st);
 }
 
 template <typename E, int D>

@@ -290,7 +290,9 @@ def check(B, H, N, M, D, side, col_stats, grid=148, seed=0, force_chunks=0, dual
         chunks = -(-col_tiles // tpc)
         assert chunks == -(-cols // chunk_len)          # the partial slots the reduction reads
     else:
-        col_tiles = -(-cols // KT)
+        # the synthesis token side (one accumulator after merging) takes wide jobs
+        kt = KT_WIDE if (NW == 2 and not dual) else KT
+        col_tiles = -(-cols // kt)
         tpc = col_tiles
         chunks = 1
     p = dict(NW=NW, NST=4, QS=1 if dual else 2, row_groups=rg, chunks=chunks, chunk_tiles=tpc,
