@@ -864,10 +864,5 @@ int launch_bwd_d(const Launch& L, cudaStream_t st) {
     }
 }
 
-// Number of partial-sum slots a latent-row pass writes (its column chunks).
-inline int partial_chunks(const Launch& L) {
-    return chunks_of(L.N, L.chunk_len > 0 ? L.chunk_len : plan_chunk_len(L.B, L.H, L.M, L.N, L.D, 0));
-}
-
 }  // namespace bwd_tc
 }  // namespace flarepp
