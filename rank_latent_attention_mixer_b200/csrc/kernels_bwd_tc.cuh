@@ -567,7 +567,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sfree[wg]);
+                tc::mbar_arrive_if(&sfree[wg], lane == 0);
 
                 const int st = g % kNST;
                 if (DUAL || p.stats_per_col) {
@@ -672,7 +672,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&pfull[wg]);
+                tc::mbar_arrive_if(&pfull[wg], lane == 0);
                 ++jobs_done;
             }
             if (!ok) break;

@@ -97,6 +97,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive on `bar` from the threads where `pred` holds, without a branch.
+__device__ __forceinline__ void mbar_arrive_if(uint64_t* bar, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}"
+                 ::"r"(smem_u32(bar)), "r"((uint32_t)pred) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -805,7 +811,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sfree[wg]);
+                mbar_arrive_if(&sfree[wg], lane == 0);
 
                 const int valid = p.kv_rows - t * KT;             // key/value rows of this tile that exist
                 if (__builtin_expect(valid < KT, 0)) {            // ragged last tile only (warp-uniform)
@@ -891,7 +897,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pfull[wg]);
+                mbar_arrive_if(&pfull[wg], lane == 0);
                 ++jobs_done;
                 ++njobs;
             }
