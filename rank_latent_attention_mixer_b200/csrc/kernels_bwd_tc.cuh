@@ -37,7 +37,12 @@
 //                     next job are issued before the accumulating MMAs of the
 //                     current one, so the tensor core runs ahead of the softmax
 // TMEM per warpgroup: S and dP (KT columns each), acc1 and acc2 (max(D, 32)
-// each), P and dS as packed 16-bit pairs (KT/2 each).
+// each), P and dS as packed 16-bit pairs (KT/2 each).  A job is KT = 32
+// columns, or 64 where the job's products need one accumulator (AccForm):
+// the latent sides of the encode and the synthesis (dq only), and the
+// synthesis token side, whose two products are one gradient (dS is scaled
+// before it is packed and both products add into acc1).  The dual launch
+// defers each item's epilogue into the next item's first job.
 // Every mbarrier wait is bounded as in the forward kernel (timeout recorded in
 // the device status word, CTA-wide abort, bounded drain, TMEM freed).
 #pragma once
