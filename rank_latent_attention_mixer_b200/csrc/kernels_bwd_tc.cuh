@@ -466,10 +466,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CU
                 ok = issue_acc(aj);
                 next_job(aj);
             }
-            // drain: every issued MMA completes before TMEM is released
+            // drain: every issued MMA completes before TMEM is released; if that
+            // runs out, report it (the outputs are then undefined)
             tc::umma_commit(&drain[w]);
             const unsigned long long t0 = tc::globaltimer_ns();
-            while (!tc::mbar_try_wait(&drain[w], 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+            bool drained = false;
+            while (!(drained = tc::mbar_try_wait(&drain[w], 0)) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+            }
+            if (!drained) {
+                *abort_flag = 1;
+                record_status(tc::kStatusTimeout);
             }
         }
       }

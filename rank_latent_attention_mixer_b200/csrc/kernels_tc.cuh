@@ -123,13 +123,17 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 // Waits until the phase with the given parity has completed.  Returns false
 // if the CTA's abort flag is up or the wait ran past kWaitLimitNs (then it
-// raises the flag and records the timeout).
+// raises the flag and records the timeout).  After a few unsuccessful polls
+// the waiting thread sleeps between polls, so that a warp waiting for a long
+// time (the producer and MMA-issuing warps) does not take issue slots from
+// the softmax warps of its SM sub-partition.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (it > 2) __nanosleep(it > 64 ? 64 : 16);
         if ((it & 31u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns || it > (1u << 30)) {
@@ -299,6 +303,7 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 
+
 // ------------------------------------------------------------------ kernel parameters
 
 // Element strides of a tensor of D-element rows: between consecutive rows,
@@ -347,10 +352,10 @@ struct Item {
     int part;             // split mode: partial index of warpgroup 0 (interleaved: NW c, else c)
 };
 
-template <int NW>
+template <int NW, int MODE>
 __device__ __forceinline__ Item decode_item(const Params& p, int item) {
     Item it;
-    if (p.mode == kSplit) {
+    if constexpr (MODE == kSplit) {
         const int g = item % p.row_groups;
         const int rest = item / p.row_groups;
         const int c = rest % p.chunks;
@@ -418,7 +423,7 @@ struct Layout {
 
 // ------------------------------------------------------------------ the kernel
 
-template <typename E, int D, int NW, int KT, int NST, int QS>
+template <typename E, int D, int NW, int KT, int NST, int QS, int MODE>
 __global__ void __launch_bounds__(Regs<NW>::kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const Params p) {
@@ -502,7 +507,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             const uint32_t q_bytes = q_tiles * SM::kQTileBytes;
             bool ok = true;
             for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-                const Item it = decode_item<NW>(p, item);
+                const Item it = decode_item<NW, MODE>(p, item);
                 const int slot = q_load % QS;
                 ok = mbar_wait(&q_empty[slot], ((q_load / QS) & 1) ^ 1, abort_flag);
                 if (!ok) break;
@@ -513,7 +518,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
 #pragma unroll
                     for (int cb = 0; cb < LY::kBlocks; ++cb) {
                         uint8_t* dst = qdst + qt * SM::kQTileBytes + cb * LY::kQBlockBytes;
-                        if (p.mode == kDecode && p.tok_heads_inner)  // token queries, [B,N,H,D]
+                        if (MODE == kDecode && p.tok_heads_inner)  // token queries, [B,N,H,D]
                             tma_load_4d(dst, &map_q, &q_full[slot], cb * 64, it.h, qrow, it.qb);
                         else
                             tma_load_4d(dst, &map_q, &q_full[slot], cb * 64, qrow, it.h, it.qb);
@@ -537,7 +542,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     if (!ok) break;
                     mbar_expect_tx(&kv_full[st], kv_bytes);
                     uint8_t* kdst = smem + SM::kKV + st * 2 * SM::kKVTileBytes;
-                    const bool hi = p.mode == kSplit && p.tok_heads_inner;   // token keys/values, [B,N,H,D]
+                    const bool hi = MODE == kSplit && p.tok_heads_inner;   // token keys/values, [B,N,H,D]
 #pragma unroll
                     for (int cb = 0; cb < LY::kBlocks; ++cb) {
                         tma_load_4d(kdst + cb * LY::kKVBlockBytes, &map_k, &kv_full[st], cb * 64,
@@ -590,7 +595,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             // counted in the right phase); only the score cursor does that.
             auto settle = [&](Cursor& c, bool score_cursor) {
                 while (c.item < p.items) {
-                    c.info = decode_item<NW>(p, c.item);
+                    c.info = decode_item<NW, MODE>(p, c.item);
                     c.t = c.info.t_begin + tfirst;
                     c.njobs = 0;
                     if (c.t < c.info.t_end) {
@@ -700,10 +705,16 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 ok = issue_pv(pc);
                 next(pc, false);
             }
-            // drain: wait until every issued MMA has completed before TMEM is released
+            // drain: wait until every issued MMA has completed before TMEM is
+            // released; if that runs out, report it (the outputs are then undefined)
             umma_commit(&drain[w]);
             const unsigned long long t0 = globaltimer_ns();
-            while (!mbar_try_wait(&drain[w], 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            bool drained = false;
+            while (!(drained = mbar_try_wait(&drain[w], 0)) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+            if (!drained) {
+                *abort_flag = 1;
+                record_status(kStatusTimeout);
             }
         }
       }
@@ -725,7 +736,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         // Item outputs from this thread's O row (o == nullptr: the warpgroup had no
         // job in the item).  With D = 16 only the first 16 of 32 loaded columns are O.
         auto write_outputs = [&](const Item& it, int njobs, float m, float l, const uint32_t (*o)[32]) {
-            if (p.mode == kSplit) {
+            if constexpr (MODE == kSplit) {
                 const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
                 const int part = p.interleave ? it.part + wg : it.part;
                 if (r < p.M) {
@@ -790,15 +801,19 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             tmem_wait_ld();
             write_outputs(it, njobs, m, l, o);
         };
-        // The epilogue of an item is deferred into the next item's first job:
-        // its last value MMA finishes while the next exponentials are computed,
-        // and its O row is read just before the next value MMA overwrites it.
+        // Decode: the epilogue of an item (a few jobs long) is deferred into the
+        // next item's first job, so its last value MMA finishes while the next
+        // exponentials are computed and its O row is read just before the next
+        // value MMA overwrites it.  Split passes (items of hundreds of jobs):
+        // the epilogue runs at the end of the item, which keeps the job loop
+        // free of the pending item's state.
+        constexpr bool kDefer = MODE == kDecode;
         bool pend = false;
         Item pend_it{};
         int pend_jobs = 0;
         float pend_m = 0.f, pend_l = 0.f;
         for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-            const Item it = decode_item<NW>(p, item);
+            const Item it = decode_item<NW, MODE>(p, item);
             float m_run = -INFINITY, l_run = 0.f;
             int njobs = 0;
             for (int t = it.t_begin + tfirst; t < it.t_end; t += tstep) {
@@ -821,7 +836,9 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         for (int j = 0; j < 32; ++j)
                             if (c * 32 + j >= valid) sr[c][j] = __float_as_uint(-INFINITY);
                 }
-                // row max: one chain of 3-input maxima per 32-column chunk (short dependency chains)
+                // row max: one chain of 3-input maxima per 32-column chunk (a
+                // tree of maxima measured slower here: 1.47 against 1.39 ms per
+                // split launch at the 1M-token workload)
                 float mc[LY::kChunks];
 #pragma unroll
                 for (int c = 0; c < LY::kChunks; ++c) {
@@ -877,10 +894,12 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
                 // Rare work on O, after P is out of the registers and before the
                 // value MMA of this job adds to O: the previous item's O row (first
-                // job of an item), or the O rescale of a grown running max.
-                if (__builtin_expect(pend, 0)) {
-                    flush(pend_it, pend_jobs, pend_m, pend_l);
-                    pend = false;
+                // job of a decode item), or the O rescale of a grown running max.
+                if constexpr (kDefer) {
+                    if (__builtin_expect(pend, 0)) {
+                        flush(pend_it, pend_jobs, pend_m, pend_l);
+                        pend = false;
+                    }
                 }
                 if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0)) {
                     const float f = njobs > 0 ? factor : 1.f;
@@ -903,18 +922,26 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             }
             if (!ok) break;
 
-            // ---------------- end of the item: defer its epilogue
-            if (njobs > 0) {
+            // ---------------- end of the item: its epilogue (deferred in the decode)
+            if (njobs == 0) {
+                write_outputs(it, 0, m_run, l_run, nullptr);
+            } else if constexpr (kDefer) {
                 pend = true;
                 pend_it = it;
                 pend_jobs = njobs;
                 pend_m = m_run;
                 pend_l = l_run;
             } else {
-                write_outputs(it, 0, m_run, l_run, nullptr);
+                while (pfree_waits < jobs_done) {
+                    if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
+                    ++pfree_waits;
+                }
+                if (!ok) break;
+                tc_fence_after();
+                flush(it, njobs, m_run, l_run);
             }
         }
-        if (ok && pend) {
+        if (kDefer && ok && pend) {
             while (pfree_waits < jobs_done) {
                 if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
                 ++pfree_waits;
@@ -1099,7 +1126,7 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
                 cudaStream_t st) {
     using C = Config<D, NW, KT, DECODE>;
     if (prm.interleave && C::NST % C::NW != 0) return 2;      // one stage ring per warpgroup needs NW | NST
-    auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS>;
+    auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS, DECODE ? kDecode : kSplit>;
     static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
         return 3;
@@ -1110,13 +1137,13 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
                : 3;
 }
 
-template <typename E, int NW, int KT>
+template <typename E, int NW, int KT, bool DECODE>
 inline int launch_attn_d(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const Params& prm, cudaStream_t st) {
     switch (D) {
-        case 16: return launch_attn<E, 16, NW, KT>(mq, mk, mv, prm, st);
-        case 32: return launch_attn<E, 32, NW, KT>(mq, mk, mv, prm, st);
-        case 64: return launch_attn<E, 64, NW, KT>(mq, mk, mv, prm, st);
+        case 16: return launch_attn<E, 16, NW, KT, DECODE>(mq, mk, mv, prm, st);
+        case 32: return launch_attn<E, 32, NW, KT, DECODE>(mq, mk, mv, prm, st);
+        case 64: return launch_attn<E, 64, NW, KT, DECODE>(mq, mk, mv, prm, st);
         default: return 2;
     }
 }
@@ -1125,14 +1152,14 @@ template <typename E>
 inline int launch_split(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const Params& prm, cudaStream_t st) {
     if (D == 128) return launch_attn<E, 128, 2, 64>(mq, mk, mv, prm, st);
-    return launch_attn_d<E, kSplitNW, kSplitKT>(D, mq, mk, mv, prm, st);
+    return launch_attn_d<E, kSplitNW, kSplitKT, false>(D, mq, mk, mv, prm, st);
 }
 
 template <typename E>
 inline int launch_decode(int D, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const Params& prm, cudaStream_t st) {
     if (D == 128) return launch_attn<E, 128, 2, 64, true>(mq, mk, mv, prm, st);
-    return launch_attn_d<E, kDecodeNW, kDecodeKT>(D, mq, mk, mv, prm, st);
+    return launch_attn_d<E, kDecodeNW, kDecodeKT, true>(D, mq, mk, mv, prm, st);
 }
 
 template <typename E, int D>
