@@ -41,7 +41,8 @@ def _stale() -> bool:
 # split is sized for exactly 65536 / threads registers per thread at launch
 # (rounded down to a multiple of 8); a smaller launch allocation would leave
 # the growing warpgroups waiting, so the build refuses any other count.  The
-# kernel's template arguments are <D, NW, KT, NST, QS>, threads = (NW+1)*128.
+# kernel's template arguments are <D, NW, KT, NST, QS, MODE, CS>, threads =
+# (NW*CS+1)*128.
 
 
 # The backward kernel bwd_kernel<E, D, NW, DUAL> splits its registers the same
@@ -55,11 +56,14 @@ def expected_launch_regs(kernel_name: str):
             raise RuntimeError(f"cannot read the warpgroup count from {kernel_name}")
         nw = int(m.group(2))
         return (65536 // ((nw + 1) * 128)) // 8 * 8 if nw == 2 else None
-    m = re.search(r"attn_kernelI\d+\w+?Li(\d+)ELi(\d+)ELi(\d+)E", kernel_name)
+    # attn_kernel<E, D, NW, KT, NST, QS, MODE, CS>: NW row tiles x CS column
+    # shares softmax warpgroups and one producer warpgroup
+    m = re.search(r"attn_kernelI\d+\w+?((?:Li\d+E){7})", kernel_name)
     if not m:
         raise RuntimeError(f"cannot read the warpgroup count from {kernel_name}")
-    nw = int(m.group(2))
-    return (65536 // ((nw + 1) * 128)) // 8 * 8
+    args = [int(x) for x in re.findall(r"Li(\d+)E", m.group(1))]
+    nw, cs = args[1], args[6]
+    return (65536 // ((nw * cs + 1) * 128)) // 8 * 8
 
 
 def check_registers(ptxas_log: str) -> None:

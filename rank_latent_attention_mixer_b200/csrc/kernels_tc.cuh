@@ -67,14 +67,17 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kStatusTimeout = 5;    // FLAREPP_ERR_TIMEOUT
 constexpr int kProducerRegs = 56;    // producer warpgroup after setmaxnreg.dec
 
-// Threads, launch registers and the softmax warpgroups' register share of a
-// configuration with NW softmax warpgroups.
+// Threads, launch registers and the register split of a configuration with NW
+// softmax warpgroups and one producer warpgroup: the producer gives back down
+// to kProducer and the softmax warpgroups take the rest (a producer share of
+// 32 with four softmax warpgroups measured slower: its code spills).
 template <int NW>
 struct Regs {
     static constexpr int kThreads = (NW + 1) * 128;
-    static constexpr int kLaunch = (65536 / kThreads) / 8 * 8;           // 168 (NW=2), 128 (NW=3)
-    static constexpr int kSoftmax = ((kThreads * kLaunch - 128 * kProducerRegs) / (NW * 128)) / 8 * 8;
-    static_assert(NW * 128 * kSoftmax + 128 * kProducerRegs <= kThreads * kLaunch,
+    static constexpr int kLaunch = (65536 / kThreads) / 8 * 8;           // 168 (NW=2), 128 (NW=3), 96 (NW=4)
+    static constexpr int kProducer = kProducerRegs;
+    static constexpr int kSoftmax = ((kThreads * kLaunch - 128 * kProducer) / (NW * 128)) / 8 * 8;
+    static_assert(NW * 128 * kSoftmax + 128 * kProducer <= kThreads * kLaunch,
                   "register split exceeds the launch allocation");
 };
 
@@ -381,17 +384,22 @@ __device__ __forceinline__ Item decode_item(const Params& p, int item) {
 }
 
 // Shared-memory plan: QS query slots of NW [128 x D] tiles, NST stages of a
-// [KT x D] key tile and value tile, then the barriers.
-template <int D, int NW, int KT, int NST, int QS>
+// [KT x D] key tile and value tile, then the barriers and, with the score
+// columns split between CS warps per row (CS = 2), the exchange area of their
+// half-row values: [NW row tiles][4 lane quarters][2 phases][CS][32 lanes] fp32.
+template <int D, int NW, int KT, int NST, int QS, int CS = 1>
 struct Smem {
     static constexpr int kQTileBytes = kQTile * D * 2;
     static constexpr int kKVTileBytes = KT * D * 2;
     static constexpr int kQ = 0;
     static constexpr int kKV = kQ + QS * NW * kQTileBytes;
     static constexpr int kBar = kKV + NST * 2 * kKVTileBytes;
-    // kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull, sfree, pfull, pfree, drain [NW each]
-    static constexpr int kNumBars = 2 * NST + 2 * QS + 5 * NW;
-    static constexpr int kMisc = kBar + kNumBars * 8;               // tmem base (u32), abort flag (int)
+    // kv_full[NST], kv_empty[NST], q_full[QS], q_empty[QS], sfull, sfree, pfull, pfree, drain [NW each],
+    // with CS = 2 one exchange barrier per (row tile, lane quarter) [4 NW]
+    static constexpr int kNumBars = 2 * NST + 2 * QS + 5 * NW + (CS > 1 ? 4 * NW : 0);
+    static constexpr int kX = (kBar + kNumBars * 8 + 15) / 16 * 16;
+    static constexpr int kXBytes = CS > 1 ? NW * 4 * 2 * CS * 32 * 4 : 0;
+    static constexpr int kMisc = kX + kXBytes;                      // tmem base (u32), abort flag (int)
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kLaunchBytes = kBytes + 1024;              // + alignment slack
 };
@@ -423,23 +431,25 @@ struct Layout {
 
 // ------------------------------------------------------------------ the kernel
 
-template <typename E, int D, int NW, int KT, int NST, int QS, int MODE>
-__global__ void __launch_bounds__(Regs<NW>::kThreads, 1)
+template <typename E, int D, int NW, int KT, int NST, int QS, int MODE, int CS>
+__global__ void __launch_bounds__(Regs<NW * CS>::kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const Params p) {
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "tcgen05 path covers D in {16, 32, 64, 128}");
     static_assert(KT == 64 || KT == 128, "key/value tiles of 64 or 128 rows");
     static_assert(NW >= 1 && NW <= 3, "the producer warpgroup holds one TMA warp and NW MMA warps");
     static_assert(NST >= 3, "at least three key/value stages");
+    static_assert(CS == 1 || (CS == 2 && KT == 128), "score columns are split between two warps per row only in 128-column jobs");
     // Interleaved mode (launch_attn refuses it unless NW divides NST): warpgroup w owns stages [w R, w R + R) and consumes them in
     // order, so no consumer can wait on a stage two fills ahead (a parity wait
     // cannot tell phase k+1 from phase k-1).  Shared mode: one ring of NST stages
     // that every warpgroup consumes in order.
     constexpr int R = NST / NW;
-    using SM = Smem<D, NW, KT, NST, QS>;
+    using SM = Smem<D, NW, KT, NST, QS, CS>;
     using LY = Layout<D, NW, KT>;
-    constexpr int kTmaWarp = 4 * NW;
-    constexpr int kMmaWarp0 = 4 * NW + 1;
+    constexpr int kSoftmaxWarps = 4 * NW * CS;
+    constexpr int kTmaWarp = kSoftmaxWarps;
+    constexpr int kMmaWarp0 = kSoftmaxWarps + 1;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -453,6 +463,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     uint64_t* pfull = sfree + NW;
     uint64_t* pfree = pfull + NW;
     uint64_t* drain = pfree + NW;
+    uint64_t* xbar = drain + NW;                 // CS = 2: [NW][4]
+    float* xval = reinterpret_cast<float*>(smem + SM::kX);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::kMisc + 4);
 
@@ -464,13 +476,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         // a query slot by every warpgroup
         for (int i = 0; i < NST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], p.interleave ? 1 : NW); }
         for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], NW); }
+        // the softmax side of row tile w arrives once per warp (lane 0): 4 CS warps
         for (int w = 0; w < NW; ++w) {
             mbar_init(&sfull[w], 1);
-            mbar_init(&sfree[w], 4);
-            mbar_init(&pfull[w], 4);
+            mbar_init(&sfree[w], 4 * CS);
+            mbar_init(&pfull[w], 4 * CS);
             mbar_init(&pfree[w], 1);
             mbar_init(&drain[w], 1);
         }
+        // a column-split exchange completes when every lane of both warps has arrived
+        if (CS > 1)
+            for (int i = 0; i < 4 * NW; ++i) mbar_init(&xbar[i], 32 * CS);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -494,8 +510,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     pdl_wait();
     pdl_launch_dependents();
 
-    if (warp >= 4 * NW) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp >= kSoftmaxWarps) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Regs<NW * CS>::kProducer));
       if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
@@ -719,86 +735,127 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         }
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Regs<NW>::kSoftmax));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Regs<NW * CS>::kSoftmax));
         // ---------------------------------------------------------- softmax warpgroups
-        const int wg = warp >> 2;
+        // Softmax warpgroup g = warp / 4 serves row tile wg = g / CS and takes the
+        // column share `half` = g % CS of each job: CW = KT / CS score columns, the
+        // matching CW / 2 columns of P and (D >= 64) D / CS columns of O; with
+        // D <= 32 the share 0 owns all of O.  With CS = 2 the two warps on one TMEM
+        // lane quarter exchange their half-row maxima through shared memory every
+        // job, so both take the weights against the same running maximum, and
+        // their half-row sums at the end of an item.
+        constexpr int CW = KT / CS;
+        constexpr int kCChunks = CW / 32;
+        constexpr int kOChunksRow = (D + 31) / 32;
+        constexpr int kOChunks = D >= 64 ? kOChunksRow / CS : kOChunksRow;   // O chunks of an owning share
+        constexpr int kOCols = D >= 64 ? D / CS : D;                         // O values of an owning share
+        const int g = warp >> 2;
+        const int wg = g / CS;
+        const int half = g % CS;
+        const bool owns_o = D >= 64 || half == 0;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_base + wg * KT;
-        const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride;
-        const uint32_t tP = tmem + lane_base + LY::kPCol + wg * (KT / 2);
+        const uint32_t tS = tmem + lane_base + wg * KT + half * CW;
+        const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride + (D >= 64 ? half * kOCols : 0);
+        const uint32_t tP = tmem + lane_base + LY::kPCol + wg * (KT / 2) + half * (CW / 2);
         const float sl2 = p.scale_log2;
         const int tstep = p.interleave ? NW : 1;
         const int tfirst = p.interleave ? wg : 0;
-        uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0;
+        uint32_t sfull_waits = 0, pfree_waits = 0, jobs_done = 0, xph = 0;
         bool ok = true;
-        // Item outputs from this thread's O row (o == nullptr: the warpgroup had no
-        // job in the item).  With D = 16 only the first 16 of 32 loaded columns are O.
+        // CS = 2: the other share's value of this thread's row (both shares call
+        // this in the same order: once per job and once per finished item)
+        uint64_t* my_xbar = xbar + (wg * 4 + wq);
+        float* my_xval = xval + (wg * 4 + wq) * 2 * CS * 32;
+        auto exchange = [&](float v) -> float {
+            if constexpr (CS == 1) {
+                return v;
+            } else {
+                float* slot = my_xval + (xph & 1) * CS * 32;
+                slot[half * 32 + lane] = v;
+                mbar_arrive(my_xbar);
+                if (!mbar_wait(my_xbar, xph & 1, abort_flag)) ok = false;
+                ++xph;
+                return slot[(half ^ 1) * 32 + lane];
+            }
+        };
+        // Item outputs from this thread's share of its O row (o == nullptr: the
+        // warpgroup had no job in the item).  With D = 16 only the first 16 of 32
+        // loaded columns are O.
         auto write_outputs = [&](const Item& it, int njobs, float m, float l, const uint32_t (*o)[32]) {
             if constexpr (MODE == kSplit) {
                 const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
                 const int part = p.interleave ? it.part + wg : it.part;
                 if (r < p.M) {
                     const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
-                    p.part_ml[ridx] = make_float2(njobs > 0 ? m : -INFINITY, l);
-                    float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D);
+                    if (half == 0) p.part_ml[ridx] = make_float2(njobs > 0 ? m : -INFINITY, l);
+                    if (owns_o) {
+                        float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D + (D >= 64 ? half * kOCols : 0));
 #pragma unroll
-                    for (int i = 0; i < D / 4; ++i)
-                        dst[i] = o ? make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
-                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
-                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
-                                                 __uint_as_float(o[i / 8][(i % 8) * 4 + 3]))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int i = 0; i < kOCols / 4; ++i)
+                            dst[i] = o ? make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
+                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
+                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
+                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 3]))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
                 }
             } else {
+                // decode: this share's columns of y (every lane of both shares takes
+                // part in the <dy, y> exchange, also for rows past N)
                 const int n = it.qrow0 + wg * kQTile + row;
-                if (n < p.N && o) {
-                    const float inv = 1.f / l;
-                    const int64_t off = (int64_t)(it.bh / p.H) * p.y_b + (int64_t)it.h * p.y_h + (int64_t)n * p.y_row;
-                    if (p.y) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + off);
+                const bool valid_row = n < p.N && o != nullptr;
+                const float inv = 1.f / l;
+                const int64_t off = (int64_t)(it.bh / p.H) * p.y_b + (int64_t)it.h * p.y_h + (int64_t)n * p.y_row +
+                                    (D >= 64 ? half * kOCols : 0);
+                if (valid_row && owns_o && p.y) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + off);
 #pragma unroll
-                        for (int i = 0; i < D / 8; ++i) {
-                            const int c = i / 4, j = (i % 4) * 8;
-                            dst[i] = make_uint4(
-                                pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
-                                pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
-                                pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
-                                pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
-                        }
+                    for (int i = 0; i < kOCols / 8; ++i) {
+                        const int c = i / 4, j = (i % 4) * 8;
+                        dst[i] = make_uint4(
+                            pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
+                            pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
                     }
-                    if (__builtin_expect(p.tok_stats != nullptr, 0)) {
-                        // the backward's per-token statistics: the softmax's log-sum-exp
-                        // (log2 units, against the same running max as l) and <dy, y>
-                        // (0 when no dy is given: a forward that saves its state)
-                        float dsum = 0.f;
-                        if (p.dy) {
-                            const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
+                }
+                if (__builtin_expect(p.tok_stats != nullptr, 0)) {
+                    // the backward's per-token statistics: the softmax's log-sum-exp
+                    // (log2 units, against the same running max as l) and <dy, y>
+                    // (0 when no dy is given: a forward that saves its state)
+                    float dsum = 0.f;
+                    if (valid_row && owns_o && p.dy) {
+                        const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
 #pragma unroll
-                            for (int i = 0; i < D / 8; ++i) {
-                                const uint4 v = g4[i];
-                                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                                const int c = i / 4, j = (i % 4) * 8;
+                        for (int i = 0; i < kOCols / 8; ++i) {
+                            const uint4 v = g4[i];
+                            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                            const int c = i / 4, j = (i % 4) * 8;
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const float2 g2 = unpack2<E>(w4[e]);
-                                    dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
-                                    dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
-                                }
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 g2 = unpack2<E>(w4[e]);
+                                dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
+                                dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
                             }
                         }
-                        p.tok_stats[(int64_t)it.bh * p.tok_stats_stride + n] = make_float2(m + log2f(l), dsum * inv);
                     }
+                    if constexpr (CS > 1) dsum += exchange(dsum);
+                    if (valid_row && half == 0)
+                        p.tok_stats[(int64_t)it.bh * p.tok_stats_stride + n] = make_float2(m + log2f(l), dsum * inv);
                 }
             }
         };
-        // O row of the finished item -> outputs (every value MMA of the item has completed)
+        // this share of the O row of the finished item -> outputs (every value MMA
+        // of the item has completed)
         auto flush = [&](const Item& it, int njobs, float m, float l) {
-            uint32_t o[(D + 31) / 32][32];
+            uint32_t o[kOChunks][32];
+            if (owns_o) {
 #pragma unroll
-            for (int c = 0; c < (D + 31) / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
-            tmem_wait_ld();
+                for (int c = 0; c < kOChunks; ++c) tmem_ld32(tO + c * 32, o[c]);
+                tmem_wait_ld();
+            }
             write_outputs(it, njobs, m, l, o);
         };
         // Decode: the epilogue of an item (a few jobs long) is deferred into the
@@ -820,28 +877,28 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 if (!mbar_wait(&sfull[wg], sfull_waits & 1, abort_flag)) { ok = false; break; }
                 ++sfull_waits;
                 tc_fence_after();
-                uint32_t sr[LY::kChunks][32];
+                uint32_t sr[kCChunks][32];
 #pragma unroll
-                for (int c = 0; c < LY::kChunks; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                for (int c = 0; c < kCChunks; ++c) tmem_ld32(tS + c * 32, sr[c]);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 mbar_arrive_if(&sfree[wg], lane == 0);
 
-                const int valid = p.kv_rows - t * KT;             // key/value rows of this tile that exist
-                if (__builtin_expect(valid < KT, 0)) {            // ragged last tile only (warp-uniform)
+                // key/value rows of this tile that exist, counted from this share's first column
+                const int valid = p.kv_rows - t * KT - half * CW;
+                if (__builtin_expect(valid < CW, 0)) {            // ragged last tile only (warp-uniform)
 #pragma unroll
-                    for (int c = 0; c < LY::kChunks; ++c)
+                    for (int c = 0; c < kCChunks; ++c)
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (c * 32 + j >= valid) sr[c][j] = __float_as_uint(-INFINITY);
                 }
-                // row max: one chain of 3-input maxima per 32-column chunk (a
-                // tree of maxima measured slower here: 1.47 against 1.39 ms per
-                // split launch at the 1M-token workload)
-                float mc[LY::kChunks];
+                // row max: one chain of 3-input maxima per 32-column chunk (a tree of
+                // maxima measured slower here), then the other share's (CS = 2)
+                float mc[kCChunks];
 #pragma unroll
-                for (int c = 0; c < LY::kChunks; ++c) {
+                for (int c = 0; c < kCChunks; ++c) {
                     mc[c] = __uint_as_float(sr[c][0]);
 #pragma unroll
                     for (int j = 1; j < 31; j += 2)
@@ -850,7 +907,11 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 float mx = mc[0];
 #pragma unroll
-                for (int c = 1; c < LY::kChunks; ++c) mx = fmaxf(mx, mc[c]);
+                for (int c = 1; c < kCChunks; ++c) mx = fmaxf(mx, mc[c]);
+                if constexpr (CS > 1) {
+                    mx = fmaxf(mx, exchange(mx));
+                    if (!ok) break;
+                }
                 const float m_new = fmaxf(m_run, mx * sl2 - Elem<E>::kPBias);
                 float factor = 1.f;
                 const bool resc = m_new > m_run + kRescaleLog2;
@@ -861,16 +922,16 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 // exponent arguments in pairs (packed fp32 FMA), row sum in packed chains
                 const float2 sl2v = make_float2(sl2, sl2);
                 const float2 negm = make_float2(-m_run, -m_run);
-                float2 acc[LY::kChunks];
-                uint32_t pk[KT / 64][32];            // [half][j]: columns 64*half + 2j, 2j+1
+                float2 acc[kCChunks];
+                uint32_t pk[(CW + 63) / 64][32];          // [h][j]: this share's columns 64 h + 2 j, 2 j + 1
 #pragma unroll
-                for (int c = 0; c < LY::kChunks; ++c) {
+                for (int c = 0; c < kCChunks; ++c) {
                     acc[c] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float2 sv = make_float2(__uint_as_float(sr[c][2 * j]), __uint_as_float(sr[c][2 * j + 1]));
                         const float2 xv = __ffma2_rn(sv, sl2v, negm);
-                        const float2 pv = fma_exp_pair(c * 16 + j)
+                        const float2 pv = fma_exp_pair(half * (CW / 2) + c * 16 + j)
                                               ? ex2_fma_pair(xv)
                                               : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
@@ -879,32 +940,33 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 float2 asum = acc[0];
 #pragma unroll
-                for (int c = 1; c < LY::kChunks; ++c) asum = __fadd2_rn(asum, acc[c]);
+                for (int c = 1; c < kCChunks; ++c) asum = __fadd2_rn(asum, acc[c]);
                 l_run = l_run * factor + (asum.x + asum.y);
 
-                // the previous value MMA of this warpgroup must be done before P and O are touched
+                // the previous value MMA of this row tile must be done before P and O are touched
                 while (pfree_waits < jobs_done) {
                     if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
                     ++pfree_waits;
                 }
                 if (!ok) break;
                 tc_fence_after();
-                // P row -> TMEM (this thread's lane, KT/2 columns of packed pairs)
+                // this share of the P row -> TMEM (this thread's lane, CW/2 columns of packed pairs)
 #pragma unroll
-                for (int h = 0; h < KT / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
+                for (int h = 0; h < (CW + 63) / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
                 // Rare work on O, after P is out of the registers and before the
                 // value MMA of this job adds to O: the previous item's O row (first
-                // job of a decode item), or the O rescale of a grown running max.
+                // job of a decode item), or the O rescale of a grown running max
+                // (each share rescales its own O columns).
                 if constexpr (kDefer) {
                     if (__builtin_expect(pend, 0)) {
                         flush(pend_it, pend_jobs, pend_m, pend_l);
                         pend = false;
                     }
                 }
-                if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0)) {
+                if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0) && owns_o) {
                     const float f = njobs > 0 ? factor : 1.f;
 #pragma unroll
-                    for (int c = 0; c < D / 32 + (D % 32 ? 1 : 0); ++c) {
+                    for (int c = 0; c < kOChunks; ++c) {
                         uint32_t o[32];
                         tmem_ld32(tO + c * 32, o);
                         tmem_wait_ld();
@@ -930,15 +992,18 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 pend_it = it;
                 pend_jobs = njobs;
                 pend_m = m_run;
-                pend_l = l_run;
+                pend_l = CS > 1 ? l_run + exchange(l_run) : l_run;
+                if (!ok) break;
             } else {
+                const float l_row = CS > 1 ? l_run + exchange(l_run) : l_run;
+                if (!ok) break;
                 while (pfree_waits < jobs_done) {
                     if (!mbar_wait(&pfree[wg], pfree_waits & 1, abort_flag)) { ok = false; break; }
                     ++pfree_waits;
                 }
                 if (!ok) break;
                 tc_fence_after();
-                flush(it, njobs, m_run, l_run);
+                flush(it, njobs, m_run, l_row);
             }
         }
         if (kDefer && ok && pend) {
@@ -1006,7 +1071,13 @@ struct Config {
     // latent tiles, so the next item's query tiles load during the current one)
     static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 128 ? (DECODE ? 3 : 4) : (D == 64 ? 4 : 6));
     static constexpr int QS = D == 128 && !DECODE ? 1 : 2;
-    using SM = Smem<D, NW, KT, NST, QS>;
+    // split passes on 128-column jobs: two softmax warps per row, each taking
+    // 64 of the columns (four softmax warps per SM sub-partition; measured
+    // 3-4% faster than one warp per row at the 1M-token workload).  The decode
+    // keeps three warpgroups on 64-row latent tiles: on two warpgroups with
+    // 128-row tiles and two warps per row it ran 2.0 ms against 1.52.
+    static constexpr int CS = !DECODE && KT == 128 ? 2 : 1;
+    using SM = Smem<D, NW, KT, NST, QS, CS>;
     // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
     static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
 };
@@ -1022,6 +1093,8 @@ inline bool supported(bool io16, int D, int M) {
 // score + 128 accumulator + 32 weight columns) = 448 of 512).
 inline int split_kt(int D) { return D == 128 ? 64 : kSplitKT; }
 inline int decode_nw(int D) { return D == 128 ? 2 : kDecodeNW; }
+// latent rows per key/value tile of the decode (the box height of its latent maps)
+inline int decode_kt(int D) { return D == 128 ? 64 : kDecodeKT; }
 
 // Split-pass plan.  With one 128-row tile holding all M latents, the two
 // warpgroups share it and take the key/value tiles round-robin (interleaved,
@@ -1126,12 +1199,12 @@ int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
                 cudaStream_t st) {
     using C = Config<D, NW, KT, DECODE>;
     if (prm.interleave && C::NST % C::NW != 0) return 2;      // one stage ring per warpgroup needs NW | NST
-    auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS, DECODE ? kDecode : kSplit>;
+    auto kern = attn_kernel<E, D, C::NW, C::KT, C::NST, C::QS, DECODE ? kDecode : kSplit, C::CS>;
     static_assert(C::SM::kLaunchBytes <= 232448, "shared memory plan exceeds 227 KB");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemLaunch) != cudaSuccess)
         return 3;
     const int grid = prm.items < sm_count() ? prm.items : sm_count();
-    return launch_pdl(kern, dim3(grid), dim3(Regs<C::NW>::kThreads), C::kSmemLaunch, st, mq, mk, mv, prm) ==
+    return launch_pdl(kern, dim3(grid), dim3(Regs<C::NW * C::CS>::kThreads), C::kSmemLaunch, st, mq, mk, mv, prm) ==
                    cudaSuccess
                ? 0
                : 3;
@@ -1196,10 +1269,10 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     const CUtensorMapDataType ty = Elem<E>::kMapType;
     const RowStrides lat1 = contiguous_rows(M, H, D), latb = contiguous_rows(M, H, D), tok = pr.tok;
     bool ok = make_map(&m_qf_q, ty, q_fixed, M, H, 1, D, lat1, kQTile) &&
-              make_map(&m_qf_kv, ty, q_fixed, M, H, 1, D, lat1, kDecodeKT) &&
+              make_map(&m_qf_kv, ty, q_fixed, M, H, 1, D, lat1, decode_kt(D)) &&
               make_map(&m_q16_q, ty, bu.q16, M, H, B, D, latb, kQTile) &&
-              make_map(&m_q16_kv, ty, bu.q16, M, H, B, D, latb, kDecodeKT) &&
-              make_map(&m_z16, ty, bu.z16, M, H, B, D, latb, kDecodeKT) &&
+              make_map(&m_q16_kv, ty, bu.q16, M, H, B, D, latb, decode_kt(D)) &&
+              make_map(&m_z16, ty, bu.z16, M, H, B, D, latb, decode_kt(D)) &&
               make_map(&m_k_kv, ty, k, N, H, B, D, tok, split_kt(D)) && make_map(&m_k_q, ty, k, N, H, B, D, tok, kQTile) &&
               make_map(&m_v, ty, v, N, H, B, D, tok, split_kt(D));
     if (gated)
@@ -1256,7 +1329,7 @@ int run(const Problem& pr, const Buffers& bu, const void* q0, const void* q_fixe
     Params dp{};
     dp.mode = kDecode;
     dp.B = B; dp.H = H; dp.M = M; dp.N = N;
-    dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
+    dp.kv_rows = M; dp.kv_tiles = (M + decode_kt(D) - 1) / decode_kt(D);
     dp.q_shared = 0; dp.k_shared = gated ? 0 : 1; dp.kv_same = 0;
     dp.interleave = 0;
     dp.q_groups = (N + decode_nw(D) * kQTile - 1) / (decode_nw(D) * kQTile);
@@ -1332,13 +1405,13 @@ int cp_decode(const Problem& pr, const void* q, bool q_shared, const void* z16, 
     const CUtensorMapDataType ty = Elem<E>::kMapType;
     CUtensorMap mq, mk, mv;
     bool ok = make_map(&mq, ty, kk, N, H, B, D, pr.tok, kQTile) &&
-              make_map(&mk, ty, q, M, H, q_shared ? 1 : B, D, contiguous_rows(M, H, D), kDecodeKT) &&
-              make_map(&mv, ty, z16, M, H, B, D, contiguous_rows(M, H, D), kDecodeKT);
+              make_map(&mk, ty, q, M, H, q_shared ? 1 : B, D, contiguous_rows(M, H, D), decode_kt(D)) &&
+              make_map(&mv, ty, z16, M, H, B, D, contiguous_rows(M, H, D), decode_kt(D));
     if (!ok) return 3;
     Params dp{};
     dp.mode = kDecode;
     dp.B = B; dp.H = H; dp.M = M; dp.N = N;
-    dp.kv_rows = M; dp.kv_tiles = (M + kDecodeKT - 1) / kDecodeKT;
+    dp.kv_rows = M; dp.kv_tiles = (M + decode_kt(D) - 1) / decode_kt(D);
     dp.q_shared = 0; dp.k_shared = q_shared ? 1 : 0; dp.kv_same = 0;
     dp.interleave = 0;
     dp.q_groups = (N + decode_nw(D) * kQTile - 1) / (decode_nw(D) * kQTile);
