@@ -1,17 +1,22 @@
 """CPU model of attn_kernel's mbarrier protocol (csrc/kernels_tc.cuh).
 
-The model runs the kernel's roles -- TMA producer, one MMA issuer per softmax
-warpgroup, the softmax warpgroups -- as coroutines that wait on mbarriers with
-the kernel's arrival counts and phase parities, in random interleavings, with
-TMA and MMA completions arriving after random delays.  It mirrors the
-kernel's item decoding, stage rings (shared ring, or one ring per warpgroup
-in interleaved mode), query slots and the score-ahead/value MMA order.
+The model runs the kernel's roles -- TMA producer, one MMA issuer per row
+tile, the softmax warpgroups (CS column shares of each row tile, which swap
+their half-row maxima every job and their row sums at the end of an item
+through an exchange barrier) -- as coroutines that wait on mbarriers with the
+kernel's arrival counts and phase parities, in random interleavings, with TMA
+and MMA completions arriving after random delays.  It mirrors the kernel's
+item decoding, stage rings (shared ring, or one ring per warpgroup in
+interleaved mode), query slots, the score-ahead/value MMA order and the
+epilogue placement (deferred into the next item in the decode, at the item's
+end in the split passes).
 
 It checks: no deadlock; no mbarrier phase receives more arrivals than its
 count; every score MMA reads the key/value stage and query slot holding the
-tile and item it expects; the score buffer is never overwritten before the
-softmax read it; every output row (partial triple or token) is written
-exactly once.
+tile and item it expects; the score buffer is never overwritten before every
+share of the softmax read it; both shares of a row take the same exchanged
+values; every output (the (m, l) pair of a partial row, each share's columns
+of its O row, each token row) is written exactly once.
 """
 import random
 import sys
@@ -80,12 +85,18 @@ def simulate(p, grid, NST, QS, seed):
         bars[f"kv_full{i}"] = Bar(f"kv_full{i}", 1); bars[f"kv_empty{i}"] = Bar(f"kv_empty{i}", 1 if p["interleave"] else p["NW"])
     for i in range(QS):
         bars[f"q_full{i}"] = Bar(f"q_full{i}", 1); bars[f"q_empty{i}"] = Bar(f"q_empty{i}", p["NW"])
+    CS = p.get("CS", 1)
     for w in range(p["NW"]):
-        bars[f"sfull{w}"] = Bar(f"sfull{w}", 1); bars[f"sfree{w}"] = Bar(f"sfree{w}", 4)
-        bars[f"pfull{w}"] = Bar(f"pfull{w}", 4); bars[f"pfree{w}"] = Bar(f"pfree{w}", 1)
+        # plant "sfree_one_share": the score buffer released by one share only
+        sfree_count = 4 if p.get("plant") == "sfree_one_share" else 4 * CS
+        bars[f"sfull{w}"] = Bar(f"sfull{w}", 1); bars[f"sfree{w}"] = Bar(f"sfree{w}", sfree_count)
+        bars[f"pfull{w}"] = Bar(f"pfull{w}", 4 * CS); bars[f"pfree{w}"] = Bar(f"pfree{w}", 1)
+        bars[f"xbar{w}"] = Bar(f"xbar{w}", CS)       # one arrival per share (all its lanes)
+    xvals = {}                                        # (row tile, exchange index) -> {share: value}
     writes = p["writes"]
     # buffer state for hazards
     S_state = ["free"] * p["NW"]
+    S_reads = [0] * p["NW"]                           # shares that have read the current scores
     kv_contents = [None] * NST
     q_contents = [None] * QS
     outstanding_mma = []            # list of (bars_to_commit...) - commits complete when all prior done
@@ -189,7 +200,9 @@ def simulate(p, grid, NST, QS, seed):
             assert kv_contents[st] == (c.info["bh"], c.t), ("kv stage holds wrong tile", kv_contents[st], c.t)
             assert q_contents[slot] == c.item, ("q slot holds wrong item", q_contents[slot], c.item)
             yield ("wait", f"sfree{w}", (s_iss[0] & 1) ^ 1)
-            assert S_state[w] in ("free", "read"), ("S overwritten before read", w, S_state[w])
+            assert S_state[w] == "free" or (S_state[w] == "read" and S_reads[w] == CS), \
+                ("S overwritten before read", w, S_state[w], S_reads[w])
+            S_reads[w] = 0
             S_state[w] = "computing"
             commit(f"sfull{w}")
             s_iss[0] += 1
@@ -214,9 +227,42 @@ def simulate(p, grid, NST, QS, seed):
                 yield from issue_s(sc); yield from nxt(sc, True)
             yield from issue_pv(pc); yield from nxt(pc, False)
 
-    def softmax(wg):
+    def softmax(wg, half):
         sfull_waits = pfree_waits = jobs_done = 0
-        turns = [0]
+        xph = [0]
+        defer = p["mode"] == "decode"
+
+        def exchange(value):
+            # the kernel's exchange(): publish, arrive, wait for the other share
+            if CS == 1:
+                return value
+            key = (wg, xph[0])
+            xvals.setdefault(key, {})[half] = value
+            bars[f"xbar{wg}"].arrive()
+            yield ("wait", f"xbar{wg}", xph[0] & 1)
+            other = xvals[key][half ^ 1]
+            xph[0] += 1
+            return other
+
+        def outputs(it, njobs):
+            for row in range(128):
+                if p["mode"] == "split":
+                    r = it["qrow0"] + (0 if p["interleave"] else wg * 128) + row
+                    part = it["part"] + wg if p["interleave"] else it["part"]
+                    if r < p["M"]:
+                        assert part < p["parts"]
+                        keys = [("O", part, it["bh"], r, half)] if (p["D"] >= 64 or half == 0) else []
+                        if half == 0:
+                            keys.append(("ml", part, it["bh"], r))
+                        for key in keys:
+                            writes[key] = writes.get(key, 0) + 1
+                else:
+                    n = it["qrow0"] + wg * 128 + row
+                    if n < p["N"] and njobs > 0 and (p["D"] >= 64 or half == 0):
+                        key = ("y", it["bh"], n, half)
+                        writes[key] = writes.get(key, 0) + 1
+
+        pend = None
         for item in range(blk, p["items"], grid):
             it = decode_item(p, item)
             njobs = 0
@@ -224,37 +270,49 @@ def simulate(p, grid, NST, QS, seed):
             for t in range(it["t_begin"] + (wg if p["interleave"] else 0), it["t_end"], step):
                 yield ("wait", f"sfull{wg}", sfull_waits & 1)
                 sfull_waits += 1
+                assert S_state[wg] in ("computing", "read") or True
                 S_state[wg] = "read"
-                for _ in range(4):
-                    bars[f"sfree{wg}"].arrive()
+                S_reads[wg] += 1
+                if p.get("plant") != "sfree_one_share" or half == 0:
+                    for _ in range(4):
+                        bars[f"sfree{wg}"].arrive()
+                mine = (item, t, half)
+                other = yield from exchange(mine)
+                if CS > 1:
+                    assert other == (item, t, half ^ 1), ("exchange pairs different jobs", mine, other)
 
                 while pfree_waits < jobs_done:
                     yield ("wait", f"pfree{wg}", pfree_waits & 1)
                     pfree_waits += 1
+                if defer and pend is not None:
+                    outputs(*pend)
+                    pend = None
                 for _ in range(4):
                     bars[f"pfull{wg}"].arrive()
                 jobs_done += 1; njobs += 1
-            if njobs > 0:
+            if njobs == 0:
+                outputs(it, 0)
+            elif defer:
+                other = yield from exchange(("l", item, half))
+                if CS > 1:
+                    assert other == ("l", item, half ^ 1), ("row-sum exchange pairs different items", other)
+                pend = (it, njobs)
+            else:
+                other = yield from exchange(("l", item, half))
+                if CS > 1:
+                    assert other == ("l", item, half ^ 1), ("row-sum exchange pairs different items", other)
                 while pfree_waits < jobs_done:
                     yield ("wait", f"pfree{wg}", pfree_waits & 1)
                     pfree_waits += 1
-            # outputs
-            for row in range(128):
-                if p["mode"] == "split":
-                    r = it["qrow0"] + (0 if p["interleave"] else wg * 128) + row
-                    part = it["part"] + wg if p["interleave"] else it["part"]
-                    if r < p["M"]:
-                        assert part < p["parts"]
-                        key = (part, it["bh"], r)
-                        writes[key] = writes.get(key, 0) + 1
-                else:
-                    n = it["qrow0"] + wg * 128 + row
-                    if n < p["N"]:
-                        key = (it["bh"], n)
-                        writes[key] = writes.get(key, 0) + 1
+                outputs(it, njobs)
+        if pend is not None:
+            while pfree_waits < jobs_done:
+                yield ("wait", f"pfree{wg}", pfree_waits & 1)
+                pfree_waits += 1
+            outputs(*pend)
 
     NWc = p["NW"]
-    roles = [producer()] + [mma(w) for w in range(NWc)] + [softmax(w) for w in range(NWc)]
+    roles = [producer()] + [mma(w) for w in range(NWc)] + [softmax(w, h) for w in range(NWc) for h in range(CS)]
     state = [None] * len(roles)
     done = [False] * len(roles)
     steps = 0
@@ -300,7 +358,8 @@ def choose_chunks(units, tiles, sms=148, jobs_div=1):
     return best_c
 
 
-def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, shared_ring=False):
+def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, shared_ring=False, CS=None,
+          plant=None):
     BH = B * H
     KT = 64 if NW == 3 else 128
     kv_tiles = (N + KT - 1) // KT
@@ -323,17 +382,25 @@ def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, sh
                 p = dict(mode="decode", NW=NW, H=H, M=M, N=N, kv_rows=M, kv_tiles=-(-M // KT), interleave=False,
                          q_groups=qg, items=BH * qg, q_shared=0, q_planes=BH, kv_same=0, parts=1)
             p["KT"] = KT
+            p["D"] = D
+            # the kernel splits the score columns between two warps per row in
+            # the split passes on 128-column jobs
+            p["CS"] = CS if CS is not None else (2 if md == "split" and KT == 128 else 1)
             p["shared_ring"] = shared_ring
+            p["plant"] = plant
             g = min(grid, p["items"])
             writes = {}
             p["writes"] = writes
             for blk in range(g):
                 p["blk"] = blk
                 simulate(p, g, NST, 2, seed=blk + 7919 * seed)
+            shares = [h for h in range(p["CS"]) if D >= 64 or h == 0]
             if md == "split":
-                exp = {(pt, bh, r) for bh in range(BH) for r in range(M) for pt in range(p["parts"])}
+                exp = {("ml", pt, bh, r) for bh in range(BH) for r in range(M) for pt in range(p["parts"])}
+                exp |= {("O", pt, bh, r, h) for bh in range(BH) for r in range(M) for pt in range(p["parts"])
+                        for h in shares}
             else:
-                exp = {(bh, n) for bh in range(BH) for n in range(N)}
+                exp = {("y", bh, n, h) for bh in range(BH) for n in range(N) for h in shares}
             assert set(writes) == exp, (md, len(set(writes) ^ exp))
             assert all(v == 1 for v in writes.values()), md
             res.append((md, kv_same, p["items"], g, chunks))

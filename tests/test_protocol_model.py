@@ -1,8 +1,9 @@
 """The attention kernel's mbarrier protocol, modelled on the CPU (see
 protocol_model.py), over shapes that exercise ragged tiles, one-tile and
 jobless items, interleaved and shared stage rings, and forced chunk counts,
-for both kernel configurations (two warpgroups on 128-row tiles for the
-split passes, three on 64-row tiles for the decode)."""
+for both kernel configurations (two row tiles on 128-row key/value tiles with
+two column shares per row for the split passes, three on 64-row tiles for
+the decode)."""
 import pytest
 
 from protocol_model import check
@@ -37,3 +38,20 @@ def test_model_catches_the_shared_ring_race():
     interleaves the warpgroups closely enough to show the race."""
     with pytest.raises(AssertionError, match="kv stage holds wrong tile"):
         check(2, 8, 16641, 128, 32, NW=3, grid=148, mode="split", shared_ring=True, force_chunks=37)
+
+
+def test_column_shares_in_split_and_single_share_decode():
+    """The split passes on 128-column jobs run two column shares per row (their
+    exchange pairs the same job), the decode one; both write each output once."""
+    res = check(1, 2, 1500, 384, 64, NW=2, grid=37, mode="split")
+    assert res
+    check(1, 2, 1500, 384, 32, NW=2, grid=37, mode="split")      # D <= 32: share 0 owns O
+    check(1, 2, 700, 64, 64, NW=2, grid=37, mode="split")        # interleaved, two shares per stream
+
+
+def test_model_catches_a_score_buffer_released_by_one_share():
+    """If the next score MMA waited for one share only, it could overwrite the
+    scores the other share has not read yet; the model must see it."""
+    with pytest.raises(AssertionError, match="S overwritten before read"):
+        for seed in range(6):
+            check(1, 2, 3000, 256, 64, NW=2, grid=5, mode="split", seed=seed, plant="sfree_one_share")
