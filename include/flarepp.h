@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define FLAREPP_ABI_VERSION 4
+#define FLAREPP_ABI_VERSION 5
 
 typedef enum flarepp_dtype {
     FLAREPP_F32 = 0,
@@ -148,9 +148,34 @@ int flarepp_mixer_fwd_ex(const void* q0, const void* q_fixed, const float* gate,
 
 /* Bytes of device scratch one call needs (partial softmax triples per token
  * chunk, and q, z in fp32 and in the 16-bit I/O dtype).  gated = 0 for the closed-gate form.
- * Returns 0 for arguments the forward entries would reject. */
+ * opts (may be NULL) is the call's options: force_chunks, layout and
+ * norm_synthesis change the size.  Returns 0 for arguments the forward
+ * entries would reject. */
 size_t flarepp_workspace_bytes(int B, int H, int N, int M, int D, int dtype, int gated,
                                const flarepp_options_t* opts);
+
+/* Registers a caller-owned DEVICE scratch buffer for the current device
+ * (256-byte aligned; dev_ptr = NULL unregisters).  The forward entries that
+ * get no workspace through their options (flarepp_mixer_fwd, flare_fwd,
+ * flarepp_mixer_fwd_debug, flarepp_mixer_fwd_ex with opts->workspace = NULL)
+ * use it when it holds at least flarepp_workspace_bytes(...) bytes for the
+ * call, and allocate stream-ordered otherwise.  The caller keeps the buffer
+ * alive while it is registered; forward calls whose kernels overlap on the GPU
+ * (other streams, other host threads) race on a shared registered buffer.
+ * The per-call flarepp_options_t.workspace needs no shared state and takes
+ * precedence.  Misaligned dev_ptr -> FLAREPP_ERR_INVALID_ARG. */
+int flarepp_set_workspace(void* dev_ptr, size_t bytes);
+
+/* flarepp_mixer_fwd that also returns the intermediates for debugging and
+ * parity checks: q_out and z_out, optional DEVICE fp32 [B,H,M,D] (either may
+ * be NULL; 16-byte aligned), the routing queries q and the latents z; and
+ * force_chunks > 0 forces the number of token chunks of the synthesis and
+ * encode passes (0 = planned; < 0 -> FLAREPP_ERR_INVALID_ARG).  The same as
+ * flarepp_mixer_fwd_ex with those three options set. */
+int flarepp_mixer_fwd_debug(const void* q0, const void* q_fixed, const float* gate,
+                            const void* k0, const void* k, const void* v, void* y,
+                            int B, int H, int N, int M, int D, int dtype,
+                            float* q_out, float* z_out, int force_chunks, void* stream);
 
 /* Same operation with HOST buffers (end-to-end form): streams the (b, h)
  * slices through the GPU -- the copy-in of one slice, the forward of the

@@ -25,7 +25,8 @@ EXPORTS = ["flarepp_mixer_fwd", "flare_fwd", "flarepp_mixer_fwd_ex", "flarepp_wo
            "flarepp_mixer_fwd_host", "flarepp_selected_path", "flarepp_check_device_status",
            "flarepp_status_string", "flarepp_abi_version", "flarepp_launches_per_call",
            "flarepp_mixer_bwd", "flarepp_mixer_bwd_workspace_bytes", "flarepp_mixer_bwd_launches",
-           "flarepp_train_context_bytes", "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx"]
+           "flarepp_train_context_bytes", "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx",
+           "flarepp_set_workspace", "flarepp_mixer_fwd_debug"]
 
 
 class FlareppError(RuntimeError):
@@ -69,16 +70,19 @@ def _load() -> ctypes.CDLL:
     lib.flarepp_train_context_bytes.restype = ctypes.c_size_t
     lib.flarepp_mixer_fwd_train.argtypes = sig + [ctypes.POINTER(Options), vp, ctypes.c_size_t, vp]
     lib.flarepp_mixer_bwd_ctx.argtypes = [vp] * 14 + [i] * 6 + [ctypes.POINTER(Options), vp, ctypes.c_size_t, vp]
+    lib.flarepp_set_workspace.argtypes = [vp, ctypes.c_size_t]
+    lib.flarepp_mixer_fwd_debug.argtypes = sig + [vp, vp, i, vp]
     for name in ("flarepp_mixer_fwd", "flarepp_mixer_fwd_ex", "flarepp_mixer_fwd_host", "flare_fwd",
                  "flarepp_selected_path", "flarepp_check_device_status", "flarepp_abi_version",
                  "flarepp_launches_per_call", "flarepp_mixer_bwd", "flarepp_mixer_bwd_launches",
-                 "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx"):
+                 "flarepp_mixer_fwd_train", "flarepp_mixer_bwd_ctx", "flarepp_set_workspace",
+                 "flarepp_mixer_fwd_debug"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
 
 lib = _load()
-ABI_VERSION = 4
+ABI_VERSION = 5
 if lib.flarepp_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {lib.flarepp_abi_version()}, this binding needs {ABI_VERSION}: "
                       "rebuild it")
@@ -307,6 +311,34 @@ def mixer_fwd_plain(q0, q_fixed, gate, k0, k, v, y):
                                B, H, N, M, D, _dtype_code(k), _stream(k.device))
     _check(rc, "flarepp_mixer_fwd")
     return y
+
+
+def mixer_fwd_debug(q0, q_fixed, gate, k0, k, v, y=None, *, force_chunks: int = 0):
+    """flarepp_mixer_fwd_debug: y and the fp32 intermediates q, z [B,H,M,D]."""
+    B, H, N, M, D = _shapes(q_fixed, k)
+    _contig(q0, q_fixed, gate, k0, k, v, y)
+    if y is None:
+        y = torch.empty_like(k)
+    q_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
+    z_out = torch.empty((B, H, M, D), dtype=torch.float32, device=k.device)
+    rc = lib.flarepp_mixer_fwd_debug(_ptr(q0), _ptr(q_fixed), _ptr(gate), _ptr(k0), _ptr(k), _ptr(v), _ptr(y),
+                                     B, H, N, M, D, _dtype_code(k), q_out.data_ptr(), z_out.data_ptr(),
+                                     force_chunks, _stream(k.device))
+    _check(rc, "flarepp_mixer_fwd_debug")
+    return y, q_out, z_out
+
+
+def set_workspace(buf: Optional[torch.Tensor]):
+    """flarepp_set_workspace on the current device: a uint8 CUDA tensor the
+    forward entries without an options workspace then use (None unregisters).
+    The caller keeps the tensor alive while it is registered."""
+    if buf is None:
+        rc = lib.flarepp_set_workspace(None, 0)
+    else:
+        if not buf.is_cuda or not buf.is_contiguous():
+            raise ValueError("the registered workspace must be a contiguous CUDA tensor")
+        rc = lib.flarepp_set_workspace(buf.data_ptr(), buf.numel() * buf.element_size())
+    _check(rc, "flarepp_set_workspace")
 
 
 def flare_fwd(q, k, v, y=None):

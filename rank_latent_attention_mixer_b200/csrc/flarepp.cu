@@ -302,6 +302,28 @@ void rms_norm(const Shape& s, const void* q0, void* q0n, const void* k0, void* k
     else launch_rms_norm<__nv_bfloat16>(s, q0, q0n, k0, k0n, st);
 }
 
+// Caller-registered scratch per device (flarepp_set_workspace), used by the
+// forward entries that receive no workspace in their options.
+constexpr int kMaxDevices = 64;
+struct RegisteredWorkspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_registered_mu;
+RegisteredWorkspace g_registered[kMaxDevices];
+
+// The current device's registered scratch if it holds at least `need` bytes.
+char* registered_workspace(size_t need) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_registered_mu);
+    const RegisteredWorkspace& r = g_registered[dev];
+    return r.ptr && r.bytes >= need ? static_cast<char*>(r.ptr) : nullptr;
+}
+
 int forward(const void* q0, const void* q_fixed, const float* gate, const void* k0, const void* k,
             const void* v, void* y, int B, int H, int N, int M, int D, int dtype,
             const flarepp_options_t* opts, void* stream, const FwdExtras& ex = FwdExtras{}) {
@@ -321,7 +343,7 @@ int forward(const void* q0, const void* q_fixed, const float* gate, const void* 
         if (opts->workspace_bytes < pl.total) return FLAREPP_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(opts->workspace) % kAlign) return FLAREPP_ERR_INVALID_ARG;
         ws = static_cast<char*>(opts->workspace);
-    } else {
+    } else if ((ws = registered_workspace(pl.total)) == nullptr) {
         if (cudaMallocAsync(reinterpret_cast<void**>(&ws), pl.total, st) != cudaSuccess) {
             cudaGetLastError();
             return FLAREPP_ERR_WORKSPACE;
@@ -360,7 +382,6 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 // array's name is only a host-side stand-in, so the address is asked from the
 // runtime once per device, with that device current, and cached.
 void* static_scratch_address() {
-    constexpr int kMaxDevices = 64;
     static std::mutex mu;
     static void* addr[kMaxDevices] = {};
     int dev = -1;
@@ -1705,11 +1726,37 @@ int flare_fwd(const void* q, const void* k, const void* v, void* y, int B, int H
     return forward(nullptr, q, nullptr, nullptr, k, v, y, B, H, N, M, D, dtype, nullptr, stream);
 }
 
+int flarepp_mixer_fwd_debug(const void* q0, const void* q_fixed, const float* gate, const void* k0,
+                            const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
+                            int dtype, float* q_out, float* z_out, int force_chunks, void* stream) {
+    if (force_chunks < 0) return FLAREPP_ERR_INVALID_ARG;
+    flarepp_options_t o{};
+    o.q_out = q_out;
+    o.z_out = z_out;
+    o.force_chunks = force_chunks;
+    return forward(q0, q_fixed, gate, k0, k, v, y, B, H, N, M, D, dtype, &o, stream);
+}
+
+int flarepp_set_workspace(void* dev_ptr, size_t bytes) {
+    if (dev_ptr && (reinterpret_cast<uintptr_t>(dev_ptr) % kAlign)) return FLAREPP_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FLAREPP_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_registered_mu);
+    g_registered[dev].ptr = dev_ptr;
+    g_registered[dev].bytes = dev_ptr ? bytes : 0;
+    return FLAREPP_OK;
+}
+
 int flarepp_mixer_fwd_noalloc(const void* q0, const void* q_fixed, const float* gate, const void* k0,
                               const void* k, const void* v, void* y, int B, int H, int N, int M, int D,
                               int dtype, void* stream) {
     const Shape s{B, H, N, M, D, dtype};
     int rc = check_shape(s);
+    if (rc) return rc;
+    rc = check_pointers(s, q0, q_fixed, gate, k0, k, v, y);    // before any CUDA call
     if (rc) return rc;
     const int chunks = chunks_fitting_static_scratch(s);
     if (chunks < 1) return FLAREPP_ERR_WORKSPACE;   // needs more than FLAREPP_NOALLOC_SCRATCH_BYTES

@@ -27,6 +27,15 @@ P (dP - Delta) k that cancel: on a D = 16, M = 200 case an emulation of that
 one rounding alone moves max |dq_fixed - o| / max |o| to 1.7e-2 (all the
 backward's bf16 roundings together: 2.1e-2), against 1.3e-3 for each of the
 others (P, dS, dz, z).  fp16 keeps the factor 1/4 of the forward bounds.
+
+A softmax scale s other than the default 1/sqrt(D) (the FLARE block prints
+s = 1): the 16-bit bounds above are multiplied by max(1, s sqrt(D)).  The
+routing queries q are rounded to the I/O type as tensor-core operands, so a
+score s <q, k> carries an absolute error of about s sqrt(D) |q_d| |k_d| u (u
+the unit roundoff); at the default scale that is the error the bounds were set
+for, and it grows in proportion to s sqrt(D), and with it the error of every
+softmax weight (measured at s = 1: bf16 rel L2 stays under 0.7e-2 for y, q, z,
+max abs reaches 0.07 at D = 64-128, where the scaled bound is 0.16-0.23).
 """
 import numpy as np
 import torch
@@ -64,21 +73,27 @@ def metrics(g, o):
     }
 
 
-def assert_parity(g, o, dtype: str, what: str = "y"):
+def scale_factor(scale: float, D: int) -> float:
+    """Factor on the 16-bit bounds for a softmax scale other than 1/sqrt(D)
+    (scale <= 0 selects the default)."""
+    return 1.0 if scale <= 0 else max(1.0, scale * D ** 0.5)
+
+
+def assert_parity(g, o, dtype: str, what: str = "y", factor: float = 1.0):
     m = metrics(g, o)
     assert m["finite"], f"{what}: non-finite values"
     if dtype == "f32":
         assert m["row_max_rel"] <= FP32_MAX_REL, f"{what}: fp32 row max rel {m['row_max_rel']:.3e} > {FP32_MAX_REL} ({m})"
     elif dtype == "f16":
-        assert m["rel_l2"] <= F16_REL_L2, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} > {F16_REL_L2} ({m})"
-        assert m["max_abs"] <= F16_MAX_ABS, f"{what}: fp16 max abs {m['max_abs']:.3e} > {F16_MAX_ABS} ({m})"
+        assert m["rel_l2"] <= F16_REL_L2 * factor, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} > {F16_REL_L2 * factor} ({m})"
+        assert m["max_abs"] <= F16_MAX_ABS * factor, f"{what}: fp16 max abs {m['max_abs']:.3e} > {F16_MAX_ABS * factor} ({m})"
     else:
-        assert m["rel_l2"] <= BF16_REL_L2, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} > {BF16_REL_L2} ({m})"
-        assert m["max_abs"] <= BF16_MAX_ABS, f"{what}: bf16 max abs {m['max_abs']:.3e} > {BF16_MAX_ABS} ({m})"
+        assert m["rel_l2"] <= BF16_REL_L2 * factor, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} > {BF16_REL_L2 * factor} ({m})"
+        assert m["max_abs"] <= BF16_MAX_ABS * factor, f"{what}: bf16 max abs {m['max_abs']:.3e} > {BF16_MAX_ABS * factor} ({m})"
     return m
 
 
-def assert_grad_parity(g, o, dtype: str, what: str, zero_atol: float = 1e-5):
+def assert_grad_parity(g, o, dtype: str, what: str, zero_atol: float = 1e-5, factor: float = 1.0):
     """A gradient the mathematics makes exactly zero (e.g. the seeds' gradient
     when one token carries all the softmax weight) is held to an absolute
     bound instead: the CUDA path leaves rounding noise there."""
@@ -92,15 +107,17 @@ def assert_grad_parity(g, o, dtype: str, what: str, zero_atol: float = 1e-5):
     if dtype == "f32":
         assert m["max_abs_rel_to_max"] <= FP32_MAX_REL, f"{what}: fp32 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     elif dtype == "f16":
-        assert m["rel_l2"] <= F16_REL_L2, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} ({m})"
-        assert m["max_abs_rel_to_max"] <= GRAD_F16_MAX, f"{what}: fp16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
+        assert m["rel_l2"] <= F16_REL_L2 * factor, f"{what}: fp16 rel L2 {m['rel_l2']:.3e} ({m})"
+        assert m["max_abs_rel_to_max"] <= GRAD_F16_MAX * factor, \
+            f"{what}: fp16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     else:
-        assert m["rel_l2"] <= BF16_REL_L2, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} ({m})"
-        assert m["max_abs_rel_to_max"] <= GRAD_BF16_MAX, f"{what}: bf16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
+        assert m["rel_l2"] <= BF16_REL_L2 * factor, f"{what}: bf16 rel L2 {m['rel_l2']:.3e} ({m})"
+        assert m["max_abs_rel_to_max"] <= GRAD_BF16_MAX * factor, \
+            f"{what}: bf16 max err / max {m['max_abs_rel_to_max']:.3e} ({m})"
     return m
 
 
-def assert_dgate_parity(g, ref: dict, dtype: str, zero_atol: float = 0.0):
+def assert_dgate_parity(g, ref: dict, dtype: str, zero_atol: float = 0.0, factor: float = 1.0):
     """dgate[h] = sum over (b, m, d) of dq * q_dyn is a dot product whose terms
     cancel, so its error is bounded through dq's by Cauchy-Schwarz:
     |err_h| <= ||err(dq)_h|| ||q_dyn_h|| <= tol ||dq_h|| ||q_dyn_h||, with tol
@@ -109,7 +126,7 @@ def assert_dgate_parity(g, ref: dict, dtype: str, zero_atol: float = 0.0):
     g = to64(g)
     o = to64(ref["dgate"])
     dq, qd = to64(ref["dq"]), to64(ref["q_dyn"])
-    tol = {"f32": FP32_MAX_REL, "f16": F16_REL_L2}.get(dtype, BF16_REL_L2)
+    tol = {"f32": FP32_MAX_REL, "f16": F16_REL_L2 * factor}.get(dtype, BF16_REL_L2 * factor)
     assert np.all(np.isfinite(g)), "dgate: non-finite values"
     for h in range(o.shape[0]):
         bound = max(tol * np.linalg.norm(dq[:, h]) * np.linalg.norm(qd[:, h]), zero_atol)

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.lib.flarepp_abi_version() == 4
+    assert lib.lib.flarepp_abi_version() == 5
     assert lib.bwd_launches(True) == 14 and lib.bwd_launches(False) == 9
     assert lib.bwd_launches(True, lib.PATH_TCGEN05) == 14 and lib.bwd_launches(False, lib.PATH_TCGEN05) == 9
     assert lib.launches_per_call(True) == 5 and lib.launches_per_call(False) == 3
@@ -241,3 +241,31 @@ def test_sharded_backward_entries_checked(lib):
     p = list(ptrs)
     p[4] = None                                                       # no z state
     assert fn(1, *p, 1, 2, 64, 16, 16, 1, None, None) == 1
+
+
+def test_debug_and_workspace_entries_checked(lib):
+    L = lib.lib
+    # flarepp_mixer_fwd_debug: argument checks before any CUDA call
+    assert L.flarepp_mixer_fwd_debug(*FAKE, 1, 2, 64, 16, 16, 1, None, None, -1, None) == 1   # force_chunks < 0
+    ptrs = list(FAKE)
+    ptrs[6] = None                                                                              # y NULL
+    assert L.flarepp_mixer_fwd_debug(*ptrs, 1, 2, 64, 16, 16, 1, None, None, 0, None) == 1
+    assert L.flarepp_mixer_fwd_debug(*FAKE, 1, 2, 64, 16, 48, 1, None, None, 0, None) == 2    # D = 48
+    assert L.flarepp_mixer_fwd_debug(*FAKE, 1, 2, 64, 16, 16, 1, 0x10008, None, 0, None) == 1  # q_out misaligned
+    # flarepp_set_workspace: a misaligned buffer is refused before any CUDA call
+    assert L.flarepp_set_workspace(0x10010, 1 << 20) == 1
+
+
+def test_noalloc_checks_pointers_before_cuda(lib):
+    fn = lib.lib.flarepp_mixer_fwd_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    ptrs = list(FAKE)
+    ptrs[6] = None                                  # y NULL
+    assert fn(*ptrs, 1, 2, 64, 16, 16, 1, None) == 1
+    ptrs = list(FAKE)
+    ptrs[6] = FAKE[4]                               # y overlaps k
+    assert fn(*ptrs, 1, 2, 64, 16, 16, 1, None) == 1
+    ptrs = list(FAKE)
+    ptrs[6] = 0x70008                               # y misaligned
+    assert fn(*ptrs, 1, 2, 64, 16, 16, 1, None) == 1

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle.backward import flarepp_backward
-from parity import assert_dgate_parity, assert_grad_parity, to64
+from parity import assert_dgate_parity, assert_grad_parity, scale_factor, to64
 from rank_latent_attention_mixer_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -93,13 +93,17 @@ def test_closed_gate_is_flare_backward(dt):
     assert_dgate_parity(gz["dgate"], ref, dt)
 
 
-def test_scale_option():
-    x, dy = inputs(1, 2, 640, 40, 32, "f32", seed=11)
+@pytest.mark.parametrize("dt,D", [("f32", 32), ("bf16", 32), ("bf16", 64), ("f16", 64)])
+def test_scale_option(dt, D):
+    """The FLARE block's printed scale=1.0 through the options, on the SIMT
+    kernels (fp32) and the tensor-core kernels (bf16, fp16)."""
+    x, dy = inputs(1, 2, 640, 40, D, dt, seed=11)
     ref = oracle_grads(x, dy, scale=1.0)
     g = gpu_grads(x, dy, scale=1.0)
+    f = scale_factor(1.0, D)              # the bounds for a non-default scale (parity.py)
     for name in GRADS:
-        assert_grad_parity(g[name], ref[name], "f32", name)
-    assert_dgate_parity(g["dgate"], ref, "f32")
+        assert_grad_parity(g[name], ref[name], dt, name, factor=f)
+    assert_dgate_parity(g["dgate"], ref, dt, factor=f)
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])

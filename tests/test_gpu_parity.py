@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from parity import assert_parity, metrics, to64
+from parity import assert_parity, metrics, scale_factor, to64
 from rank_latent_attention_mixer_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -220,10 +220,88 @@ def test_permutation_equivariance_gpu():
     assert metrics(yp, y[:, :, perm.to(y.device)])["row_max_rel"] < 1e-4
 
 
-@pytest.mark.parametrize("name", ["scale1m_bf16", "scale1m_f16"])
+def test_scale1m_full():
+    """The 1M-token bf16 workload (B=1, H=8, N=1048576, M=512, D=64) in the
+    launch configuration the benchmark times, compared with the oracle in full:
+    every head's q and z and every token of y.  The oracle runs one (b, h)
+    slice at a time; the bf16 bounds are taken over the whole tensors
+    (relative L2 from the accumulated squared norms, max abs over all)."""
+    w = W.WORKLOADS["scale1m_bf16"]
+    x = W.make_inputs(w, device=DEV)
+    b = binding()
+    y, q, z = b.mixer_fwd(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], return_qz=True)
+    torch.cuda.synchronize()
+    assert b.check_device_status() == 0
+    acc = {n: [0.0, 0.0, 0.0] for n in ("y", "q", "z")}      # sum d^2, sum o^2, max |d|
+    toks = np.arange(w.N, dtype=np.int64)
+
+    def add(name, got, ref):
+        d = to64(got) - ref
+        a = acc[name]
+        a[0] += float((d * d).sum())
+        a[1] += float((ref * ref).sum())
+        a[2] = max(a[2], float(np.abs(d).max()))
+
+    for bi in range(w.B):
+        for h in range(w.H):
+            y_ref, q_ref, z_ref = oracle.flarepp_head(x["q0"][h], x["q_fixed"][h], float(x["gate"][h]),
+                                                      x["k0"][bi, h], x["k"][bi, h], x["v"][bi, h], toks)
+            add("y", y[bi, h], y_ref)
+            add("q", q[bi, h], q_ref)
+            add("z", z[bi, h], z_ref)
+            del y_ref
+    for name, (sd, so, mx) in acc.items():
+        rel = (sd / so) ** 0.5
+        print(f"scale1m_bf16 full {name}: rel_l2={rel:.3e} max_abs={mx:.3e}")
+        assert rel <= 1e-2 and mx <= 2e-2, (name, rel, mx)
+    assert bool(torch.isfinite(y.float()).all())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("gated", [True, False], ids=["gated", "closed"])
+@pytest.mark.parametrize("D,M", [(16, 64), (32, 200), (64, 300), (128, 130)], ids=lambda v: str(v))
+def test_scale_one_tensor_cores(D, M, gated, dtype):
+    """The FLARE block's printed scale=1.0 (options' scale) on the tensor-core
+    kernels: scores 4-11x larger than at 1/sqrt(D), which exercises the fp16
+    weight offset and the lazy rescale of the running maximum.  The bounds are
+    the dtype's scaled by sqrt(D) (parity.scale_factor: the error of the
+    scores from rounding q to the operand type grows with the scale)."""
+    x = W.random_inputs(1, 2, 1100, M, D, dtype=dtype, seed=D + M)
+    if gated:
+        y_ref, q_ref, z_ref = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"], scale=1.0)
+    else:
+        y_ref, q_ref, z_ref = oracle.flarepp(None, x["q_fixed"], None, None, x["k"], x["v"], scale=1.0, flare=True)
+    y, q, z = run(x, flare=not gated, scale=1.0)
+    assert binding().selected_path(1, 2, 1100, M, D, binding().BF16 if dtype == "bf16" else binding().F16) == 2
+    print(dtype, D, M, gated, "y", metrics(y, y_ref), "z", metrics(z, z_ref))
+    f = scale_factor(1.0, D)              # the bounds for a non-default scale (parity.py)
+    assert_parity(q, q_ref, dtype, "q", f)
+    assert_parity(z, z_ref, dtype, "z", f)
+    assert_parity(y, y_ref, dtype, "y", f)
+
+
+@pytest.mark.parametrize("shape,dtype", [((1, 1, 3001, 1024, 64), "bf16"), ((1, 1, 3001, 1024, 64), "f16"),
+                                         ((1, 2, 2500, 2048, 64), "bf16"), ((1, 1, 2500, 2048, 64), "f16"),
+                                         ((1, 1, 1500, 4096, 64), "bf16")],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else v)
+def test_large_latent_counts(shape, dtype):
+    """Latent ranks above 512, up to the header's limit M = 4096 (the pages use
+    M = 2048 at 1M points): more latent row groups in the split passes and more
+    latent tiles per decode item than the benchmark workloads."""
+    B, H, N, M, D = shape
+    x = W.random_inputs(B, H, N, M, D, dtype=dtype, seed=M + N)
+    y_ref, q_ref, z_ref = oracle.flarepp(x["q0"], x["q_fixed"], x["gate"], x["k0"], x["k"], x["v"])
+    y, q, z = run(x)
+    assert_parity(q, q_ref, dtype, "q")
+    assert_parity(z, z_ref, dtype, "z")
+    assert_parity(y, y_ref, dtype, "y")
+
+
+@pytest.mark.parametrize("name", ["scale1m_f16"])
 def test_scale1m_sampled(name):
-    """The 1M-token workload in the launch configuration the benchmark times:
-    one head checked in full for q and z, and 256 sampled tokens of y."""
+    """The 1M-token fp16 workload in the launch configuration the benchmark
+    times: one head checked in full for q and z, and 256 sampled tokens of y
+    (the bf16 workload is compared in full above)."""
     w = W.WORKLOADS[name]
     x = W.make_inputs(w, device=DEV)
     b = binding()
