@@ -1071,12 +1071,14 @@ struct Config {
     // latent tiles, so the next item's query tiles load during the current one)
     static constexpr int NST = NW == 3 ? (D == 64 ? 6 : 9) : (D == 128 ? (DECODE ? 3 : 4) : (D == 64 ? 4 : 6));
     static constexpr int QS = D == 128 && !DECODE ? 1 : 2;
-    // split passes on 128-column jobs: two softmax warps per row, each taking
-    // 64 of the columns (four softmax warps per SM sub-partition; measured
-    // 3-4% faster than one warp per row at the 1M-token workload).  The decode
-    // keeps three warpgroups on 64-row latent tiles: on two warpgroups with
-    // 128-row tiles and two warps per row it ran 2.0 ms against 1.52.
-    static constexpr int CS = !DECODE && KT == 128 ? 2 : 1;
+    // split passes on 128-column jobs at D = 64: two softmax warps per row,
+    // each taking 64 of the columns (four softmax warps per SM sub-partition;
+    // measured 3-4% faster than one warp per row at the 1M-token workload).
+    // At D <= 32 the column split spills registers and runs slower (40000-token
+    // cloud: split launch 0.052 against 0.042 ms), and the decode keeps three
+    // warpgroups on 64-row latent tiles (on two warpgroups with 128-row tiles
+    // and two warps per row it ran 2.0 ms against 1.52).
+    static constexpr int CS = !DECODE && KT == 128 && D == 64 ? 2 : 1;
     using SM = Smem<D, NW, KT, NST, QS, CS>;
     // at least 116 KB so that a second CTA (which would block on TMEM) never shares the SM
     static constexpr int kSmemLaunch = SM::kLaunchBytes > 118784 ? SM::kLaunchBytes : 118784;
