@@ -596,8 +596,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             const int tstep = p.interleave ? NW : 1;
             const int tfirst = p.interleave ? w : 0;
             // This warpgroup's jobs: the key/value tiles it consumes, item by item.
-            // Two cursors over the stream: `sc` issues the score MMA one job ahead
-            // of `pc`, which issues the value MMAs.
+            // One cursor over the stream issues the score MMAs one job ahead of the
+            // value MMAs; what a value MMA needs of its job (the key/value stage,
+            // whether it starts the item's accumulator) is kept from its score
+            // MMA in a two-entry record, so the issuer needs few registers.
             struct Cursor {
                 int item, t, njobs;
                 bool valid;
@@ -608,8 +610,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             // Settles on the next item (from c.item on) that has a job for this
             // warpgroup.  An item without one still takes part in freeing its
             // query slot, after the slot's load has landed (so the release is
-            // counted in the right phase); only the score cursor does that.
-            auto settle = [&](Cursor& c, bool score_cursor) {
+            // counted in the right phase).
+            auto settle = [&](Cursor& c) {
                 while (c.item < p.items) {
                     c.info = decode_item<NW, MODE>(p, c.item);
                     c.t = c.info.t_begin + tfirst;
@@ -618,7 +620,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         c.valid = true;
                         return;
                     }
-                    if (score_cursor && ok) {
+                    if (ok) {
                         const int slot = c.item_count % QS;
                         ok = mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag);
                         if (ok) umma_commit(&q_empty[slot]);
@@ -629,20 +631,20 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 }
                 c.valid = false;
             };
-            auto first = [&](Cursor& c, bool score_cursor) {
+            auto first = [&](Cursor& c) {
                 c.item = blockIdx.x;
                 c.tiles_before = 0;
                 c.item_count = 0;
-                settle(c, score_cursor);
+                settle(c);
             };
-            auto next = [&](Cursor& c, bool score_cursor) {
+            auto next = [&](Cursor& c) {
                 ++c.njobs;
                 c.t += tstep;
                 if (c.t < c.info.t_end) return;
                 c.tiles_before += c.info.t_end - c.info.t_begin;
                 ++c.item_count;
                 c.item += gridDim.x;
-                settle(c, score_cursor);
+                settle(c);
             };
             // stage and fill count of the cursor's tile: this warpgroup's own ring in
             // interleaved mode (its j-th tile), else the shared ring (global tile count)
@@ -655,7 +657,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 fill = g / NST;
                 return (int)(g % NST);
             };
-            uint32_t s_issued = 0;
+            uint32_t s_issued = 0, pv_issued = 0;
+            // the two outstanding jobs' stages and "first job of its item" flags (entry = job parity)
+            int job_st0 = 0, job_st1 = 0;
+            bool job_first0 = false, job_first1 = false;
             auto issue_s = [&](const Cursor& c) -> bool {
                 const int slot = c.item_count % QS;
                 if (c.njobs == 0 && !mbar_wait(&q_full[slot], (c.item_count / QS) & 1, abort_flag)) return false;
@@ -675,17 +680,23 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     umma_f16(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&sfull[w]);
+                if (s_issued & 1) {
+                    job_st1 = st;
+                    job_first1 = c.njobs == 0;
+                } else {
+                    job_st0 = st;
+                    job_first0 = c.njobs == 0;
+                }
                 ++s_issued;
                 // this warpgroup's last score MMA of the item releases its share of the query slot
                 if (c.t + tstep >= c.info.t_end) umma_commit(&q_empty[slot]);
                 return true;
             };
-            uint32_t pv_issued = 0;
-            auto issue_pv = [&](const Cursor& c) -> bool {
+            auto issue_pv = [&]() -> bool {
                 if (!mbar_wait(&pfull[w], pv_issued & 1, abort_flag)) return false;
                 tc_fence_after();
-                uint32_t fill;
-                const int st = stage_of(c, pv_issued, fill);
+                const int st = (pv_issued & 1) ? job_st1 : job_st0;
+                const bool first_job = (pv_issued & 1) ? job_first1 : job_first0;
                 const uint8_t* vbase = smem + SM::kKV + st * 2 * SM::kKVTileBytes + (p.kv_same ? 0 : SM::kKVTileBytes);
                 const uint32_t vaddr = smem_u32(vbase);
                 const uint32_t d_tmem = tmem + LY::kOCol + w * LY::kOStride;
@@ -698,28 +709,26 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     // (D = 128: the two 64-column blocks are the MN atoms, kKVBlockBytes apart)
                     const uint64_t bd = smem_desc(vaddr + kk * 16 * LY::kRowBytes, LY::kKVBlockBytes,
                                                   LY::kSbo, LY::kType);
-                    umma_f16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (c.njobs == 0 && kk == 0) ? 0u : 1u);
+                    umma_f16_tmem_a(d_tmem, p_tmem + kk * 8, bd, idesc_o, (first_job && kk == 0) ? 0u : 1u);
                 }
                 umma_commit(&pfree[w]);
                 ++pv_issued;
                 umma_commit(&kv_empty[st]);     // this warpgroup is done with the stage
                 return true;
             };
-            Cursor sc, pc;
-            first(sc, true);
-            first(pc, false);
+            Cursor sc;
+            first(sc);
             if (sc.valid && ok) {
                 ok = issue_s(sc);
-                next(sc, true);
+                next(sc);
             }
-            while (pc.valid && ok) {
+            while (pv_issued < s_issued && ok) {
                 if (sc.valid) {
                     ok = issue_s(sc);
                     if (!ok) break;
-                    next(sc, true);
+                    next(sc);
                 }
-                ok = issue_pv(pc);
-                next(pc, false);
+                ok = issue_pv();
             }
             // drain: wait until every issued MMA has completed before TMEM is
             // released; if that runs out, report it (the outputs are then undefined)
