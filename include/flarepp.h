@@ -238,6 +238,8 @@ const char* flarepp_status_string(int status);
 /* ---------------------------------------------------------------------------
  * Token-sharded (context-parallel) form, physicsnemo issue #2024, section 2:
  * the N tokens are split across ranks and no rank holds the whole sequence.
+ * (An extension beyond the single-GPU forward that the library's benchmark
+ * measures; the single-GPU entries above do not depend on it.)
  * Each rank runs the split softmax passes on its own tokens and reduces them
  * to one unnormalised triple (row max in log2 units, row sum, weighted sum of
  * the value rows) per latent row; the ranks' triples are all-gathered (by the
