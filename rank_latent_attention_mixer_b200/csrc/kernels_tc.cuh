@@ -223,6 +223,47 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// 16 or 8 consecutive TMEM columns of this thread's lane -> registers (the O
+// share of a row when it is narrower than 32 columns).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
+    if constexpr (N == 32) {
+        tmem_ld32(taddr, r);
+    } else if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr));
+    } else {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
+    if constexpr (N == 32) {
+        tmem_st32(taddr, r);
+    } else if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+            ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+              "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+            : "memory");
+    } else {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                     ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                       "r"(r[7])
+                     : "memory");
+    }
+}
+
 // Shared-memory matrix descriptor of tcgen05: start address, leading and
 // stride byte offsets (16-byte units), descriptor version 1, layout type.
 constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6;
@@ -439,7 +480,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
     static_assert(KT == 64 || KT == 128, "key/value tiles of 64 or 128 rows");
     static_assert(NW >= 1 && NW <= 3, "the producer warpgroup holds one TMA warp and NW MMA warps");
     static_assert(NST >= 3, "at least three key/value stages");
-    static_assert(CS == 1 || (CS == 2 && KT == 128), "score columns are split between two warps per row only in 128-column jobs");
+    static_assert(CS == 1 || CS == 2, "one or two warps per score row");
     // Interleaved mode (launch_attn refuses it unless NW divides NST): warpgroup w owns stages [w R, w R + R) and consumes them in
     // order, so no consumer can wait on a stage two fills ahead (a parity wait
     // cannot tell phase k+1 from phase k-1).  Shared mode: one ring of NST stages
@@ -748,25 +789,26 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         // ---------------------------------------------------------- softmax warpgroups
         // Softmax warpgroup g = warp / 4 serves row tile wg = g / CS and takes the
         // column share `half` = g % CS of each job: CW = KT / CS score columns, the
-        // matching CW / 2 columns of P and (D >= 64) D / CS columns of O; with
-        // D <= 32 the share 0 owns all of O.  With CS = 2 the two warps on one TMEM
+        // matching CW / 2 columns of P and D / CS columns of O.  With CS = 2 the
+        // two warps on one TMEM
         // lane quarter exchange their half-row maxima through shared memory every
         // job, so both take the weights against the same running maximum, and
         // their half-row sums at the end of an item.
         constexpr int CW = KT / CS;
         constexpr int kCChunks = CW / 32;
-        constexpr int kOChunksRow = (D + 31) / 32;
-        constexpr int kOChunks = D >= 64 ? kOChunksRow / CS : kOChunksRow;   // O chunks of an owning share
-        constexpr int kOCols = D >= 64 ? D / CS : D;                         // O values of an owning share
+        constexpr int kPSt = CW / 2 < 32 ? CW / 2 : 32;         // packed P columns per TMEM store
+        constexpr int kPChunks = CW / 2 / kPSt;
+        constexpr int kOCols = D / CS;                          // this share's O columns
+        constexpr int kOLd = kOCols < 32 ? kOCols : 32;         // O columns per TMEM load
+        constexpr int kOChunks = kOCols / kOLd;
         const int g = warp >> 2;
         const int wg = g / CS;
         const int half = g % CS;
-        const bool owns_o = D >= 64 || half == 0;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + wg * KT + half * CW;
-        const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride + (D >= 64 ? half * kOCols : 0);
+        const uint32_t tO = tmem + lane_base + LY::kOCol + wg * LY::kOStride + half * kOCols;
         const uint32_t tP = tmem + lane_base + LY::kPCol + wg * (KT / 2) + half * (CW / 2);
         const float sl2 = p.scale_log2;
         const int tstep = p.interleave ? NW : 1;
@@ -790,24 +832,22 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
             }
         };
         // Item outputs from this thread's share of its O row (o == nullptr: the
-        // warpgroup had no job in the item).  With D = 16 only the first 16 of 32
-        // loaded columns are O.
-        auto write_outputs = [&](const Item& it, int njobs, float m, float l, const uint32_t (*o)[32]) {
+        // warpgroup had no job in the item); value e of the share is o[e / kOLd][e % kOLd].
+        auto ov = [](const uint32_t (*o)[kOLd], int e) { return __uint_as_float(o[e / kOLd][e % kOLd]); };
+        auto write_outputs = [&](const Item& it, int njobs, float m, float l, const uint32_t (*o)[kOLd]) {
             if constexpr (MODE == kSplit) {
                 const int r = it.qrow0 + (p.interleave ? 0 : wg * kQTile) + row;
                 const int part = p.interleave ? it.part + wg : it.part;
                 if (r < p.M) {
                     const int64_t ridx = ((int64_t)part * p.B * p.H + it.bh) * p.M + r;
                     if (half == 0) p.part_ml[ridx] = make_float2(njobs > 0 ? m : -INFINITY, l);
-                    if (owns_o) {
-                        float4* dst = reinterpret_cast<float4*>(p.part_O + ridx * D + (D >= 64 ? half * kOCols : 0));
+                    float* dst = p.part_O + ridx * D + half * kOCols;
+                    if constexpr (kOCols >= 4) {
 #pragma unroll
                         for (int i = 0; i < kOCols / 4; ++i)
-                            dst[i] = o ? make_float4(__uint_as_float(o[i / 8][(i % 8) * 4 + 0]),
-                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 1]),
-                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 2]),
-                                                     __uint_as_float(o[i / 8][(i % 8) * 4 + 3]))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                            reinterpret_cast<float4*>(dst)[i] =
+                                o ? make_float4(ov(o, 4 * i), ov(o, 4 * i + 1), ov(o, 4 * i + 2), ov(o, 4 * i + 3))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
                 }
             } else {
@@ -817,17 +857,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const bool valid_row = n < p.N && o != nullptr;
                 const float inv = 1.f / l;
                 const int64_t off = (int64_t)(it.bh / p.H) * p.y_b + (int64_t)it.h * p.y_h + (int64_t)n * p.y_row +
-                                    (D >= 64 ? half * kOCols : 0);
-                if (valid_row && owns_o && p.y) {
+                                    half * kOCols;
+                static_assert(kOCols % 8 == 0, "16-byte stores of y");
+                if (valid_row && p.y) {
                     uint4* dst = reinterpret_cast<uint4*>(static_cast<E*>(p.y) + off);
 #pragma unroll
                     for (int i = 0; i < kOCols / 8; ++i) {
-                        const int c = i / 4, j = (i % 4) * 8;
-                        dst[i] = make_uint4(
-                            pack2<E>(__uint_as_float(o[c][j + 0]) * inv, __uint_as_float(o[c][j + 1]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 2]) * inv, __uint_as_float(o[c][j + 3]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 4]) * inv, __uint_as_float(o[c][j + 5]) * inv),
-                            pack2<E>(__uint_as_float(o[c][j + 6]) * inv, __uint_as_float(o[c][j + 7]) * inv));
+                        const int e = 8 * i;
+                        dst[i] = make_uint4(pack2<E>(ov(o, e + 0) * inv, ov(o, e + 1) * inv),
+                                            pack2<E>(ov(o, e + 2) * inv, ov(o, e + 3) * inv),
+                                            pack2<E>(ov(o, e + 4) * inv, ov(o, e + 5) * inv),
+                                            pack2<E>(ov(o, e + 6) * inv, ov(o, e + 7) * inv));
                     }
                 }
                 if (__builtin_expect(p.tok_stats != nullptr, 0)) {
@@ -835,18 +875,17 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                     // (log2 units, against the same running max as l) and <dy, y>
                     // (0 when no dy is given: a forward that saves its state)
                     float dsum = 0.f;
-                    if (valid_row && owns_o && p.dy) {
+                    if (valid_row && p.dy) {
                         const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const E*>(p.dy) + off);
 #pragma unroll
                         for (int i = 0; i < kOCols / 8; ++i) {
                             const uint4 v = g4[i];
                             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                            const int c = i / 4, j = (i % 4) * 8;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const float2 g2 = unpack2<E>(w4[e]);
-                                dsum = fmaf(g2.x, __uint_as_float(o[c][j + 2 * e]), dsum);
-                                dsum = fmaf(g2.y, __uint_as_float(o[c][j + 2 * e + 1]), dsum);
+                                dsum = fmaf(g2.x, ov(o, 8 * i + 2 * e), dsum);
+                                dsum = fmaf(g2.y, ov(o, 8 * i + 2 * e + 1), dsum);
                             }
                         }
                     }
@@ -859,12 +898,10 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
         // this share of the O row of the finished item -> outputs (every value MMA
         // of the item has completed)
         auto flush = [&](const Item& it, int njobs, float m, float l) {
-            uint32_t o[kOChunks][32];
-            if (owns_o) {
+            uint32_t o[kOChunks][kOLd];
 #pragma unroll
-                for (int c = 0; c < kOChunks; ++c) tmem_ld32(tO + c * 32, o[c]);
-                tmem_wait_ld();
-            }
+            for (int c = 0; c < kOChunks; ++c) tmem_ld_cols<kOLd>(tO + c * kOLd, o[c]);
+            tmem_wait_ld();
             write_outputs(it, njobs, m, l, o);
         };
         // Decode: the epilogue of an item (a few jobs long) is deferred into the
@@ -932,7 +969,8 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 const float2 sl2v = make_float2(sl2, sl2);
                 const float2 negm = make_float2(-m_run, -m_run);
                 float2 acc[kCChunks];
-                uint32_t pk[(CW + 63) / 64][32];          // [h][j]: this share's columns 64 h + 2 j, 2 j + 1
+                // packed weight column q (this share's columns 2 q, 2 q + 1) -> pk[q / kPSt][q % kPSt]
+                uint32_t pk[kPChunks][kPSt];
 #pragma unroll
                 for (int c = 0; c < kCChunks; ++c) {
                     acc[c] = make_float2(0.f, 0.f);
@@ -944,7 +982,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                                               ? ex2_fma_pair(xv)
                                               : make_float2(ex2_mufu(xv.x), ex2_mufu(xv.y));
                         acc[c] = __fadd2_rn(acc[c], pv);
-                        pk[c >> 1][(c & 1) * 16 + j] = pack2<E>(pv.x, pv.y);
+                        pk[(c * 16 + j) / kPSt][(c * 16 + j) % kPSt] = pack2<E>(pv.x, pv.y);
                     }
                 }
                 float2 asum = acc[0];
@@ -961,7 +999,7 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                 tc_fence_after();
                 // this share of the P row -> TMEM (this thread's lane, CW/2 columns of packed pairs)
 #pragma unroll
-                for (int h = 0; h < (CW + 63) / 64; ++h) tmem_st32(tP + h * 32, pk[h]);
+                for (int h = 0; h < kPChunks; ++h) tmem_st_cols<kPSt>(tP + h * kPSt, pk[h]);
                 // Rare work on O, after P is out of the registers and before the
                 // value MMA of this job adds to O: the previous item's O row (first
                 // job of a decode item), or the O rescale of a grown running max
@@ -972,16 +1010,16 @@ attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ C
                         pend = false;
                     }
                 }
-                if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0) && owns_o) {
+                if (__builtin_expect(__any_sync(0xffffffffu, resc && njobs > 0), 0)) {
                     const float f = njobs > 0 ? factor : 1.f;
 #pragma unroll
                     for (int c = 0; c < kOChunks; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
+                        uint32_t o[kOLd];
+                        tmem_ld_cols<kOLd>(tO + c * kOLd, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-                        tmem_st32(tO + c * 32, o);
+                        for (int j = 0; j < kOLd; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+                        tmem_st_cols<kOLd>(tO + c * kOLd, o);
                     }
                 }
                 tmem_wait_st();
@@ -1083,8 +1121,9 @@ struct Config {
     // split passes on 128-column jobs at D = 64: two softmax warps per row,
     // each taking 64 of the columns (four softmax warps per SM sub-partition;
     // measured 3-4% faster than one warp per row at the 1M-token workload).
-    // At D <= 32 the column split spills registers and runs slower (40000-token
-    // cloud: split launch 0.052 against 0.042 ms), and the decode keeps three
+    // At D <= 32 the column split (O divided between the shares, no spills)
+    // still ran 3-7% slower (40000-token cloud: split launch 0.0416 against
+    // 0.0402 ms; 16641-token grid: 0.0249 against 0.0232), and the decode keeps three
     // warpgroups on 64-row latent tiles (on two warpgroups with 128-row tiles
     // and two warps per row it ran 2.0 ms against 1.52).
     static constexpr int CS = !DECODE && KT == 128 && D == 64 ? 2 : 1;
