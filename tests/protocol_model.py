@@ -251,14 +251,14 @@ def simulate(p, grid, NST, QS, seed):
                     part = it["part"] + wg if p["interleave"] else it["part"]
                     if r < p["M"]:
                         assert part < p["parts"]
-                        keys = [("O", part, it["bh"], r, half)] if (p["D"] >= 64 or half == 0) else []
+                        keys = [("O", part, it["bh"], r, half)]          # each share its D / CS columns
                         if half == 0:
                             keys.append(("ml", part, it["bh"], r))
                         for key in keys:
                             writes[key] = writes.get(key, 0) + 1
                 else:
                     n = it["qrow0"] + wg * 128 + row
-                    if n < p["N"] and njobs > 0 and (p["D"] >= 64 or half == 0):
+                    if n < p["N"] and njobs > 0:
                         key = ("y", it["bh"], n, half)
                         writes[key] = writes.get(key, 0) + 1
 
@@ -384,8 +384,8 @@ def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, sh
             p["KT"] = KT
             p["D"] = D
             # the kernel splits the score columns between two warps per row in
-            # the split passes on 128-column jobs
-            p["CS"] = CS if CS is not None else (2 if md == "split" and KT == 128 else 1)
+            # the split passes on 128-column jobs at D = 64
+            p["CS"] = CS if CS is not None else (2 if md == "split" and KT == 128 and D == 64 else 1)
             p["shared_ring"] = shared_ring
             p["plant"] = plant
             g = min(grid, p["items"])
@@ -394,7 +394,7 @@ def check(B, H, N, M, D, grid=148, mode="both", seed=0, force_chunks=0, NW=3, sh
             for blk in range(g):
                 p["blk"] = blk
                 simulate(p, g, NST, 2, seed=blk + 7919 * seed)
-            shares = [h for h in range(p["CS"]) if D >= 64 or h == 0]
+            shares = list(range(p["CS"]))
             if md == "split":
                 exp = {("ml", pt, bh, r) for bh in range(BH) for r in range(M) for pt in range(p["parts"])}
                 exp |= {("O", pt, bh, r, h) for bh in range(BH) for r in range(M) for pt in range(p["parts"])

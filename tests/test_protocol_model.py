@@ -45,7 +45,8 @@ def test_column_shares_in_split_and_single_share_decode():
     exchange pairs the same job), the decode one; both write each output once."""
     res = check(1, 2, 1500, 384, 64, NW=2, grid=37, mode="split")
     assert res
-    check(1, 2, 1500, 384, 32, NW=2, grid=37, mode="split")      # D <= 32: share 0 owns O
+    check(1, 2, 1500, 384, 32, NW=2, grid=37, mode="split")      # D <= 32: one warp per row
+    check(1, 2, 1500, 384, 32, NW=2, grid=37, mode="split", CS=2)  # two shares at D = 32 (not launched)
     check(1, 2, 700, 64, 64, NW=2, grid=37, mode="split")        # interleaved, two shares per stream
 
 
