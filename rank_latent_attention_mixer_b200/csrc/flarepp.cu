@@ -185,7 +185,7 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
     const dim3 split_grid(pl.chunks, (unsigned)s.bh(), pl.row_blocks);
     const int64_t rows = s.bh() * s.M;
     const dim3 merge_grid((unsigned)((rows + 7) / 8));
-    const dim3 dec_grid((unsigned)((s.N + kSimtThreads - 1) / kSimtThreads), (unsigned)s.bh());
+    const dim3 dec_grid((unsigned)((s.N + simt_decode_rows(s.D) - 1) / simt_decode_rows(s.D)), (unsigned)s.bh());
 
     SplitParams sp{};
     sp.tok_row = pl.tok.row; sp.tok_h = pl.tok.h; sp.tok_b = pl.tok.b;
@@ -205,18 +205,18 @@ int run_simt(const Shape& s, const Plan& pl, const void* q0, const void* q_fixed
         ev.mark(st);                                                                               \
         if (gated) {                                                                               \
             sp.Q = q0; sp.q_batch_heads = 0; sp.K = k0; sp.V = k0;                                 \
-            split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
+            split_partial_simt<T, T, DD><<<split_grid, simt_split_threads(DD), 0, st>>>(sp);                 \
             ev.mark(st);                                                                           \
             mp.mode = kMergeSynthesis; mp.out_f32 = q32; mp.out_16 = q16; mp.user_out = q_out;   \
             mp.q_copy_out = nullptr; mp.lse_out = ex.lse_syn; mp.pregate_out = ex.qdyn;           \
             merge_partials<T, DD><<<merge_grid, 256, 0, st>>>(mp);                                 \
             ev.mark(st);                                                                           \
             sp.Q = q32; sp.q_batch_heads = s.H; sp.K = k; sp.V = v;                                \
-            split_partial_simt<float, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);             \
+            split_partial_simt<float, T, DD><<<split_grid, simt_split_threads(DD), 0, st>>>(sp);             \
             ev.mark(st);                                                                           \
         } else {                                                                                   \
             sp.Q = q_fixed; sp.q_batch_heads = 0; sp.K = k; sp.V = v;                              \
-            split_partial_simt<T, T, DD><<<split_grid, kSimtThreads, 0, st>>>(sp);                 \
+            split_partial_simt<T, T, DD><<<split_grid, simt_split_threads(DD), 0, st>>>(sp);                 \
             ev.mark(st);                                                                           \
         }                                                                                          \
         mp.mode = kMergeEncode; mp.out_f32 = z32; mp.out_16 = z16; mp.user_out = z_out;          \
@@ -640,8 +640,8 @@ int simt_cp_partials(const Shape& s, const Plan& pl, const void* q, bool q_share
     const dim3 grid(pl.chunks, (unsigned)s.bh(), pl.row_blocks);
 #define FLAREPP_CP_SPLIT(DD)                                                                       \
     case DD:                                                                                       \
-        if (q_shared) split_partial_simt<T, T, DD><<<grid, kSimtThreads, 0, st>>>(sp);             \
-        else split_partial_simt<float, T, DD><<<grid, kSimtThreads, 0, st>>>(sp);                  \
+        if (q_shared) split_partial_simt<T, T, DD><<<grid, simt_split_threads(DD), 0, st>>>(sp);             \
+        else split_partial_simt<float, T, DD><<<grid, simt_split_threads(DD), 0, st>>>(sp);                  \
         break;
     switch (s.D) {
         FLAREPP_CP_SPLIT(16)
@@ -663,7 +663,7 @@ int simt_cp_decode(const Shape& s, const Plan& pl, const void* q, bool q_shared,
     dp.B = s.B; dp.H = s.H; dp.N = s.N; dp.M = s.M;
     dp.tok_row = pl.tok.row; dp.tok_h = pl.tok.h; dp.tok_b = pl.tok.b;
     dp.scale_log2 = pl.scale_log2;
-    const dim3 grid((unsigned)((s.N + kSimtThreads - 1) / kSimtThreads), (unsigned)s.bh());
+    const dim3 grid((unsigned)((s.N + simt_decode_rows(s.D) - 1) / simt_decode_rows(s.D)), (unsigned)s.bh());
 #define FLAREPP_CP_DEC(DD)                                                                         \
     case DD:                                                                                       \
         if (q_shared) decode_simt<T, T, DD><<<grid, kSimtThreads, 0, st>>>(dp);                    \
