@@ -5,7 +5,7 @@ pipe instead of the MUFU unit: 2^x = 2^n * 2^f with n = round(x) (Cody-Waite
 range reduction, here with a single exact step since the base is 2) and
 2^f from this cubic.  The cubic is the minimax approximation of 2^f for
 RELATIVE error on [-1/2, 1/2], found by the Remez exchange algorithm below
-(fp64, numpy); its maximum relative error is about 8.8e-5, far below the
+(fp64, numpy); its maximum relative error is about 7.5e-5, far below the
 bf16 rounding (2^-9 = 2e-3) the softmax weights then take.
 
 Run `python -m rank_latent_attention_mixer_b200.exp2_poly` to print the
