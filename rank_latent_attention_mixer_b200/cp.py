@@ -39,17 +39,15 @@ def shard_bounds(N: int, ranks: int, rank: int):
 
 
 def _all_gather(t: torch.Tensor, group) -> torch.Tensor:
-    """The ranks' buffers back to back in rank order (one collective)."""
+    """The ranks' buffers back to back in rank order, flat: one
+    all_gather_into_tensor, the same call on NCCL (device buffers) and on gloo
+    (host buffers, as in the multi-process tests)."""
     if not dist.is_initialized():
-        return t
+        return t.reshape(-1)
     ranks = dist.get_world_size(group)
-    if dist.get_backend(group) == "nccl":
-        out = torch.empty(ranks * t.numel(), dtype=t.dtype, device=t.device)
-        dist.all_gather_into_tensor(out, t, group=group)
-        return out
-    parts = [torch.empty_like(t) for _ in range(ranks)]
-    dist.all_gather(parts, t, group=group)
-    return torch.cat(parts)
+    out = torch.empty(ranks * t.numel(), dtype=t.dtype, device=t.device)
+    dist.all_gather_into_tensor(out, t.contiguous().reshape(-1), group=group)
+    return out
 
 
 def _all_reduce(t: torch.Tensor, group) -> torch.Tensor:
