@@ -115,14 +115,40 @@ def load_peaks():
 KERNEL_SOURCES = {"split_partial": ["common.cuh", "kernels_tc.cuh"]}
 
 
+def code_only(src: str) -> str:
+    """C++/CUDA source without its comments, whitespace runs collapsed to one
+    space; string and character literals are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest(kernel: str = "split_partial") -> str:
-    """Digest of the source files that define a kernel (so a recorded ncu
-    traffic figure is used only for the kernel it was measured on)."""
+    """Digest of the code of the source files that define a kernel, comments
+    left out (so a recorded ncu traffic figure is used only for the code it was
+    measured on, and an edited comment does not retire it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_latent_attention_mixer_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update((name + "\n" + code_only(f.read())).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,29 +14,33 @@
 //                    key/value rows are the M latents of q and z, and the
 //                    output is the normalised y row in E.
 //
-// Per CTA (persistent, one per SM): NW softmax warpgroups and one producer
-// warpgroup, (NW + 1) x 128 threads.
-//   warps 0 .. 4NW-1   softmax warpgroup w = warp / 4 (query-row tile, TMEM lanes
-//                      32 (warp % 4) .. +31)
-//   warp  4NW          TMA producer: query tiles and a ring of key/value tiles of
-//                      KT rows
-//   warps 4NW+1 ..     one MMA issuer per softmax warpgroup w:
-//                      S_w = Q_w K^T and O_w += P_w V, into TMEM
+// Per CTA (persistent, one per SM): NW query-row tiles of 128 rows, each served
+// by CS softmax warpgroups (column shares: CS = 2 in the split passes at
+// D = 64, else 1), and one producer warpgroup, (NW CS + 1) x 128 threads.
+//   warps 0 .. 4NW CS-1  softmax warpgroup g = warp / 4 serves row tile g / CS
+//                        and column share g % CS (TMEM lanes 32 (warp % 4) .. +31)
+//   warp  4NW CS         TMA producer: query tiles and a ring of key/value tiles
+//                        of KT rows
+//   next NW warps        one MMA issuer per row tile w:
+//                        S_w = Q_w K^T and O_w += P_w V, into TMEM
 // TMEM columns: S_w at KT w, O_w at NW KT + OS w (OS = max(D, 32)), P_w (KT
 // 16-bit values = KT/2 columns) after them; NW (KT + OS + KT/2) <= 512.
-// Each softmax thread owns one query row: it reads its KT scores from TMEM,
+// Each softmax thread owns one query row (with CS = 2, KT/2 of its score
+// columns, the matching P columns and D/2 of its O columns; the two warps on a
+// lane quarter swap their half-row maxima through shared memory every job and
+// their half-row sums at the end of an item): it reads its scores from TMEM,
 // takes exponentials base 2, writes the weights P back to TMEM in E (the value
-// MMA reads its A operand from TMEM), and rescales its O row in TMEM only when
-// its running max grows by more than 2^8 (the final normalisation uses the
+// MMA reads its A operand from TMEM), and rescales its O columns in TMEM only
+// when its running max grows by more than 2^8 (the final normalisation uses the
 // same stale max, so the result is exact up to rounding).  Each MMA warp
-// issues its warpgroup's next score MMA as soon as the softmax has read the
+// issues its row tile's next score MMA as soon as the softmax has read the
 // previous scores, before that job's value MMA, so the tensor core works ahead
-// of the softmax; the warpgroups run independently.
+// of the softmax; the row tiles run independently.
 // Query tiles and key/value tiles are shared in one of two ways:
 //   * shared key/value tiles (decode, and split with one 128-latent group per
-//     warpgroup): each warpgroup has its own query tile and every warpgroup
+//     row tile): each row tile has its own query tile and every row tile
 //     consumes every key/value tile of the item;
-//   * interleaved (split otherwise): the warpgroups share one query tile and
+//   * interleaved (split with M <= 128): the row tiles share one query tile and
 //     take the item's key/value tiles round-robin, each writing its own
 //     partial triple.
 // The launch gives every thread R0 = 65536 / threads registers; the producer

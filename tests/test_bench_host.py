@@ -39,6 +39,16 @@ def test_source_digest_is_stable():
     assert b.source_digest("split_partial") == d
 
 
+def test_code_digest_ignores_comments_only():
+    b = _bench()
+    a = 'int f(int x) { // doubles\n  return 2 * x; /* no "//" here */ }\nconst char* s = "a // b";'
+    c = 'int f(int x) {\n\n  return 2 * x;   }\n// another comment\nconst char* s = "a // b";'
+    assert b.code_only(a) == b.code_only(c)
+    assert '"a // b"' in b.code_only(a)              # string literals are code
+    assert b.code_only(a) != b.code_only(a.replace("2 * x", "3 * x"))
+    assert b.code_only(a) != b.code_only(a.replace('"a // b"', '"a / b"'))
+
+
 def test_traffic_is_reported_only_for_the_recorded_sources():
     b = _bench()
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
