@@ -172,7 +172,7 @@ class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
-    def __init__(self, device_index: int, period: float = 0.05):
+    def __init__(self, device_index: int, period: float = 0.005):
         self.period = period
         self.samples = []
         self.error = None
